@@ -1,0 +1,247 @@
+/*
+ * lq.h - C ABI of liblq, the quantized linear-layer GEMM ("scaled_mm") for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What it computes
+ * ----------------
+ *   C[m, n] = bf16( sum_k dequant(A_q)[m, k] * dequant(B_q)[k, n] )
+ *
+ * in the three formats that the PyTorch blog post "Building a
+ * High-Performance and Portable vLLM Linear Backend with Helion" defines in
+ * its section "Helion Linear Backend > Scope":
+ *
+ *   LQ_FP8_DYNAMIC : e4m3 codes, one fp32 scale per token (row of A) and one
+ *                    per output channel (row n of the stored weight);
+ *   LQ_W8A8_INT8   : int8 codes, the same scale granularity, int32 sums;
+ *   LQ_BLOCK_FP8   : e4m3 codes, one activation scale per 1x128 K-group and
+ *                    one weight scale per 128x128 (n, k) block.
+ *
+ * The algorithmic variants Standard, Split-K and Swap-AB of the same page's
+ * section "Kernel Implementation" are selected per call by an lq_variant (or
+ * by the dispatch table when the caller passes NULL); every variant computes
+ * the same C.
+ *
+ * Conventions shared by all entry points
+ * --------------------------------------
+ *  - Every pointer argument except file paths and lq_variant* is a DEVICE
+ *    pointer of the current CUDA device, owned by the caller.  Arrays are
+ *    dense and row-major with the shapes given below.
+ *  - A is [M, K], one row per token.  B is stored [N, K] (one row per output
+ *    channel, K contiguous), i.e. the pages' logical b[k, n] transposed, as a
+ *    linear layer stores its weight.  C is [M, N] bf16.
+ *  - e4m3 codes are OCP E4M3 "fn" bytes; int8 codes are two's complement.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and never synchronise.  They may be captured into a
+ *    CUDA graph once the device has been initialised (lq_init_device, or any
+ *    earlier non-captured call on that device).
+ *  - All arguments are checked before anything is launched; a failed check
+ *    launches nothing and returns an error code.  No C++ exception crosses
+ *    this interface.
+ *  - The library allocates device memory only in lq_init_device,
+ *    lq_reserve_workspace and, outside stream capture, when a Split-K call
+ *    needs more workspace than it holds.
+ */
+#ifndef LQ_H_
+#define LQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, spelled without the CUDA headers. */
+typedef struct CUstream_st *lq_stream_t;
+
+typedef enum {
+  LQ_FP8_DYNAMIC = 0,
+  LQ_W8A8_INT8 = 1,
+  LQ_BLOCK_FP8 = 2
+} lq_fmt;
+
+typedef enum {
+  LQ_OK = 0,
+  LQ_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, bad variant field */
+  LQ_ERR_ALIGNMENT = 2,         /* a pointer is not aligned as required      */
+  LQ_ERR_UNSUPPORTED_SHAPE = 3, /* a size breaks a divisibility/limit rule   */
+  LQ_ERR_WORKSPACE = 4,         /* Split-K workspace would have to grow during
+                                   stream capture, or allocation failed      */
+  LQ_ERR_CUDA = 5,              /* a CUDA runtime/driver call failed          */
+  LQ_ERR_DEVICE_TIMEOUT = 6,    /* a kernel gave up on a bounded wait         */
+  LQ_ERR_TABLE = 7              /* dispatch table file missing or malformed   */
+} lq_status;
+
+/*
+ * One point of the variant space (the blog's tunables split_k and swap_ab,
+ * plus the tile and pipeline choices of this implementation).
+ *
+ *  swap_ab : 0 = Standard: tokens on the tensor-core M side (128-row tiles of
+ *            A), weights on the N side (tile_n rows of B per tile);
+ *            1 = Swap-AB: C^T = B . A^T is computed, 128 weight rows on the M
+ *            side and tile_n tokens on the N side; the epilogue transposes
+ *            back on store.
+ *  split_k : 1, 2, 4, ..., 256.  Split s owns the 128-wide K tiles
+ *            [floor(s*T/S), floor((s+1)*T/S)), T = ceil(K/128); a split may
+ *            be empty.  Partials are summed in the fixed order s = 0..S-1,
+ *            so results are reproducible bit for bit.
+ *  tile_n  : Standard: 64, 128 or 256 (Block_FP8: 64 or 128);
+ *            Swap-AB: 16, 32 or 64.
+ *  stages  : depth of the shared-memory ring (2..16), 0 = the deepest that
+ *            fits.
+ *  reduce  : for split_k > 1: 0 = a separate reduction kernel, 1 = the last
+ *            CTA to finish a tile reduces it (arrival counter).
+ *  pdl     : 0 = plain launch;
+ *            1 = programmatic dependent launch: the kernel's set-up overlaps
+ *            the tail of the previous kernel on the stream, and all of its
+ *            global-memory accesses wait until that kernel has completed;
+ *            2 = as 1, and the first weight tiles (B) are streamed before
+ *            that wait.  With 2 the caller guarantees that B and b_scales
+ *            are not being written by any kernel that may still be running
+ *            when the call is launched (true of model weights, which are
+ *            written once before inference).
+ */
+typedef struct {
+  int32_t swap_ab;
+  int32_t split_k;
+  int32_t tile_n;
+  int32_t stages;
+  int32_t reduce;
+  int32_t pdl;
+} lq_variant;
+
+/*
+ * scaled_mm: C = dequant(A) . dequant(B)^T in bf16 (round to nearest even).
+ *
+ * Defined by: PyTorch blog "Building a High-Performance and Portable vLLM
+ * Linear Backend with Helion", sections "Helion Linear Backend > Scope"
+ * (formats, scale granularity) and "Kernel Implementation" (variants).
+ *
+ *   fmt      : LQ_FP8_DYNAMIC, LQ_W8A8_INT8 or LQ_BLOCK_FP8.
+ *   A        : [M, K] codes (uint8 e4m3 or int8), 16-byte aligned.
+ *   a_scales : fp32; [M] for FP8_DYNAMIC/W8A8_INT8, [M, K/128] for BLOCK_FP8.
+ *   B        : [N, K] codes, 16-byte aligned.
+ *   b_scales : fp32; [N] for FP8_DYNAMIC/W8A8_INT8, [N/128, K/128] for
+ *              BLOCK_FP8.
+ *   C        : [M, N] bf16 output, 16-byte aligned.
+ *   M, N, K  : M >= 0, N >= 0, K >= 0; K % 16 == 0 and N % 8 == 0;
+ *              BLOCK_FP8 also needs K % 128 == 0 and N % 128 == 0.
+ *              M == 0 or N == 0 is a no-op; K == 0 writes C = 0.
+ *   variant  : NULL = the dispatch table's choice for (fmt, M, N, K).
+ *   stream   : CUDA stream.
+ *
+ * Errors: LQ_ERR_INVALID_ARG / LQ_ERR_ALIGNMENT / LQ_ERR_UNSUPPORTED_SHAPE
+ * before any launch; LQ_ERR_WORKSPACE when split_k > 1 needs a larger
+ * workspace while `stream` is capturing; LQ_ERR_CUDA when a launch fails.
+ * A Split-K call uses the library's per-device workspace: Split-K calls on
+ * different streams of one device must not overlap in time.
+ */
+lq_status lq_scaled_mm(lq_fmt fmt, const void *A, const float *a_scales,
+                       const void *B, const float *b_scales, void *C,
+                       int64_t M, int64_t N, int64_t K,
+                       const lq_variant *variant, lq_stream_t stream);
+
+/*
+ * Test hook for W8A8_INT8: as lq_scaled_mm(LQ_W8A8_INT8, ...) and also
+ * writes the exact int32 accumulator sum_k A[m,k]*B[n,k] to acc_out [M, N]
+ * (device, 16-byte aligned), so that it can be compared bit for bit with an
+ * exact integer reference.  Same arguments and errors as lq_scaled_mm.
+ */
+lq_status lq_scaled_mm_i32acc(const void *A, const float *a_scales,
+                              const void *B, const float *b_scales, void *C,
+                              int32_t *acc_out, int64_t M, int64_t N, int64_t K,
+                              const lq_variant *variant, lq_stream_t stream);
+
+/*
+ * Dynamic per-token activation quantization (the blog's integrated kernel
+ * dynamic_per_token_scaled_fp8_quant, as listed in the 24-ai.news report,
+ * section "kernels integrated into vLLM"; the int8 form serves W8A8_INT8).
+ *
+ *   fmt    : LQ_FP8_DYNAMIC (e4m3, Q = 448) or LQ_W8A8_INT8 (int8, Q = 127).
+ *   x      : [M, K] bf16, 16-byte aligned.
+ *   q      : [M, K] codes out, 8-byte aligned.
+ *   scales : [M] fp32 out.  s = max(fp32(amax_row / Q), 2^-126),
+ *            q = encode(fp32(x / s)) with a correctly rounded division,
+ *            e4m3 round-to-nearest-even with saturation to +-448, int8
+ *            round-half-even clamped to +-127.
+ *   K % 16 == 0.  M == 0 is a no-op.
+ * The same call quantizes a weight [N, K] per output channel.
+ */
+lq_status lq_quant_per_token(lq_fmt fmt, const void *x, void *q, float *scales,
+                             int64_t M, int64_t K, lq_stream_t stream);
+
+/*
+ * 1x128 group quantization of Block_FP8 activations (the blog's
+ * per_token_group_fp8_quant): one scale per (row, 128-wide K group).
+ *   x [M, K] bf16 (16-byte aligned) -> q [M, K] e4m3, scales [M, K/128] fp32.
+ *   K % 128 == 0.  Same rule as lq_quant_per_token with Q = 448.
+ */
+lq_status lq_quant_per_token_group128(const void *x, void *q, float *scales,
+                                      int64_t M, int64_t K, lq_stream_t stream);
+
+/*
+ * 128x128 block quantization of a Block_FP8 weight stored [N, K]: one scale
+ * per (n-block, k-block) from the amax over the whole block.
+ *   w [N, K] bf16 (16-byte aligned) -> q [N, K] e4m3, scales [N/128, K/128].
+ *   N % 128 == 0 and K % 128 == 0.
+ */
+lq_status lq_quant_weight_block128(const void *w, void *q, float *scales,
+                                   int64_t N, int64_t K, lq_stream_t stream);
+
+/*
+ * The variant that lq_scaled_mm uses for (fmt, M, N, K) when given NULL:
+ * the dispatch-table entry for the token bucket of M (the next of
+ * 1,2,4,8,16,24,32, then powers of two), else a built-in heuristic.
+ * Host-only; writes *out.  Errors: LQ_ERR_INVALID_ARG.
+ */
+lq_status lq_select_variant(lq_fmt fmt, int64_t M, int64_t N, int64_t K,
+                            lq_variant *out);
+
+/*
+ * Replace the dispatch table by the entries of a text file (one entry per
+ * line: "fmt m_bucket N K swap_ab split_k tile_n stages reduce pdl", '#'
+ * starts a comment).  path == NULL restores the compiled-in table.  On error
+ * the current table is kept and LQ_ERR_TABLE is returned.  Not thread-safe
+ * with concurrent lq_scaled_mm calls that pass variant == NULL.
+ */
+lq_status lq_load_dispatch_table(const char *path);
+
+/* Number of entries in the current dispatch table. */
+int64_t lq_dispatch_table_size(void);
+
+/*
+ * Create the per-device state of `device` (status word, Split-K arrival
+ * counters) if it does not exist yet.  Call it before capturing a CUDA graph
+ * that contains lq calls.  Errors: LQ_ERR_CUDA.
+ */
+lq_status lq_init_device(int device);
+
+/*
+ * Make sure the per-device Split-K workspace holds at least `bytes` bytes
+ * (a Split-K call needs split_k * M * N * 4).  Synchronises the device when
+ * it has to replace a smaller workspace.  Call it before stream capture.
+ */
+lq_status lq_reserve_workspace(int device, size_t bytes);
+
+/* Workspace bytes that lq_scaled_mm needs for (fmt, M, N, K, variant). */
+size_t lq_workspace_bytes(lq_fmt fmt, int64_t M, int64_t N, int64_t K,
+                          const lq_variant *variant);
+
+/*
+ * Read and clear the device status word of `device`: LQ_OK, or
+ * LQ_ERR_DEVICE_TIMEOUT if a kernel since the last read gave up on a
+ * bounded wait (its output is then undefined).  Synchronises the device.
+ */
+lq_status lq_device_status(int device);
+
+/* Human-readable name of a status code (static storage). */
+const char *lq_status_string(lq_status status);
+
+/* Library version string (static storage). */
+const char *lq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LQ_H_ */

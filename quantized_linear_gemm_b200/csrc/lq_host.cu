@@ -1,0 +1,559 @@
+// Host side of liblq: argument checks, variant selection (dispatch table +
+// heuristic), per-device state (status word, Split-K workspace and arrival
+// counters), TMA descriptor encoding and kernel launches.
+//
+// The variant space is the one of the blog's unified GEMM (PyTorch blog
+// "Building a High-Performance and Portable vLLM Linear Backend with Helion",
+// "Kernel Implementation": tunables split_k in {1, 2, ..., 256} and swap_ab),
+// extended by the tile / pipeline choices of this implementation.  Instead of
+// an online autotuner the library reads a static table keyed by
+// (format, token bucket, N, K) that an offline on-device sweep writes; the
+// token buckets are the decode sizes 1, 2, 4, 8, 16, 24, 32 for which the
+// techfeed.io summary of the blog (section on hybrid dispatch, Fig. 2) says
+// configs are tuned, followed by powers of two for larger M.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cerrno>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <fstream>
+#include <memory>
+#include <mutex>
+#include <sstream>
+#include <string>
+#include <vector>
+
+#include "../../include/lq.h"
+#include "lq_kernels.h"
+
+namespace {
+
+using lq::GemmLaunch;
+using lq::GemmParams;
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxSmemPerCta = 227 * 1024;
+constexpr size_t kCounterCapacity = size_t(1) << 20;   // Split-K arrival counters per device
+constexpr int kNumSms = 148;
+
+// ---------------------------------------------------------------- devices
+struct DeviceState {
+  bool ready = false;
+  int* status = nullptr;       // one int, bit i set when wait site i timed out
+  int* counters = nullptr;     // kCounterCapacity ints, zero between calls
+  void* ws = nullptr;          // Split-K partials
+  size_t ws_bytes = 0;
+};
+
+std::mutex g_dev_mutex;
+DeviceState g_dev[kMaxDevices];
+
+uint64_t wait_limit_ns() {
+  static uint64_t v = [] {
+    const char* e = std::getenv("LQ_WAIT_LIMIT_NS");
+    if (e && *e) {
+      char* end = nullptr;
+      unsigned long long x = std::strtoull(e, &end, 10);
+      if (end != e && x > 0) return static_cast<uint64_t>(x);
+    }
+    return static_cast<uint64_t>(2000000000ull);   // 2 s
+  }();
+  return v;
+}
+
+bool stream_capturing(cudaStream_t s) {
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &st) != cudaSuccess) return false;
+  return st != cudaStreamCaptureStatusNone;
+}
+
+lq_status init_device_locked(int dev) {
+  DeviceState& d = g_dev[dev];
+  if (d.ready) return LQ_OK;
+  int prev = 0;
+  if (cudaGetDevice(&prev) != cudaSuccess) return LQ_ERR_CUDA;
+  if (cudaSetDevice(dev) != cudaSuccess) return LQ_ERR_CUDA;
+  lq_status rc = LQ_OK;
+  if (cudaMalloc(&d.status, sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&d.counters, kCounterCapacity * sizeof(int)) != cudaSuccess ||
+      cudaMemset(d.status, 0, sizeof(int)) != cudaSuccess ||
+      cudaMemset(d.counters, 0, kCounterCapacity * sizeof(int)) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
+    rc = LQ_ERR_CUDA;
+  } else {
+    d.ready = true;
+  }
+  cudaSetDevice(prev);
+  return rc;
+}
+
+// The state of the current device, created on first use (refused while the
+// stream is being captured, since creation allocates and synchronises).
+lq_status device_state(cudaStream_t stream, DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return LQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mutex);
+  if (!g_dev[dev].ready) {
+    if (stream_capturing(stream)) return LQ_ERR_WORKSPACE;
+    lq_status rc = init_device_locked(dev);
+    if (rc != LQ_OK) return rc;
+  }
+  *out = &g_dev[dev];
+  return LQ_OK;
+}
+
+lq_status ensure_workspace(DeviceState* d, size_t bytes, cudaStream_t stream) {
+  if (bytes <= d->ws_bytes) return LQ_OK;
+  if (stream_capturing(stream)) return LQ_ERR_WORKSPACE;
+  if (d->ws) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return LQ_ERR_CUDA;
+    cudaFree(d->ws);
+    d->ws = nullptr;
+    d->ws_bytes = 0;
+  }
+  const size_t rounded = (bytes + (size_t(1) << 21) - 1) & ~((size_t(1) << 21) - 1);
+  if (cudaMalloc(&d->ws, rounded) != cudaSuccess) {
+    cudaGetLastError();
+    return LQ_ERR_WORKSPACE;
+  }
+  d->ws_bytes = rounded;
+  return LQ_OK;
+}
+
+// ---------------------------------------------------------- TMA encoding
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// K-major operand [rows, K] of bytes, tiles of box_rows x 128 bytes with the
+// 128-byte swizzle; out-of-range rows / K are zero-filled by the TMA unit.
+bool encode_operand(CUtensorMap* map, const void* ptr, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// --------------------------------------------------------- dispatch table
+struct TableEntry {
+  int fmt;
+  int64_t m_bucket, N, K;
+  lq_variant v;
+};
+
+#include "dispatch_table.inc"   // kDefaultTable[], kDefaultTableSize
+
+std::shared_ptr<const std::vector<TableEntry>> default_table() {
+  auto t = std::make_shared<std::vector<TableEntry>>();
+  for (size_t i = 0; i < kDefaultTableSize; ++i) t->push_back(kDefaultTable[i]);
+  return t;
+}
+
+std::shared_ptr<const std::vector<TableEntry>>& table_slot() {
+  static std::shared_ptr<const std::vector<TableEntry>> t = default_table();
+  return t;
+}
+std::mutex g_table_mutex;
+
+std::shared_ptr<const std::vector<TableEntry>> current_table() {
+  std::lock_guard<std::mutex> lk(g_table_mutex);
+  return table_slot();
+}
+
+int64_t m_bucket(int64_t M) {
+  static const int64_t pts[] = {1, 2, 4, 8, 16, 24, 32};
+  for (int64_t p : pts)
+    if (M <= p) return p;
+  int64_t b = 64;
+  while (b < M && b < (int64_t(1) << 40)) b <<= 1;
+  return b;
+}
+
+// Deepest ring that fits when `ctas_per_sm` CTAs share one SM's shared memory.
+int max_stages_fit(int tile_n, int ctas_per_sm) {
+  const int share = (228 * 1024) / ctas_per_sm - 1024;
+  const int budget = share < kMaxSmemPerCta ? share : kMaxSmemPerCta;
+  int best = 2;
+  for (int s = 2; s <= 16; ++s)
+    if (lq::gemm_smem_bytes_for(tile_n, s) <= budget) best = s;
+  return best;
+}
+
+lq_variant heuristic_variant(int fmt, int64_t M, int64_t N, int64_t K) {
+  lq_variant v{};
+  const int64_t T = (K + 127) / 128;
+  v.reduce = 1;
+  v.pdl = 1;
+  if (M <= 64) {
+    v.swap_ab = 1;
+    v.tile_n = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    const int64_t tiles = ((N + 127) / 128) * ((M + v.tile_n - 1) / v.tile_n);
+    int S = 1;
+    while (S < 256 && tiles * S * 2 <= 2 * kNumSms && T / (S * 2) >= 2) S *= 2;
+    v.split_k = S;
+    const int per_split = static_cast<int>((T + S - 1) / S);
+    const int cap = max_stages_fit(v.tile_n, 2);
+    v.stages = per_split < 2 ? 2 : (per_split > cap ? cap : per_split);
+  } else {
+    v.swap_ab = 0;
+    v.tile_n = fmt == lq::kFmtBlock ? 128 : 256;
+    const int64_t tiles = ((M + 127) / 128) * ((N + v.tile_n - 1) / v.tile_n);
+    int S = 1;
+    while (S < 256 && tiles * S < kNumSms && T / (S * 2) >= 4) S *= 2;
+    v.split_k = S;
+    v.stages = max_stages_fit(v.tile_n, 1);
+  }
+  return v;
+}
+
+bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, lq_variant* out) {
+  auto t = current_table();
+  const int64_t mb = m_bucket(M);
+  for (const TableEntry& e : *t) {
+    if (e.fmt == fmt && e.m_bucket == mb && e.N == N && e.K == K) {
+      *out = e.v;
+      return true;
+    }
+  }
+  return false;
+}
+
+// --------------------------------------------------------------- checks
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+lq_status check_variant(int fmt, const lq_variant& v) {
+  if (v.swap_ab != 0 && v.swap_ab != 1) return LQ_ERR_INVALID_ARG;
+  if (!is_pow2(v.split_k) || v.split_k > 256) return LQ_ERR_INVALID_ARG;
+  if (v.reduce != 0 && v.reduce != 1) return LQ_ERR_INVALID_ARG;
+  if (v.pdl < 0 || v.pdl > 2) return LQ_ERR_INVALID_ARG;
+  if (v.swap_ab) {
+    if (v.tile_n != 16 && v.tile_n != 32 && v.tile_n != 64) return LQ_ERR_INVALID_ARG;
+  } else {
+    if (v.tile_n != 64 && v.tile_n != 128 && v.tile_n != 256) return LQ_ERR_INVALID_ARG;
+    if (fmt == lq::kFmtBlock && v.tile_n == 256) return LQ_ERR_INVALID_ARG;
+  }
+  if (v.stages != 0 && (v.stages < 2 || v.stages > 16)) return LQ_ERR_INVALID_ARG;
+  if (v.stages != 0 && lq::gemm_smem_bytes_for(v.tile_n, v.stages) > kMaxSmemPerCta) return LQ_ERR_INVALID_ARG;
+  return LQ_OK;
+}
+
+lq_status check_gemm_args(int fmt, const void* A, const float* a_s, const void* B, const float* b_s, const void* C,
+                          int64_t M, int64_t N, int64_t K) {
+  if (fmt < 0 || fmt > 2) return LQ_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return LQ_OK;
+  if (!C) return LQ_ERR_INVALID_ARG;
+  if (!aligned(C, 16)) return LQ_ERR_ALIGNMENT;
+  if (K == 0) return LQ_OK;
+  if (!A || !B || !a_s || !b_s) return LQ_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(B, 16)) return LQ_ERR_ALIGNMENT;
+  if (!aligned(a_s, 4) || !aligned(b_s, 4)) return LQ_ERR_ALIGNMENT;
+  if (K % 16 != 0 || N % 8 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (fmt == lq::kFmtBlock && (K % 128 != 0 || N % 128 != 0)) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1)
+    return LQ_ERR_UNSUPPORTED_SHAPE;
+  return LQ_OK;
+}
+
+lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B, const float* b_s, void* C,
+                         int32_t* acc_out, int64_t M, int64_t N, int64_t K, const lq_variant* variant,
+                         cudaStream_t stream) {
+  lq_status rc = check_gemm_args(fmt, A, a_s, B, b_s, C, M, N, K);
+  if (rc != LQ_OK) return rc;
+  if (acc_out && !aligned(acc_out, 16)) return LQ_ERR_ALIGNMENT;
+  if (M == 0 || N == 0) return LQ_OK;
+  if (K == 0) {
+    if (acc_out && cudaMemsetAsync(acc_out, 0, static_cast<size_t>(M * N) * sizeof(int32_t), stream) != cudaSuccess)
+      return LQ_ERR_CUDA;
+    return lq::launch_fill_zero_bf16(static_cast<__nv_bfloat16*>(C), M * N, stream) == cudaSuccess ? LQ_OK
+                                                                                                  : LQ_ERR_CUDA;
+  }
+  lq_variant v{};
+  if (variant) {
+    v = *variant;
+  } else if (!lookup_table(fmt, M, N, K, &v)) {
+    v = heuristic_variant(fmt, M, N, K);
+  }
+  rc = check_variant(fmt, v);
+  if (rc != LQ_OK) return rc;
+  if (v.stages == 0) v.stages = max_stages_fit(v.tile_n, 1);
+
+  const int64_t x_rows = v.swap_ab ? N : M;
+  const int64_t y_rows = v.swap_ab ? M : N;
+  const int64_t gx = (x_rows + 127) / 128;
+  const int64_t gy = (y_rows + v.tile_n - 1) / v.tile_n;
+  if (gy > 65535 || gx > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+
+  DeviceState* d = nullptr;
+  rc = device_state(stream, &d);
+  if (rc != LQ_OK) return rc;
+
+  GemmLaunch l;
+  std::memset(&l, 0, sizeof(l));
+  GemmParams& p = l.p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.T = static_cast<int>((K + 127) / 128);
+  p.KB = static_cast<int>(K / 128);
+  p.S = v.split_k;
+  p.stages = v.stages;
+  p.reduce_in_kernel = v.reduce;
+  p.early_weights = v.pdl == 2 ? 1 : 0;
+  p.a_s = a_s;
+  p.b_s = b_s;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.acc_out = acc_out;
+  p.status = d->status;
+  p.wait_limit_ns = wait_limit_ns();
+  if (v.split_k > 1) {
+    const size_t need = static_cast<size_t>(v.split_k) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
+    rc = ensure_workspace(d, need, stream);
+    if (rc != LQ_OK) return rc;
+    if (static_cast<size_t>(gx * gy) > kCounterCapacity) return LQ_ERR_UNSUPPORTED_SHAPE;
+    p.ws = d->ws;
+    p.counters = d->counters;
+  }
+  const void* x_ptr = v.swap_ab ? B : A;
+  const void* y_ptr = v.swap_ab ? A : B;
+  if (!encode_operand(&l.tmX, x_ptr, x_rows, K, 128) || !encode_operand(&l.tmY, y_ptr, y_rows, K, v.tile_n))
+    return LQ_ERR_CUDA;
+  l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
+  l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages);
+  l.pdl = v.pdl != 0;
+  l.stream = stream;
+
+  cudaError_t e;
+  switch (fmt) {
+    case lq::kFmtFp8: e = lq::launch_scaled_mm_fp8(l, v.swap_ab, v.tile_n); break;
+    case lq::kFmtInt8: e = lq::launch_scaled_mm_int8(l, v.swap_ab, v.tile_n); break;
+    default: e = lq::launch_scaled_mm_block(l, v.swap_ab, v.tile_n); break;
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return LQ_ERR_CUDA;
+  }
+  if (v.split_k > 1 && !v.reduce) {
+    e = lq::launch_splitk_reduce(fmt, p, v.pdl != 0, stream);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return LQ_ERR_CUDA;
+    }
+  }
+  return LQ_OK;
+}
+
+bool parse_table_file(const char* path, std::vector<TableEntry>* out, std::string* err) {
+  std::ifstream f(path);
+  if (!f) {
+    *err = "cannot open";
+    return false;
+  }
+  std::string line;
+  int lineno = 0;
+  while (std::getline(f, line)) {
+    ++lineno;
+    const size_t hash = line.find('#');
+    if (hash != std::string::npos) line.resize(hash);
+    std::istringstream is(line);
+    std::string fmt_s;
+    if (!(is >> fmt_s)) continue;
+    TableEntry e{};
+    if (fmt_s == "fp8_dynamic" || fmt_s == "0") e.fmt = 0;
+    else if (fmt_s == "w8a8_int8" || fmt_s == "1") e.fmt = 1;
+    else if (fmt_s == "block_fp8" || fmt_s == "2") e.fmt = 2;
+    else {
+      *err = "bad format at line " + std::to_string(lineno);
+      return false;
+    }
+    long long mb, n, k;
+    int sw, sk, tn, st, rd, pdl;
+    if (!(is >> mb >> n >> k >> sw >> sk >> tn >> st >> rd >> pdl)) {
+      *err = "short entry at line " + std::to_string(lineno);
+      return false;
+    }
+    e.m_bucket = mb;
+    e.N = n;
+    e.K = k;
+    e.v = lq_variant{sw, sk, tn, st, rd, pdl};
+    if (check_variant(e.fmt, e.v) != LQ_OK) {
+      *err = "invalid variant at line " + std::to_string(lineno);
+      return false;
+    }
+    out->push_back(e);
+  }
+  return true;
+}
+
+}  // namespace
+
+// ======================================================================
+extern "C" {
+
+const char* lq_status_string(lq_status s) {
+  switch (s) {
+    case LQ_OK: return "LQ_OK";
+    case LQ_ERR_INVALID_ARG: return "LQ_ERR_INVALID_ARG";
+    case LQ_ERR_ALIGNMENT: return "LQ_ERR_ALIGNMENT";
+    case LQ_ERR_UNSUPPORTED_SHAPE: return "LQ_ERR_UNSUPPORTED_SHAPE";
+    case LQ_ERR_WORKSPACE: return "LQ_ERR_WORKSPACE";
+    case LQ_ERR_CUDA: return "LQ_ERR_CUDA";
+    case LQ_ERR_DEVICE_TIMEOUT: return "LQ_ERR_DEVICE_TIMEOUT";
+    case LQ_ERR_TABLE: return "LQ_ERR_TABLE";
+  }
+  return "LQ_ERR_UNKNOWN";
+}
+
+const char* lq_version(void) { return "lq 0.1.0 (sm_100a)"; }
+
+lq_status lq_scaled_mm(lq_fmt fmt, const void* A, const float* a_scales, const void* B, const float* b_scales,
+                       void* C, int64_t M, int64_t N, int64_t K, const lq_variant* variant, lq_stream_t stream) {
+  return scaled_mm_impl(static_cast<int>(fmt), A, a_scales, B, b_scales, C, nullptr, M, N, K, variant,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+lq_status lq_scaled_mm_i32acc(const void* A, const float* a_scales, const void* B, const float* b_scales, void* C,
+                              int32_t* acc_out, int64_t M, int64_t N, int64_t K, const lq_variant* variant,
+                              lq_stream_t stream) {
+  if (!acc_out && M > 0 && N > 0) return LQ_ERR_INVALID_ARG;
+  return scaled_mm_impl(lq::kFmtInt8, A, a_scales, B, b_scales, C, acc_out, M, N, K, variant,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+lq_status lq_quant_per_token(lq_fmt fmt, const void* x, void* q, float* scales, int64_t M, int64_t K,
+                             lq_stream_t stream) {
+  if (fmt != LQ_FP8_DYNAMIC && fmt != LQ_W8A8_INT8) return LQ_ERR_INVALID_ARG;
+  if (M < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (M == 0) return LQ_OK;
+  if (!x || !q || !scales) return LQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 8) || !aligned(scales, 4)) return LQ_ERR_ALIGNMENT;
+  if (K % 16 != 0 || M > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+  return lq::launch_quant_per_token(static_cast<int>(fmt), x, q, scales, M, K,
+                                    reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LQ_OK
+             : LQ_ERR_CUDA;
+}
+
+lq_status lq_quant_per_token_group128(const void* x, void* q, float* scales, int64_t M, int64_t K,
+                                      lq_stream_t stream) {
+  if (M < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (M == 0 || K == 0) return LQ_OK;
+  if (!x || !q || !scales) return LQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 8) || !aligned(scales, 4)) return LQ_ERR_ALIGNMENT;
+  if (K % 128 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if ((M * (K / 128) + 15) / 16 > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+  return lq::launch_quant_group128(x, q, scales, M, K, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LQ_OK
+             : LQ_ERR_CUDA;
+}
+
+lq_status lq_quant_weight_block128(const void* w, void* q, float* scales, int64_t N, int64_t K,
+                                   lq_stream_t stream) {
+  if (N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (N == 0 || K == 0) return LQ_OK;
+  if (!w || !q || !scales) return LQ_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(q, 8) || !aligned(scales, 4)) return LQ_ERR_ALIGNMENT;
+  if (N % 128 != 0 || K % 128 != 0 || N / 128 > 65535 || K / 128 > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+  return lq::launch_quant_weight_block128(w, q, scales, N, K, reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? LQ_OK
+             : LQ_ERR_CUDA;
+}
+
+lq_status lq_select_variant(lq_fmt fmt, int64_t M, int64_t N, int64_t K, lq_variant* out) {
+  if (!out || fmt < 0 || fmt > 2 || M < 0 || N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (!lookup_table(static_cast<int>(fmt), M, N, K, out)) *out = heuristic_variant(static_cast<int>(fmt), M, N, K);
+  return LQ_OK;
+}
+
+lq_status lq_load_dispatch_table(const char* path) {
+  if (!path) {
+    std::lock_guard<std::mutex> lk(g_table_mutex);
+    table_slot() = default_table();
+    return LQ_OK;
+  }
+  auto t = std::make_shared<std::vector<TableEntry>>();
+  std::string err;
+  if (!parse_table_file(path, t.get(), &err)) return LQ_ERR_TABLE;
+  std::lock_guard<std::mutex> lk(g_table_mutex);
+  table_slot() = t;
+  return LQ_OK;
+}
+
+int64_t lq_dispatch_table_size(void) { return static_cast<int64_t>(current_table()->size()); }
+
+lq_status lq_init_device(int device) {
+  if (device < 0 || device >= kMaxDevices) return LQ_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_dev_mutex);
+  return init_device_locked(device);
+}
+
+lq_status lq_reserve_workspace(int device, size_t bytes) {
+  if (device < 0 || device >= kMaxDevices) return LQ_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_dev_mutex);
+  lq_status rc = init_device_locked(device);
+  if (rc != LQ_OK) return rc;
+  int prev = 0;
+  if (cudaGetDevice(&prev) != cudaSuccess || cudaSetDevice(device) != cudaSuccess) return LQ_ERR_CUDA;
+  rc = ensure_workspace(&g_dev[device], bytes, nullptr);
+  cudaSetDevice(prev);
+  return rc;
+}
+
+size_t lq_workspace_bytes(lq_fmt fmt, int64_t M, int64_t N, int64_t K, const lq_variant* variant) {
+  if (M <= 0 || N <= 0 || K <= 0 || fmt < 0 || fmt > 2) return 0;
+  lq_variant v{};
+  if (variant) v = *variant;
+  else if (!lookup_table(static_cast<int>(fmt), M, N, K, &v)) v = heuristic_variant(static_cast<int>(fmt), M, N, K);
+  if (v.split_k <= 1) return 0;
+  return static_cast<size_t>(v.split_k) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
+}
+
+lq_status lq_device_status(int device) {
+  if (device < 0 || device >= kMaxDevices) return LQ_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_dev_mutex);
+  DeviceState& d = g_dev[device];
+  if (!d.ready) return LQ_OK;
+  int prev = 0;
+  if (cudaGetDevice(&prev) != cudaSuccess || cudaSetDevice(device) != cudaSuccess) return LQ_ERR_CUDA;
+  int word = 0;
+  lq_status rc = LQ_OK;
+  if (cudaDeviceSynchronize() != cudaSuccess || cudaMemcpy(&word, d.status, sizeof(int), cudaMemcpyDeviceToHost) !=
+                                                    cudaSuccess ||
+      cudaMemset(d.status, 0, sizeof(int)) != cudaSuccess) {
+    rc = LQ_ERR_CUDA;
+  } else if (word != 0) {
+    // A CTA that gave up did not count itself: clear the Split-K arrival
+    // counters so that later calls start from zero.
+    cudaMemset(d.counters, 0, kCounterCapacity * sizeof(int));
+    cudaDeviceSynchronize();
+    rc = LQ_ERR_DEVICE_TIMEOUT;
+  }
+  cudaSetDevice(prev);
+  return rc;
+}
+
+}  // extern "C"

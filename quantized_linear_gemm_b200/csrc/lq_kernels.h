@@ -1,0 +1,65 @@
+// Internal interface between the host library (lq_host.cu) and the kernel
+// translation units.  Not part of the public C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace lq {
+
+constexpr int kFmtFp8 = 0;    // LQ_FP8_DYNAMIC
+constexpr int kFmtInt8 = 1;   // LQ_W8A8_INT8
+constexpr int kFmtBlock = 2;  // LQ_BLOCK_FP8
+
+struct GemmParams {
+  int64_t M, N, K;
+  int T;               // number of 128-wide K tiles, ceil(K / 128)
+  int KB;              // K / 128 (Block_FP8 scale row length)
+  int S;               // split_k
+  int stages;          // shared-memory ring depth
+  int reduce_in_kernel;
+  int early_weights;   // stream weight tiles before the grid dependency wait
+  const float* a_s;
+  const float* b_s;
+  __nv_bfloat16* C;
+  void* ws;            // Split-K partials [S, M, N] (f32, or s32 for INT8)
+  int* counters;       // Split-K arrival counters, one per output tile
+  int32_t* acc_out;    // optional exact INT8 accumulators [M, N]
+  int* status;         // device status word (bit set per timed-out wait site)
+  uint64_t wait_limit_ns;
+};
+
+// Launch description filled by the host library.
+struct GemmLaunch {
+  CUtensorMap tmX;     // operand on the MMA M side (128-row tiles)
+  CUtensorMap tmY;     // operand on the MMA N side (tile_n-row tiles)
+  GemmParams p;
+  dim3 grid;
+  int smem_bytes;
+  int pdl;
+  cudaStream_t stream;
+};
+
+// Implemented in scaled_mm_{fp8,int8,block}.cu: launches the instantiation
+// (swap_ab, tile_n) of the format.  Returns cudaErrorInvalidValue for a
+// (swap_ab, tile_n) pair that is not instantiated.
+cudaError_t launch_scaled_mm_fp8(const GemmLaunch& l, int swap_ab, int tile_n);
+cudaError_t launch_scaled_mm_int8(const GemmLaunch& l, int swap_ab, int tile_n);
+cudaError_t launch_scaled_mm_block(const GemmLaunch& l, int swap_ab, int tile_n);
+cudaError_t launch_splitk_reduce(int fmt, const GemmParams& p, int pdl, cudaStream_t stream);
+
+// Largest dynamic shared memory the GEMM kernel may use for (swap_ab, tile_n, stages).
+int gemm_smem_bytes_for(int tile_n, int stages);
+
+// Quantization kernels (quant_kernels.cu).
+cudaError_t launch_quant_per_token(int fmt, const void* x, void* q, float* scales, int64_t M, int64_t K,
+                                   cudaStream_t stream);
+cudaError_t launch_quant_group128(const void* x, void* q, float* scales, int64_t M, int64_t K,
+                                  cudaStream_t stream);
+cudaError_t launch_quant_weight_block128(const void* w, void* q, float* scales, int64_t N, int64_t K,
+                                         cudaStream_t stream);
+cudaError_t launch_fill_zero_bf16(__nv_bfloat16* C, int64_t count, cudaStream_t stream);
+
+}  // namespace lq

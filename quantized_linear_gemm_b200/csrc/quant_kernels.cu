@@ -1,0 +1,227 @@
+// Dynamic activation quantizers and the offline weight quantizer.
+//
+// Rule (formats of the PyTorch blog "Building a High-Performance and Portable
+// vLLM Linear Backend with Helion", "Helion Linear Backend > Scope"; kernels
+// dynamic_per_token_scaled_fp8_quant and per_token_group_fp8_quant of the
+// 24-ai.news report, "kernels integrated into vLLM"):
+//
+//   s = max(fp32(amax / Q), 2^-126),   q = encode(fp32(x / s))
+//
+// with Q = 448 (e4m3, round to nearest even, saturating) or 127 (int8,
+// round half to even, clamped to +-127).  The division is the correctly
+// rounded __fdiv_rn (not a reciprocal multiply), so codes and scales are
+// reproducible bit for bit.
+//
+// These kernels are bandwidth / launch bound: each reads bf16 once per pass
+// with 16-byte loads and writes 8-byte code chunks.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <cfloat>
+#include <cstdint>
+
+#include "lq_kernels.h"
+#include "ptx.cuh"
+
+namespace lq {
+namespace {
+
+constexpr float kE4m3Max = 448.0f;
+constexpr float kInt8Max = 127.0f;
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ float amax8(const float (&f)[8]) {
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(f[i]));
+  return a;
+}
+
+__device__ __forceinline__ float scale_from_amax(float amax, float qmax) {
+  return fmaxf(__fdiv_rn(amax, qmax), FLT_MIN);
+}
+
+// 8 values -> 8 e4m3 bytes (lowest address first).
+__device__ __forceinline__ uint2 encode8_e4m3(const float (&f)[8], float s) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 pr = make_float2(__fdiv_rn(f[2 * i], s), __fdiv_rn(f[2 * i + 1], s));
+    w[i] = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3));
+  }
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+// 8 values -> 8 int8 bytes.
+__device__ __forceinline__ uint2 encode8_int8(const float (&f)[8], float s) {
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int v = __float2int_rn(__fdiv_rn(f[i], s));
+    v = v > 127 ? 127 : (v < -127 ? -127 : v);
+    b[i] = static_cast<uint32_t>(v) & 0xFFu;
+  }
+  return make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24),
+                    b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
+}
+
+template <int kThreadsPerRow>
+__device__ __forceinline__ float block_max(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = lane < kThreadsPerRow / 32 ? red[lane] : 0.f;
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) red[0] = v;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+// One CTA per row.  Two passes over the row (the second hits L1/L2).
+template <bool kInt8>
+__global__ void __launch_bounds__(256) quant_per_token_kernel(const __nv_bfloat16* __restrict__ x,
+                                                               uint8_t* __restrict__ q, float* __restrict__ scales,
+                                                               int64_t K) {
+  __shared__ float red[32];
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int64_t row = blockIdx.x;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
+  const int64_t nvec = K / 8;
+  float a = 0.f;
+  for (int64_t i = threadIdx.x; i < nvec; i += blockDim.x) {
+    float f[8];
+    bf16x8_to_f32(__ldg(xr + i), f);
+    a = fmaxf(a, amax8(f));
+  }
+  const float amax = block_max<256>(a, red);
+  const float s = scale_from_amax(amax, kInt8 ? kInt8Max : kE4m3Max);
+  if (threadIdx.x == 0) scales[row] = s;
+  uint2* qr = reinterpret_cast<uint2*>(q + row * K);
+  for (int64_t i = threadIdx.x; i < nvec; i += blockDim.x) {
+    float f[8];
+    bf16x8_to_f32(__ldg(xr + i), f);
+    qr[i] = kInt8 ? encode8_int8(f, s) : encode8_e4m3(f, s);
+  }
+}
+
+// 16 threads per 128-element group, 8 elements each; 16 groups per CTA.
+__global__ void __launch_bounds__(256) quant_group128_kernel(const __nv_bfloat16* __restrict__ x,
+                                                              uint8_t* __restrict__ q, float* __restrict__ scales,
+                                                              int64_t M, int64_t K) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int64_t KB = K / 128;
+  const int64_t g = blockIdx.x * 16ll + (threadIdx.x >> 4);
+  const int sub = threadIdx.x & 15;
+  const bool valid = g < M * KB;
+  const int64_t row = valid ? g / KB : 0;
+  const int64_t kb = valid ? g - row * KB : 0;
+  const int64_t off = row * K + kb * 128 + sub * 8;
+  float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (valid) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(x + off)), f);
+  float a = amax8(f);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));   // within 16 lanes
+  const float s = scale_from_amax(a, kE4m3Max);
+  if (valid) {
+    if (sub == 0) scales[row * KB + kb] = s;
+    *reinterpret_cast<uint2*>(q + off) = encode8_e4m3(f, s);
+  }
+}
+
+// One CTA per 128x128 block of W[N, K]; thread t covers row t/2, 64 columns.
+__global__ void __launch_bounds__(256) quant_weight_block128_kernel(const __nv_bfloat16* __restrict__ w,
+                                                                     uint8_t* __restrict__ q,
+                                                                     float* __restrict__ scales, int64_t K) {
+  __shared__ float red[32];
+  const int64_t KB = K / 128;
+  const int64_t nb = blockIdx.y, kb = blockIdx.x;
+  const int64_t row = nb * 128 + (threadIdx.x >> 1);
+  const int64_t col = kb * 128 + (threadIdx.x & 1) * 64;
+  const uint4* src = reinterpret_cast<const uint4*>(w + row * K + col);
+  float f[8][8];
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    bf16x8_to_f32(__ldg(src + i), f[i]);
+    a = fmaxf(a, amax8(f[i]));
+  }
+  const float amax = block_max<256>(a, red);
+  const float s = scale_from_amax(amax, kE4m3Max);
+  if (threadIdx.x == 0) scales[nb * KB + kb] = s;
+  uint2* dst = reinterpret_cast<uint2*>(q + row * K + col);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dst[i] = encode8_e4m3(f[i], s);
+}
+
+__global__ void fill_zero_bf16_kernel(__nv_bfloat16* __restrict__ C, int64_t count) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    C[i] = __float2bfloat16_rn(0.f);
+}
+
+cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, cudaStream_t stream, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+}  // namespace
+
+cudaError_t launch_quant_per_token(int fmt, const void* x, void* q, float* scales, int64_t M, int64_t K,
+                                   cudaStream_t stream) {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(dim3(static_cast<unsigned>(M)), dim3(256), stream, attr);
+  const auto* xp = static_cast<const __nv_bfloat16*>(x);
+  auto* qp = static_cast<uint8_t*>(q);
+  if (fmt == kFmtInt8) return cudaLaunchKernelEx(&cfg, quant_per_token_kernel<true>, xp, qp, scales, K);
+  return cudaLaunchKernelEx(&cfg, quant_per_token_kernel<false>, xp, qp, scales, K);
+}
+
+cudaError_t launch_quant_group128(const void* x, void* q, float* scales, int64_t M, int64_t K,
+                                  cudaStream_t stream) {
+  const int64_t groups = M * (K / 128);
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(dim3(static_cast<unsigned>((groups + 15) / 16)), dim3(256), stream, attr);
+  return cudaLaunchKernelEx(&cfg, quant_group128_kernel, static_cast<const __nv_bfloat16*>(x),
+                            static_cast<uint8_t*>(q), scales, M, K);
+}
+
+cudaError_t launch_quant_weight_block128(const void* w, void* q, float* scales, int64_t N, int64_t K,
+                                         cudaStream_t stream) {
+  quant_weight_block128_kernel<<<dim3(static_cast<unsigned>(K / 128), static_cast<unsigned>(N / 128)), 256, 0,
+                                  stream>>>(static_cast<const __nv_bfloat16*>(w), static_cast<uint8_t*>(q), scales,
+                                            K);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_zero_bf16(__nv_bfloat16* C, int64_t count, cudaStream_t stream) {
+  int64_t blocks = (count + 255) / 256;
+  if (blocks > 148 * 4) blocks = 148 * 4;
+  if (blocks < 1) blocks = 1;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(dim3(static_cast<unsigned>(blocks)), dim3(256), stream, attr);
+  return cudaLaunchKernelEx(&cfg, fill_zero_bf16_kernel, C, count);
+}
+
+}  // namespace lq

@@ -1,0 +1,40 @@
+// Block_FP8 instantiations of the scaled_mm kernel and the Split-K reduction.
+#include "scaled_mm_launch.cuh"
+namespace lq {
+cudaError_t launch_scaled_mm_block(const GemmLaunch& l, int swap_ab, int tile_n) {
+  return launch_format<kFmtBlock>(l, swap_ab, tile_n);
+}
+
+int gemm_smem_bytes_for(int tile_n, int stages) {
+  switch (tile_n) {
+    case 16: return gemm_smem_bytes<16>(stages);
+    case 32: return gemm_smem_bytes<32>(stages);
+    case 64: return gemm_smem_bytes<64>(stages);
+    case 128: return gemm_smem_bytes<128>(stages);
+    case 256: return gemm_smem_bytes<256>(stages);
+    default: return -1;
+  }
+}
+
+cudaError_t launch_splitk_reduce(int fmt, const GemmParams& p, int pdl, cudaStream_t stream) {
+  const int64_t work = p.M * p.N / 4;
+  int64_t blocks = (work + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (blocks < 1) blocks = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  switch (fmt) {
+    case kFmtFp8: return cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<kFmtFp8>, p);
+    case kFmtInt8: return cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<kFmtInt8>, p);
+    case kFmtBlock: return cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<kFmtBlock>, p);
+    default: return cudaErrorInvalidValue;
+  }
+}
+}  // namespace lq

@@ -1,0 +1,538 @@
+// scaled_mm on sm_100a: a TMA -> shared-memory ring -> tcgen05.mma -> TMEM
+// pipeline, one output tile per CTA.
+//
+// Operation (PyTorch blog "Building a High-Performance and Portable vLLM
+// Linear Backend with Helion", "Helion Linear Backend > Scope" for the
+// formats and "Kernel Implementation" for the variants):
+//
+//   C[m, n] = bf16( a_s . b_s . sum_k A[m, k] B[n, k] )          FP8 / INT8
+//   C[m, n] = bf16( sum_kb a_s[m, kb] b_s[n/128, kb]
+//                          sum_{k in kb} A[m, k] B[n, k] )         Block_FP8
+//
+// The tensor core computes D[128 x TN] = X[128 x Kt] . Y[TN x Kt]^T from two
+// K-major shared-memory tiles:
+//   Standard : X = 128 rows of A (tokens), Y = TN rows of B (weights);
+//   Swap-AB  : X = 128 rows of B (weights), Y = TN rows of A (tokens), i.e.
+//              the blog's (B^T A^T)^T; the epilogue stores D transposed.
+// Split-K: blockIdx.z = s owns K tiles [floor(s T / S), floor((s+1) T / S)).
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
+// MMA issuer, warps 2..5 = epilogue (warp w reads TMEM lanes 32 (w % 4) ..).
+// Every wait is bounded; a timeout sets the device status word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "lq_kernels.h"
+#include "ptx.cuh"
+
+namespace lq {
+
+constexpr int kTileM = 128;      // MMA M (rows of X)
+constexpr int kTileK = 128;      // K elements (bytes) per pipeline stage
+constexpr int kMmaK = 32;        // K per tcgen05.mma for 8-bit operands
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+
+template <int TN>
+struct TileShape {
+  static constexpr int kXBytes = kTileM * kTileK;   // 16 KB
+  static constexpr int kYBytes = TN * kTileK;       // multiple of 1 KB for TN % 8 == 0
+  static constexpr int kStageBytes = kXBytes + kYBytes;
+};
+
+__host__ __device__ constexpr int tmem_cols_for(int cols) {
+  return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
+}
+
+// Shared-memory bytes the kernel needs for `stages` ring slots.
+template <int TN>
+__host__ __device__ constexpr int gemm_smem_bytes(int stages) {
+  return 1024 /* alignment slack */ + stages * TileShape<TN>::kStageBytes + 64 * 8 /* barriers */ + 64;
+}
+
+struct SmemCtl {
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;     // [2]
+  uint64_t* tempty;    // [2]
+  uint64_t* mma_done;  // [1]
+  uint32_t* tmem_slot;
+  volatile int* abort_flag;
+  volatile int* last_flag;
+};
+
+__device__ __forceinline__ void report_timeout(const GemmParams& p, int where) {
+  if (p.status) atomicOr(p.status, 1 << where);
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const GemmParams& p, const SmemCtl& c,
+                                         int where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*c.abort_flag) return false;
+    if (global_timer_ns() - t0 > p.wait_limit_ns) {
+      *c.abort_flag = 1;
+      report_timeout(p, where);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ---------------------------------------------------------------------------
+// The GEMM kernel
+// ---------------------------------------------------------------------------
+template <int FMT, bool SWAP, int TN>
+__global__ void __launch_bounds__(kThreads, 1)
+    scaled_mm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                        const GemmParams p) {
+  using Shape = TileShape<TN>;
+  constexpr bool kInt8 = FMT == kFmtInt8;
+  constexpr bool kBlocked = FMT == kFmtBlock;
+  constexpr int kAccBufs = kBlocked ? 2 : 1;
+  constexpr int kTmemCols = tmem_cols_for(TN * kAccBufs);
+  constexpr int CH = TN < 32 ? TN : 32;   // TMEM columns per tcgen05.ld
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+  const int stages = p.stages;
+  uint8_t* ring = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + stages * Shape::kStageBytes);
+  SmemCtl c;
+  c.full = bars;
+  c.empty = bars + stages;
+  c.tfull = bars + 2 * stages;
+  c.tempty = c.tfull + 2;
+  c.mma_done = c.tempty + 2;
+  c.tmem_slot = reinterpret_cast<uint32_t*>(c.mma_done + 1);
+  c.abort_flag = reinterpret_cast<volatile int*>(c.tmem_slot + 1);
+  c.last_flag = c.abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int split = blockIdx.z;
+  const int kb_lo = static_cast<int>((static_cast<int64_t>(split) * p.T) / p.S);
+  const int kb_hi = static_cast<int>((static_cast<int64_t>(split + 1) * p.T) / p.S);
+  const int nkb = kb_hi - kb_lo;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&c.full[s], 1);
+      mbar_init(&c.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&c.tfull[b], 1);
+      mbar_init(&c.tempty[b], kEpiThreads / 32);
+    }
+    mbar_init(c.mma_done, 1);
+    *c.abort_flag = 0;
+    *c.last_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensor_map(&tmX);
+    prefetch_tensor_map(&tmY);
+  }
+  if (warp == 1) {
+    tmem_alloc(c.tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *c.tmem_slot;
+
+  // Let the next kernel on the stream start its own prologue / weight stream.
+  grid_launch_dependents();
+
+  const int x_row0 = blockIdx.x * kTileM;
+  const int y_row0 = blockIdx.y * TN;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();   // weights: streamed once
+      const uint64_t pol_a = policy_evict_last();    // activations: re-read by many CTAs
+      const CUtensorMap* tmW = SWAP ? &tmX : &tmY;
+      const CUtensorMap* tmA = SWAP ? &tmY : &tmX;
+      const int w_row0 = SWAP ? x_row0 : y_row0;
+      const int a_row0 = SWAP ? y_row0 : x_row0;
+      const int w_off = SWAP ? 0 : Shape::kXBytes;   // byte offset of the weight tile in a stage
+      const int a_off = SWAP ? Shape::kXBytes : 0;
+      const int pre = nkb < stages ? nkb : stages;
+      if (p.early_weights) {
+        // The caller guarantees that the weights are not written by a kernel
+        // that may still run: start streaming them before waiting for the
+        // previous kernel on the stream (programmatic dependent launch).
+        for (int i = 0; i < pre; ++i) {
+          uint8_t* st = ring + i * Shape::kStageBytes;
+          mbar_arrive_expect_tx(&c.full[i], Shape::kStageBytes);
+          tma_load_2d(tmW, &c.full[i], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
+        }
+        grid_dependency_wait();
+      } else {
+        grid_dependency_wait();
+        for (int i = 0; i < pre; ++i) {
+          uint8_t* st = ring + i * Shape::kStageBytes;
+          mbar_arrive_expect_tx(&c.full[i], Shape::kStageBytes);
+          tma_load_2d(tmW, &c.full[i], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
+        }
+      }
+      for (int i = 0; i < pre; ++i) {
+        uint8_t* st = ring + i * Shape::kStageBytes;
+        tma_load_2d(tmA, &c.full[i], st + a_off, (kb_lo + i) * kTileK, a_row0, pol_a);
+      }
+      int issued = pre;
+      for (int i = pre; i < nkb; ++i) {
+        const int s = i % stages;
+        const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
+        if (!wait_bar(&c.empty[s], ph ^ 1u, p, c, 0)) break;
+        uint8_t* st = ring + s * Shape::kStageBytes;
+        mbar_arrive_expect_tx(&c.full[s], Shape::kStageBytes);
+        tma_load_2d(tmW, &c.full[s], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
+        tma_load_2d(tmA, &c.full[s], st + a_off, (kb_lo + i) * kTileK, a_row0, pol_a);
+        issued = i + 1;
+      }
+      if (*c.abort_flag) {
+        // Drain: wait (bounded) for the copies still in flight into shared memory.
+        const int first = issued > stages ? issued - stages : 0;
+        for (int j = first; j < issued; ++j) {
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&c.full[j % stages], static_cast<uint32_t>(j / stages) & 1u) &&
+                 global_timer_ns() - t0 < p.wait_limit_ns) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    grid_dependency_wait();
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc<kInt8>(kTileM, TN);
+      bool issued_any = false;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % stages;
+        const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
+        uint32_t d_tmem = tmem_base;
+        if (kBlocked) {
+          const int buf = i & 1;
+          const uint32_t use = static_cast<uint32_t>(i >> 1);
+          if (!wait_bar(&c.tempty[buf], (use & 1u) ^ 1u, p, c, 1)) break;
+          d_tmem += static_cast<uint32_t>(buf * TN);
+        }
+        if (!wait_bar(&c.full[s], ph, p, c, 2)) break;
+        tc_fence_after_sync();
+        uint8_t* st = ring + s * Shape::kStageBytes;
+        const uint64_t xd = smem_desc_k_sw128(st);
+        const uint64_t yd = smem_desc_k_sw128(st + Shape::kXBytes);
+#pragma unroll
+        for (int kk = 0; kk < kTileK / kMmaK; ++kk) {
+          // +32 bytes along K inside the 128-byte swizzle row = +2 in the 16-byte address field
+          const uint32_t acc = kBlocked ? (kk > 0) : (i > 0 || kk > 0);
+          if (kInt8)
+            mma_i8(d_tmem, xd + 2 * kk, yd + 2 * kk, idesc, acc);
+          else
+            mma_f8f6f4(d_tmem, xd + 2 * kk, yd + 2 * kk, idesc, acc);
+        }
+        issued_any = true;
+        mma_commit(&c.empty[s]);
+        if (kBlocked) mma_commit(&c.tfull[i & 1]);
+      }
+      if (!kBlocked && nkb > 0 && !*c.abort_flag) mma_commit(&c.tfull[0]);
+      if (issued_any) {
+        // All MMAs must be complete before TMEM is released at teardown.
+        mma_commit(c.mma_done);
+        wait_bar(c.mma_done, 0, p, c, 3);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    grid_dependency_wait();
+    const int q = warp & 3;                    // TMEM lane quarter of this warp
+    const int r = q * 32 + lane;               // accumulator row (TMEM lane)
+    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    // (m, n) of accumulator element (r, j): Standard (x_row0 + r, y_row0 + j),
+    // Swap-AB (y_row0 + j, x_row0 + r).
+    const int64_t M = p.M, N = p.N;
+
+    float accr[kBlocked ? TN : 1];
+#pragma unroll
+    for (int j = 0; j < (kBlocked ? TN : 1); ++j) accr[j] = 0.f;
+
+    bool ok = true;
+    if (kBlocked) {
+      // Per-128-K-block promotion: D_kb from TMEM times a_s[m,kb] b_s[nb,kb].
+      const int nb = SWAP ? (x_row0 + r) / 128 : y_row0 / 128;
+      const int64_t m_thread = SWAP ? 0 : x_row0 + r;
+      for (int i = 0; i < nkb; ++i) {
+        const int buf = i & 1;
+        const uint32_t use = static_cast<uint32_t>(i >> 1);
+        // warp-uniform decision: the tcgen05.ld below is .sync.aligned
+        if (!__all_sync(0xffffffffu, wait_bar(&c.tfull[buf], use & 1u, p, c, 4))) { ok = false; break; }
+        tc_fence_after_sync();
+        const int kb = kb_lo + i;
+        const bool n_ok = SWAP ? (x_row0 + r) < N : true;
+        const float sb = (SWAP ? n_ok : true) ? __ldg(p.b_s + static_cast<int64_t>(nb) * p.KB + kb) : 0.f;
+        float sa_row = 0.f;
+        if (!SWAP) sa_row = m_thread < M ? __ldg(p.a_s + m_thread * p.KB + kb) : 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < TN; c0 += CH) {
+          uint32_t v[CH];
+          if constexpr (CH == 32)
+            tmem_ld_32x32b_x32(t_row + buf * TN + c0, v);
+          else
+            tmem_ld_32x32b_x16(t_row + buf * TN + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < CH; ++j) {
+            float scale;
+            if (SWAP) {
+              const int64_t m = y_row0 + c0 + j;
+              scale = (m < M ? __ldg(p.a_s + m * p.KB + kb) : 0.f) * sb;
+            } else {
+              scale = sa_row * sb;
+            }
+            accr[c0 + j] = fmaf(__uint_as_float(v[j]), scale, accr[c0 + j]);
+          }
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.tempty[buf]);
+      }
+    } else if (nkb > 0) {
+      ok = wait_bar(&c.tfull[0], 0, p, c, 5);
+      tc_fence_after_sync();
+    }
+    ok = __all_sync(0xffffffffu, ok && !*c.abort_flag);
+
+    if (ok) {
+      float* wsf = reinterpret_cast<float*>(p.ws);
+      int32_t* wsi = reinterpret_cast<int32_t*>(p.ws);
+      const bool split_mode = p.S > 1;
+
+#pragma unroll
+      for (int c0 = 0; c0 < TN; c0 += CH) {
+        uint32_t v[CH];
+        if (kBlocked) {
+#pragma unroll
+          for (int j = 0; j < CH; ++j) v[j] = __float_as_uint(accr[c0 + j]);
+        } else if (nkb > 0) {
+          if constexpr (CH == 32)
+            tmem_ld_32x32b_x32(t_row + c0, v);
+          else
+            tmem_ld_32x32b_x16(t_row + c0, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < CH; ++j) v[j] = 0u;   // empty split: zero partial
+        }
+
+        if (SWAP) {
+          const int64_t n = x_row0 + r;
+          if (n < N) {
+            const float bsn = (!kBlocked && !split_mode) ? __ldg(p.b_s + n) : 1.f;
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+              const int64_t m = y_row0 + c0 + j;
+              if (m < M) {
+                const int64_t idx = m * N + n;
+                if (split_mode) {
+                  const int64_t widx = (static_cast<int64_t>(split) * M + m) * N + n;
+                  if (kInt8) wsi[widx] = static_cast<int32_t>(v[j]);
+                  else wsf[widx] = __uint_as_float(v[j]);
+                } else {
+                  float val;
+                  if (kBlocked) {
+                    val = __uint_as_float(v[j]);
+                  } else {
+                    const float a = kInt8 ? static_cast<float>(static_cast<int32_t>(v[j])) : __uint_as_float(v[j]);
+                    val = a * __ldg(p.a_s + m) * bsn;
+                  }
+                  p.C[idx] = __float2bfloat16_rn(val);
+                  if (kInt8 && p.acc_out) p.acc_out[idx] = static_cast<int32_t>(v[j]);
+                }
+              }
+            }
+          }
+        } else {
+          const int64_t m = x_row0 + r;
+          if (m < M) {
+            const float asm_ = (!kBlocked && !split_mode) ? __ldg(p.a_s + m) : 1.f;
+#pragma unroll
+            for (int j8 = 0; j8 < CH; j8 += 8) {
+              const int64_t n = y_row0 + c0 + j8;
+              if (n < N) {   // N % 8 == 0: the 8-wide group is fully inside or outside
+                if (split_mode) {
+                  const int64_t widx = (static_cast<int64_t>(split) * M + m) * N + n;
+                  uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint32_t*>(p.ws) + widx);
+                  dst[0] = make_uint4(v[j8 + 0], v[j8 + 1], v[j8 + 2], v[j8 + 3]);
+                  dst[1] = make_uint4(v[j8 + 4], v[j8 + 5], v[j8 + 6], v[j8 + 7]);
+                } else {
+                  float f[8];
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    if (kBlocked) {
+                      f[e] = __uint_as_float(v[j8 + e]);
+                    } else {
+                      const float a =
+                          kInt8 ? static_cast<float>(static_cast<int32_t>(v[j8 + e])) : __uint_as_float(v[j8 + e]);
+                      f[e] = a * asm_ * __ldg(p.b_s + n + e);
+                    }
+                  }
+                  uint4 pk = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                                        pack_bf16x2(f[6], f[7]));
+                  *reinterpret_cast<uint4*>(p.C + m * N + n) = pk;
+                  if (kInt8 && p.acc_out) {
+                    uint4* ao = reinterpret_cast<uint4*>(p.acc_out + m * N + n);
+                    ao[0] = make_uint4(v[j8 + 0], v[j8 + 1], v[j8 + 2], v[j8 + 3]);
+                    ao[1] = make_uint4(v[j8 + 4], v[j8 + 5], v[j8 + 6], v[j8 + 7]);
+                  }
+                }
+              }
+            }
+          }
+        }
+      }
+
+    }
+
+    // -------------------------------------------- in-kernel Split-K reduce
+    // Every epilogue thread reaches both named barriers, also after a
+    // timeout (then this CTA does not count itself and no CTA reduces).
+    if (p.S > 1 && p.reduce_in_kernel) {
+      float* wsf = reinterpret_cast<float*>(p.ws);
+      int32_t* wsi = reinterpret_cast<int32_t*>(p.ws);
+      __threadfence();
+      named_barrier_sync(1, kEpiThreads);
+      const int tile_id = blockIdx.x + blockIdx.y * gridDim.x;
+      if (warp == 2 && lane == 0) {
+        int last = 0;
+        if (!*c.abort_flag) last = atomicAdd(p.counters + tile_id, 1) == p.S - 1;
+        *c.last_flag = last;
+      }
+      named_barrier_sync(1, kEpiThreads);
+      if (*c.last_flag) {
+        __threadfence();
+        if (SWAP) {
+          const int64_t n = x_row0 + r;
+          if (n < N) {
+            const float bsn = kBlocked ? 1.f : __ldg(p.b_s + n);
+            for (int j = 0; j < TN; ++j) {
+              const int64_t m = y_row0 + j;
+              if (m >= M) break;
+              float sf = 0.f;
+              int32_t si = 0;
+              for (int s = 0; s < p.S; ++s) {
+                const int64_t widx = (static_cast<int64_t>(s) * M + m) * N + n;
+                if (kInt8) si += __ldcg(wsi + widx);
+                else sf += __ldcg(wsf + widx);
+              }
+              float val;
+              if (kBlocked) val = sf;
+              else val = (kInt8 ? static_cast<float>(si) : sf) * __ldg(p.a_s + m) * bsn;
+              p.C[m * N + n] = __float2bfloat16_rn(val);
+              if (kInt8 && p.acc_out) p.acc_out[m * N + n] = si;
+            }
+          }
+        } else {
+          const int64_t m = x_row0 + r;
+          if (m < M) {
+            const float asm_ = kBlocked ? 1.f : __ldg(p.a_s + m);
+            for (int j4 = 0; j4 < TN; j4 += 4) {
+              const int64_t n = y_row0 + j4;
+              if (n >= N) break;
+              float4 sf = make_float4(0.f, 0.f, 0.f, 0.f);
+              int4 si = make_int4(0, 0, 0, 0);
+              for (int s = 0; s < p.S; ++s) {
+                const int64_t widx = (static_cast<int64_t>(s) * M + m) * N + n;
+                if (kInt8) {
+                  const int4 t = __ldcg(reinterpret_cast<const int4*>(wsi + widx));
+                  si.x += t.x; si.y += t.y; si.z += t.z; si.w += t.w;
+                } else {
+                  const float4 t = __ldcg(reinterpret_cast<const float4*>(wsf + widx));
+                  sf.x += t.x; sf.y += t.y; sf.z += t.z; sf.w += t.w;
+                }
+              }
+              float f[4];
+              if (kInt8) { f[0] = si.x; f[1] = si.y; f[2] = si.z; f[3] = si.w; }
+              else { f[0] = sf.x; f[1] = sf.y; f[2] = sf.z; f[3] = sf.w; }
+              if (!kBlocked) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * __ldg(p.b_s + n + e);
+              }
+              uint2 pk = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+              *reinterpret_cast<uint2*>(p.C + m * N + n) = pk;
+              if (kInt8 && p.acc_out) *reinterpret_cast<int4*>(p.acc_out + m * N + n) = si;
+            }
+          }
+        }
+        if (warp == 2 && lane == 0) p.counters[tile_id] = 0;   // ready for the next launch / replay
+      }
+    }
+  }
+
+  // -------------------------------------------------------------- teardown
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Separate fixed-order Split-K reduction: C = scale(sum_{s=0..S-1} ws[s]).
+// One thread per 4 consecutive outputs (N % 8 == 0).
+// ---------------------------------------------------------------------------
+template <int FMT>
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmParams p) {
+  constexpr bool kInt8 = FMT == kFmtInt8;
+  constexpr bool kBlocked = FMT == kFmtBlock;
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int64_t MN4 = p.M * p.N / 4;
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < MN4;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t e0 = t * 4;
+    const int64_t m = e0 / p.N;
+    const int64_t n = e0 - m * p.N;
+    float f[4];
+    int4 si = make_int4(0, 0, 0, 0);
+    if (kInt8) {
+      const int32_t* ws = reinterpret_cast<const int32_t*>(p.ws);
+      for (int s = 0; s < p.S; ++s) {
+        const int4 v = __ldcg(reinterpret_cast<const int4*>(ws + s * p.M * p.N + e0));
+        si.x += v.x; si.y += v.y; si.z += v.z; si.w += v.w;
+      }
+      f[0] = si.x; f[1] = si.y; f[2] = si.z; f[3] = si.w;
+    } else {
+      const float* ws = reinterpret_cast<const float*>(p.ws);
+      float4 sf = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s = 0; s < p.S; ++s) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(ws + s * p.M * p.N + e0));
+        sf.x += v.x; sf.y += v.y; sf.z += v.z; sf.w += v.w;
+      }
+      f[0] = sf.x; f[1] = sf.y; f[2] = sf.z; f[3] = sf.w;
+    }
+    if (!kBlocked) {
+      const float a = __ldg(p.a_s + m);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f[e] = f[e] * a * __ldg(p.b_s + n + e);
+    }
+    *reinterpret_cast<uint2*>(p.C + e0) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+    if (kInt8 && p.acc_out) *reinterpret_cast<int4*>(p.acc_out + e0) = si;
+  }
+}
+
+}  // namespace lq

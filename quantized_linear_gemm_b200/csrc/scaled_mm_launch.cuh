@@ -1,0 +1,50 @@
+// Launch helper shared by the per-format instantiation files.
+#pragma once
+
+#include "scaled_mm_kernel.cuh"
+
+namespace lq {
+
+template <int FMT, bool SWAP, int TN>
+cudaError_t launch_tc(const GemmLaunch& l) {
+  auto kern = scaled_mm_tc_kernel<FMT, SWAP, TN>;
+  static int configured = 0;   // max dynamic smem set once per instantiation and process
+  if (configured < l.smem_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    configured = 227 * 1024;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = l.grid;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(l.smem_bytes);
+  cfg.stream = l.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = l.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, l.tmX, l.tmY, l.p);
+}
+
+template <int FMT>
+cudaError_t launch_format(const GemmLaunch& l, int swap_ab, int tile_n) {
+  if (swap_ab) {
+    switch (tile_n) {
+      case 16: return launch_tc<FMT, true, 16>(l);
+      case 32: return launch_tc<FMT, true, 32>(l);
+      case 64: return launch_tc<FMT, true, 64>(l);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  switch (tile_n) {
+    case 64: return launch_tc<FMT, false, 64>(l);
+    case 128: return launch_tc<FMT, false, 128>(l);
+    case 256:
+      if constexpr (FMT != kFmtBlock) return launch_tc<FMT, false, 256>(l);
+      return cudaErrorInvalidValue;
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace lq

@@ -1,0 +1,282 @@
+"""Python binding of liblq (ctypes).  Argument marshalling only.
+
+Every function here checks tensor devices / dtypes / contiguity, then calls
+the C function of the same name in ``liblq.so`` on torch's current CUDA
+stream.  All arithmetic runs in the library's CUDA kernels; there is no
+fallback.  If ``liblq.so`` is missing the first call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblq.so")
+
+FP8_DYNAMIC = 0
+W8A8_INT8 = 1
+BLOCK_FP8 = 2
+FORMATS = {"fp8_dynamic": FP8_DYNAMIC, "w8a8_int8": W8A8_INT8, "block_fp8": BLOCK_FP8}
+
+STATUS = {
+    0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_ALIGNMENT", 3: "LQ_ERR_UNSUPPORTED_SHAPE",
+    4: "LQ_ERR_WORKSPACE", 5: "LQ_ERR_CUDA", 6: "LQ_ERR_DEVICE_TIMEOUT", 7: "LQ_ERR_TABLE",
+}
+
+# every symbol that include/lq.h declares
+EXPORTED = (
+    "lq_scaled_mm", "lq_scaled_mm_i32acc", "lq_quant_per_token", "lq_quant_per_token_group128",
+    "lq_quant_weight_block128", "lq_select_variant", "lq_load_dispatch_table", "lq_dispatch_table_size",
+    "lq_init_device", "lq_reserve_workspace", "lq_workspace_bytes", "lq_device_status",
+    "lq_status_string", "lq_version",
+)
+
+
+class LQError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Variant(ctypes.Structure):
+    _fields_ = [("swap_ab", ctypes.c_int32), ("split_k", ctypes.c_int32), ("tile_n", ctypes.c_int32),
+                ("stages", ctypes.c_int32), ("reduce", ctypes.c_int32), ("pdl", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {f: int(getattr(self, f)) for f, _ in self._fields_}
+
+
+def make_variant(swap_ab=0, split_k=1, tile_n=None, stages=0, reduce=1, pdl=1) -> Variant:
+    if tile_n is None:
+        tile_n = 32 if swap_ab else 128
+    return Variant(int(swap_ab), int(split_k), int(tile_n), int(stages), int(reduce), int(pdl))
+
+
+_lib = None
+_lock = threading.Lock()
+
+_vp, _i64, _i32, _st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded liblq.so (loaded on first use)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m quantized_linear_gemm_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            L.lq_scaled_mm.argtypes = [_i32, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.POINTER(Variant), _st]
+            L.lq_scaled_mm_i32acc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                              ctypes.POINTER(Variant), _st]
+            L.lq_quant_per_token.argtypes = [_i32, _vp, _vp, _vp, _i64, _i64, _st]
+            L.lq_quant_per_token_group128.argtypes = [_vp, _vp, _vp, _i64, _i64, _st]
+            L.lq_quant_weight_block128.argtypes = [_vp, _vp, _vp, _i64, _i64, _st]
+            L.lq_select_variant.argtypes = [_i32, _i64, _i64, _i64, ctypes.POINTER(Variant)]
+            L.lq_load_dispatch_table.argtypes = [ctypes.c_char_p]
+            L.lq_dispatch_table_size.argtypes = []
+            L.lq_dispatch_table_size.restype = _i64
+            L.lq_init_device.argtypes = [_i32]
+            L.lq_reserve_workspace.argtypes = [_i32, ctypes.c_size_t]
+            L.lq_workspace_bytes.argtypes = [_i32, _i64, _i64, _i64, ctypes.POINTER(Variant)]
+            L.lq_workspace_bytes.restype = ctypes.c_size_t
+            L.lq_device_status.argtypes = [_i32]
+            L.lq_status_string.argtypes = [_i32]
+            L.lq_status_string.restype = ctypes.c_char_p
+            L.lq_version.argtypes = []
+            L.lq_version.restype = ctypes.c_char_p
+            for name in ("lq_scaled_mm", "lq_scaled_mm_i32acc", "lq_quant_per_token", "lq_quant_per_token_group128",
+                         "lq_quant_weight_block128", "lq_select_variant", "lq_load_dispatch_table",
+                         "lq_init_device", "lq_reserve_workspace", "lq_device_status"):
+                getattr(L, name).restype = _i32
+            _lib = L
+    return _lib
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        raise LQError(fn, rc)
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _fmt(fmt) -> int:
+    if isinstance(fmt, str):
+        return FORMATS[fmt]
+    return int(fmt)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtypes, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+_CODE_DTYPES = (torch.uint8, torch.int8, torch.float8_e4m3fn)
+
+
+def scaled_mm(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor, b_scales: torch.Tensor,
+              C: torch.Tensor | None = None, variant: Variant | None = None, stream=None) -> torch.Tensor:
+    """C[M, N] (bf16) = dequant(A[M, K]) @ dequant(B[N, K])^T through ``lq_scaled_mm``."""
+    f = _fmt(fmt)
+    _need(A, "A", _CODE_DTYPES, 2)
+    _need(B, "B", _CODE_DTYPES, 2)
+    _need(a_scales, "a_scales", (torch.float32,), 2 if f == BLOCK_FP8 else 1)
+    _need(b_scales, "b_scales", (torch.float32,), 2 if f == BLOCK_FP8 else 1)
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] != K:
+        raise ValueError("A and B disagree on K")
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _need(C, "C", (torch.bfloat16,), 2)
+    if tuple(C.shape) != (M, N):
+        raise ValueError("C has the wrong shape")
+    rc = lib().lq_scaled_mm(f, _ptr(A), _ptr(a_scales), _ptr(B), _ptr(b_scales), _ptr(C), M, N, K,
+                            ctypes.byref(variant) if variant is not None else None, _stream(stream))
+    _check("lq_scaled_mm", rc)
+    return C
+
+
+def scaled_mm_i32acc(A, a_scales, B, b_scales, C=None, acc=None, variant: Variant | None = None, stream=None):
+    """W8A8_INT8 scaled_mm that also returns the exact int32 accumulators."""
+    _need(A, "A", (torch.int8,), 2)
+    _need(B, "B", (torch.int8,), 2)
+    M, K = A.shape
+    N = B.shape[0]
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=A.device)
+    _need(acc, "acc", (torch.int32,), 2)
+    rc = lib().lq_scaled_mm_i32acc(_ptr(A), _ptr(a_scales), _ptr(B), _ptr(b_scales), _ptr(C), _ptr(acc), M, N, K,
+                                   ctypes.byref(variant) if variant is not None else None, _stream(stream))
+    _check("lq_scaled_mm_i32acc", rc)
+    return C, acc
+
+
+def quant_per_token(fmt, x: torch.Tensor, q: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                    stream=None):
+    """(codes [M, K], scales [M]) of a bf16 [M, K] tensor; e4m3 codes as uint8, int8 codes as int8."""
+    f = _fmt(fmt)
+    _need(x, "x", (torch.bfloat16,), 2)
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.int8 if f == W8A8_INT8 else torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((M,), dtype=torch.float32, device=x.device)
+    rc = lib().lq_quant_per_token(f, _ptr(x), _ptr(q), _ptr(scales), M, K, _stream(stream))
+    _check("lq_quant_per_token", rc)
+    return q, scales
+
+
+def quant_per_token_group128(x: torch.Tensor, q=None, scales=None, stream=None):
+    """(e4m3 codes [M, K], scales [M, K/128]) of a bf16 [M, K] tensor."""
+    _need(x, "x", (torch.bfloat16,), 2)
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((M, max(K // 128, 0)), dtype=torch.float32, device=x.device)
+    rc = lib().lq_quant_per_token_group128(_ptr(x), _ptr(q), _ptr(scales), M, K, _stream(stream))
+    _check("lq_quant_per_token_group128", rc)
+    return q, scales
+
+
+def quant_weight_block128(w: torch.Tensor, q=None, scales=None, stream=None):
+    """(e4m3 codes [N, K], scales [N/128, K/128]) of a bf16 weight [N, K]."""
+    _need(w, "w", (torch.bfloat16,), 2)
+    N, K = w.shape
+    if q is None:
+        q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty((max(N // 128, 0), max(K // 128, 0)), dtype=torch.float32, device=w.device)
+    rc = lib().lq_quant_weight_block128(_ptr(w), _ptr(q), _ptr(scales), N, K, _stream(stream))
+    _check("lq_quant_weight_block128", rc)
+    return q, scales
+
+
+def select_variant(fmt, M: int, N: int, K: int) -> Variant:
+    v = Variant()
+    _check("lq_select_variant", lib().lq_select_variant(_fmt(fmt), M, N, K, ctypes.byref(v)))
+    return v
+
+
+def load_dispatch_table(path: str | None) -> None:
+    _check("lq_load_dispatch_table", lib().lq_load_dispatch_table(None if path is None else path.encode()))
+
+
+def dispatch_table_size() -> int:
+    return int(lib().lq_dispatch_table_size())
+
+
+def init_device(device: int = 0) -> None:
+    _check("lq_init_device", lib().lq_init_device(device))
+
+
+def reserve_workspace(device: int, nbytes: int) -> None:
+    _check("lq_reserve_workspace", lib().lq_reserve_workspace(device, nbytes))
+
+
+def workspace_bytes(fmt, M, N, K, variant: Variant | None = None) -> int:
+    return int(lib().lq_workspace_bytes(_fmt(fmt), M, N, K, ctypes.byref(variant) if variant is not None else None))
+
+
+def device_status(device: int = 0) -> int:
+    """Read and clear the device status word: 0, or LQ_ERR_DEVICE_TIMEOUT (6)."""
+    return int(lib().lq_device_status(device))
+
+
+def status_string(code: int) -> str:
+    return lib().lq_status_string(code).decode()
+
+
+def version() -> str:
+    return lib().lq_version().decode()
+
+
+def call_raw(name: str, *args) -> int:
+    """Call a C entry point with raw arguments (for argument-check tests)."""
+    return int(getattr(lib(), name)(*args))
+
+
+@dataclass(frozen=True)
+class Problem:
+    """A (format, M, N, K) GEMM shape."""
+    fmt: int
+    M: int
+    N: int
+    K: int
+
+    @property
+    def flops(self) -> int:
+        return 2 * self.M * self.N * self.K
+
+    @property
+    def bytes(self) -> int:
+        """Algorithmic HBM bytes: weights + activations + scales + bf16 output."""
+        if self.fmt == BLOCK_FP8:
+            scales = 4 * (self.M * (self.K // 128) + (self.N // 128) * (self.K // 128))
+        else:
+            scales = 4 * (self.M + self.N)
+        return self.N * self.K + self.M * self.K + scales + 2 * self.M * self.N

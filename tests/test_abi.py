@@ -1,0 +1,153 @@
+"""CPU tests of the C ABI: the library loads, exports every symbol that
+include/lq.h declares, and rejects bad arguments with status codes before it
+touches the GPU.  No call here launches a kernel."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantized_linear_gemm_b200 import lq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lq.h")
+
+OK, INVALID, ALIGN, SHAPE, TABLE = 0, 1, 2, 3, 7
+FAKE = 0x10000          # 16-byte aligned non-null "device pointer"; never dereferenced
+MISALIGNED = 0x10008
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_what_binding_lists():
+    assert declared_functions() == sorted(lq.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    L = lq.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_version_and_status_strings():
+    assert lq.version().startswith("lq ")
+    for code, name in lq.STATUS.items():
+        assert lq.status_string(code) == name
+
+
+def _mm(fmt=0, A=FAKE, a_s=FAKE, B=FAKE, b_s=FAKE, C=FAKE, M=16, N=128, K=128, variant=None):
+    return lq.lib().lq_scaled_mm(fmt, A, a_s, B, b_s, C, M, N, K,
+                                 ctypes.byref(variant) if variant is not None else None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(fmt=3), INVALID), (dict(fmt=-1), INVALID),
+    (dict(A=None), INVALID), (dict(B=None), INVALID), (dict(C=None), INVALID),
+    (dict(a_s=None), INVALID), (dict(b_s=None), INVALID),
+    (dict(M=-1), INVALID), (dict(K=-16), INVALID),
+    (dict(A=MISALIGNED), ALIGN), (dict(B=MISALIGNED), ALIGN), (dict(C=MISALIGNED), ALIGN),
+    (dict(K=120), SHAPE), (dict(N=100), SHAPE),
+    (dict(fmt=2, K=192), SHAPE), (dict(fmt=2, N=192), SHAPE),
+])
+def test_scaled_mm_argument_checks(kw, code):
+    assert _mm(**kw) == code
+
+
+def test_empty_problem_is_a_noop():
+    # M == 0 or N == 0: nothing to do, no pointer is needed
+    assert _mm(M=0, A=None, B=None, C=None, a_s=None, b_s=None) == OK
+    assert _mm(N=0, A=None, B=None, C=None, a_s=None, b_s=None) == OK
+
+
+@pytest.mark.parametrize("field,value", [
+    ("split_k", 3), ("split_k", 512), ("split_k", 0), ("swap_ab", 2), ("tile_n", 48),
+    ("stages", 1), ("stages", 17), ("reduce", 2), ("pdl", 5),
+])
+def test_variant_checks(field, value):
+    v = lq.make_variant(swap_ab=1, split_k=2, tile_n=32)
+    setattr(v, field, value)
+    assert _mm(variant=v) == INVALID
+
+
+def test_variant_tile_rules():
+    assert _mm(variant=lq.make_variant(swap_ab=1, tile_n=128)) == INVALID      # swap tiles are 16/32/64
+    assert _mm(variant=lq.make_variant(swap_ab=0, tile_n=16)) == INVALID       # standard tiles are 64/128/256
+    assert _mm(fmt=2, variant=lq.make_variant(swap_ab=0, tile_n=256)) == INVALID
+    assert _mm(variant=lq.make_variant(swap_ab=0, tile_n=256, stages=5)) == INVALID   # > 227 KB smem
+
+
+def test_quant_argument_checks():
+    L = lq.lib()
+    assert L.lq_quant_per_token(2, FAKE, FAKE, FAKE, 4, 128, None) == INVALID    # block fmt not per-token
+    assert L.lq_quant_per_token(0, None, FAKE, FAKE, 4, 128, None) == INVALID
+    assert L.lq_quant_per_token(0, MISALIGNED, FAKE, FAKE, 4, 128, None) == ALIGN
+    assert L.lq_quant_per_token(0, FAKE, FAKE, FAKE, 4, 120, None) == SHAPE
+    assert L.lq_quant_per_token(0, FAKE, FAKE, FAKE, 0, 128, None) == OK
+    assert L.lq_quant_per_token_group128(FAKE, FAKE, FAKE, 4, 192, None) == SHAPE
+    assert L.lq_quant_per_token_group128(None, FAKE, FAKE, 4, 256, None) == INVALID
+    assert L.lq_quant_weight_block128(FAKE, FAKE, FAKE, 192, 256, None) == SHAPE
+    assert L.lq_quant_weight_block128(FAKE, FAKE, FAKE, 0, 256, None) == OK
+
+
+def test_i32acc_needs_an_output():
+    L = lq.lib()
+    assert L.lq_scaled_mm_i32acc(FAKE, FAKE, FAKE, FAKE, FAKE, None, 4, 128, 128, None, None) == INVALID
+    assert L.lq_scaled_mm_i32acc(FAKE, FAKE, FAKE, FAKE, FAKE, MISALIGNED, 4, 128, 128, None, None) == ALIGN
+
+
+def test_heuristic_variant_shapes():
+    v = lq.select_variant("fp8_dynamic", 1, 4096, 4096)
+    assert v.swap_ab == 1 and v.tile_n == 16 and v.split_k >= 2
+    v = lq.select_variant("fp8_dynamic", 24, 4096, 4096)
+    assert v.swap_ab == 1 and v.tile_n == 32
+    v = lq.select_variant("w8a8_int8", 8192, 5120, 25600)
+    assert v.swap_ab == 0 and v.tile_n == 256 and v.split_k == 1
+    v = lq.select_variant("block_fp8", 2048, 51200, 5120)
+    assert v.swap_ab == 0 and v.tile_n == 128
+    for M in (1, 2, 3, 17, 33, 64, 100, 4096):
+        v = lq.select_variant("block_fp8", M, 5120, 25600)
+        assert v.split_k & (v.split_k - 1) == 0 and 1 <= v.split_k <= 256
+
+
+def test_dispatch_table_file(tmp_path):
+    p = tmp_path / "table.txt"
+    p.write_text("# fmt m_bucket N K swap split tile stages reduce pdl\n"
+                 "fp8_dynamic 8 4096 4096 1 8 16 4 0 1\n"
+                 "w8a8_int8 32 6144 4096 0 2 64 6 1 0   # trailing comment\n")
+    try:
+        lq.load_dispatch_table(str(p))
+        assert lq.dispatch_table_size() == 2
+        v = lq.select_variant("fp8_dynamic", 5, 4096, 4096)      # M=5 -> bucket 8
+        assert v.as_dict() == dict(swap_ab=1, split_k=8, tile_n=16, stages=4, reduce=0, pdl=1)
+        v = lq.select_variant("w8a8_int8", 32, 6144, 4096)
+        assert v.as_dict() == dict(swap_ab=0, split_k=2, tile_n=64, stages=6, reduce=1, pdl=0)
+        # workspace need follows the selected variant
+        assert lq.workspace_bytes("fp8_dynamic", 5, 4096, 4096) == 8 * 5 * 4096 * 4
+        bad = tmp_path / "bad.txt"
+        bad.write_text("fp8_dynamic 8 4096 4096 1 3 16 4 0 1\n")   # split_k 3 is not a power of two
+        with pytest.raises(lq.LQError) as e:
+            lq.load_dispatch_table(str(bad))
+        assert e.value.code == TABLE
+        assert lq.dispatch_table_size() == 2                       # the table in force is kept
+        with pytest.raises(lq.LQError):
+            lq.load_dispatch_table(str(tmp_path / "missing.txt"))
+    finally:
+        lq.load_dispatch_table(None)
+
+
+def test_token_buckets(tmp_path):
+    """M rounds up to the next tuned decode size (1,2,4,8,16,24,32), then to powers of two."""
+    buckets = (1, 2, 4, 8, 16, 24, 32, 64, 128)
+    p = tmp_path / "buckets.txt"
+    p.write_text("".join(f"fp8_dynamic {mb} 4096 4096 1 2 16 {2 + i} 1 1\n" for i, mb in enumerate(buckets)))
+    try:
+        lq.load_dispatch_table(str(p))
+        for M, mb in [(1, 1), (2, 2), (3, 4), (5, 8), (9, 16), (17, 24), (25, 32), (33, 64), (65, 128)]:
+            assert lq.select_variant("fp8_dynamic", M, 4096, 4096).stages == 2 + buckets.index(mb), M
+    finally:
+        lq.load_dispatch_table(None)
