@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized linear-layer GEMM hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl lq|reference]
+
+One step = one pass of the whole hot path over one batch: for every decode
+size M in {1, 2, 4, 8, 16, 24, 32} and every linear of a Qwen3 layer, the
+bf16 activations are quantized (lq_quant_per_token / _group128) and
+multiplied with the pre-quantized weights (lq_scaled_mm, variant from the
+dispatch table).  The step is captured once in a CUDA graph and replayed.
+Weights are kept in several copies that are rotated between M points so
+that every weight read comes from HBM (more than 2x the L2 capacity passes
+between two reads of one copy).
+
+The metric is HBM throughput of algorithmic bytes (weights + activations +
+scales + outputs, plus the quantizers' reads and writes) per second; TFLOP/s
+and the per-shape breakdown are reported beside it.  Multi-GPU runs are
+replicas (each rank runs the whole step on its own GPU; no collective is
+part of the hot path) and report the aggregate.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from quantized_linear_gemm_b200 import inputs, lq  # noqa: E402
+
+CONFIGS = {
+    # name: (format, model shapes, M list)
+    "qwen3-8b-fp8-decode": ("fp8_dynamic", inputs.QWEN3_8B, inputs.DECODE_M),
+    "qwen3-8b-int8-decode": ("w8a8_int8", inputs.QWEN3_8B, inputs.DECODE_M),
+    "qwen3-32b-block-decode": ("block_fp8", inputs.QWEN3_32B, inputs.DECODE_M),
+    "qwen3-32b-fp8-prefill": ("fp8_dynamic", {k: inputs.QWEN3_32B[k] for k in ("gate_up", "down")}, inputs.PREFILL_M),
+    "qwen3-32b-int8-prefill": ("w8a8_int8", {k: inputs.QWEN3_32B[k] for k in ("gate_up", "down")}, inputs.PREFILL_M),
+    "qwen3-32b-block-prefill": ("block_fp8", {k: inputs.QWEN3_32B[k] for k in ("gate_up", "down")}, inputs.PREFILL_M),
+}
+DEFAULT_CONFIG = "qwen3-8b-fp8-decode"
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ sizes
+def gemm_bytes(fmt: str, M: int, N: int, K: int) -> int:
+    return lq.Problem(lq.FORMATS[fmt], M, N, K).bytes
+
+
+def quant_bytes(fmt: str, M: int, K: int) -> int:
+    """bf16 read + codes written + scales written."""
+    scales = 4 * M * (K // 128) if fmt == "block_fp8" else 4 * M
+    return 2 * M * K + M * K + scales
+
+
+# -------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the GPU works."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        exe = shutil.which("nvidia-smi")
+        if not exe:
+            return
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        self.proc = subprocess.Popen([exe, "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                      "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 active=parts[4], hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(loaded), "power_w_max": max(r["power"] for r in rows)}
+
+
+# ------------------------------------------------------------ workload
+class Workload:
+    """Device buffers of one configuration: rotated weight copies, bf16
+    activations, codes, scales and outputs of every (M, layer) call."""
+
+    def __init__(self, config: str, device: torch.device, copies: int = 3, seed: int = 0):
+        self.config = config
+        self.fmt, self.layers, self.ms = CONFIGS[config]
+        self.device = device
+        self.copies = copies
+        f = self.fmt
+        self.weights = {}   # layer -> list of (codes, scales)
+        for li, (layer, (K, N)) in enumerate(self.layers.items()):
+            w = inputs.weights(N, K, seed=inputs.stable_seed(config, "W", layer, seed)).to(device)
+            if f == "block_fp8":
+                q, s = lq.quant_weight_block128(w)
+            else:
+                q, s = lq.quant_per_token(f, w)
+            reps = [(q, s)]
+            for _ in range(copies - 1):
+                reps.append((q.clone(), s.clone()))
+            self.weights[layer] = reps
+            del w
+        # one flat bf16 buffer for every activation, one for every output
+        self.calls = []
+        x_off = c_off = 0
+        for M in self.ms:
+            for layer, (K, N) in self.layers.items():
+                self.calls.append(dict(M=M, layer=layer, K=K, N=N, x_off=x_off, c_off=c_off))
+                x_off += -(-M * K // 64) * 64
+                c_off += -(-M * N // 64) * 64
+        self.x_all = torch.empty(x_off, dtype=torch.bfloat16, device=device)
+        self.c_all = torch.empty(c_off, dtype=torch.bfloat16, device=device)
+        code_dt = torch.int8 if f == "w8a8_int8" else torch.uint8
+        for i, c in enumerate(self.calls):
+            M, K, N = c["M"], c["K"], c["N"]
+            x = inputs.activations(M, K, seed=inputs.stable_seed(config, "A", c["layer"], M, seed))
+            c["x"] = self.x_all[c["x_off"]:c["x_off"] + M * K].view(M, K)
+            c["x"].copy_(x)
+            c["C"] = self.c_all[c["c_off"]:c["c_off"] + M * N].view(M, N)
+            c["q"] = torch.empty((M, K), dtype=code_dt, device=device)
+            c["s"] = torch.empty((M, K // 128) if f == "block_fp8" else (M,), dtype=torch.float32, device=device)
+            c["copy"] = self.ms.index(M) % copies
+            c["variant"] = lq.select_variant(f, M, N, K)
+        self.x_host = torch.empty(self.x_all.shape, dtype=torch.bfloat16, pin_memory=True)
+        self.x_host.copy_(self.x_all)
+        self.c_host = torch.empty(self.c_all.shape, dtype=torch.bfloat16, pin_memory=True)
+        ws = max(lq.workspace_bytes(f, c["M"], c["N"], c["K"], c["variant"]) for c in self.calls)
+        lq.reserve_workspace(device.index, ws)
+
+    # bytes / flops of one step
+    @property
+    def gemm_bytes(self) -> int:
+        return sum(gemm_bytes(self.fmt, c["M"], c["N"], c["K"]) for c in self.calls)
+
+    @property
+    def quant_bytes(self) -> int:
+        return sum(quant_bytes(self.fmt, c["M"], c["K"]) for c in self.calls)
+
+    @property
+    def flops(self) -> int:
+        return sum(2 * c["M"] * c["N"] * c["K"] for c in self.calls)
+
+    def launches_per_step(self, gemm=True, quant=True) -> int:
+        n = 0
+        for c in self.calls:
+            v = c["variant"]
+            if quant:
+                n += 1
+            if gemm:
+                n += 1 + (1 if (v.split_k > 1 and v.reduce == 0) else 0)
+        return n
+
+    def quant(self, c, stream):
+        if self.fmt == "block_fp8":
+            lq.quant_per_token_group128(c["x"], c["q"], c["s"], stream=stream)
+        else:
+            lq.quant_per_token(self.fmt, c["x"], c["q"], c["s"], stream=stream)
+
+    def gemm(self, c, stream, copy=None):
+        qb, sb = self.weights[c["layer"]][c["copy"] if copy is None else copy]
+        lq.scaled_mm(self.fmt, c["q"], c["s"], qb, sb, C=c["C"], variant=c["variant"], stream=stream)
+
+    def step(self, stream, gemm=True, quant=True):
+        for c in self.calls:
+            if quant:
+                self.quant(c, stream)
+            if gemm:
+                self.gemm(c, stream)
+
+
+def capture(fn, stream) -> torch.cuda.CUDAGraph:
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn()   # eager run once (allocations, lazy module loads)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_replays(g: torch.cuda.CUDAGraph, n: int, stream, pre=None, post=None) -> float:
+    """Total ms of n replays, measured with CUDA events on `stream`."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(n):
+            if pre:
+                pre()
+            g.replay()
+            if post:
+                post()
+        end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
+# ----------------------------------------------------------- CPU leg
+def cpu_baseline(config: str, budget_s: float = 20.0) -> dict:
+    """The oracle, as it stands, on a bounded sample of the same workload:
+    every linear at the middle decode size (activation quantization plus the
+    exact product), repeated until about `budget_s` seconds have passed."""
+    import numpy as np
+    from oracle import lq_oracle as O
+
+    fmt, layers, ms = CONFIGS[config]
+    M = ms[len(ms) // 2]
+    prepared = []
+    for layer, (K, N) in layers.items():
+        w = inputs.weights(N, K, seed=inputs.stable_seed(config, "W", layer, 0)).float().numpy()
+        if fmt == "block_fp8":
+            qb, sb = O.quant_weight_block128(w)
+        else:
+            qb, sb = O.quant_per_channel(w, fmt)
+        x = inputs.activations(M, K, seed=inputs.stable_seed(config, "A", layer, M, 0)).float().numpy()
+        prepared.append((M, N, K, x, qb, sb))
+    nbytes = 0
+    t0 = time.perf_counter()
+    rounds = 0
+    while True:
+        for (M_, N, K, x, qb, sb) in prepared:
+            if fmt == "block_fp8":
+                qa, sa = O.quant_per_token_group128(x)
+            else:
+                qa, sa = O.quant_per_token(x, fmt)
+            O.scaled_mm_ref(fmt, qa, sa, qb, sb)
+            nbytes += gemm_bytes(fmt, M_, N, K) + quant_bytes(fmt, M_, K)
+        rounds += 1
+        if time.perf_counter() - t0 > budget_s or rounds >= 50:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{config}: all {len(layers)} linears at M={M}, quantize + exact product, {rounds} round(s), "
+                      f"{dt:.1f} s (numpy int64 matmul, single thread)"}
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = args.config
+    per_step_budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(cfg, budget_s=per_step_budget)
+    vals = []
+    t0 = time.perf_counter()
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline(cfg, budget_s=per_step_budget)
+        vals.append(last["value"])
+    dt = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(1, args.steps),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE[CONFIGS[cfg][0]],
+           "data": "synthetic", "config": {"workload": cfg, "sample": last["sample"]},
+           "cpu_baseline": {"value": value, "unit": "GB/s", "cores": last["cores"], "kind": "oracle",
+                            "sample": last["sample"]},
+           "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+METRIC = "scaled_mm HBM GB/s (algorithmic bytes) at M=1..32 on Qwen3 linear shapes"
+DTYPE = {"fp8_dynamic": "e4m3 x e4m3 -> f32", "w8a8_int8": "s8 x s8 -> s32", "block_fp8": "e4m3 x e4m3 -> f32"}
+
+
+# ---------------------------------------------------------------- main
+def main() -> None:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="lq", choices=["lq", "reference"])
+    ap.add_argument("--copies", type=int, default=3, help="weight copies rotated to defeat L2 reuse")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-shape-reps", type=int, default=30)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    lq.init_device(local)
+    peaks = load_peaks()
+
+    wl = Workload(args.config, device, copies=args.copies)
+    stream = torch.cuda.Stream(device=device)
+    stream.wait_stream(torch.cuda.current_stream())
+
+    # one CUDA graph per step (quant + GEMM of every call), and GEMM-only / quant-only graphs
+    g_step = capture(lambda: wl.step(stream), stream)
+    g_gemm = capture(lambda: wl.step(stream, quant=False), stream)
+    g_quant = capture(lambda: wl.step(stream, gemm=False), stream)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    # warm-up, kept running for at least ~1 s so that clocks settle under load
+    t_warm = time.perf_counter()
+    time_replays(g_step, args.warmup, stream)
+    while time.perf_counter() - t_warm < 1.0:
+        time_replays(g_step, 20, stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ms_total = time_replays(g_step, args.steps, stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+
+    step_bytes = wl.gemm_bytes + wl.quant_bytes
+    value = world * step_bytes * args.steps / (ms_total * 1e-3) / 1e9
+    tflops = world * wl.flops * args.steps / (ms_total * 1e-3) / 1e12
+
+    # dominant kernel: scaled_mm, all launches of a step, timed on its own
+    n_gemm_reps = max(50, min(args.steps, 500))
+    time_replays(g_gemm, 10, stream)
+    ms_gemm = time_replays(g_gemm, n_gemm_reps, stream) / n_gemm_reps
+    time_replays(g_quant, 10, stream)
+    ms_quant = time_replays(g_quant, n_gemm_reps, stream) / n_gemm_reps
+    gemm_gbs = wl.gemm_bytes / (ms_gemm * 1e-3) / 1e9
+
+    # per-shape breakdown: R calls of one shape per graph, rotating weight copies
+    per_shape = []
+    reps = args.per_shape_reps
+    for c in wl.calls:
+        def one(c=c):
+            for r in range(reps):
+                wl.gemm(c, stream, copy=r % wl.copies)
+        g = capture(one, stream)
+        time_replays(g, 3, stream)
+        ms = time_replays(g, 10, stream) / (10 * reps)
+        b = gemm_bytes(wl.fmt, c["M"], c["N"], c["K"])
+        per_shape.append({"layer": c["layer"], "M": c["M"], "N": c["N"], "K": c["K"], "us": round(ms * 1e3, 3),
+                          "GB/s": round(b / (ms * 1e-3) / 1e9, 1), "TFLOP/s": round(2 * c["M"] * c["N"] * c["K"] / (ms * 1e-3) / 1e12, 2),
+                          "frac_hbm": round(b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+                          "variant": c["variant"].as_dict()})
+        del g
+
+    # end to end through the public API: H2D of the step's activations from
+    # pinned host memory, the step, D2H of every output
+    def h2d():
+        wl.x_all.copy_(wl.x_host, non_blocking=True)
+
+    def d2h():
+        wl.c_host.copy_(wl.c_all, non_blocking=True)
+
+    time_replays(g_step, 3, stream, pre=h2d, post=d2h)
+    e2e_n = max(20, min(args.steps, 500))
+    ms_e2e = time_replays(g_step, e2e_n, stream, pre=h2d, post=d2h) / e2e_n
+    e2e_val = world * step_bytes / (ms_e2e * 1e-3) / 1e9
+
+    del g_step, g_gemm, g_quant
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = cpu_baseline(args.config, budget_s=15.0)
+
+    layers = ",".join(f"{k}({K}x{N})" for k, (K, N) in wl.layers.items())
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": DTYPE[wl.fmt],
+        "data": "synthetic",
+        "config": {"workload": args.config, "format": wl.fmt, "layers": layers, "M": list(wl.ms),
+                   "calls_per_step": len(wl.calls), "parallelism": f"replicas x{world}",
+                   "l2": f"{wl.copies} weight copies rotated per M point (> 2x L2 between reuses)",
+                   "graph": "one CUDA graph per step"},
+        "tflops": round(tflops, 3),
+        "frac_hbm_step": round(value / world / peaks["hbm_gbs"], 4),
+        "roofline": {"bound": "hbm", "kernel": "scaled_mm (all launches of one step)",
+                     "achieved": round(gemm_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gemm_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                     "algorithmic_bytes_per_step": wl.gemm_bytes, "launches_per_step": wl.launches_per_step(quant=False),
+                     "us_per_step": round(ms_gemm * 1e3, 2), "peak_source": peaks["source"]},
+        "quant_us_per_step": round(ms_quant * 1e3, 2),
+        "clocks": clocks,
+        "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "ms_per_step": round(ms_e2e, 5),
+                "h2d_bytes_per_step": wl.x_all.numel() * 2, "d2h_bytes_per_step": wl.c_all.numel() * 2},
+        "gpu_launches": wl.launches_per_step() * args.steps,
+        "per_shape": per_shape,
+    }
+    if cpu is not None:
+        out["cpu_baseline"] = cpu
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()
