@@ -89,8 +89,13 @@ typedef enum {
  *            Swap-AB: 16, 32 or 64.
  *  stages  : depth of the shared-memory ring (2..16), 0 = the deepest that
  *            fits.
- *  reduce  : for split_k > 1: 0 = a separate reduction kernel, 1 = the last
- *            CTA to finish a tile reduces it (arrival counter).
+ *  reduce  : for split_k > 1: 0 = partials to a global workspace and a
+ *            separate reduction kernel; 1 = partials to the workspace and the
+ *            last CTA to finish a tile reduces it (arrival counter); 2 = the
+ *            split_k CTAs of a tile form a thread-block cluster and reduce
+ *            through distributed shared memory, each finishing a slice of the
+ *            tile (split_k <= 16, no workspace).  All three sum the partials
+ *            in the order s = 0..split_k-1 and give identical results.
  *  pdl     : 0 = plain launch;
  *            1 = programmatic dependent launch: the kernel's set-up overlaps
  *            the tail of the previous kernel on the stream, and all of its
@@ -133,8 +138,8 @@ typedef struct {
  * Errors: LQ_ERR_INVALID_ARG / LQ_ERR_ALIGNMENT / LQ_ERR_UNSUPPORTED_SHAPE
  * before any launch; LQ_ERR_WORKSPACE when split_k > 1 needs a larger
  * workspace while `stream` is capturing; LQ_ERR_CUDA when a launch fails.
- * A Split-K call uses the library's per-device workspace: Split-K calls on
- * different streams of one device must not overlap in time.
+ * A Split-K call with reduce 0 or 1 uses the library's per-device workspace:
+ * such calls on different streams of one device must not overlap in time.
  */
 lq_status lq_scaled_mm(lq_fmt fmt, const void *A, const float *a_scales,
                        const void *B, const float *b_scales, void *C,
@@ -200,7 +205,9 @@ lq_status lq_select_variant(lq_fmt fmt, int64_t M, int64_t N, int64_t K,
 /*
  * Replace the dispatch table by the entries of a text file (one entry per
  * line: "fmt m_bucket N K swap_ab split_k tile_n stages reduce pdl", '#'
- * starts a comment).  path == NULL restores the compiled-in table.  On error
+ * starts a comment).  path == NULL restores the compiled-in table.  At
+ * start-up the environment variable LQ_DISPATCH_TABLE, when set, names a
+ * file that replaces the compiled-in table.  On error
  * the current table is kept and LQ_ERR_TABLE is returned.  Not thread-safe
  * with concurrent lq_scaled_mm calls that pass variant == NULL.
  */
@@ -223,7 +230,8 @@ lq_status lq_init_device(int device);
  */
 lq_status lq_reserve_workspace(int device, size_t bytes);
 
-/* Workspace bytes that lq_scaled_mm needs for (fmt, M, N, K, variant). */
+/* Workspace bytes that lq_scaled_mm needs for (fmt, M, N, K, variant):
+ * split_k * M * N * 4 for reduce 0 or 1, else 0. */
 size_t lq_workspace_bytes(lq_fmt fmt, int64_t M, int64_t N, int64_t K,
                           const lq_variant *variant);
 

@@ -171,8 +171,21 @@ std::shared_ptr<const std::vector<TableEntry>> default_table() {
   return t;
 }
 
+bool parse_table_file(const char* path, std::vector<TableEntry>* out, std::string* err);
+
+// The table in force: the file named by LQ_DISPATCH_TABLE when it is set and
+// valid, else the compiled-in table.
 std::shared_ptr<const std::vector<TableEntry>>& table_slot() {
-  static std::shared_ptr<const std::vector<TableEntry>> t = default_table();
+  static std::shared_ptr<const std::vector<TableEntry>> t = [] {
+    const char* env = std::getenv("LQ_DISPATCH_TABLE");
+    if (env && *env) {
+      auto f = std::make_shared<std::vector<TableEntry>>();
+      std::string err;
+      if (parse_table_file(env, f.get(), &err)) return std::shared_ptr<const std::vector<TableEntry>>(f);
+      std::fprintf(stderr, "lq: LQ_DISPATCH_TABLE=%s not used (%s)\n", env, err.c_str());
+    }
+    return default_table();
+  }();
   return t;
 }
 std::mutex g_table_mutex;
@@ -213,6 +226,7 @@ lq_variant heuristic_variant(int fmt, int64_t M, int64_t N, int64_t K) {
     int S = 1;
     while (S < 256 && tiles * S * 2 <= 2 * kNumSms && T / (S * 2) >= 2) S *= 2;
     v.split_k = S;
+    v.reduce = S <= 16 ? 2 : 1;
     const int per_split = static_cast<int>((T + S - 1) / S);
     const int cap = max_stages_fit(v.tile_n, 2);
     v.stages = per_split < 2 ? 2 : (per_split > cap ? cap : per_split);
@@ -223,6 +237,7 @@ lq_variant heuristic_variant(int fmt, int64_t M, int64_t N, int64_t K) {
     int S = 1;
     while (S < 256 && tiles * S < kNumSms && T / (S * 2) >= 4) S *= 2;
     v.split_k = S;
+    v.reduce = S <= 16 ? 2 : 1;
     v.stages = max_stages_fit(v.tile_n, 1);
   }
   return v;
@@ -247,7 +262,8 @@ bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
 lq_status check_variant(int fmt, const lq_variant& v) {
   if (v.swap_ab != 0 && v.swap_ab != 1) return LQ_ERR_INVALID_ARG;
   if (!is_pow2(v.split_k) || v.split_k > 256) return LQ_ERR_INVALID_ARG;
-  if (v.reduce != 0 && v.reduce != 1) return LQ_ERR_INVALID_ARG;
+  if (v.reduce < 0 || v.reduce > 2) return LQ_ERR_INVALID_ARG;
+  if (v.reduce == 2 && v.split_k > 16) return LQ_ERR_INVALID_ARG;   // a cluster holds at most 16 CTAs
   if (v.pdl < 0 || v.pdl > 2) return LQ_ERR_INVALID_ARG;
   if (v.swap_ab) {
     if (v.tile_n != 16 && v.tile_n != 32 && v.tile_n != 64) return LQ_ERR_INVALID_ARG;
@@ -321,7 +337,7 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   p.KB = static_cast<int>(K / 128);
   p.S = v.split_k;
   p.stages = v.stages;
-  p.reduce_in_kernel = v.reduce;
+  p.reduce_mode = v.reduce;
   p.early_weights = v.pdl == 2 ? 1 : 0;
   p.a_s = a_s;
   p.b_s = b_s;
@@ -329,7 +345,7 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   p.acc_out = acc_out;
   p.status = d->status;
   p.wait_limit_ns = wait_limit_ns();
-  if (v.split_k > 1) {
+  if (v.split_k > 1 && v.reduce != 2) {   // the cluster reduction needs no global workspace
     const size_t need = static_cast<size_t>(v.split_k) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
     rc = ensure_workspace(d, need, stream);
     if (rc != LQ_OK) return rc;
@@ -344,6 +360,7 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
   l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages);
   l.pdl = v.pdl != 0;
+  l.cluster_z = (v.split_k > 1 && v.reduce == 2) ? v.split_k : 1;
   l.stream = stream;
 
   cudaError_t e;
@@ -356,7 +373,7 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
     cudaGetLastError();
     return LQ_ERR_CUDA;
   }
-  if (v.split_k > 1 && !v.reduce) {
+  if (v.split_k > 1 && v.reduce == 0) {
     e = lq::launch_splitk_reduce(fmt, p, v.pdl != 0, stream);
     if (e != cudaSuccess) {
       cudaGetLastError();
@@ -528,7 +545,7 @@ size_t lq_workspace_bytes(lq_fmt fmt, int64_t M, int64_t N, int64_t K, const lq_
   lq_variant v{};
   if (variant) v = *variant;
   else if (!lookup_table(static_cast<int>(fmt), M, N, K, &v)) v = heuristic_variant(static_cast<int>(fmt), M, N, K);
-  if (v.split_k <= 1) return 0;
+  if (v.split_k <= 1 || v.reduce == 2) return 0;
   return static_cast<size_t>(v.split_k) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
 }
 

@@ -19,7 +19,7 @@ struct GemmParams {
   int KB;              // K / 128 (Block_FP8 scale row length)
   int S;               // split_k
   int stages;          // shared-memory ring depth
-  int reduce_in_kernel;
+  int reduce_mode;     // S > 1: 0 separate kernel, 1 last-arriver (global), 2 cluster (DSMEM)
   int early_weights;   // stream weight tiles before the grid dependency wait
   const float* a_s;
   const float* b_s;
@@ -39,6 +39,7 @@ struct GemmLaunch {
   dim3 grid;
   int smem_bytes;
   int pdl;
+  int cluster_z;       // > 1: launch clusters of (1, 1, cluster_z) CTAs
   cudaStream_t stream;
 };
 

@@ -47,10 +47,18 @@ __host__ __device__ constexpr int tmem_cols_for(int cols) {
   return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
 }
 
+// Bytes of the ring region: `stages` slots, and at least the 128 x TN 32-bit
+// partial tile that the cluster Split-K reduction stages there afterwards.
+template <int TN>
+__host__ __device__ constexpr int ring_bytes(int stages) {
+  return stages * TileShape<TN>::kStageBytes > TN * kTileM * 4 ? stages * TileShape<TN>::kStageBytes
+                                                                 : TN * kTileM * 4;
+}
+
 // Shared-memory bytes the kernel needs for `stages` ring slots.
 template <int TN>
 __host__ __device__ constexpr int gemm_smem_bytes(int stages) {
-  return 1024 /* alignment slack */ + stages * TileShape<TN>::kStageBytes + 64 * 8 /* barriers */ + 64;
+  return 1024 /* alignment slack */ + ring_bytes<TN>(stages) + 64 * 8 /* barriers */ + 64;
 }
 
 struct SmemCtl {
@@ -108,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
   const int stages = p.stages;
   uint8_t* ring = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + stages * Shape::kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + ring_bytes<TN>(stages));
   SmemCtl c;
   c.full = bars;
   c.empty = bars + stages;
@@ -316,10 +324,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ok = __all_sync(0xffffffffu, ok && !*c.abort_flag);
 
+    const bool cluster_mode = p.S > 1 && p.reduce_mode == 2;
+    // The ring's last readers were the tensor core (async proxy); order them
+    // before the generic-proxy stores of the cluster partial tile.
+    if (cluster_mode) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (ok) {
       float* wsf = reinterpret_cast<float*>(p.ws);
       int32_t* wsi = reinterpret_cast<int32_t*>(p.ws);
-      const bool split_mode = p.S > 1;
+      const bool split_mode = p.S > 1 && !cluster_mode;   // partials to the global workspace
 
 #pragma unroll
       for (int c0 = 0; c0 < TN; c0 += CH) {
@@ -336,6 +348,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int j = 0; j < CH; ++j) v[j] = 0u;   // empty split: zero partial
+        }
+
+        if (cluster_mode) {
+          // partial tile -> own shared memory, [column j][row r] (the ring is free now)
+          uint32_t* red = reinterpret_cast<uint32_t*>(ring);
+#pragma unroll
+          for (int j = 0; j < CH; ++j) red[(c0 + j) * kTileM + r] = v[j];
+          continue;
         }
 
         if (SWAP) {
@@ -410,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------- in-kernel Split-K reduce
     // Every epilogue thread reaches both named barriers, also after a
     // timeout (then this CTA does not count itself and no CTA reduces).
-    if (p.S > 1 && p.reduce_in_kernel) {
+    if (p.S > 1 && p.reduce_mode == 1) {
       float* wsf = reinterpret_cast<float*>(p.ws);
       int32_t* wsi = reinterpret_cast<int32_t*>(p.ws);
       __threadfence();
@@ -480,6 +500,96 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (warp == 2 && lane == 0) p.counters[tile_id] = 0;   // ready for the next launch / replay
       }
     }
+  }
+
+  // ------------------------------------------------ cluster Split-K reduce
+  // The S CTAs of a tile form one cluster (cluster rank == split index).
+  // After the first cluster barrier every partial tile sits in its CTA's
+  // shared memory; CTA s sums columns [s TN/S, (s+1) TN/S) of all S partials
+  // in the fixed order 0..S-1 (the order of the other reduction modes, so the
+  // result is the same bit for bit), scales and stores them.  The second
+  // barrier keeps every CTA alive until the others have read its partial.
+  // All threads of all CTAs execute both barriers on every path.
+  if (p.S > 1 && p.reduce_mode == 2) {
+    __syncwarp();
+    cluster_sync_all();
+    if (warp >= 2 && !*c.abort_flag) {
+      const int q = warp & 3;
+      const int r = q * 32 + lane;
+      const int S = p.S;
+      const int W = TN / S;
+      const int j0 = split * W;
+      const int64_t M = p.M, N = p.N;
+      uint32_t rb[16];
+      const uint32_t local = smem_addr(ring);
+#pragma unroll
+      for (int s = 0; s < 16; ++s) rb[s] = s < S ? dsmem_map(local, static_cast<uint32_t>(s)) : 0u;
+      if (SWAP) {
+        const int64_t n = x_row0 + r;
+        const float bsn = (!kBlocked && n < N) ? __ldg(p.b_s + n) : 1.f;
+        for (int j = j0; j < j0 + W; ++j) {
+          const uint32_t off = static_cast<uint32_t>((j * kTileM + r) * 4);
+          uint32_t u[16];
+#pragma unroll
+          for (int s = 0; s < 16; ++s)
+            if (s < S) u[s] = dsmem_ld_u32(rb[s] + off);
+          float sf = 0.f;
+          int32_t si = 0;
+#pragma unroll
+          for (int s = 0; s < 16; ++s)
+            if (s < S) {
+              if (kInt8) si += static_cast<int32_t>(u[s]);
+              else sf += __uint_as_float(u[s]);
+            }
+          const int64_t m = y_row0 + j;
+          if (n < N && m < M) {
+            float val;
+            if (kBlocked) val = sf;
+            else val = (kInt8 ? static_cast<float>(si) : sf) * __ldg(p.a_s + m) * bsn;
+            p.C[m * N + n] = __float2bfloat16_rn(val);
+            if (kInt8 && p.acc_out) p.acc_out[m * N + n] = si;
+          }
+        }
+      } else {
+        const int64_t m = x_row0 + r;
+        const float asm_ = (!kBlocked && m < M) ? __ldg(p.a_s + m) : 1.f;
+        for (int j = j0; j < j0 + W; j += 4) {   // W >= 4 for Standard tiles (TN >= 64, S <= 16)
+          uint32_t u[4][16];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int s = 0; s < 16; ++s)
+              if (s < S) u[e][s] = dsmem_ld_u32(rb[s] + static_cast<uint32_t>(((j + e) * kTileM + r) * 4));
+          float f[4];
+          int32_t iv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float sf = 0.f;
+            int32_t si = 0;
+#pragma unroll
+            for (int s = 0; s < 16; ++s)
+              if (s < S) {
+                if (kInt8) si += static_cast<int32_t>(u[e][s]);
+                else sf += __uint_as_float(u[e][s]);
+              }
+            iv[e] = si;
+            f[e] = kInt8 ? static_cast<float>(si) : sf;
+          }
+          const int64_t n = y_row0 + j;
+          if (m < M && n < N) {
+            if (!kBlocked) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * __ldg(p.b_s + n + e);
+            }
+            *reinterpret_cast<uint2*>(p.C + m * N + n) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+            if (kInt8 && p.acc_out)
+              *reinterpret_cast<int4*>(p.acc_out + m * N + n) = make_int4(iv[0], iv[1], iv[2], iv[3]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();
   }
 
   // -------------------------------------------------------------- teardown

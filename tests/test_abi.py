@@ -66,7 +66,7 @@ def test_empty_problem_is_a_noop():
 
 @pytest.mark.parametrize("field,value", [
     ("split_k", 3), ("split_k", 512), ("split_k", 0), ("swap_ab", 2), ("tile_n", 48),
-    ("stages", 1), ("stages", 17), ("reduce", 2), ("pdl", 5),
+    ("stages", 1), ("stages", 17), ("reduce", 3), ("pdl", 5),
 ])
 def test_variant_checks(field, value):
     v = lq.make_variant(swap_ab=1, split_k=2, tile_n=32)

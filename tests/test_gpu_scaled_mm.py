@@ -27,6 +27,12 @@ for tn in (16, 32, 64):
     VARIANTS.append(dict(swap_ab=1, tile_n=tn, split_k=2, stages=2, reduce=0))
     VARIANTS.append(dict(swap_ab=1, tile_n=tn, split_k=8, stages=4, reduce=1))
 VARIANTS.append(dict(swap_ab=1, tile_n=32, split_k=16, stages=0, reduce=1, pdl=0))
+for tn in (16, 32, 64):
+    VARIANTS.append(dict(swap_ab=1, tile_n=tn, split_k=4, stages=2, reduce=2))
+VARIANTS.append(dict(swap_ab=1, tile_n=16, split_k=16, stages=2, reduce=2, pdl=2))
+for tn in (64, 128, 256):
+    VARIANTS.append(dict(swap_ab=0, tile_n=tn, split_k=2, stages=0, reduce=2))
+VARIANTS.append(dict(swap_ab=0, tile_n=64, split_k=16, stages=3, reduce=2))
 VARIANTS.append(dict(swap_ab=0, tile_n=128, split_k=16, stages=4, reduce=0, pdl=0))
 
 
@@ -193,3 +199,24 @@ def test_default_variant_selection_runs(cuda_device):
         for M in (1, 24, 100):
             prob = make_problem(fmt, M, 256, 1024, seed=14)
             assert_close(_run(prob, None), prob.reference(), f"default fmt={fmt} M={M}")
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
+@pytest.mark.parametrize("swap,tn", [(1, 16), (1, 32), (1, 64), (0, 64), (0, 128), (0, 256)])
+def test_reduce_modes_bitwise_identical(cuda_device, fmt, swap, tn):
+    """Separate kernel, last arriver and cluster reduction sum the same
+    partials in the same order: identical bits, and within tolerance."""
+    if fmt == lq.BLOCK_FP8 and not swap and tn == 256:
+        pytest.skip("Block_FP8 Standard tiles stop at 128")
+    prob = make_problem(fmt, 40, 512, 2304, seed=15)
+    A, sa, B, sb = prob.device()
+    ref = prob.reference()
+    for S in (2, 4, 8, 16):
+        outs = []
+        for red in (0, 1, 2):
+            v = lq.make_variant(swap_ab=swap, tile_n=tn, split_k=S, stages=2, reduce=red)
+            outs.append(lq.scaled_mm(fmt, A, sa, B, sb, variant=v).clone())
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2]), f"S={S}"
+        assert_close(outs[2], ref, f"cluster S={S}")
+    assert lq.device_status(0) == 0
