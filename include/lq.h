@@ -242,6 +242,21 @@ size_t lq_workspace_bytes(lq_fmt fmt, int64_t M, int64_t N, int64_t K,
  */
 lq_status lq_device_status(int device);
 
+/*
+ * Diagnostics: while `device_buffer` is non-NULL, every scaled_mm kernel
+ * launched afterwards writes 12 %globaltimer stamps (ns) per CTA to
+ * device_buffer[cta * 12 + i], cta = x + gx * (y + gy * z) over the launch
+ * grid: 0 entry, 1 set-up done, 2 producer past the wait for the previous
+ * kernel, 3 first operand stage landed, 4 last MMA issued, 5 accumulator
+ * ready, 6 outputs or partials written, 7 exit, and for the cluster Split-K
+ * reduction 8 past its first barrier, 9 reduced tile stored, 10 past its
+ * second barrier (slots a launch does not reach keep their old contents).
+ * The buffer must hold 12 uint64 per CTA of every traced launch.  A launch
+ * captured into a CUDA graph keeps the pointer that was set at capture
+ * time.  NULL turns tracing off.
+ */
+lq_status lq_set_trace(uint64_t *device_buffer);
+
 /* Human-readable name of a status code (static storage). */
 const char *lq_status_string(lq_status status);
 

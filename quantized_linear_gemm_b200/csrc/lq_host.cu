@@ -50,6 +50,7 @@ struct DeviceState {
 
 std::mutex g_dev_mutex;
 DeviceState g_dev[kMaxDevices];
+std::atomic<uint64_t*> g_trace{nullptr};   // diagnostics: per-CTA stamps of the next launches
 
 uint64_t wait_limit_ns() {
   static uint64_t v = [] {
@@ -205,12 +206,12 @@ int64_t m_bucket(int64_t M) {
 }
 
 // Deepest ring that fits when `ctas_per_sm` CTAs share one SM's shared memory.
-int max_stages_fit(int tile_n, int ctas_per_sm) {
+int max_stages_fit(int tile_n, int ctas_per_sm, bool cluster_reduce) {
   const int share = (228 * 1024) / ctas_per_sm - 1024;
   const int budget = share < kMaxSmemPerCta ? share : kMaxSmemPerCta;
   int best = 2;
   for (int s = 2; s <= 16; ++s)
-    if (lq::gemm_smem_bytes_for(tile_n, s) <= budget) best = s;
+    if (lq::gemm_smem_bytes_for(tile_n, s, cluster_reduce) <= budget) best = s;
   return best;
 }
 
@@ -228,7 +229,7 @@ lq_variant heuristic_variant(int fmt, int64_t M, int64_t N, int64_t K) {
     v.split_k = S;
     v.reduce = S <= 16 ? 2 : 1;
     const int per_split = static_cast<int>((T + S - 1) / S);
-    const int cap = max_stages_fit(v.tile_n, 2);
+    const int cap = max_stages_fit(v.tile_n, 2, S > 1 && v.reduce == 2);
     v.stages = per_split < 2 ? 2 : (per_split > cap ? cap : per_split);
   } else {
     v.swap_ab = 0;
@@ -238,7 +239,7 @@ lq_variant heuristic_variant(int fmt, int64_t M, int64_t N, int64_t K) {
     while (S < 256 && tiles * S < kNumSms && T / (S * 2) >= 4) S *= 2;
     v.split_k = S;
     v.reduce = S <= 16 ? 2 : 1;
-    v.stages = max_stages_fit(v.tile_n, 1);
+    v.stages = max_stages_fit(v.tile_n, 1, S > 1 && v.reduce == 2);
   }
   return v;
 }
@@ -272,7 +273,9 @@ lq_status check_variant(int fmt, const lq_variant& v) {
     if (fmt == lq::kFmtBlock && v.tile_n == 256) return LQ_ERR_INVALID_ARG;
   }
   if (v.stages != 0 && (v.stages < 2 || v.stages > 16)) return LQ_ERR_INVALID_ARG;
-  if (v.stages != 0 && lq::gemm_smem_bytes_for(v.tile_n, v.stages) > kMaxSmemPerCta) return LQ_ERR_INVALID_ARG;
+  if (v.stages != 0 &&
+      lq::gemm_smem_bytes_for(v.tile_n, v.stages, v.split_k > 1 && v.reduce == 2) > kMaxSmemPerCta)
+    return LQ_ERR_INVALID_ARG;
   return LQ_OK;
 }
 
@@ -315,7 +318,8 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   }
   rc = check_variant(fmt, v);
   if (rc != LQ_OK) return rc;
-  if (v.stages == 0) v.stages = max_stages_fit(v.tile_n, 1);
+  const bool cluster_reduce = v.split_k > 1 && v.reduce == 2;
+  if (v.stages == 0) v.stages = max_stages_fit(v.tile_n, 1, cluster_reduce);
 
   const int64_t x_rows = v.swap_ab ? N : M;
   const int64_t y_rows = v.swap_ab ? M : N;
@@ -345,6 +349,7 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   p.acc_out = acc_out;
   p.status = d->status;
   p.wait_limit_ns = wait_limit_ns();
+  p.trace = g_trace.load();
   if (v.split_k > 1 && v.reduce != 2) {   // the cluster reduction needs no global workspace
     const size_t need = static_cast<size_t>(v.split_k) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
     rc = ensure_workspace(d, need, stream);
@@ -358,7 +363,7 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   if (!encode_operand(&l.tmX, x_ptr, x_rows, K, 128) || !encode_operand(&l.tmY, y_ptr, y_rows, K, v.tile_n))
     return LQ_ERR_CUDA;
   l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
-  l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages);
+  l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce);
   l.pdl = v.pdl != 0;
   l.cluster_z = (v.split_k > 1 && v.reduce == 2) ? v.split_k : 1;
   l.stream = stream;
@@ -445,6 +450,11 @@ const char* lq_status_string(lq_status s) {
 }
 
 const char* lq_version(void) { return "lq 0.1.0 (sm_100a)"; }
+
+lq_status lq_set_trace(uint64_t* device_buffer) {
+  g_trace.store(device_buffer);
+  return LQ_OK;
+}
 
 lq_status lq_scaled_mm(lq_fmt fmt, const void* A, const float* a_scales, const void* B, const float* b_scales,
                        void* C, int64_t M, int64_t N, int64_t K, const lq_variant* variant, lq_stream_t stream) {

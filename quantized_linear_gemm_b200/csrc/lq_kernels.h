@@ -29,7 +29,10 @@ struct GemmParams {
   int32_t* acc_out;    // optional exact INT8 accumulators [M, N]
   int* status;         // device status word (bit set per timed-out wait site)
   uint64_t wait_limit_ns;
+  uint64_t* trace;     // optional: kTraceSlots globaltimer stamps per CTA
 };
+
+constexpr int kTraceSlots = 12;
 
 // Launch description filled by the host library.
 struct GemmLaunch {
@@ -51,8 +54,9 @@ cudaError_t launch_scaled_mm_int8(const GemmLaunch& l, int swap_ab, int tile_n);
 cudaError_t launch_scaled_mm_block(const GemmLaunch& l, int swap_ab, int tile_n);
 cudaError_t launch_splitk_reduce(int fmt, const GemmParams& p, int pdl, cudaStream_t stream);
 
-// Largest dynamic shared memory the GEMM kernel may use for (swap_ab, tile_n, stages).
-int gemm_smem_bytes_for(int tile_n, int stages);
+// Dynamic shared memory of the GEMM kernel for (tile_n, stages), with or
+// without the cluster Split-K reduction (reduce mode 2 with split_k > 1).
+int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce);
 
 // Quantization kernels (quant_kernels.cu).
 cudaError_t launch_quant_per_token(int fmt, const void* x, void* q, float* scales, int64_t M, int64_t K,

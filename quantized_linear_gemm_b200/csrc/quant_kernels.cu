@@ -88,7 +88,48 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return red[0];
 }
 
-// One CTA per row.  Two passes over the row (the second hits L1/L2).
+// One CTA per row, the row held in registers (VPT 16-byte vectors per
+// thread): one global read, a block-wide amax, then quantization.
+template <bool kInt8, int VPT>
+__global__ void __launch_bounds__(256) quant_per_token_reg_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                   uint8_t* __restrict__ q,
+                                                                   float* __restrict__ scales, int64_t K) {
+  __shared__ float red[32];
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int64_t row = blockIdx.x;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
+  const int nvec = static_cast<int>(K / 8);
+  uint4 v[VPT];
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * 256;
+    v[i] = idx < nvec ? __ldg(xr + idx) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    float f[8];
+    bf16x8_to_f32(v[i], f);
+    a = fmaxf(a, amax8(f));
+  }
+  const float amax = block_max<256>(a, red);
+  const float s = scale_from_amax(amax, kInt8 ? kInt8Max : kE4m3Max);
+  if (threadIdx.x == 0) scales[row] = s;
+  uint2* qr = reinterpret_cast<uint2*>(q + row * K);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * 256;
+    if (idx < nvec) {
+      float f[8];
+      bf16x8_to_f32(v[i], f);
+      qr[idx] = kInt8 ? encode8_int8(f, s) : encode8_e4m3(f, s);
+    }
+  }
+}
+
+// One CTA per row.  Two passes over the row (the second hits L1/L2); used
+// for rows longer than the register-resident kernel holds.
 template <bool kInt8>
 __global__ void __launch_bounds__(256) quant_per_token_kernel(const __nv_bfloat16* __restrict__ x,
                                                                uint8_t* __restrict__ q, float* __restrict__ scales,
@@ -194,7 +235,19 @@ cudaError_t launch_quant_per_token(int fmt, const void* x, void* q, float* scale
   cudaLaunchConfig_t cfg = pdl_config(dim3(static_cast<unsigned>(M)), dim3(256), stream, attr);
   const auto* xp = static_cast<const __nv_bfloat16*>(x);
   auto* qp = static_cast<uint8_t*>(q);
-  if (fmt == kFmtInt8) return cudaLaunchKernelEx(&cfg, quant_per_token_kernel<true>, xp, qp, scales, K);
+  const bool i8 = fmt == kFmtInt8;
+  const int64_t nvec = K / 8;
+#define LQ_QROW(V)                                                                                     \
+  if (nvec <= 256 * (V))                                                                               \
+    return i8 ? cudaLaunchKernelEx(&cfg, quant_per_token_reg_kernel<true, V>, xp, qp, scales, K)       \
+              : cudaLaunchKernelEx(&cfg, quant_per_token_reg_kernel<false, V>, xp, qp, scales, K);
+  LQ_QROW(1)
+  LQ_QROW(2)
+  LQ_QROW(4)
+  LQ_QROW(8)
+  LQ_QROW(16)
+#undef LQ_QROW
+  if (i8) return cudaLaunchKernelEx(&cfg, quant_per_token_kernel<true>, xp, qp, scales, K);
   return cudaLaunchKernelEx(&cfg, quant_per_token_kernel<false>, xp, qp, scales, K);
 }
 

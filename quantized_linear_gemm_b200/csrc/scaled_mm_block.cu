@@ -5,13 +5,13 @@ cudaError_t launch_scaled_mm_block(const GemmLaunch& l, int swap_ab, int tile_n)
   return launch_format<kFmtBlock>(l, swap_ab, tile_n);
 }
 
-int gemm_smem_bytes_for(int tile_n, int stages) {
+int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce) {
   switch (tile_n) {
-    case 16: return gemm_smem_bytes<16>(stages);
-    case 32: return gemm_smem_bytes<32>(stages);
-    case 64: return gemm_smem_bytes<64>(stages);
-    case 128: return gemm_smem_bytes<128>(stages);
-    case 256: return gemm_smem_bytes<256>(stages);
+    case 16: return gemm_smem_bytes<16>(stages, cluster_reduce);
+    case 32: return gemm_smem_bytes<32>(stages, cluster_reduce);
+    case 64: return gemm_smem_bytes<64>(stages, cluster_reduce);
+    case 128: return gemm_smem_bytes<128>(stages, cluster_reduce);
+    case 256: return gemm_smem_bytes<256>(stages, cluster_reduce);
     default: return -1;
   }
 }

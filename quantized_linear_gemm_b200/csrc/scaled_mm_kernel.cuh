@@ -35,6 +35,9 @@ constexpr int kTileK = 128;      // K elements (bytes) per pipeline stage
 constexpr int kMmaK = 32;        // K per tcgen05.mma for 8-bit operands
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
+constexpr int kCtlBytes = 64 * 8 + 64;     // mbarriers, TMEM address, flags
+constexpr int kScaleBytes = 1024 * 4;      // staged scales: [0,256) per column, [256,384) per row,
+                                           // [512,1024) two per-K-block buffers (Block_FP8)
 
 template <int TN>
 struct TileShape {
@@ -47,18 +50,33 @@ __host__ __device__ constexpr int tmem_cols_for(int cols) {
   return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
 }
 
-// Bytes of the ring region: `stages` slots, and at least the 128 x TN 32-bit
-// partial tile that the cluster Split-K reduction stages there afterwards.
+// Cluster Split-K reduction.  Tiles up to 64 wide push: every CTA sends its
+// partial columns, from registers, into slots in the shared memory of the
+// CTA that owns those columns (st.async, completion counted in bytes on the
+// owner's mbarrier); the slots are a region of their own.  Wider tiles pull:
+// each CTA parks its partial in its ring once the ring is free and the
+// owners read them remotely between two cluster barriers.
+template <int TN>
+struct ClusterReduce {
+  static constexpr bool kPush = TN <= 64;
+  static constexpr int kSlotBytes = TN * 128 * 4;   // S partials of W = TN / S columns
+};
+
+// Bytes of the ring region: `stages` slots, and for the pull reduction at
+// least the 128 x TN 32-bit partial tile it parks there.
 template <int TN>
 __host__ __device__ constexpr int ring_bytes(int stages) {
-  return stages * TileShape<TN>::kStageBytes > TN * kTileM * 4 ? stages * TileShape<TN>::kStageBytes
-                                                                 : TN * kTileM * 4;
+  return (ClusterReduce<TN>::kPush || stages * TileShape<TN>::kStageBytes > TN * kTileM * 4)
+             ? stages * TileShape<TN>::kStageBytes
+             : TN * kTileM * 4;
 }
 
-// Shared-memory bytes the kernel needs for `stages` ring slots.
+// Shared-memory bytes of the kernel for `stages` ring slots; `cluster`: the
+// launch uses the cluster Split-K reduction (adds the push slots).
 template <int TN>
-__host__ __device__ constexpr int gemm_smem_bytes(int stages) {
-  return 1024 /* alignment slack */ + ring_bytes<TN>(stages) + 64 * 8 /* barriers */ + 64;
+__host__ __device__ constexpr int gemm_smem_bytes(int stages, bool cluster) {
+  return 1024 /* alignment slack */ + ring_bytes<TN>(stages) +
+         ((cluster && ClusterReduce<TN>::kPush) ? ClusterReduce<TN>::kSlotBytes : 0) + kCtlBytes + kScaleBytes;
 }
 
 struct SmemCtl {
@@ -67,6 +85,7 @@ struct SmemCtl {
   uint64_t* tfull;     // [2]
   uint64_t* tempty;    // [2]
   uint64_t* mma_done;  // [1]
+  uint64_t* red_bar;   // [1] push reduction: partial columns received
   uint32_t* tmem_slot;
   volatile int* abort_flag;
   volatile int* last_flag;
@@ -76,20 +95,35 @@ __device__ __forceinline__ void report_timeout(const GemmParams& p, int where) {
   if (p.status) atomicOr(p.status, 1 << where);
 }
 
+template <bool kClusterScope = false>
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const GemmParams& p, const SmemCtl& c,
                                          int where) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto try_once = [&]() { return kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (try_once()) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+      if (try_once()) return true;
     if (*c.abort_flag) return false;
     if (global_timer_ns() - t0 > p.wait_limit_ns) {
       *c.abort_flag = 1;
       report_timeout(p, where);
       return false;
     }
+  }
+}
+
+// Trace stamp i of this CTA (diagnostics; off when p.trace is null).
+//   0 entry, 1 set-up done, 2 producer past the grid dependency wait,
+//   3 first stage landed, 4 last MMA issued, 5 accumulator ready in TMEM,
+//   6 outputs / partials written, 7 exit, 8 / 9 / 10 cluster reduction:
+//   push: past the start barrier / all partials received / reduced tile
+//   stored; pull: past the first barrier / tile stored / past the second
+__device__ __forceinline__ void trace_stamp(const GemmParams& p, int i) {
+  if (p.trace) {
+    const uint64_t cta = blockIdx.x + static_cast<uint64_t>(gridDim.x) * (blockIdx.y + static_cast<uint64_t>(gridDim.y) * blockIdx.z);
+    p.trace[cta * kTraceSlots + i] = global_timer_ns();
   }
 }
 
@@ -116,16 +150,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
   const int stages = p.stages;
   uint8_t* ring = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + ring_bytes<TN>(stages));
+  const bool cluster_launch = p.S > 1 && p.reduce_mode == 2;
+  const bool push_mode = ClusterReduce<TN>::kPush && cluster_launch;
+  uint32_t* slots = reinterpret_cast<uint32_t*>(ring + ring_bytes<TN>(stages));   // push slots [src][row][col]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + ring_bytes<TN>(stages) +
+                                               (push_mode ? ClusterReduce<TN>::kSlotBytes : 0));
   SmemCtl c;
   c.full = bars;
   c.empty = bars + stages;
   c.tfull = bars + 2 * stages;
   c.tempty = c.tfull + 2;
   c.mma_done = c.tempty + 2;
-  c.tmem_slot = reinterpret_cast<uint32_t*>(c.mma_done + 1);
+  c.red_bar = c.mma_done + 1;
+  c.tmem_slot = reinterpret_cast<uint32_t*>(c.red_bar + 1);
   c.abort_flag = reinterpret_cast<volatile int*>(c.tmem_slot + 1);
   c.last_flag = c.abort_flag + 1;
+  float* sc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kCtlBytes);
+  float* colsc = sc;          // a_s (Swap-AB) or b_s (Standard) of each tile column
+  float* rowsc = sc + 256;    // b_s (Swap-AB) or a_s (Standard) of each accumulator row
+  float* blksc = sc + 512;    // Block_FP8: [2][256] per-K-block scale products
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -134,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kb_hi = static_cast<int>((static_cast<int64_t>(split + 1) * p.T) / p.S);
   const int nkb = kb_hi - kb_lo;
 
+  if (threadIdx.x == 0) trace_stamp(p, 0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&c.full[s], 1);
@@ -144,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&c.tempty[b], kEpiThreads / 32);
     }
     mbar_init(c.mma_done, 1);
+    mbar_init(c.red_bar, 1);
     *c.abort_flag = 0;
     *c.last_flag = 0;
     fence_barrier_init();
@@ -160,6 +205,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *c.tmem_slot;
+  if (threadIdx.x == 0) trace_stamp(p, 1);
+  // Push reduction: announce (cluster-wide, release) that this CTA's barriers
+  // exist; the epilogue waits for the whole cluster before pushing.
+  if (push_mode) cluster_arrive_release();
 
   // Let the next kernel on the stream start its own prologue / weight stream.
   grid_launch_dependents();
@@ -197,6 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(tmW, &c.full[i], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
         }
       }
+      trace_stamp(p, 2);
       for (int i = 0; i < pre; ++i) {
         uint8_t* st = ring + i * Shape::kStageBytes;
         tma_load_2d(tmA, &c.full[i], st + a_off, (kb_lo + i) * kTileK, a_row0, pol_a);
@@ -241,6 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!wait_bar(&c.full[s], ph, p, c, 2)) break;
         tc_fence_after_sync();
+        if (i == 0) trace_stamp(p, 3);
         uint8_t* st = ring + s * Shape::kStageBytes;
         const uint64_t xd = smem_desc_k_sw128(st);
         const uint64_t yd = smem_desc_k_sw128(st + Shape::kXBytes);
@@ -257,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&c.empty[s]);
         if (kBlocked) mma_commit(&c.tfull[i & 1]);
       }
+      trace_stamp(p, 4);
       if (!kBlocked && nkb > 0 && !*c.abort_flag) mma_commit(&c.tfull[0]);
       if (issued_any) {
         // All MMAs must be complete before TMEM is released at teardown.
@@ -278,56 +330,91 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int j = 0; j < (kBlocked ? TN : 1); ++j) accr[j] = 0.f;
 
+    if (!kBlocked) {
+      // Scales do not depend on the accumulator: load them while the mainloop
+      // runs (these warps are idle until then).
+      for (int j = r; j < TN; j += kEpiThreads) {
+        const int64_t col = y_row0 + j;
+        colsc[j] = SWAP ? (col < M ? __ldg(p.a_s + col) : 0.f) : (col < N ? __ldg(p.b_s + col) : 0.f);
+      }
+      const int64_t row = x_row0 + r;
+      rowsc[r] = SWAP ? (row < N ? __ldg(p.b_s + row) : 0.f) : (row < M ? __ldg(p.a_s + row) : 0.f);
+      named_barrier_sync(2, kEpiThreads);
+    }
+
     bool ok = true;
     if (kBlocked) {
-      // Per-128-K-block promotion: D_kb from TMEM times a_s[m,kb] b_s[nb,kb].
-      const int nb = SWAP ? (x_row0 + r) / 128 : y_row0 / 128;
-      const int64_t m_thread = SWAP ? 0 : x_row0 + r;
+      // Per-128-K-block promotion: acc += D_kb * a_s[m, kb] * b_s[nb, kb].
+      // The scale products of block kb+1 are loaded while block kb is
+      // waited for and promoted (double buffer blksc, one named barrier per
+      // block).  Every thread runs every iteration (also after a timeout),
+      // so the named barriers always match.
+      const int nb = SWAP ? x_row0 / 128 : y_row0 / 128;
+      const int64_t m_thread = x_row0 + r;   // Standard: this thread's token
+      auto load_scale = [&](int kb) -> float {
+        const float sb = __ldg(p.b_s + static_cast<int64_t>(nb) * p.KB + kb);
+        if (SWAP) {
+          const int64_t m = y_row0 + r;     // column r of the tile (r < TN)
+          return (m < M ? __ldg(p.a_s + m * p.KB + kb) : 0.f) * sb;
+        }
+        return (m_thread < M ? __ldg(p.a_s + m_thread * p.KB + kb) : 0.f) * sb;
+      };
+      const bool loader = SWAP ? (r < TN) : true;
+      float cur = 0.f;   // Standard: this thread's scale product of the current block
+      if (nkb > 0 && loader) {
+        cur = load_scale(kb_lo);
+        if (SWAP) blksc[r] = cur;
+      }
+      if (SWAP) named_barrier_sync(2, kEpiThreads);
       for (int i = 0; i < nkb; ++i) {
         const int buf = i & 1;
         const uint32_t use = static_cast<uint32_t>(i >> 1);
+        const float nxt = (loader && i + 1 < nkb) ? load_scale(kb_lo + i + 1) : 0.f;
         // warp-uniform decision: the tcgen05.ld below is .sync.aligned
-        if (!__all_sync(0xffffffffu, wait_bar(&c.tfull[buf], use & 1u, p, c, 4))) { ok = false; break; }
-        tc_fence_after_sync();
-        const int kb = kb_lo + i;
-        const bool n_ok = SWAP ? (x_row0 + r) < N : true;
-        const float sb = (SWAP ? n_ok : true) ? __ldg(p.b_s + static_cast<int64_t>(nb) * p.KB + kb) : 0.f;
-        float sa_row = 0.f;
-        if (!SWAP) sa_row = m_thread < M ? __ldg(p.a_s + m_thread * p.KB + kb) : 0.f;
+        if (ok) ok = __all_sync(0xffffffffu, wait_bar(&c.tfull[buf], use & 1u, p, c, 4));
+        if (ok) {
+          tc_fence_after_sync();
+          const float* bs = blksc + (i & 1) * 256;
 #pragma unroll
-        for (int c0 = 0; c0 < TN; c0 += CH) {
-          uint32_t v[CH];
-          if constexpr (CH == 32)
-            tmem_ld_32x32b_x32(t_row + buf * TN + c0, v);
-          else
-            tmem_ld_32x32b_x16(t_row + buf * TN + c0, v);
-          tmem_ld_wait();
+          for (int c0 = 0; c0 < TN; c0 += CH) {
+            uint32_t v[CH];
+            if constexpr (CH == 32)
+              tmem_ld_32x32b_x32(t_row + buf * TN + c0, v);
+            else
+              tmem_ld_32x32b_x16(t_row + buf * TN + c0, v);
+            tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < CH; ++j) {
-            float scale;
-            if (SWAP) {
-              const int64_t m = y_row0 + c0 + j;
-              scale = (m < M ? __ldg(p.a_s + m * p.KB + kb) : 0.f) * sb;
-            } else {
-              scale = sa_row * sb;
-            }
-            accr[c0 + j] = fmaf(__uint_as_float(v[j]), scale, accr[c0 + j]);
+            for (int j = 0; j < CH; ++j)
+              accr[c0 + j] = fmaf(__uint_as_float(v[j]), SWAP ? bs[c0 + j] : cur, accr[c0 + j]);
           }
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c.tempty[buf]);
         }
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c.tempty[buf]);
+        cur = nxt;
+        if (SWAP) {
+          if (loader && i + 1 < nkb) blksc[((i + 1) & 1) * 256 + r] = nxt;
+          named_barrier_sync(2, kEpiThreads);
+        }
       }
     } else if (nkb > 0) {
       ok = wait_bar(&c.tfull[0], 0, p, c, 5);
       tc_fence_after_sync();
     }
     ok = __all_sync(0xffffffffu, ok && !*c.abort_flag);
+    if (warp == 2 && lane == 0) trace_stamp(p, 5);
 
-    const bool cluster_mode = p.S > 1 && p.reduce_mode == 2;
+    const bool cluster_mode = cluster_launch;
     // The ring's last readers were the tensor core (async proxy); order them
-    // before the generic-proxy stores of the cluster partial tile.
-    if (cluster_mode) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    // before the generic-proxy stores of the pulled partial tile.
+    if (cluster_mode && !push_mode) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (push_mode) {
+      cluster_wait_acquire();   // every CTA of the cluster has initialised its barriers
+      if (warp == 2 && lane == 0) {
+        trace_stamp(p, 8);
+        mbar_arrive_expect_tx(c.red_bar, static_cast<uint32_t>(ClusterReduce<TN>::kSlotBytes));
+      }
+    }
     if (ok) {
       float* wsf = reinterpret_cast<float*>(p.ws);
       int32_t* wsi = reinterpret_cast<int32_t*>(p.ws);
@@ -350,6 +437,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < CH; ++j) v[j] = 0u;   // empty split: zero partial
         }
 
+        if (push_mode) {
+          // columns [o W, (o+1) W) go to CTA o, slot [split][r][0..W)
+          const int W = TN / p.S;
+          const uint32_t slot_row = static_cast<uint32_t>((split * kTileM + r) * W) * 4u;
+          const uint32_t slots_local = smem_addr(slots);
+          const uint32_t bar_local = smem_addr(c.red_bar);
+          if (W >= 4) {
+#pragma unroll
+            for (int j = 0; j < CH; j += 4) {
+              const int owner = (c0 + j) / W;
+              const int jj = (c0 + j) - owner * W;
+              st_async_v4(dsmem_map(slots_local, owner) + slot_row + jj * 4u, v[j], v[j + 1], v[j + 2], v[j + 3],
+                          dsmem_map(bar_local, owner));
+            }
+          } else if (W == 2) {
+#pragma unroll
+            for (int j = 0; j < CH; j += 2) {
+              const int owner = (c0 + j) / 2;
+              st_async_v2(dsmem_map(slots_local, owner) + slot_row, v[j], v[j + 1], dsmem_map(bar_local, owner));
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < CH; ++j)
+              st_async_b32(dsmem_map(slots_local, c0 + j) + slot_row, v[j], dsmem_map(bar_local, c0 + j));
+          }
+          continue;
+        }
         if (cluster_mode) {
           // partial tile -> own shared memory, [column j][row r] (the ring is free now)
           uint32_t* red = reinterpret_cast<uint32_t*>(ring);
@@ -361,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (SWAP) {
           const int64_t n = x_row0 + r;
           if (n < N) {
-            const float bsn = (!kBlocked && !split_mode) ? __ldg(p.b_s + n) : 1.f;
+            const float bsn = (!kBlocked && !split_mode) ? rowsc[r] : 1.f;
 #pragma unroll
             for (int j = 0; j < CH; ++j) {
               const int64_t m = y_row0 + c0 + j;
@@ -377,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     val = __uint_as_float(v[j]);
                   } else {
                     const float a = kInt8 ? static_cast<float>(static_cast<int32_t>(v[j])) : __uint_as_float(v[j]);
-                    val = a * __ldg(p.a_s + m) * bsn;
+                    val = a * colsc[c0 + j] * bsn;
                   }
                   p.C[idx] = __float2bfloat16_rn(val);
                   if (kInt8 && p.acc_out) p.acc_out[idx] = static_cast<int32_t>(v[j]);
@@ -388,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const int64_t m = x_row0 + r;
           if (m < M) {
-            const float asm_ = (!kBlocked && !split_mode) ? __ldg(p.a_s + m) : 1.f;
+            const float asm_ = (!kBlocked && !split_mode) ? rowsc[r] : 1.f;
 #pragma unroll
             for (int j8 = 0; j8 < CH; j8 += 8) {
               const int64_t n = y_row0 + c0 + j8;
@@ -407,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                       const float a =
                           kInt8 ? static_cast<float>(static_cast<int32_t>(v[j8 + e])) : __uint_as_float(v[j8 + e]);
-                      f[e] = a * asm_ * __ldg(p.b_s + n + e);
+                      f[e] = a * asm_ * colsc[c0 + j8 + e];
                     }
                   }
                   uint4 pk = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
@@ -426,6 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
     }
+
+    if (warp == 2 && lane == 0) trace_stamp(p, 6);
 
     // -------------------------------------------- in-kernel Split-K reduce
     // Every epilogue thread reaches both named barriers, also after a
@@ -447,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (SWAP) {
           const int64_t n = x_row0 + r;
           if (n < N) {
-            const float bsn = kBlocked ? 1.f : __ldg(p.b_s + n);
+            const float bsn = kBlocked ? 1.f : rowsc[r];
             for (int j = 0; j < TN; ++j) {
               const int64_t m = y_row0 + j;
               if (m >= M) break;
@@ -460,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               float val;
               if (kBlocked) val = sf;
-              else val = (kInt8 ? static_cast<float>(si) : sf) * __ldg(p.a_s + m) * bsn;
+              else val = (kInt8 ? static_cast<float>(si) : sf) * colsc[j] * bsn;
               p.C[m * N + n] = __float2bfloat16_rn(val);
               if (kInt8 && p.acc_out) p.acc_out[m * N + n] = si;
             }
@@ -468,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const int64_t m = x_row0 + r;
           if (m < M) {
-            const float asm_ = kBlocked ? 1.f : __ldg(p.a_s + m);
+            const float asm_ = kBlocked ? 1.f : rowsc[r];
             for (int j4 = 0; j4 < TN; j4 += 4) {
               const int64_t n = y_row0 + j4;
               if (n >= N) break;
@@ -489,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               else { f[0] = sf.x; f[1] = sf.y; f[2] = sf.z; f[3] = sf.w; }
               if (!kBlocked) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * __ldg(p.b_s + n + e);
+                for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * colsc[j4 + e];
               }
               uint2 pk = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
               *reinterpret_cast<uint2*>(p.C + m * N + n) = pk;
@@ -499,6 +615,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (warp == 2 && lane == 0) p.counters[tile_id] = 0;   // ready for the next launch / replay
       }
+    }
+
+    // --------------------------------------- push-mode cluster reduce (owner)
+    if (push_mode) {
+      const bool got = __all_sync(0xffffffffu, wait_bar<true>(c.red_bar, 0, p, c, 6));
+      if (warp == 2 && lane == 0) trace_stamp(p, 9);
+      if (got && !*c.abort_flag) {
+        const int S = p.S;
+        const int W = TN / S;
+        const int j0 = split * W;
+        const int64_t M = p.M, N = p.N;
+        // partial of split s for column j0 + jj of this thread's row
+        auto slot = [&](int s, int jj) -> uint32_t { return slots[(s * kTileM + r) * W + jj]; };
+        if (SWAP) {
+          const int64_t n = x_row0 + r;
+          const float bsn = !kBlocked ? rowsc[r] : 1.f;
+          for (int jj = 0; jj < W; ++jj) {
+            float sf = 0.f;
+            int32_t si = 0;
+#pragma unroll
+            for (int s = 0; s < 16; ++s)
+              if (s < S) {
+                const uint32_t u = slot(s, jj);
+                if (kInt8) si += static_cast<int32_t>(u);
+                else sf += __uint_as_float(u);
+              }
+            const int64_t m = y_row0 + j0 + jj;
+            if (n < N && m < M) {
+              float val;
+              if (kBlocked) val = sf;
+              else val = (kInt8 ? static_cast<float>(si) : sf) * colsc[j0 + jj] * bsn;
+              p.C[m * N + n] = __float2bfloat16_rn(val);
+              if (kInt8 && p.acc_out) p.acc_out[m * N + n] = si;
+            }
+          }
+        } else {
+          const int64_t m = x_row0 + r;
+          const float asm_ = !kBlocked ? rowsc[r] : 1.f;
+          for (int jj = 0; jj < W; jj += 4) {   // W >= 4 for Standard tiles (TN >= 64, S <= 16)
+            float f[4];
+            int32_t iv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float sf = 0.f;
+              int32_t si = 0;
+#pragma unroll
+              for (int s = 0; s < 16; ++s)
+                if (s < S) {
+                  const uint32_t u = slot(s, jj + e);
+                  if (kInt8) si += static_cast<int32_t>(u);
+                  else sf += __uint_as_float(u);
+                }
+              iv[e] = si;
+              f[e] = kInt8 ? static_cast<float>(si) : sf;
+            }
+            const int64_t n = y_row0 + j0 + jj;
+            if (m < M && n < N) {
+              if (!kBlocked) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * colsc[j0 + jj + e];
+              }
+              *reinterpret_cast<uint2*>(p.C + m * N + n) =
+                  make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+              if (kInt8 && p.acc_out)
+                *reinterpret_cast<int4*>(p.acc_out + m * N + n) = make_int4(iv[0], iv[1], iv[2], iv[3]);
+            }
+          }
+        }
+      }
+      if (warp == 2 && lane == 0) trace_stamp(p, 10);
     }
   }
 
@@ -510,9 +696,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // result is the same bit for bit), scales and stores them.  The second
   // barrier keeps every CTA alive until the others have read its partial.
   // All threads of all CTAs execute both barriers on every path.
-  if (p.S > 1 && p.reduce_mode == 2) {
+  if (push_mode && warp < 2) {
+    __syncwarp();
+    cluster_wait_acquire();   // pairs with the arrive after set-up
+  }
+  if (cluster_launch && !push_mode) {
     __syncwarp();
     cluster_sync_all();
+    if (warp == 2 && lane == 0) trace_stamp(p, 8);
     if (warp >= 2 && !*c.abort_flag) {
       const int q = warp & 3;
       const int r = q * 32 + lane;
@@ -526,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < 16; ++s) rb[s] = s < S ? dsmem_map(local, static_cast<uint32_t>(s)) : 0u;
       if (SWAP) {
         const int64_t n = x_row0 + r;
-        const float bsn = (!kBlocked && n < N) ? __ldg(p.b_s + n) : 1.f;
+        const float bsn = !kBlocked ? rowsc[r] : 1.f;
         for (int j = j0; j < j0 + W; ++j) {
           const uint32_t off = static_cast<uint32_t>((j * kTileM + r) * 4);
           uint32_t u[16];
@@ -545,14 +736,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (n < N && m < M) {
             float val;
             if (kBlocked) val = sf;
-            else val = (kInt8 ? static_cast<float>(si) : sf) * __ldg(p.a_s + m) * bsn;
+            else val = (kInt8 ? static_cast<float>(si) : sf) * colsc[j] * bsn;
             p.C[m * N + n] = __float2bfloat16_rn(val);
             if (kInt8 && p.acc_out) p.acc_out[m * N + n] = si;
           }
         }
       } else {
         const int64_t m = x_row0 + r;
-        const float asm_ = (!kBlocked && m < M) ? __ldg(p.a_s + m) : 1.f;
+        const float asm_ = !kBlocked ? rowsc[r] : 1.f;
         for (int j = j0; j < j0 + W; j += 4) {   // W >= 4 for Standard tiles (TN >= 64, S <= 16)
           uint32_t u[4][16];
 #pragma unroll
@@ -579,7 +770,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (m < M && n < N) {
             if (!kBlocked) {
 #pragma unroll
-              for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * __ldg(p.b_s + n + e);
+              for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * colsc[j + e];
             }
             *reinterpret_cast<uint2*>(p.C + m * N + n) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
             if (kInt8 && p.acc_out)
@@ -588,13 +779,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if (warp == 2 && lane == 0) trace_stamp(p, 9);
     __syncwarp();
     cluster_sync_all();
+    if (warp == 2 && lane == 0) trace_stamp(p, 10);
   }
 
   // -------------------------------------------------------------- teardown
   tc_fence_before_sync();
   __syncthreads();
+  if (threadIdx.x == 0) trace_stamp(p, 7);
   if (warp == 1) {
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, kTmemCols);

@@ -33,7 +33,7 @@ EXPORTED = (
     "lq_scaled_mm", "lq_scaled_mm_i32acc", "lq_quant_per_token", "lq_quant_per_token_group128",
     "lq_quant_weight_block128", "lq_select_variant", "lq_load_dispatch_table", "lq_dispatch_table_size",
     "lq_init_device", "lq_reserve_workspace", "lq_workspace_bytes", "lq_device_status",
-    "lq_status_string", "lq_version",
+    "lq_status_string", "lq_version", "lq_set_trace",
 )
 
 
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
             L.lq_device_status.argtypes = [_i32]
             L.lq_status_string.argtypes = [_i32]
             L.lq_status_string.restype = ctypes.c_char_p
+            L.lq_set_trace.argtypes = [_vp]
+            L.lq_set_trace.restype = _i32
             L.lq_version.argtypes = []
             L.lq_version.restype = ctypes.c_char_p
             for name in ("lq_scaled_mm", "lq_scaled_mm_i32acc", "lq_quant_per_token", "lq_quant_per_token_group128",
@@ -245,6 +247,12 @@ def workspace_bytes(fmt, M, N, K, variant: Variant | None = None) -> int:
 def device_status(device: int = 0) -> int:
     """Read and clear the device status word: 0, or LQ_ERR_DEVICE_TIMEOUT (6)."""
     return int(lib().lq_device_status(device))
+
+
+def set_trace(buf: torch.Tensor | None) -> None:
+    """Record 12 globaltimer stamps per CTA of the following scaled_mm launches
+    into ``buf`` (int64 CUDA tensor with 12 entries per CTA), or stop (None)."""
+    lib().lq_set_trace(None if buf is None else buf.data_ptr())
 
 
 def status_string(code: int) -> str:

@@ -10,7 +10,7 @@ from quantized_linear_gemm_b200 import inputs, lq
 
 pytestmark = pytest.mark.gpu
 
-PER_TOKEN_SHAPES = [(1, 16), (3, 128), (16, 2048), (32, 4096), (7, 4112), (24, 12288), (64, 25600), (300, 1024)]
+PER_TOKEN_SHAPES = [(1, 16), (3, 128), (16, 2048), (32, 4096), (7, 4112), (24, 12288), (64, 25600), (300, 1024), (2, 40960), (5, 2064)]
 
 
 def _x(M, K, seed, outliers=True):
