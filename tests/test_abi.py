@@ -100,7 +100,17 @@ def test_i32acc_needs_an_output():
     assert L.lq_scaled_mm_i32acc(FAKE, FAKE, FAKE, FAKE, FAKE, MISALIGNED, 4, 128, 128, None, None) == ALIGN
 
 
-def test_heuristic_variant_shapes():
+def test_heuristic_variant_shapes(tmp_path):
+    empty = tmp_path / "empty.txt"
+    empty.write_text("# no entries: every lookup falls back to the heuristic\n")
+    lq.load_dispatch_table(str(empty))
+    try:
+        _check_heuristic()
+    finally:
+        lq.load_dispatch_table(None)
+
+
+def _check_heuristic():
     v = lq.select_variant("fp8_dynamic", 1, 4096, 4096)
     assert v.swap_ab == 1 and v.tile_n == 16 and v.split_k >= 2
     v = lq.select_variant("fp8_dynamic", 24, 4096, 4096)
