@@ -158,6 +158,39 @@ lq_status lq_scaled_mm_i32acc(const void *A, const float *a_scales,
                               const lq_variant *variant, lq_stream_t stream);
 
 /*
+ * Allocation-free scaled_mm, for callers that cannot call cudaMalloc when
+ * they run a GEMM: code running while a CUDA graph is captured with the
+ * global capture mode (an allocation is an unsafe call there), frameworks
+ * whose device memory comes only from their own pool allocator, and
+ * latency-critical services that must not allocate or synchronise after
+ * start-up.  lq_scaled_mm may allocate its per-device state and Split-K
+ * workspace on first use; this entry point never calls cudaMalloc, cudaFree
+ * or any allocating routine.  The pages have no counterpart: it is an
+ * interface of this library only.
+ *
+ * Same arguments, layouts and results as lq_scaled_mm.  Differences:
+ *  - With split_k > 1 the partial sums go to a fixed 16 MiB array in device
+ *    memory that the library reserves when it is loaded (every GPU that
+ *    loads the library holds it until the process exits), and are summed by
+ *    the separate fixed-order reduction kernel (the variant's reduce field is
+ *    ignored).  A call whose split_k * M * N * 4 bytes exceed 16 MiB returns
+ *    LQ_ERR_WORKSPACE before launching anything.
+ *  - Every call shares that array and it keeps the last call's partials, so
+ *    calls that overlap on the GPU (different streams without ordering, or
+ *    concurrent graph branches) race and give wrong results.  Calls ordered
+ *    on one stream are safe.  Nothing in the array needs to start at zero.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress with that device current); make that first call
+ *    before capturing a CUDA graph.
+ *  - A kernel that gives up on a bounded wait leaves C undefined; this entry
+ *    point has no status word, so lq_device_status does not report it.
+ */
+lq_status lq_scaled_mm_noalloc(lq_fmt fmt, const void *A, const float *a_scales,
+                               const void *B, const float *b_scales, void *C,
+                               int64_t M, int64_t N, int64_t K,
+                               const lq_variant *variant, lq_stream_t stream);
+
+/*
  * Dynamic per-token activation quantization (the blog's integrated kernel
  * dynamic_per_token_scaled_fp8_quant, as listed in the 24-ai.news report,
  * section "kernels integrated into vLLM"; the int8 form serves W8A8_INT8).

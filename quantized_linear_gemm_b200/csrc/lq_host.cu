@@ -584,3 +584,126 @@ lq_status lq_device_status(int device) {
 }
 
 }  // extern "C"
+
+// ======================================================================
+// Allocation-free scaled_mm.
+//
+// Some callers cannot call cudaMalloc when they run a GEMM: code that runs
+// while a CUDA graph is being captured with the global capture mode (where
+// an allocation is an unsafe call), frameworks whose memory is handed out
+// only by their own pool allocator, and latency-critical services that must
+// not allocate or synchronise after start-up.  lq_scaled_mm may allocate its
+// per-device state and Split-K workspace on first use; the entry point below
+// never does.  Its Split-K partials live in a fixed array in device memory
+// that the library reserves when it is loaded.
+namespace {
+
+// Split-K partial sums of lq_scaled_mm_noalloc: [split_k, M, N] fp32 / int32.
+// Every GPU that loads the library holds these bytes until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};   // device address of g_noalloc_scratch per device
+
+// Device address of the scratch array on the current device.  The first call
+// on a device looks it up (cudaGetSymbolAddress, with that device current).
+lq_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return LQ_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return LQ_OK;
+}
+
+}  // namespace
+
+extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const float* a_scales, const void* B,
+                                          const float* b_scales, void* C, int64_t M, int64_t N, int64_t K,
+                                          const lq_variant* variant, lq_stream_t stream_) {
+  const int fmt = static_cast<int>(fmt_);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  lq_status rc = check_gemm_args(fmt, A, a_scales, B, b_scales, C, M, N, K);
+  if (rc != LQ_OK) return rc;
+  if (M == 0 || N == 0) return LQ_OK;
+  if (K == 0)
+    return lq::launch_fill_zero_bf16(static_cast<__nv_bfloat16*>(C), M * N, stream) == cudaSuccess ? LQ_OK
+                                                                                                  : LQ_ERR_CUDA;
+  lq_variant v{};
+  if (variant) {
+    v = *variant;
+  } else if (!lookup_table(fmt, M, N, K, &v)) {
+    v = heuristic_variant(fmt, M, N, K);
+  }
+  // Split-K partials always go through the scratch array and the separate
+  // fixed-order reduction kernel (no arrival counters, nothing to re-arm).
+  if (v.split_k > 1) v.reduce = 0;
+  rc = check_variant(fmt, v);
+  if (rc != LQ_OK) return rc;
+  const size_t need = v.split_k > 1 ? static_cast<size_t>(v.split_k) * static_cast<size_t>(M) *
+                                          static_cast<size_t>(N) * 4u
+                                    : 0;
+  if (need > kNoAllocScratchBytes) return LQ_ERR_WORKSPACE;
+  if (v.stages == 0) v.stages = max_stages_fit(v.tile_n, 1, false);
+
+  const int64_t x_rows = v.swap_ab ? N : M;
+  const int64_t y_rows = v.swap_ab ? M : N;
+  const int64_t gx = (x_rows + 127) / 128;
+  const int64_t gy = (y_rows + v.tile_n - 1) / v.tile_n;
+  if (gy > 65535 || gx > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc != LQ_OK) return rc;
+
+  GemmLaunch l;
+  std::memset(&l, 0, sizeof(l));
+  GemmParams& p = l.p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.T = static_cast<int>((K + 127) / 128);
+  p.KB = static_cast<int>(K / 128);
+  p.S = v.split_k;
+  p.stages = v.stages;
+  p.reduce_mode = 0;
+  p.early_weights = v.pdl == 2 ? 1 : 0;
+  p.a_s = a_scales;
+  p.b_s = b_scales;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.ws = v.split_k > 1 ? scratch : nullptr;
+  p.counters = nullptr;
+  p.acc_out = nullptr;
+  p.status = nullptr;   // a timed-out wait leaves C undefined and is not reported here
+  p.wait_limit_ns = wait_limit_ns();
+  p.trace = nullptr;
+  const void* x_ptr = v.swap_ab ? B : A;
+  const void* y_ptr = v.swap_ab ? A : B;
+  if (!encode_operand(&l.tmX, x_ptr, x_rows, K, 128) || !encode_operand(&l.tmY, y_ptr, y_rows, K, v.tile_n))
+    return LQ_ERR_CUDA;
+  l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
+  l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, false);
+  l.pdl = v.pdl != 0;
+  l.cluster_z = 1;
+  l.stream = stream;
+  cudaError_t e;
+  switch (fmt) {
+    case lq::kFmtFp8: e = lq::launch_scaled_mm_fp8(l, v.swap_ab, v.tile_n); break;
+    case lq::kFmtInt8: e = lq::launch_scaled_mm_int8(l, v.swap_ab, v.tile_n); break;
+    default: e = lq::launch_scaled_mm_block(l, v.swap_ab, v.tile_n); break;
+  }
+  if (e == cudaSuccess && v.split_k > 1) e = lq::launch_splitk_reduce(fmt, p, v.pdl != 0, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return LQ_ERR_CUDA;
+  }
+  return LQ_OK;
+}

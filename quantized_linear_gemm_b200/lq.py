@@ -33,7 +33,7 @@ EXPORTED = (
     "lq_scaled_mm", "lq_scaled_mm_i32acc", "lq_quant_per_token", "lq_quant_per_token_group128",
     "lq_quant_weight_block128", "lq_select_variant", "lq_load_dispatch_table", "lq_dispatch_table_size",
     "lq_init_device", "lq_reserve_workspace", "lq_workspace_bytes", "lq_device_status",
-    "lq_status_string", "lq_version", "lq_set_trace",
+    "lq_status_string", "lq_version", "lq_set_trace", "lq_scaled_mm_noalloc",
 )
 
 
@@ -75,6 +75,9 @@ def lib() -> ctypes.CDLL:
                                    "`python -m quantized_linear_gemm_b200.build`")
             L = ctypes.CDLL(LIB_PATH)
             L.lq_scaled_mm.argtypes = [_i32, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.POINTER(Variant), _st]
+            L.lq_scaled_mm_noalloc.argtypes = [_i32, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                               ctypes.POINTER(Variant), _st]
+            L.lq_scaled_mm_noalloc.restype = _i32
             L.lq_scaled_mm_i32acc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                                               ctypes.POINTER(Variant), _st]
             L.lq_quant_per_token.argtypes = [_i32, _vp, _vp, _vp, _i64, _i64, _st]
@@ -157,6 +160,24 @@ def scaled_mm(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor, b_s
     rc = lib().lq_scaled_mm(f, _ptr(A), _ptr(a_scales), _ptr(B), _ptr(b_scales), _ptr(C), M, N, K,
                             ctypes.byref(variant) if variant is not None else None, _stream(stream))
     _check("lq_scaled_mm", rc)
+    return C
+
+
+def scaled_mm_noalloc(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor, b_scales: torch.Tensor,
+                      C: torch.Tensor | None = None, variant: Variant | None = None, stream=None) -> torch.Tensor:
+    """``lq_scaled_mm_noalloc``: scaled_mm whose Split-K partials use the library's
+    fixed device array instead of allocated workspace (see include/lq.h)."""
+    f = _fmt(fmt)
+    _need(A, "A", _CODE_DTYPES, 2)
+    _need(B, "B", _CODE_DTYPES, 2)
+    M, K = A.shape
+    N = B.shape[0]
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _need(C, "C", (torch.bfloat16,), 2)
+    rc = lib().lq_scaled_mm_noalloc(f, _ptr(A), _ptr(a_scales), _ptr(B), _ptr(b_scales), _ptr(C), M, N, K,
+                                    ctypes.byref(variant) if variant is not None else None, _stream(stream))
+    _check("lq_scaled_mm_noalloc", rc)
     return C
 
 
