@@ -290,6 +290,19 @@ lq_status lq_device_status(int device);
  */
 lq_status lq_set_trace(uint64_t *device_buffer);
 
+/*
+ * Test hook for failure detection.  While k_tile >= 0, every scaled_mm
+ * kernel launched afterwards leaves the k_tile-th K tile of each CTA
+ * unloaded, so the tensor-core warp's bounded wait for it runs out: the
+ * kernel sets the device status word, drains its copies, frees its tensor
+ * memory and returns (C undefined), and lq_device_status reports
+ * LQ_ERR_DEVICE_TIMEOUT.  Nothing faults or hangs.  wait_limit_ns > 0
+ * replaces the bound of every wait (default 2 s, or LQ_WAIT_LIMIT_NS) until
+ * the hook is called again with 0.  k_tile = -1 turns the hook off.
+ * Errors: LQ_ERR_INVALID_ARG for k_tile < -1.
+ */
+lq_status lq_test_inject_stall(int k_tile, uint64_t wait_limit_ns);
+
 /* Human-readable name of a status code (static storage). */
 const char *lq_status_string(lq_status status);
 

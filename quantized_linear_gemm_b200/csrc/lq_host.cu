@@ -51,8 +51,12 @@ struct DeviceState {
 std::mutex g_dev_mutex;
 DeviceState g_dev[kMaxDevices];
 std::atomic<uint64_t*> g_trace{nullptr};   // diagnostics: per-CTA stamps of the next launches
+std::atomic<int> g_skip_stage{-1};          // test hook: K tile the producer never fills
+std::atomic<uint64_t> g_wait_limit_override{0};
 
 uint64_t wait_limit_ns() {
+  const uint64_t o = g_wait_limit_override.load();
+  if (o) return o;
   static uint64_t v = [] {
     const char* e = std::getenv("LQ_WAIT_LIMIT_NS");
     if (e && *e) {
@@ -350,6 +354,7 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   p.status = d->status;
   p.wait_limit_ns = wait_limit_ns();
   p.trace = g_trace.load();
+  p.skip_stage = g_skip_stage.load();
   if (v.split_k > 1 && v.reduce != 2) {   // the cluster reduction needs no global workspace
     const size_t need = static_cast<size_t>(v.split_k) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
     rc = ensure_workspace(d, need, stream);
@@ -450,6 +455,13 @@ const char* lq_status_string(lq_status s) {
 }
 
 const char* lq_version(void) { return "lq 0.1.0 (sm_100a)"; }
+
+lq_status lq_test_inject_stall(int k_tile, uint64_t wait_limit_ns) {
+  if (k_tile < -1) return LQ_ERR_INVALID_ARG;
+  g_skip_stage.store(k_tile);
+  g_wait_limit_override.store(wait_limit_ns);
+  return LQ_OK;
+}
 
 lq_status lq_set_trace(uint64_t* device_buffer) {
   g_trace.store(device_buffer);
@@ -685,6 +697,7 @@ extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const floa
   p.status = nullptr;   // a timed-out wait leaves C undefined and is not reported here
   p.wait_limit_ns = wait_limit_ns();
   p.trace = nullptr;
+  p.skip_stage = -1;
   const void* x_ptr = v.swap_ab ? B : A;
   const void* y_ptr = v.swap_ab ? A : B;
   if (!encode_operand(&l.tmX, x_ptr, x_rows, K, 128) || !encode_operand(&l.tmY, y_ptr, y_rows, K, v.tile_n))

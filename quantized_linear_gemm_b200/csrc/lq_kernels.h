@@ -30,6 +30,7 @@ struct GemmParams {
   int* status;         // device status word (bit set per timed-out wait site)
   uint64_t wait_limit_ns;
   uint64_t* trace;     // optional: kTraceSlots globaltimer stamps per CTA
+  int skip_stage;      // test hook: >= 0 = the producer never fills this K tile (a wait runs out)
 };
 
 constexpr int kTraceSlots = 12;

@@ -233,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // that may still run: start streaming them before waiting for the
         // previous kernel on the stream (programmatic dependent launch).
         for (int i = 0; i < pre; ++i) {
+          if (i == p.skip_stage) continue;
           uint8_t* st = ring + i * Shape::kStageBytes;
           mbar_arrive_expect_tx(&c.full[i], Shape::kStageBytes);
           tma_load_2d(tmW, &c.full[i], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
@@ -241,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         grid_dependency_wait();
         for (int i = 0; i < pre; ++i) {
+          if (i == p.skip_stage) continue;
           uint8_t* st = ring + i * Shape::kStageBytes;
           mbar_arrive_expect_tx(&c.full[i], Shape::kStageBytes);
           tma_load_2d(tmW, &c.full[i], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
@@ -248,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       trace_stamp(p, 2);
       for (int i = 0; i < pre; ++i) {
+        if (i == p.skip_stage) continue;
         uint8_t* st = ring + i * Shape::kStageBytes;
         tma_load_2d(tmA, &c.full[i], st + a_off, (kb_lo + i) * kTileK, a_row0, pol_a);
       }
@@ -256,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = i % stages;
         const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
         if (!wait_bar(&c.empty[s], ph ^ 1u, p, c, 0)) break;
+        if (i == p.skip_stage) continue;
         uint8_t* st = ring + s * Shape::kStageBytes;
         mbar_arrive_expect_tx(&c.full[s], Shape::kStageBytes);
         tma_load_2d(tmW, &c.full[s], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
@@ -266,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Drain: wait (bounded) for the copies still in flight into shared memory.
         const int first = issued > stages ? issued - stages : 0;
         for (int j = first; j < issued; ++j) {
+          if (j == p.skip_stage) continue;   // never armed
           const uint64_t t0 = global_timer_ns();
           while (!mbar_try_wait(&c.full[j % stages], static_cast<uint32_t>(j / stages) & 1u) &&
                  global_timer_ns() - t0 < p.wait_limit_ns) {

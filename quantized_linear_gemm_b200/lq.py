@@ -33,7 +33,7 @@ EXPORTED = (
     "lq_scaled_mm", "lq_scaled_mm_i32acc", "lq_quant_per_token", "lq_quant_per_token_group128",
     "lq_quant_weight_block128", "lq_select_variant", "lq_load_dispatch_table", "lq_dispatch_table_size",
     "lq_init_device", "lq_reserve_workspace", "lq_workspace_bytes", "lq_device_status",
-    "lq_status_string", "lq_version", "lq_set_trace", "lq_scaled_mm_noalloc",
+    "lq_status_string", "lq_version", "lq_set_trace", "lq_scaled_mm_noalloc", "lq_test_inject_stall",
 )
 
 
@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
             L.lq_device_status.argtypes = [_i32]
             L.lq_status_string.argtypes = [_i32]
             L.lq_status_string.restype = ctypes.c_char_p
+            L.lq_test_inject_stall.argtypes = [_i32, ctypes.c_uint64]
+            L.lq_test_inject_stall.restype = _i32
             L.lq_set_trace.argtypes = [_vp]
             L.lq_set_trace.restype = _i32
             L.lq_version.argtypes = []
@@ -274,6 +276,12 @@ def set_trace(buf: torch.Tensor | None) -> None:
     """Record 12 globaltimer stamps per CTA of the following scaled_mm launches
     into ``buf`` (int64 CUDA tensor with 12 entries per CTA), or stop (None)."""
     lib().lq_set_trace(None if buf is None else buf.data_ptr())
+
+
+def test_inject_stall(k_tile: int, wait_limit_ns: int = 0) -> None:
+    """Test hook: leave K tile `k_tile` of every CTA unloaded so that a bounded
+    wait runs out (-1 = off); `wait_limit_ns` > 0 shortens every wait."""
+    _check("lq_test_inject_stall", lib().lq_test_inject_stall(int(k_tile), int(wait_limit_ns)))
 
 
 def status_string(code: int) -> str:

@@ -94,6 +94,11 @@ def test_quant_argument_checks():
     assert L.lq_quant_weight_block128(FAKE, FAKE, FAKE, 0, 256, None) == OK
 
 
+def test_stall_hook_argument_check():
+    assert lq.lib().lq_test_inject_stall(-2, 0) == INVALID
+    assert lq.lib().lq_test_inject_stall(-1, 0) == OK
+
+
 def test_i32acc_needs_an_output():
     L = lq.lib()
     assert L.lq_scaled_mm_i32acc(FAKE, FAKE, FAKE, FAKE, FAKE, None, 4, 128, 128, None, None) == INVALID
