@@ -81,16 +81,17 @@ def kernel_sources_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(config: str):
-    """DRAM bytes per step of the scaled_mm launches from the committed ncu
-    summary, or None when there is none or the kernels changed since."""
-    p = os.path.join(ROOT, "profiles", f"traffic_{config.replace('-', '_')}.json")
+def recorded_traffic(config: str, kernel: str):
+    """DRAM bytes per step of the step's `kernel` launches ("fused" or
+    "scaled_mm") from the committed ncu summary, or None when there is none
+    or the kernel sources changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", f"traffic_{config.replace('-', '_')}_{kernel}.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     if d.get("kernel_sources_sha256_16") != kernel_sources_digest():
         return None
-    return int(d["scaled_mm_dram_bytes_per_step"])
+    return int(d["dram_bytes_per_step"])
 
 
 # ------------------------------------------------------- multi-rank timing
@@ -240,9 +241,14 @@ class Workload:
     def flops(self) -> int:
         return sum(2 * c["M"] * c["N"] * c["K"] for c in self.calls)
 
-    def launches_per_step(self, gemm=True, quant=True) -> int:
+    def launches_per_step(self, gemm=True, quant=True, fused=False) -> int:
         n = 0
         for c in self.calls:
+            if fused:
+                v = c["variant"]
+                fusable = v.swap_ab == 1 and v.split_k <= 16 and v.split_k * v.tile_n <= 512
+                n += 1 if fusable else 2
+                continue
             v = c["variant"]
             if quant:
                 n += 1
@@ -268,8 +274,16 @@ class Workload:
         qb, sb = reps[c["copy"] if copy is None else copy % len(reps)]
         lq.scaled_mm(self.fmt, c["q"], c["s"], qb, sb, C=c["C"], variant=c["variant"], stream=stream)
 
-    def step(self, stream, gemm=True, quant=True):
+    def fused(self, c, stream):
+        qb, sb = self.weights[c["layer"]][c["copy"]]
+        lq.quant_scaled_mm(self.fmt, c["x"], qb, sb, C=c["C"], q=c["q"], s=c["s"], variant=c["variant"],
+                           stream=stream)
+
+    def step(self, stream, gemm=True, quant=True, fused=False):
         for c in self.calls:
+            if fused:
+                self.fused(c, stream)
+                continue
             if quant:
                 self.quant(c, stream)
             if gemm:
@@ -425,6 +439,9 @@ def main() -> None:
     ap.add_argument("--copies", type=int, default=3, help="weight copies rotated to defeat L2 reuse")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--per-shape-reps", type=int, default=30)
+    ap.add_argument("--path", default="separate", choices=["fused", "separate"],
+                    help="fused: one lq_quant_scaled_mm per linear (quantization inside the GEMM kernel); "
+                         "separate: lq_quant_per_token then lq_scaled_mm")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -450,7 +467,8 @@ def main() -> None:
     stream.wait_stream(torch.cuda.current_stream())
 
     # one CUDA graph per step (quant + GEMM of every call), and GEMM-only / quant-only graphs
-    g_step = capture(lambda: wl.step(stream), stream)
+    use_fused = args.path == "fused" and wl.fmt != "block_fp8"
+    g_step = capture(lambda: wl.step(stream, fused=use_fused), stream)
     g_gemm = capture(lambda: wl.step(stream, quant=False), stream)
     g_quant = capture(lambda: wl.step(stream, gemm=False), stream)
 
@@ -512,7 +530,7 @@ def main() -> None:
     g_e2e = []
     for b in range(2):
         wl.bind(x_bufs[b], c_bufs[b])
-        g_e2e.append(capture(lambda: wl.step(stream), stream))
+        g_e2e.append(capture(lambda: wl.step(stream, fused=use_fused), stream))
     wl.bind(x_bufs[0], c_bufs[0])
     h2d_s = torch.cuda.Stream(device=device)
     d2h_s = torch.cuda.Stream(device=device)
@@ -567,6 +585,23 @@ def main() -> None:
         cpu = cpu_baseline(args.config, budget_s=15.0)
 
     layers = ",".join(f"{k}({K}x{N})" for k, (K, N) in wl.layers.items())
+    if use_fused:
+        # the dominant (and only) kernel of the step: the fused quantize + GEMM kernel
+        roofline = {"bound": "hbm", "kernel": "lq_quant_scaled_mm fused kernel (all launches of one step)",
+                    "achieved": round(value / world, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(value / world / peaks["hbm_gbs"], 4),
+                    "traffic": recorded_traffic(args.config, "fused"),
+                    "traffic_unit": "DRAM bytes per step of the fused launches (ncu)",
+                    "algorithmic_bytes_per_step": step_bytes, "launches_per_step": wl.launches_per_step(fused=True),
+                    "us_per_step": round(ms_step * 1e3, 2), "peak_source": peaks["source"]}
+    else:
+        roofline = {"bound": "hbm", "kernel": "scaled_mm (all launches of one step)",
+                    "achieved": round(gemm_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(gemm_gbs / peaks["hbm_gbs"], 4),
+                    "traffic": recorded_traffic(args.config, "scaled_mm"),
+                    "traffic_unit": "DRAM bytes per step of scaled_mm launches (ncu)",
+                    "algorithmic_bytes_per_step": wl.gemm_bytes, "launches_per_step": wl.launches_per_step(quant=False),
+                    "us_per_step": round(ms_gemm * 1e3, 2), "peak_source": peaks["source"]}
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -583,21 +618,21 @@ def main() -> None:
         "config": {"workload": args.config, "format": wl.fmt, "layers": layers, "M": list(wl.ms),
                    "calls_per_step": len(wl.calls), "parallelism": f"replicas x{world}",
                    "l2": "weight copies rotated so that > 2x L2 is streamed between two reads of one copy",
-                   "graph": "one CUDA graph per step"},
+                   "graph": "one CUDA graph per step",
+                   "path": "lq_quant_scaled_mm (activation quantization fused into the GEMM kernel)" if use_fused
+                   else "lq_quant_per_token + lq_scaled_mm"},
         "tflops": round(tflops, 3),
         "frac_hbm_step": round(value / world / peaks["hbm_gbs"], 4),
-        "roofline": {"bound": "hbm", "kernel": "scaled_mm (all launches of one step)",
-                     "achieved": round(gemm_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(gemm_gbs / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(args.config),
-                     "traffic_unit": "DRAM bytes per step of scaled_mm launches (ncu)",
-                     "algorithmic_bytes_per_step": wl.gemm_bytes, "launches_per_step": wl.launches_per_step(quant=False),
-                     "us_per_step": round(ms_gemm * 1e3, 2), "peak_source": peaks["source"]},
+        "roofline": roofline,
+        "scaled_mm_only": {"GB/s": round(gemm_gbs, 1), "frac": round(gemm_gbs / peaks["hbm_gbs"], 4),
+                           "us_per_step": round(ms_gemm * 1e3, 2), "algorithmic_bytes_per_step": wl.gemm_bytes,
+                           "what": "the step's 28 lq_scaled_mm calls alone (codes already quantized)"},
         "quant_us_per_step": round(ms_quant * 1e3, 2),
         "clocks": clocks,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "ms_per_step": round(ms_e2e, 5),
                 "pipeline": "H2D / step / D2H on three streams, double-buffered",
                 "h2d_bytes_per_step": wl.x_all.numel() * 2, "d2h_bytes_per_step": wl.c_all.numel() * 2},
-        "gpu_launches": wl.launches_per_step() * args.steps,
+        "gpu_launches": wl.launches_per_step(fused=use_fused) * args.steps,
         "per_shape": per_shape,
     }
     if cpu is not None:

@@ -158,6 +158,32 @@ lq_status lq_scaled_mm_i32acc(const void *A, const float *a_scales,
                               const lq_variant *variant, lq_stream_t stream);
 
 /*
+ * Quantize the activations and multiply, in one kernel where possible: the
+ * per-token dynamic quantization of lq_quant_per_token fused with
+ * lq_scaled_mm (the in-GEMM activation quantization that the pages' fused
+ * quantization kernels motivate; 24-ai.news report, section "kernels
+ * integrated into vLLM", and the blog's aim of fewer kernel calls per
+ * forward pass).
+ *
+ *   fmt      : LQ_FP8_DYNAMIC or LQ_W8A8_INT8.
+ *   x        : [M, K] bf16 activations, 16-byte aligned.
+ *   B, b_scales, C, M, N, K : as lq_scaled_mm.
+ *   a_codes  : [M, K] out, the activation codes (16-byte aligned).
+ *   a_scales : [M] out, the per-token scales.
+ *   variant  : NULL = the dispatch table's choice for (fmt, M, N, K).
+ * a_codes, a_scales and C equal, bit for bit, those of lq_quant_per_token
+ * followed by lq_scaled_mm with the same variant.  With a Swap-AB variant
+ * (split_k <= 16 and split_k * tile_n <= 512) one kernel does both: its
+ * Split-K CTAs form a cluster (reduce is forced to 2) and exchange the
+ * per-token amax; other variants run the two kernels.  Errors as
+ * lq_scaled_mm; LQ_ERR_INVALID_ARG for Block_FP8.
+ */
+lq_status lq_quant_scaled_mm(lq_fmt fmt, const void *x, const void *B,
+                             const float *b_scales, void *C, void *a_codes,
+                             float *a_scales, int64_t M, int64_t N, int64_t K,
+                             const lq_variant *variant, lq_stream_t stream);
+
+/*
  * Allocation-free scaled_mm, for callers that cannot call cudaMalloc when
  * they run a GEMM: code running while a CUDA graph is captured with the
  * global capture mode (an allocation is an unsafe call there), frameworks

@@ -303,8 +303,10 @@ lq_status check_gemm_args(int fmt, const void* A, const float* a_s, const void* 
 
 lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B, const float* b_s, void* C,
                          int32_t* acc_out, int64_t M, int64_t N, int64_t K, const lq_variant* variant,
-                         cudaStream_t stream) {
-  lq_status rc = check_gemm_args(fmt, A, a_s, B, b_s, C, M, N, K);
+                         cudaStream_t stream, const void* x_fused = nullptr, void* codes_out = nullptr,
+                         float* scales_out = nullptr) {
+  const bool fused = x_fused != nullptr;
+  lq_status rc = fused ? LQ_OK : check_gemm_args(fmt, A, a_s, B, b_s, C, M, N, K);
   if (rc != LQ_OK) return rc;
   if (acc_out && !aligned(acc_out, 16)) return LQ_ERR_ALIGNMENT;
   if (M == 0 || N == 0) return LQ_OK;
@@ -355,6 +357,9 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   p.wait_limit_ns = wait_limit_ns();
   p.trace = g_trace.load();
   p.skip_stage = g_skip_stage.load();
+  p.x = static_cast<const __nv_bfloat16*>(x_fused);
+  p.a_codes_out = static_cast<uint8_t*>(codes_out);
+  p.a_scales_out = scales_out;
   if (v.split_k > 1 && v.reduce != 2) {   // the cluster reduction needs no global workspace
     const size_t need = static_cast<size_t>(v.split_k) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
     rc = ensure_workspace(d, need, stream);
@@ -365,8 +370,10 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   }
   const void* x_ptr = v.swap_ab ? B : A;
   const void* y_ptr = v.swap_ab ? A : B;
-  if (!encode_operand(&l.tmX, x_ptr, x_rows, K, 128) || !encode_operand(&l.tmY, y_ptr, y_rows, K, v.tile_n))
-    return LQ_ERR_CUDA;
+  if (!encode_operand(&l.tmX, x_ptr, x_rows, K, 128)) return LQ_ERR_CUDA;
+  if (fused) l.tmY = l.tmX;   // the activation operand is produced in the kernel, not loaded by TMA
+  else if (!encode_operand(&l.tmY, y_ptr, y_rows, K, v.tile_n)) return LQ_ERR_CUDA;
+  l.fuse = fused ? 1 : 0;
   l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
   l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce);
   l.pdl = v.pdl != 0;
@@ -480,6 +487,37 @@ lq_status lq_scaled_mm_i32acc(const void* A, const float* a_scales, const void* 
   if (!acc_out && M > 0 && N > 0) return LQ_ERR_INVALID_ARG;
   return scaled_mm_impl(lq::kFmtInt8, A, a_scales, B, b_scales, C, acc_out, M, N, K, variant,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+lq_status lq_quant_scaled_mm(lq_fmt fmt_, const void* x, const void* B, const float* b_scales, void* C,
+                             void* a_codes, float* a_scales, int64_t M, int64_t N, int64_t K,
+                             const lq_variant* variant, lq_stream_t stream_) {
+  const int fmt = static_cast<int>(fmt_);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (fmt != lq::kFmtFp8 && fmt != lq::kFmtInt8) return LQ_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return LQ_OK;
+  if (!x || !B || !b_scales || !C || !a_codes || !a_scales) return LQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(a_codes, 16) || !aligned(a_scales, 4) ||
+      !aligned(b_scales, 4))
+    return LQ_ERR_ALIGNMENT;
+  if (K % 16 != 0 || N % 8 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+  lq_variant v{};
+  if (variant) v = *variant;
+  else if (!lookup_table(fmt, M, N, K, &v)) v = heuristic_variant(fmt, M, N, K);
+  if (v.split_k > 1) v.reduce = 2;   // the per-token amax is exchanged inside the Split-K cluster
+  const bool fusable = K > 0 && v.swap_ab == 1 && v.split_k <= 16 && v.split_k * v.tile_n <= 512;
+  if (!fusable) {
+    // quantize, then scaled_mm (same codes, scales and result as the fused kernel)
+    if (M > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+    if (lq::launch_quant_per_token(fmt, x, a_codes, a_scales, M, K, stream) != cudaSuccess) {
+      cudaGetLastError();
+      return LQ_ERR_CUDA;
+    }
+    return scaled_mm_impl(fmt, a_codes, a_scales, B, b_scales, C, nullptr, M, N, K, variant ? &v : nullptr, stream);
+  }
+  return scaled_mm_impl(fmt, a_codes, a_scales, B, b_scales, C, nullptr, M, N, K, &v, stream, x, a_codes, a_scales);
 }
 
 lq_status lq_quant_per_token(lq_fmt fmt, const void* x, void* q, float* scales, int64_t M, int64_t K,

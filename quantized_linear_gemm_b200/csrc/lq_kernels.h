@@ -31,6 +31,10 @@ struct GemmParams {
   uint64_t wait_limit_ns;
   uint64_t* trace;     // optional: kTraceSlots globaltimer stamps per CTA
   int skip_stage;      // test hook: >= 0 = the producer never fills this K tile (a wait runs out)
+  // fused activation quantization (Swap-AB, FP8_Dynamic / W8A8_INT8)
+  const __nv_bfloat16* x;   // bf16 activations [M, K]
+  uint8_t* a_codes_out;     // [M, K] codes written by the first n-tile's CTAs
+  float* a_scales_out;      // [M] per-token scales
 };
 
 constexpr int kTraceSlots = 12;
@@ -44,6 +48,7 @@ struct GemmLaunch {
   int smem_bytes;
   int pdl;
   int cluster_z;       // > 1: launch clusters of (1, 1, cluster_z) CTAs
+  int fuse;            // fused activation quantization (Swap-AB only)
   cudaStream_t stream;
 };
 

@@ -27,6 +27,7 @@
 
 #include "lq_kernels.h"
 #include "ptx.cuh"
+#include "quant_common.cuh"
 
 namespace lq {
 
@@ -86,6 +87,7 @@ struct SmemCtl {
   uint64_t* tempty;    // [2]
   uint64_t* mma_done;  // [1]
   uint64_t* red_bar;   // [1] push reduction: partial columns received
+  uint64_t* amax_bar;  // [1] fused quantization: per-token partial amax of every split received
   uint32_t* tmem_slot;
   volatile int* abort_flag;
   volatile int* last_flag;
@@ -135,11 +137,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---------------------------------------------------------------------------
 // The GEMM kernel
 // ---------------------------------------------------------------------------
-template <int FMT, bool SWAP, int TN>
+// FUSE (Swap-AB, FP8_Dynamic / W8A8_INT8 only): the activations arrive as
+// bf16; the epilogue warps, idle during the mainloop, quantize them per
+// token into the ring's activation slots (see the A-producer below).
+template <int FMT, bool SWAP, int TN, bool FUSE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     scaled_mm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                         const GemmParams p) {
+  static_assert(!FUSE || (SWAP && FMT != kFmtBlock && TN <= 64), "fused quantization: Swap-AB FP8/INT8 tiles");
   using Shape = TileShape<TN>;
+  // bytes the TMA delivers per stage (the fused path writes the activation slot itself)
+  constexpr uint32_t kTmaStageBytes = FUSE ? Shape::kXBytes : Shape::kStageBytes;
   constexpr bool kInt8 = FMT == kFmtInt8;
   constexpr bool kBlocked = FMT == kFmtBlock;
   constexpr int kAccBufs = kBlocked ? 2 : 1;
@@ -162,7 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   c.tempty = c.tfull + 2;
   c.mma_done = c.tempty + 2;
   c.red_bar = c.mma_done + 1;
-  c.tmem_slot = reinterpret_cast<uint32_t*>(c.red_bar + 1);
+  c.amax_bar = c.red_bar + 1;
+  c.tmem_slot = reinterpret_cast<uint32_t*>(c.amax_bar + 1);
   c.abort_flag = reinterpret_cast<volatile int*>(c.tmem_slot + 1);
   c.last_flag = c.abort_flag + 1;
   float* sc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kCtlBytes);
@@ -180,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) trace_stamp(p, 0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
-      mbar_init(&c.full[s], 1);
+      mbar_init(&c.full[s], FUSE ? 1 + kEpiThreads / 32 : 1);   // TMA (+ the four A-producer warps)
       mbar_init(&c.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -189,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(c.mma_done, 1);
     mbar_init(c.red_bar, 1);
+    mbar_init(c.amax_bar, 1);
     *c.abort_flag = 0;
     *c.last_flag = 0;
     fence_barrier_init();
@@ -235,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < pre; ++i) {
           if (i == p.skip_stage) continue;
           uint8_t* st = ring + i * Shape::kStageBytes;
-          mbar_arrive_expect_tx(&c.full[i], Shape::kStageBytes);
+          mbar_arrive_expect_tx(&c.full[i], kTmaStageBytes);
           tma_load_2d(tmW, &c.full[i], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
         }
         grid_dependency_wait();
@@ -244,13 +254,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < pre; ++i) {
           if (i == p.skip_stage) continue;
           uint8_t* st = ring + i * Shape::kStageBytes;
-          mbar_arrive_expect_tx(&c.full[i], Shape::kStageBytes);
+          mbar_arrive_expect_tx(&c.full[i], kTmaStageBytes);
           tma_load_2d(tmW, &c.full[i], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
         }
       }
       trace_stamp(p, 2);
       for (int i = 0; i < pre; ++i) {
-        if (i == p.skip_stage) continue;
+        if (FUSE || i == p.skip_stage) continue;
         uint8_t* st = ring + i * Shape::kStageBytes;
         tma_load_2d(tmA, &c.full[i], st + a_off, (kb_lo + i) * kTileK, a_row0, pol_a);
       }
@@ -261,9 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_bar(&c.empty[s], ph ^ 1u, p, c, 0)) break;
         if (i == p.skip_stage) continue;
         uint8_t* st = ring + s * Shape::kStageBytes;
-        mbar_arrive_expect_tx(&c.full[s], Shape::kStageBytes);
+        mbar_arrive_expect_tx(&c.full[s], kTmaStageBytes);
         tma_load_2d(tmW, &c.full[s], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
-        tma_load_2d(tmA, &c.full[s], st + a_off, (kb_lo + i) * kTileK, a_row0, pol_a);
+        if (!FUSE) tma_load_2d(tmA, &c.full[s], st + a_off, (kb_lo + i) * kTileK, a_row0, pol_a);
         issued = i + 1;
       }
       if (*c.abort_flag) {
@@ -337,14 +347,136 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (!kBlocked) {
       // Scales do not depend on the accumulator: load them while the mainloop
-      // runs (these warps are idle until then).
-      for (int j = r; j < TN; j += kEpiThreads) {
-        const int64_t col = y_row0 + j;
-        colsc[j] = SWAP ? (col < M ? __ldg(p.a_s + col) : 0.f) : (col < N ? __ldg(p.b_s + col) : 0.f);
+      // runs (these warps are idle until then).  The fused path computes the
+      // token scales itself below.
+      if (!FUSE) {
+        for (int j = r; j < TN; j += kEpiThreads) {
+          const int64_t col = y_row0 + j;
+          colsc[j] = SWAP ? (col < M ? __ldg(p.a_s + col) : 0.f) : (col < N ? __ldg(p.b_s + col) : 0.f);
+        }
       }
       const int64_t row = x_row0 + r;
       rowsc[r] = SWAP ? (row < N ? __ldg(p.b_s + row) : 0.f) : (row < M ? __ldg(p.a_s + row) : 0.f);
       named_barrier_sync(2, kEpiThreads);
+    }
+
+    bool cluster_waited = false;
+    if constexpr (FUSE) {
+      // ------------------------------------------------ A-producer (fused)
+      // 1. partial amax of each token over this CTA's K range;
+      // 2. Split-K cluster: every CTA sends its partials to every CTA
+      //    (st.async, counted in bytes on amax_bar) and takes the max, so all
+      //    CTAs of a tile derive the same per-token scale;
+      // 3. s = max(fp32(amax / Q), 2^-126); q = enc(fp32(x / s)) for each K
+      //    tile, written in the 128-byte-swizzled K-major layout that the
+      //    tensor core reads, into the stage's activation slot; the four
+      //    warps' arrivals (with the weight TMA) complete the stage.
+      // Codes and scales equal those of lq_quant_per_token bit for bit.
+      constexpr int kChunks = TN * 8 / kEpiThreads;   // 16-byte code chunks per thread per K tile (TN >= 16)
+      const int e = warp - 2;                         // epilogue warp 0..3
+      const int tid = e * 32 + lane;                  // epilogue thread 0..127
+      float* pa = sc + 384;                           // [TN] this CTA's partial amax
+      float* slots_amax = sc + 512;                   // [S][TN] partial amax of every split
+      const int64_t k_lo = static_cast<int64_t>(kb_lo) * kTileK;
+      const int64_t k_hi = min(static_cast<int64_t>(kb_hi) * kTileK, p.K);
+      const float qmax = kInt8 ? kInt8Max : kE4m3Max;
+      for (int j = e; j < TN; j += 4) {
+        const int64_t m = y_row0 + j;
+        float a = 0.f;
+        if (m < M) {
+          const uint4* xr = reinterpret_cast<const uint4*>(p.x + m * p.K);
+#pragma unroll 4
+          for (int64_t v = k_lo / 8 + lane; v < k_hi / 8; v += 32) {
+            float f[8];
+            bf16x8_to_f32(__ldg(xr + v), f);
+            a = fmaxf(a, amax8(f));
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        if (lane == 0) pa[j] = a;
+      }
+      named_barrier_sync(2, kEpiThreads);
+      if (p.S > 1) {
+        cluster_wait_acquire();   // every CTA of the cluster has initialised its barriers
+        cluster_waited = true;
+        if (tid == 0) mbar_arrive_expect_tx(c.amax_bar, static_cast<uint32_t>(p.S * TN * 4));
+        if (tid < p.S) {
+          const uint32_t dst = dsmem_map(smem_addr(slots_amax), static_cast<uint32_t>(tid)) +
+                               static_cast<uint32_t>(split * TN * 4);
+          const uint32_t bar = dsmem_map(smem_addr(c.amax_bar), static_cast<uint32_t>(tid));
+#pragma unroll
+          for (int j = 0; j < TN; j += 4)
+            st_async_v4(dst + j * 4, __float_as_uint(pa[j]), __float_as_uint(pa[j + 1]), __float_as_uint(pa[j + 2]),
+                        __float_as_uint(pa[j + 3]), bar);
+        }
+        wait_bar<true>(c.amax_bar, 0, p, c, 8);
+      }
+      if (tid < TN) {
+        float a = pa[tid];
+        if (p.S > 1) {
+          a = 0.f;
+          for (int s2 = 0; s2 < p.S; ++s2) a = fmaxf(a, slots_amax[s2 * TN + tid]);
+        }
+        const int64_t m = y_row0 + tid;
+        const float sm = scale_from_amax(a, qmax);
+        colsc[tid] = sm;
+        if (p.a_scales_out && blockIdx.x == 0 && split == 0 && m < M) p.a_scales_out[m] = sm;
+      }
+      named_barrier_sync(2, kEpiThreads);
+
+      // 4. produce the activation tiles, loads of tile i+1 in flight while tile i is encoded
+      auto load_tile = [&](int i, uint4 (&buf)[2 * kChunks]) {
+#pragma unroll
+        for (int u = 0; u < kChunks; ++u) {
+          const int t = tid + u * kEpiThreads;
+          const int j = t >> 3, cc = t & 7;
+          const int64_t m = y_row0 + j;
+          const int64_t k0 = static_cast<int64_t>(kb_lo + i) * kTileK + cc * 16;
+          if (m < M && k0 < p.K) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.x + m * p.K + k0);
+            buf[2 * u] = __ldg(src);
+            buf[2 * u + 1] = __ldg(src + 1);
+          } else {
+            buf[2 * u] = make_uint4(0u, 0u, 0u, 0u);
+            buf[2 * u + 1] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+      };
+      uint4 cur[2 * kChunks], nxt[2 * kChunks];
+      if (nkb > 0) load_tile(0, cur);
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % stages;
+        if (i + 1 < nkb) load_tile(i + 1, nxt);
+        if (i >= stages) {
+          const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
+          if (!wait_bar(&c.empty[s], ph ^ 1u, p, c, 9)) break;   // the MMA has released this slot
+        }
+        uint8_t* slot = ring + s * Shape::kStageBytes + Shape::kXBytes;
+#pragma unroll
+        for (int u = 0; u < kChunks; ++u) {
+          const int t = tid + u * kEpiThreads;
+          const int j = t >> 3, cc = t & 7;
+          const float sm = colsc[j];
+          float f0[8], f1[8];
+          bf16x8_to_f32(cur[2 * u], f0);
+          bf16x8_to_f32(cur[2 * u + 1], f1);
+          const uint2 q0 = kInt8 ? encode8_int8(f0, sm) : encode8_e4m3(f0, sm);
+          const uint2 q1 = kInt8 ? encode8_int8(f1, sm) : encode8_e4m3(f1, sm);
+          const uint4 qv = make_uint4(q0.x, q0.y, q1.x, q1.y);
+          // row j of the slot, 16-byte chunk cc placed at cc ^ (j % 8) (128-byte swizzle)
+          *reinterpret_cast<uint4*>(slot + j * kTileK + ((cc ^ (j & 7)) << 4)) = qv;
+          const int64_t m = y_row0 + j;
+          const int64_t k0 = static_cast<int64_t>(kb_lo + i) * kTileK + cc * 16;
+          if (p.a_codes_out && blockIdx.x == 0 && m < M && k0 < p.K)
+            *reinterpret_cast<uint4*>(p.a_codes_out + m * p.K + k0) = qv;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // generic stores -> tensor core
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.full[s]);
+#pragma unroll
+        for (int u = 0; u < 2 * kChunks; ++u) cur[u] = nxt[u];
+      }
     }
 
     bool ok = true;
@@ -414,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // before the generic-proxy stores of the pulled partial tile.
     if (cluster_mode && !push_mode) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (push_mode) {
-      cluster_wait_acquire();   // every CTA of the cluster has initialised its barriers
+      if (!cluster_waited) cluster_wait_acquire();   // every CTA of the cluster has initialised its barriers
       if (warp == 2 && lane == 0) {
         trace_stamp(p, 8);
         mbar_arrive_expect_tx(c.red_bar, static_cast<uint32_t>(ClusterReduce<TN>::kSlotBytes));

@@ -5,9 +5,9 @@
 
 namespace lq {
 
-template <int FMT, bool SWAP, int TN>
+template <int FMT, bool SWAP, int TN, bool FUSE = false>
 cudaError_t launch_tc(const GemmLaunch& l) {
-  auto kern = scaled_mm_tc_kernel<FMT, SWAP, TN>;
+  auto kern = scaled_mm_tc_kernel<FMT, SWAP, TN, FUSE>;
   static int configured = 0;   // max dynamic smem set once per instantiation and process
   if (configured < l.smem_bytes) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
@@ -44,6 +44,18 @@ cudaError_t launch_tc(const GemmLaunch& l) {
 
 template <int FMT>
 cudaError_t launch_format(const GemmLaunch& l, int swap_ab, int tile_n) {
+  if (l.fuse) {
+    if constexpr (FMT != kFmtBlock) {
+      if (!swap_ab) return cudaErrorInvalidValue;
+      switch (tile_n) {
+        case 16: return launch_tc<FMT, true, 16, true>(l);
+        case 32: return launch_tc<FMT, true, 32, true>(l);
+        case 64: return launch_tc<FMT, true, 64, true>(l);
+        default: return cudaErrorInvalidValue;
+      }
+    }
+    return cudaErrorInvalidValue;
+  }
   if (swap_ab) {
     switch (tile_n) {
       case 16: return launch_tc<FMT, true, 16>(l);

@@ -34,6 +34,7 @@ EXPORTED = (
     "lq_quant_weight_block128", "lq_select_variant", "lq_load_dispatch_table", "lq_dispatch_table_size",
     "lq_init_device", "lq_reserve_workspace", "lq_workspace_bytes", "lq_device_status",
     "lq_status_string", "lq_version", "lq_set_trace", "lq_scaled_mm_noalloc", "lq_test_inject_stall",
+    "lq_quant_scaled_mm",
 )
 
 
@@ -75,6 +76,9 @@ def lib() -> ctypes.CDLL:
                                    "`python -m quantized_linear_gemm_b200.build`")
             L = ctypes.CDLL(LIB_PATH)
             L.lq_scaled_mm.argtypes = [_i32, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.POINTER(Variant), _st]
+            L.lq_quant_scaled_mm.argtypes = [_i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                             ctypes.POINTER(Variant), _st]
+            L.lq_quant_scaled_mm.restype = _i32
             L.lq_scaled_mm_noalloc.argtypes = [_i32, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                                                ctypes.POINTER(Variant), _st]
             L.lq_scaled_mm_noalloc.restype = _i32
@@ -163,6 +167,27 @@ def scaled_mm(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor, b_s
                             ctypes.byref(variant) if variant is not None else None, _stream(stream))
     _check("lq_scaled_mm", rc)
     return C
+
+
+def quant_scaled_mm(fmt, x: torch.Tensor, B: torch.Tensor, b_scales: torch.Tensor, C=None, q=None, s=None,
+                    variant: Variant | None = None, stream=None):
+    """``lq_quant_scaled_mm``: per-token quantization of bf16 ``x`` fused with
+    scaled_mm.  Returns (C, codes, scales)."""
+    f = _fmt(fmt)
+    _need(x, "x", (torch.bfloat16,), 2)
+    _need(B, "B", _CODE_DTYPES, 2)
+    M, K = x.shape
+    N = B.shape[0]
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.int8 if f == W8A8_INT8 else torch.uint8, device=x.device)
+    if s is None:
+        s = torch.empty((M,), dtype=torch.float32, device=x.device)
+    rc = lib().lq_quant_scaled_mm(f, _ptr(x), _ptr(B), _ptr(b_scales), _ptr(C), _ptr(q), _ptr(s), M, N, K,
+                                  ctypes.byref(variant) if variant is not None else None, _stream(stream))
+    _check("lq_quant_scaled_mm", rc)
+    return C, q, s
 
 
 def scaled_mm_noalloc(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor, b_scales: torch.Tensor,

@@ -94,6 +94,16 @@ def test_quant_argument_checks():
     assert L.lq_quant_weight_block128(FAKE, FAKE, FAKE, 0, 256, None) == OK
 
 
+def test_quant_scaled_mm_argument_checks():
+    L = lq.lib()
+    assert L.lq_quant_scaled_mm(2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 128, 128, None, None) == INVALID  # block
+    assert L.lq_quant_scaled_mm(0, None, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 128, 128, None, None) == INVALID
+    assert L.lq_quant_scaled_mm(0, FAKE, FAKE, FAKE, FAKE, None, FAKE, 4, 128, 128, None, None) == INVALID
+    assert L.lq_quant_scaled_mm(0, MISALIGNED, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 128, 128, None, None) == ALIGN
+    assert L.lq_quant_scaled_mm(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 100, 128, None, None) == SHAPE
+    assert L.lq_quant_scaled_mm(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 128, 128, None, None) == OK
+
+
 def test_stall_hook_argument_check():
     assert lq.lib().lq_test_inject_stall(-2, 0) == INVALID
     assert lq.lib().lq_test_inject_stall(-1, 0) == OK
