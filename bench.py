@@ -468,6 +468,8 @@ def main() -> None:
 
     # one CUDA graph per step (quant + GEMM of every call), and GEMM-only / quant-only graphs
     use_fused = args.path == "fused" and wl.fmt != "block_fp8"
+    if use_fused:
+        lq.set_fuse_limit(1 << 40)   # every fusable call takes the one-kernel path
     g_step = capture(lambda: wl.step(stream, fused=use_fused), stream)
     g_gemm = capture(lambda: wl.step(stream, quant=False), stream)
     g_quant = capture(lambda: wl.step(stream, gemm=False), stream)

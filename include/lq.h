@@ -87,7 +87,7 @@ typedef enum {
  *            so results are reproducible bit for bit.
  *  tile_n  : Standard: 64, 128 or 256 (Block_FP8: 64 or 128);
  *            Swap-AB: 16, 32 or 64.
- *  stages  : depth of the shared-memory ring (2..16), 0 = the deepest that
+ *  stages  : depth of the shared-memory ring (2..14), 0 = the deepest that
  *            fits.
  *  reduce  : for split_k > 1: 0 = partials to a global workspace and a
  *            separate reduction kernel; 1 = partials to the workspace and the
@@ -172,16 +172,31 @@ lq_status lq_scaled_mm_i32acc(const void *A, const float *a_scales,
  *   a_scales : [M] out, the per-token scales.
  *   variant  : NULL = the dispatch table's choice for (fmt, M, N, K).
  * a_codes, a_scales and C equal, bit for bit, those of lq_quant_per_token
- * followed by lq_scaled_mm with the same variant.  With a Swap-AB variant
- * (split_k <= 16 and split_k * tile_n <= 512) one kernel does both: its
- * Split-K CTAs form a cluster (reduce is forced to 2) and exchange the
- * per-token amax; other variants run the two kernels.  Errors as
- * lq_scaled_mm; LQ_ERR_INVALID_ARG for Block_FP8.
+ * followed by lq_scaled_mm with the same variant.  By default the two
+ * kernels run (lq_quant_per_token, then lq_scaled_mm).  With a Swap-AB
+ * variant (split_k <= 16 and split_k * tile_n <= 512) whose CTAs each see an
+ * activation slice (min(M, tile_n) x ceil(K / 128 / split_k) x 128 bf16
+ * values) no larger than a limit that is 0 by default (raise it with
+ * lq_set_fuse_limit or the environment variable LQ_FUSE_MAX_SLICE_BYTES,
+ * read once), one kernel does both: the TMA stages each bf16 activation tile
+ * beside the weight tile, the CTA's idle epilogue warps quantize it into the
+ * tensor core's operand slot, and the Split-K CTAs form a cluster (reduce is
+ * forced to 2) that exchanges the per-token amax.  Errors as lq_scaled_mm;
+ * LQ_ERR_INVALID_ARG for Block_FP8.
  */
 lq_status lq_quant_scaled_mm(lq_fmt fmt, const void *x, const void *B,
                              const float *b_scales, void *C, void *a_codes,
                              float *a_scales, int64_t M, int64_t N, int64_t K,
                              const lq_variant *variant, lq_stream_t stream);
+
+/*
+ * Sets, for this process, the largest per-CTA activation slice (bytes) for
+ * which lq_quant_scaled_mm uses its one-kernel path; 0 = never fuse, a
+ * negative value restores the default (0, or LQ_FUSE_MAX_SLICE_BYTES).
+ * Returns the limit in force before the call.  A tuning and test hook: it
+ * changes which kernels run, never the results.
+ */
+int64_t lq_set_fuse_limit(int64_t max_slice_bytes);
 
 /*
  * Allocation-free scaled_mm, for callers that cannot call cudaMalloc when

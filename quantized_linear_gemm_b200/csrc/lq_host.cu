@@ -38,6 +38,14 @@ constexpr int kMaxDevices = 64;
 constexpr int kMaxSmemPerCta = 227 * 1024;
 constexpr size_t kCounterCapacity = size_t(1) << 20;   // Split-K arrival counters per device
 constexpr int kNumSms = 148;
+constexpr int kMaxStages = 14;   // the kernel's control block holds 4 x stages + 7 mbarriers (64 at most)
+// 0: lq_quant_scaled_mm runs the quantization kernel and the GEMM unless a
+// caller raises the limit.  Measured on B200 (Qwen3-8B decode shapes, FP8):
+// the one-kernel path saves up to 1.2 us per call at M = 1 on the down
+// projection but loses 0.3 - 2 us elsewhere, since its first MMA waits for
+// the per-token amax (a pass over the CTA's slice of x plus a cluster
+// exchange) that the separate kernel overlaps with the GEMM's weight stream.
+constexpr int64_t kFuseMaxSliceBytes = 0;
 
 // ---------------------------------------------------------------- devices
 struct DeviceState {
@@ -53,6 +61,25 @@ DeviceState g_dev[kMaxDevices];
 std::atomic<uint64_t*> g_trace{nullptr};   // diagnostics: per-CTA stamps of the next launches
 std::atomic<int> g_skip_stage{-1};          // test hook: K tile the producer never fills
 std::atomic<uint64_t> g_wait_limit_override{0};
+
+// Largest per-CTA activation slice (tokens x K range x 2 bytes) for which
+// lq_quant_scaled_mm uses the fused kernel; LQ_FUSE_MAX_SLICE_BYTES overrides.
+std::atomic<int64_t> g_fuse_limit_override{-1};
+
+int64_t fuse_max_slice_bytes() {
+  const int64_t o = g_fuse_limit_override.load();
+  if (o >= 0) return o;
+  static int64_t v = [] {
+    const char* e = std::getenv("LQ_FUSE_MAX_SLICE_BYTES");
+    if (e && *e) {
+      char* end = nullptr;
+      long long x = std::strtoll(e, &end, 10);
+      if (end != e && x >= 0) return static_cast<int64_t>(x);
+    }
+    return static_cast<int64_t>(kFuseMaxSliceBytes);
+  }();
+  return v;
+}
 
 uint64_t wait_limit_ns() {
   const uint64_t o = g_wait_limit_override.load();
@@ -161,6 +188,21 @@ bool encode_operand(CUtensorMap* map, const void* ptr, int64_t rows, int64_t K, 
   return r == CUDA_SUCCESS;
 }
 
+// Row-major bf16 activations [rows, K], tiles of box_rows x 128 elements
+// (256 bytes, no swizzle); out-of-range rows / K are zero-filled.
+bool encode_bf16_rows(CUtensorMap* map, const void* ptr, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2u};
+  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // --------------------------------------------------------- dispatch table
 struct TableEntry {
   int fmt;
@@ -210,12 +252,12 @@ int64_t m_bucket(int64_t M) {
 }
 
 // Deepest ring that fits when `ctas_per_sm` CTAs share one SM's shared memory.
-int max_stages_fit(int tile_n, int ctas_per_sm, bool cluster_reduce) {
+int max_stages_fit(int tile_n, int ctas_per_sm, bool cluster_reduce, bool fuse = false) {
   const int share = (228 * 1024) / ctas_per_sm - 1024;
   const int budget = share < kMaxSmemPerCta ? share : kMaxSmemPerCta;
   int best = 2;
-  for (int s = 2; s <= 16; ++s)
-    if (lq::gemm_smem_bytes_for(tile_n, s, cluster_reduce) <= budget) best = s;
+  for (int s = 2; s <= kMaxStages; ++s)
+    if (lq::gemm_smem_bytes_for(tile_n, s, cluster_reduce, fuse) <= budget) best = s;
   return best;
 }
 
@@ -276,7 +318,7 @@ lq_status check_variant(int fmt, const lq_variant& v) {
     if (v.tile_n != 64 && v.tile_n != 128 && v.tile_n != 256) return LQ_ERR_INVALID_ARG;
     if (fmt == lq::kFmtBlock && v.tile_n == 256) return LQ_ERR_INVALID_ARG;
   }
-  if (v.stages != 0 && (v.stages < 2 || v.stages > 16)) return LQ_ERR_INVALID_ARG;
+  if (v.stages != 0 && (v.stages < 2 || v.stages > kMaxStages)) return LQ_ERR_INVALID_ARG;
   if (v.stages != 0 &&
       lq::gemm_smem_bytes_for(v.tile_n, v.stages, v.split_k > 1 && v.reduce == 2) > kMaxSmemPerCta)
     return LQ_ERR_INVALID_ARG;
@@ -325,7 +367,9 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   rc = check_variant(fmt, v);
   if (rc != LQ_OK) return rc;
   const bool cluster_reduce = v.split_k > 1 && v.reduce == 2;
-  if (v.stages == 0) v.stages = max_stages_fit(v.tile_n, 1, cluster_reduce);
+  if (v.stages == 0) v.stages = max_stages_fit(v.tile_n, 1, cluster_reduce, fused);
+  if (fused && lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce, true) > kMaxSmemPerCta)
+    v.stages = max_stages_fit(v.tile_n, 1, cluster_reduce, true);
 
   const int64_t x_rows = v.swap_ab ? N : M;
   const int64_t y_rows = v.swap_ab ? M : N;
@@ -371,11 +415,15 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   const void* x_ptr = v.swap_ab ? B : A;
   const void* y_ptr = v.swap_ab ? A : B;
   if (!encode_operand(&l.tmX, x_ptr, x_rows, K, 128)) return LQ_ERR_CUDA;
-  if (fused) l.tmY = l.tmX;   // the activation operand is produced in the kernel, not loaded by TMA
-  else if (!encode_operand(&l.tmY, y_ptr, y_rows, K, v.tile_n)) return LQ_ERR_CUDA;
+  if (fused) {
+    // the kernel stages the bf16 activations and quantizes them itself
+    if (!encode_bf16_rows(&l.tmY, x_fused, M, K, v.tile_n)) return LQ_ERR_CUDA;
+  } else if (!encode_operand(&l.tmY, y_ptr, y_rows, K, v.tile_n)) {
+    return LQ_ERR_CUDA;
+  }
   l.fuse = fused ? 1 : 0;
   l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
-  l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce);
+  l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce, fused);
   l.pdl = v.pdl != 0;
   l.cluster_z = (v.split_k > 1 && v.reduce == 2) ? v.split_k : 1;
   l.stream = stream;
@@ -507,7 +555,13 @@ lq_status lq_quant_scaled_mm(lq_fmt fmt_, const void* x, const void* B, const fl
   if (variant) v = *variant;
   else if (!lookup_table(fmt, M, N, K, &v)) v = heuristic_variant(fmt, M, N, K);
   if (v.split_k > 1) v.reduce = 2;   // the per-token amax is exchanged inside the Split-K cluster
-  const bool fusable = K > 0 && v.swap_ab == 1 && v.split_k <= 16 && v.split_k * v.tile_n <= 512;
+  // Each CTA of the fused kernel reads its tokens' slice of x once more to
+  // find the per-token amax before any code exists; that read sits on the
+  // critical path, so the kernel is used only while the slice is small.
+  const int64_t T = (K + 127) / 128;
+  const int64_t slice_bytes = (M < v.tile_n ? M : v.tile_n) * ((T + v.split_k - 1) / v.split_k) * 128 * 2;
+  const bool fusable = K > 0 && v.swap_ab == 1 && v.split_k <= 16 && v.split_k * v.tile_n <= 512 &&
+                       slice_bytes <= fuse_max_slice_bytes();
   if (!fusable) {
     // quantize, then scaled_mm (same codes, scales and result as the fused kernel)
     if (M > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
@@ -518,6 +572,12 @@ lq_status lq_quant_scaled_mm(lq_fmt fmt_, const void* x, const void* B, const fl
     return scaled_mm_impl(fmt, a_codes, a_scales, B, b_scales, C, nullptr, M, N, K, variant ? &v : nullptr, stream);
   }
   return scaled_mm_impl(fmt, a_codes, a_scales, B, b_scales, C, nullptr, M, N, K, &v, stream, x, a_codes, a_scales);
+}
+
+int64_t lq_set_fuse_limit(int64_t max_slice_bytes) {
+  const int64_t prev = fuse_max_slice_bytes();
+  g_fuse_limit_override.store(max_slice_bytes < 0 ? -1 : max_slice_bytes);
+  return prev;
 }
 
 lq_status lq_quant_per_token(lq_fmt fmt, const void* x, void* q, float* scales, int64_t M, int64_t K,

@@ -62,7 +62,9 @@ cudaError_t launch_splitk_reduce(int fmt, const GemmParams& p, int pdl, cudaStre
 
 // Dynamic shared memory of the GEMM kernel for (tile_n, stages), with or
 // without the cluster Split-K reduction (reduce mode 2 with split_k > 1).
-int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce);
+// Dynamic shared memory of the GEMM kernel; `fuse`: the fused-quantization
+// instantiation (each ring slot also stages a bf16 activation tile).
+int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce, bool fuse = false);
 
 // Quantization kernels (quant_kernels.cu).
 cudaError_t launch_quant_per_token(int fmt, const void* x, void* q, float* scales, int64_t M, int64_t K,

@@ -69,6 +69,7 @@ __global__ void __launch_bounds__(256) quant_per_token_reg_kernel(const __nv_bfl
   }
   const float amax = block_max<256>(a, red);
   const float s = scale_from_amax(amax, kInt8 ? kInt8Max : kE4m3Max);
+  const Divisor d = make_divisor(amax, s);
   if (threadIdx.x == 0) scales[row] = s;
   uint2* qr = reinterpret_cast<uint2*>(q + row * K);
 #pragma unroll
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(256) quant_per_token_reg_kernel(const __nv_bfl
     if (idx < nvec) {
       float f[8];
       bf16x8_to_f32(v[i], f);
-      qr[idx] = kInt8 ? encode8_int8(f, s) : encode8_e4m3(f, s);
+      qr[idx] = kInt8 ? encode8_int8(f, d) : encode8_e4m3(f, d);
     }
   }
 }
@@ -102,12 +103,13 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const __nv_bfloat1
   }
   const float amax = block_max<256>(a, red);
   const float s = scale_from_amax(amax, kInt8 ? kInt8Max : kE4m3Max);
+  const Divisor d = make_divisor(amax, s);
   if (threadIdx.x == 0) scales[row] = s;
   uint2* qr = reinterpret_cast<uint2*>(q + row * K);
   for (int64_t i = threadIdx.x; i < nvec; i += blockDim.x) {
     float f[8];
     bf16x8_to_f32(__ldg(xr + i), f);
-    qr[i] = kInt8 ? encode8_int8(f, s) : encode8_e4m3(f, s);
+    qr[i] = kInt8 ? encode8_int8(f, d) : encode8_e4m3(f, d);
   }
 }
 
@@ -132,7 +134,7 @@ __global__ void __launch_bounds__(256) quant_group128_kernel(const __nv_bfloat16
   const float s = scale_from_amax(a, kE4m3Max);
   if (valid) {
     if (sub == 0) scales[row * KB + kb] = s;
-    *reinterpret_cast<uint2*>(q + off) = encode8_e4m3(f, s);
+    *reinterpret_cast<uint2*>(q + off) = encode8_e4m3(f, make_divisor(a, s));
   }
 }
 
@@ -155,10 +157,11 @@ __global__ void __launch_bounds__(256) quant_weight_block128_kernel(const __nv_b
   }
   const float amax = block_max<256>(a, red);
   const float s = scale_from_amax(amax, kE4m3Max);
+  const Divisor d = make_divisor(amax, s);
   if (threadIdx.x == 0) scales[nb * KB + kb] = s;
   uint2* dst = reinterpret_cast<uint2*>(q + row * K + col);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) dst[i] = encode8_e4m3(f[i], s);
+  for (int i = 0; i < 8; ++i) dst[i] = encode8_e4m3(f[i], d);
 }
 
 __global__ void fill_zero_bf16_kernel(__nv_bfloat16* __restrict__ C, int64_t count) {

@@ -5,7 +5,15 @@ cudaError_t launch_scaled_mm_block(const GemmLaunch& l, int swap_ab, int tile_n)
   return launch_format<kFmtBlock>(l, swap_ab, tile_n);
 }
 
-int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce) {
+int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce, bool fuse) {
+  if (fuse) {
+    switch (tile_n) {
+      case 16: return gemm_smem_bytes<16, true>(stages, cluster_reduce);
+      case 32: return gemm_smem_bytes<32, true>(stages, cluster_reduce);
+      case 64: return gemm_smem_bytes<64, true>(stages, cluster_reduce);
+      default: return -1;
+    }
+  }
   switch (tile_n) {
     case 16: return gemm_smem_bytes<16>(stages, cluster_reduce);
     case 32: return gemm_smem_bytes<32>(stages, cluster_reduce);

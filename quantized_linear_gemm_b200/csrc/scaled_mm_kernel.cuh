@@ -40,11 +40,14 @@ constexpr int kCtlBytes = 64 * 8 + 64;     // mbarriers, TMEM address, flags
 constexpr int kScaleBytes = 1024 * 4;      // staged scales: [0,256) per column, [256,384) per row,
                                            // [512,1024) two per-K-block buffers (Block_FP8)
 
-template <int TN>
+// One ring slot: the X tile, the Y tile and, for the fused quantization, the
+// bf16 activation tile (TN x 128, row-major, no swizzle) the codes come from.
+template <int TN, bool FUSE = false>
 struct TileShape {
-  static constexpr int kXBytes = kTileM * kTileK;   // 16 KB
-  static constexpr int kYBytes = TN * kTileK;       // multiple of 1 KB for TN % 8 == 0
-  static constexpr int kStageBytes = kXBytes + kYBytes;
+  static constexpr int kXBytes = kTileM * kTileK;                 // 16 KB
+  static constexpr int kYBytes = TN * kTileK;                     // multiple of 1 KB for TN % 8 == 0
+  static constexpr int kStagingBytes = FUSE ? TN * kTileK * 2 : 0;   // multiple of 1 KB as well
+  static constexpr int kStageBytes = kXBytes + kYBytes + kStagingBytes;
 };
 
 __host__ __device__ constexpr int tmem_cols_for(int cols) {
@@ -65,24 +68,27 @@ struct ClusterReduce {
 
 // Bytes of the ring region: `stages` slots, and for the pull reduction at
 // least the 128 x TN 32-bit partial tile it parks there.
-template <int TN>
+template <int TN, bool FUSE = false>
 __host__ __device__ constexpr int ring_bytes(int stages) {
-  return (ClusterReduce<TN>::kPush || stages * TileShape<TN>::kStageBytes > TN * kTileM * 4)
-             ? stages * TileShape<TN>::kStageBytes
+  return (ClusterReduce<TN>::kPush || stages * TileShape<TN, FUSE>::kStageBytes > TN * kTileM * 4)
+             ? stages * TileShape<TN, FUSE>::kStageBytes
              : TN * kTileM * 4;
 }
 
 // Shared-memory bytes of the kernel for `stages` ring slots; `cluster`: the
 // launch uses the cluster Split-K reduction (adds the push slots).
-template <int TN>
+template <int TN, bool FUSE = false>
 __host__ __device__ constexpr int gemm_smem_bytes(int stages, bool cluster) {
-  return 1024 /* alignment slack */ + ring_bytes<TN>(stages) +
+  return 1024 /* alignment slack */ + ring_bytes<TN, FUSE>(stages) +
          ((cluster && ClusterReduce<TN>::kPush) ? ClusterReduce<TN>::kSlotBytes : 0) + kCtlBytes + kScaleBytes;
 }
 
 struct SmemCtl {
   uint64_t* full;
   uint64_t* empty;
+  uint64_t* xfull;     // [stages] fused quantization: the bf16 activation tile has landed
+  uint64_t* wfull;     // [stages] fused quantization: the weight tile has landed
+                       // (full[] then counts the four A-producer warps only)
   uint64_t* tfull;     // [2]
   uint64_t* tempty;    // [2]
   uint64_t* mma_done;  // [1]
@@ -138,14 +144,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // The GEMM kernel
 // ---------------------------------------------------------------------------
 // FUSE (Swap-AB, FP8_Dynamic / W8A8_INT8 only): the activations arrive as
-// bf16; the epilogue warps, idle during the mainloop, quantize them per
-// token into the ring's activation slots (see the A-producer below).
+// bf16 (tmY maps them: [M, K] bf16, boxes of TN rows x 128); the TMA stages
+// each K tile of them beside the weights, and the epilogue warps, idle during
+// the mainloop, quantize it per token into the ring's activation slot (see
+// the A-producer below).
 template <int FMT, bool SWAP, int TN, bool FUSE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     scaled_mm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                         const GemmParams p) {
   static_assert(!FUSE || (SWAP && FMT != kFmtBlock && TN <= 64), "fused quantization: Swap-AB FP8/INT8 tiles");
-  using Shape = TileShape<TN>;
+  using Shape = TileShape<TN, FUSE>;
   // bytes the TMA delivers per stage (the fused path writes the activation slot itself)
   constexpr uint32_t kTmaStageBytes = FUSE ? Shape::kXBytes : Shape::kStageBytes;
   constexpr bool kInt8 = FMT == kFmtInt8;
@@ -160,13 +168,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ring = smem;
   const bool cluster_launch = p.S > 1 && p.reduce_mode == 2;
   const bool push_mode = ClusterReduce<TN>::kPush && cluster_launch;
-  uint32_t* slots = reinterpret_cast<uint32_t*>(ring + ring_bytes<TN>(stages));   // push slots [src][row][col]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + ring_bytes<TN>(stages) +
+  uint32_t* slots = reinterpret_cast<uint32_t*>(ring + ring_bytes<TN, FUSE>(stages));   // push slots [src][row][col]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + ring_bytes<TN, FUSE>(stages) +
                                                (push_mode ? ClusterReduce<TN>::kSlotBytes : 0));
   SmemCtl c;
   c.full = bars;
   c.empty = bars + stages;
-  c.tfull = bars + 2 * stages;
+  c.xfull = bars + 2 * stages;
+  c.wfull = bars + 3 * stages;
+  c.tfull = bars + 4 * stages;
   c.tempty = c.tfull + 2;
   c.mma_done = c.tempty + 2;
   c.red_bar = c.mma_done + 1;
@@ -189,8 +199,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) trace_stamp(p, 0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
-      mbar_init(&c.full[s], FUSE ? 1 + kEpiThreads / 32 : 1);   // TMA (+ the four A-producer warps)
+      mbar_init(&c.full[s], FUSE ? kEpiThreads / 32 : 1);   // the TMA, or the four A-producer warps
       mbar_init(&c.empty[s], 1);
+      mbar_init(&c.xfull[s], 1);
+      mbar_init(&c.wfull[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&c.tfull[b], 1);
@@ -237,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int a_row0 = SWAP ? y_row0 : x_row0;
       const int w_off = SWAP ? 0 : Shape::kXBytes;   // byte offset of the weight tile in a stage
       const int a_off = SWAP ? Shape::kXBytes : 0;
+      constexpr int kStagingOff = Shape::kXBytes + Shape::kYBytes;   // fused: the bf16 activation tile
       const int pre = nkb < stages ? nkb : stages;
       if (p.early_weights) {
         // The caller guarantees that the weights are not written by a kernel
@@ -245,8 +258,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < pre; ++i) {
           if (i == p.skip_stage) continue;
           uint8_t* st = ring + i * Shape::kStageBytes;
-          mbar_arrive_expect_tx(&c.full[i], kTmaStageBytes);
-          tma_load_2d(tmW, &c.full[i], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
+          uint64_t* wb = FUSE ? &c.wfull[i] : &c.full[i];
+          mbar_arrive_expect_tx(wb, kTmaStageBytes);
+          tma_load_2d(tmW, wb, st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
         }
         grid_dependency_wait();
       } else {
@@ -254,15 +268,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < pre; ++i) {
           if (i == p.skip_stage) continue;
           uint8_t* st = ring + i * Shape::kStageBytes;
-          mbar_arrive_expect_tx(&c.full[i], kTmaStageBytes);
-          tma_load_2d(tmW, &c.full[i], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
+          uint64_t* wb = FUSE ? &c.wfull[i] : &c.full[i];
+          mbar_arrive_expect_tx(wb, kTmaStageBytes);
+          tma_load_2d(tmW, wb, st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
         }
       }
       trace_stamp(p, 2);
       for (int i = 0; i < pre; ++i) {
-        if (FUSE || i == p.skip_stage) continue;
+        if (i == p.skip_stage) continue;
         uint8_t* st = ring + i * Shape::kStageBytes;
-        tma_load_2d(tmA, &c.full[i], st + a_off, (kb_lo + i) * kTileK, a_row0, pol_a);
+        if constexpr (FUSE) {
+          mbar_arrive_expect_tx(&c.xfull[i], Shape::kStagingBytes);
+          tma_load_2d(tmA, &c.xfull[i], st + kStagingOff, (kb_lo + i) * kTileK, a_row0, pol_a);
+        } else {
+          tma_load_2d(tmA, &c.full[i], st + a_off, (kb_lo + i) * kTileK, a_row0, pol_a);
+        }
       }
       int issued = pre;
       for (int i = pre; i < nkb; ++i) {
@@ -271,9 +291,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_bar(&c.empty[s], ph ^ 1u, p, c, 0)) break;
         if (i == p.skip_stage) continue;
         uint8_t* st = ring + s * Shape::kStageBytes;
-        mbar_arrive_expect_tx(&c.full[s], kTmaStageBytes);
-        tma_load_2d(tmW, &c.full[s], st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
-        if (!FUSE) tma_load_2d(tmA, &c.full[s], st + a_off, (kb_lo + i) * kTileK, a_row0, pol_a);
+        uint64_t* wb = FUSE ? &c.wfull[s] : &c.full[s];
+        mbar_arrive_expect_tx(wb, kTmaStageBytes);
+        tma_load_2d(tmW, wb, st + w_off, (kb_lo + i) * kTileK, w_row0, pol_w);
+        if constexpr (FUSE) {
+          mbar_arrive_expect_tx(&c.xfull[s], Shape::kStagingBytes);
+          tma_load_2d(tmA, &c.xfull[s], st + kStagingOff, (kb_lo + i) * kTileK, a_row0, pol_a);
+        } else {
+          tma_load_2d(tmA, &c.full[s], st + a_off, (kb_lo + i) * kTileK, a_row0, pol_a);
+        }
         issued = i + 1;
       }
       if (*c.abort_flag) {
@@ -281,9 +307,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int first = issued > stages ? issued - stages : 0;
         for (int j = first; j < issued; ++j) {
           if (j == p.skip_stage) continue;   // never armed
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(&c.full[j % stages], static_cast<uint32_t>(j / stages) & 1u) &&
-                 global_timer_ns() - t0 < p.wait_limit_ns) {
+          const uint32_t par = static_cast<uint32_t>(j / stages) & 1u;
+          uint64_t* bars_tx[2] = {FUSE ? &c.wfull[j % stages] : &c.full[j % stages], &c.xfull[j % stages]};
+          for (int b = 0; b < (FUSE ? 2 : 1); ++b) {
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bars_tx[b], par) && global_timer_ns() - t0 < p.wait_limit_ns) {
+            }
           }
         }
       }
@@ -304,6 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!wait_bar(&c.tempty[buf], (use & 1u) ^ 1u, p, c, 1)) break;
           d_tmem += static_cast<uint32_t>(buf * TN);
         }
+        if (FUSE && !wait_bar(&c.wfull[s], ph, p, c, 2)) break;
         if (!wait_bar(&c.full[s], ph, p, c, 2)) break;
         tc_fence_after_sync();
         if (i == 0) trace_stamp(p, 3);
@@ -363,38 +393,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool cluster_waited = false;
     if constexpr (FUSE) {
       // ------------------------------------------------ A-producer (fused)
-      // 1. partial amax of each token over this CTA's K range;
+      // 1. partial amax of each token over this CTA's K range (read straight
+      //    from global memory, eight 16-byte loads in flight per lane; when
+      //    the tile has fewer than four tokens, the warps split the range);
       // 2. Split-K cluster: every CTA sends its partials to every CTA
       //    (st.async, counted in bytes on amax_bar) and takes the max, so all
       //    CTAs of a tile derive the same per-token scale;
       // 3. s = max(fp32(amax / Q), 2^-126); q = enc(fp32(x / s)) for each K
-      //    tile, written in the 128-byte-swizzled K-major layout that the
-      //    tensor core reads, into the stage's activation slot; the four
-      //    warps' arrivals (with the weight TMA) complete the stage.
+      //    tile, read from the bf16 tile the TMA staged in the slot and
+      //    written in the 128-byte-swizzled K-major layout that the tensor
+      //    core reads, into the slot's activation tile; the four warps'
+      //    arrivals complete the stage.
       // Codes and scales equal those of lq_quant_per_token bit for bit.
       constexpr int kChunks = TN * 8 / kEpiThreads;   // 16-byte code chunks per thread per K tile (TN >= 16)
       const int e = warp - 2;                         // epilogue warp 0..3
       const int tid = e * 32 + lane;                  // epilogue thread 0..127
       float* pa = sc + 384;                           // [TN] this CTA's partial amax
       float* slots_amax = sc + 512;                   // [S][TN] partial amax of every split
+      float* rcp = sc + 128;                          // [TN] Divisor reciprocal of each token (colsc
+                                                      // holds only TN <= 64 entries here)
       const int64_t k_lo = static_cast<int64_t>(kb_lo) * kTileK;
       const int64_t k_hi = min(static_cast<int64_t>(kb_hi) * kTileK, p.K);
       const float qmax = kInt8 ? kInt8Max : kE4m3Max;
-      for (int j = e; j < TN; j += 4) {
-        const int64_t m = y_row0 + j;
-        float a = 0.f;
-        if (m < M) {
-          const uint4* xr = reinterpret_cast<const uint4*>(p.x + m * p.K);
-#pragma unroll 4
-          for (int64_t v = k_lo / 8 + lane; v < k_hi / 8; v += 32) {
-            float f[8];
-            bf16x8_to_f32(__ldg(xr + v), f);
-            a = fmaxf(a, amax8(f));
-          }
-        }
+      const int mv = (M - y_row0) < TN ? static_cast<int>(M - y_row0) : TN;   // tokens of this tile (>= 1)
+      for (int j = tid; j < TN; j += kEpiThreads) pa[j] = 0.f;
+      named_barrier_sync(2, kEpiThreads);
+      {
+        const int64_t nch = (k_hi - k_lo) / 8;   // 16-byte chunks of one token in the K range
+        const int parts = mv >= 4 ? 1 : 4 / mv;
+        for (int u = e; u < mv * parts; u += 4) {
+          const int j = u / parts, part = u - j * parts;
+          const int64_t c_lo = nch * part / parts, c_hi = nch * (part + 1) / parts;
+          const uint4* xr = reinterpret_cast<const uint4*>(p.x + (y_row0 + j) * p.K + k_lo);
+          float a = 0.f;
+          for (int64_t v = c_lo + lane; v < c_hi; v += 32 * 8) {
+            uint4 buf[8];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        if (lane == 0) pa[j] = a;
+            for (int w = 0; w < 8; ++w)
+              buf[w] = v + 32 * w < c_hi ? __ldg(xr + v + 32 * w) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+              float f[8];
+              bf16x8_to_f32(buf[w], f);
+              a = fmaxf(a, amax8(f));
+            }
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+          // a >= 0, so the order of the float bits is the order of the values
+          if (lane == 0) atomicMax(reinterpret_cast<int*>(pa) + j, __float_as_int(a));
+        }
       }
       named_barrier_sync(2, kEpiThreads);
       if (p.S > 1) {
@@ -421,61 +469,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t m = y_row0 + tid;
         const float sm = scale_from_amax(a, qmax);
         colsc[tid] = sm;
+        rcp[tid] = make_divisor(a, sm).y;
         if (p.a_scales_out && blockIdx.x == 0 && split == 0 && m < M) p.a_scales_out[m] = sm;
       }
       named_barrier_sync(2, kEpiThreads);
 
-      // 4. produce the activation tiles, loads of tile i+1 in flight while tile i is encoded
-      auto load_tile = [&](int i, uint4 (&buf)[2 * kChunks]) {
-#pragma unroll
-        for (int u = 0; u < kChunks; ++u) {
-          const int t = tid + u * kEpiThreads;
-          const int j = t >> 3, cc = t & 7;
-          const int64_t m = y_row0 + j;
-          const int64_t k0 = static_cast<int64_t>(kb_lo + i) * kTileK + cc * 16;
-          if (m < M && k0 < p.K) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.x + m * p.K + k0);
-            buf[2 * u] = __ldg(src);
-            buf[2 * u + 1] = __ldg(src + 1);
-          } else {
-            buf[2 * u] = make_uint4(0u, 0u, 0u, 0u);
-            buf[2 * u + 1] = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-      };
-      uint4 cur[2 * kChunks], nxt[2 * kChunks];
-      if (nkb > 0) load_tile(0, cur);
+      // 4. encode the staged tiles stage by stage.  The TMA refills a slot
+      //    only after the MMA has released it (empty), so xfull[s] landing
+      //    means the activation tile of slot s is free to overwrite as well.
       for (int i = 0; i < nkb; ++i) {
         const int s = i % stages;
-        if (i + 1 < nkb) load_tile(i + 1, nxt);
-        if (i >= stages) {
-          const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
-          if (!wait_bar(&c.empty[s], ph ^ 1u, p, c, 9)) break;   // the MMA has released this slot
-        }
+        const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
+        if (!wait_bar(&c.xfull[s], ph, p, c, 9)) break;
         uint8_t* slot = ring + s * Shape::kStageBytes + Shape::kXBytes;
+        const uint8_t* staged = slot + Shape::kYBytes;
 #pragma unroll
         for (int u = 0; u < kChunks; ++u) {
           const int t = tid + u * kEpiThreads;
           const int j = t >> 3, cc = t & 7;
-          const float sm = colsc[j];
-          float f0[8], f1[8];
-          bf16x8_to_f32(cur[2 * u], f0);
-          bf16x8_to_f32(cur[2 * u + 1], f1);
-          const uint2 q0 = kInt8 ? encode8_int8(f0, sm) : encode8_e4m3(f0, sm);
-          const uint2 q1 = kInt8 ? encode8_int8(f1, sm) : encode8_e4m3(f1, sm);
-          const uint4 qv = make_uint4(q0.x, q0.y, q1.x, q1.y);
+          uint4 qv = make_uint4(0u, 0u, 0u, 0u);   // rows past the last token: any code, their columns are dropped
+          if (j < mv) {
+            const Divisor d{colsc[j], rcp[j]};
+            const uint4* src = reinterpret_cast<const uint4*>(staged + j * (kTileK * 2) + cc * 32);
+            float f0[8], f1[8];
+            bf16x8_to_f32(src[0], f0);
+            bf16x8_to_f32(src[1], f1);
+            const uint2 q0 = kInt8 ? encode8_int8(f0, d) : encode8_e4m3(f0, d);
+            const uint2 q1 = kInt8 ? encode8_int8(f1, d) : encode8_e4m3(f1, d);
+            qv = make_uint4(q0.x, q0.y, q1.x, q1.y);
+            const int64_t k0 = static_cast<int64_t>(kb_lo + i) * kTileK + cc * 16;
+            if (p.a_codes_out && blockIdx.x == 0 && k0 < p.K)
+              *reinterpret_cast<uint4*>(p.a_codes_out + (y_row0 + j) * p.K + k0) = qv;
+          }
           // row j of the slot, 16-byte chunk cc placed at cc ^ (j % 8) (128-byte swizzle)
           *reinterpret_cast<uint4*>(slot + j * kTileK + ((cc ^ (j & 7)) << 4)) = qv;
-          const int64_t m = y_row0 + j;
-          const int64_t k0 = static_cast<int64_t>(kb_lo + i) * kTileK + cc * 16;
-          if (p.a_codes_out && blockIdx.x == 0 && m < M && k0 < p.K)
-            *reinterpret_cast<uint4*>(p.a_codes_out + m * p.K + k0) = qv;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // generic stores -> tensor core
         __syncwarp();
         if (lane == 0) mbar_arrive(&c.full[s]);
-#pragma unroll
-        for (int u = 0; u < 2 * kChunks; ++u) cur[u] = nxt[u];
       }
     }
 

@@ -34,7 +34,7 @@ EXPORTED = (
     "lq_quant_weight_block128", "lq_select_variant", "lq_load_dispatch_table", "lq_dispatch_table_size",
     "lq_init_device", "lq_reserve_workspace", "lq_workspace_bytes", "lq_device_status",
     "lq_status_string", "lq_version", "lq_set_trace", "lq_scaled_mm_noalloc", "lq_test_inject_stall",
-    "lq_quant_scaled_mm",
+    "lq_quant_scaled_mm", "lq_set_fuse_limit",
 )
 
 
@@ -102,6 +102,8 @@ def lib() -> ctypes.CDLL:
             L.lq_test_inject_stall.restype = _i32
             L.lq_set_trace.argtypes = [_vp]
             L.lq_set_trace.restype = _i32
+            L.lq_set_fuse_limit.argtypes = [ctypes.c_int64]
+            L.lq_set_fuse_limit.restype = ctypes.c_int64
             L.lq_version.argtypes = []
             L.lq_version.restype = ctypes.c_char_p
             for name in ("lq_scaled_mm", "lq_scaled_mm_i32acc", "lq_quant_per_token", "lq_quant_per_token_group128",
@@ -301,6 +303,12 @@ def set_trace(buf: torch.Tensor | None) -> None:
     """Record 12 globaltimer stamps per CTA of the following scaled_mm launches
     into ``buf`` (int64 CUDA tensor with 12 entries per CTA), or stop (None)."""
     lib().lq_set_trace(None if buf is None else buf.data_ptr())
+
+
+def set_fuse_limit(max_slice_bytes: int) -> int:
+    """Largest per-CTA activation slice (bytes) for which quant_scaled_mm
+    runs one kernel (0 = never, negative = default); returns the old limit."""
+    return int(lib().lq_set_fuse_limit(int(max_slice_bytes)))
 
 
 def test_inject_stall(k_tile: int, wait_limit_ns: int = 0) -> None:

@@ -84,3 +84,27 @@ def assert_close(C_gpu: torch.Tensor, C_ref: np.ndarray, what: str = "", rms_of=
         i = np.unravel_index(np.argmax(err), err.shape)
         raise AssertionError(f"{what}: outside tolerance, worst ratio {worst:.3g} at {i}: gpu {C[i]!r} ref {C_ref[i]!r}")
     return worst
+
+
+def wide_range_rows(K: int, seed: int) -> torch.Tensor:
+    """bf16 rows that exercise both ways the kernels divide by the scale: the
+    FMA-corrected reciprocal (amax >= 2^-80) and the plain division (smaller
+    amax), around the 2^-80 boundary, with elements down to bf16 subnormals
+    and up to 2^120, and rows whose every scale is extreme."""
+    g = np.random.default_rng(seed)
+    rows = []
+    def row(lo, hi, amax=None):
+        e = g.uniform(lo, hi, K)
+        v = np.where(g.random(K) < 0.5, -1.0, 1.0)
+        r = v * (1.0 + g.random(K)) * np.exp2(e)
+        if amax is not None:
+            r[g.integers(K)] = amax
+        return r
+    rows.append(row(-140, -81, amax=2.0 ** -80))                 # amax exactly 2^-80: fast path
+    rows.append(row(-140, -82, amax=-(2.0 ** -80) * (1 - 2 ** -8)))   # just below: division
+    rows.append(row(-133, -100))                                # all tiny, subnormals included
+    rows.append(row(-130, 100))                                 # 230 binades in one row
+    rows.append(row(60, 120, amax=3.0e38))                      # scale near the top of fp32
+    rows.append(row(-20, 5))
+    x = torch.from_numpy(np.stack(rows)).to(torch.bfloat16)
+    return x

@@ -66,7 +66,7 @@ def test_empty_problem_is_a_noop():
 
 @pytest.mark.parametrize("field,value", [
     ("split_k", 3), ("split_k", 512), ("split_k", 0), ("swap_ab", 2), ("tile_n", 48),
-    ("stages", 1), ("stages", 17), ("reduce", 3), ("pdl", 5),
+    ("stages", 1), ("stages", 15), ("reduce", 3), ("pdl", 5),
 ])
 def test_variant_checks(field, value):
     v = lq.make_variant(swap_ab=1, split_k=2, tile_n=32)
@@ -176,3 +176,13 @@ def test_token_buckets(tmp_path):
             assert lq.select_variant("fp8_dynamic", M, 4096, 4096).stages == 2 + buckets.index(mb), M
     finally:
         lq.load_dispatch_table(None)
+
+
+def test_fuse_limit_hook():
+    """lq_set_fuse_limit returns the limit in force and restores the default."""
+    default = lq.set_fuse_limit(-1)
+    assert default == 0 or os.environ.get("LQ_FUSE_MAX_SLICE_BYTES")
+    assert lq.set_fuse_limit(0) == default
+    assert lq.set_fuse_limit(4096) == 0
+    assert lq.set_fuse_limit(-1) == 4096
+    assert lq.set_fuse_limit(-1) == default

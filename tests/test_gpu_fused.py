@@ -24,9 +24,18 @@ def _vid(v):
     return f"tn{v['tile_n']}-s{v['split_k']}"
 
 
+@pytest.fixture
+def always_fuse():
+    """Every fusable variant takes the one-kernel path, whatever its slice."""
+    old = lq.set_fuse_limit(1 << 40)
+    yield
+    lq.set_fuse_limit(-1)
+    assert old == lq.set_fuse_limit(-1)
+
+
 @pytest.mark.parametrize("fmt", [lq.FP8_DYNAMIC, lq.W8A8_INT8], ids=["fp8", "int8"])
 @pytest.mark.parametrize("vd", VARIANTS, ids=_vid)
-def test_fused_matches_oracle_and_two_step(cuda_device, fmt, vd):
+def test_fused_matches_oracle_and_two_step(cuda_device, always_fuse, fmt, vd):
     name = FMT_NAME[fmt]
     for (M, N, K) in SHAPES:
         if vd["split_k"] * vd["tile_n"] > 512:
@@ -66,8 +75,18 @@ def test_fused_default_variant_and_fallback(cuda_device):
             assert torch.equal(q, q2) and torch.equal(s, s2) and torch.equal(C, C2)
 
 
-def test_fused_qwen_shapes_against_two_step(cuda_device):
-    """Full decode shapes with the table's variants."""
+@pytest.mark.parametrize("limit", [-1, 1 << 40], ids=["default-limit", "always-fuse"])
+def test_fused_qwen_shapes_against_two_step(cuda_device, limit):
+    """Full decode shapes with the table's variants, with the default fusion
+    limit and with every fusable variant fused."""
+    lq.set_fuse_limit(limit)
+    try:
+        _qwen_shapes()
+    finally:
+        lq.set_fuse_limit(-1)
+
+
+def _qwen_shapes():
     for (K, N) in inputs.QWEN3_8B.values():
         for M in (1, 16, 32):
             x = inputs.activations(M, K, seed=M + K).cuda()
@@ -79,3 +98,26 @@ def test_fused_qwen_shapes_against_two_step(cuda_device):
             torch.cuda.synchronize()
             assert torch.equal(q, q2) and torch.equal(s, s2)
             assert torch.equal(C, C2), (M, N, K)
+
+
+@pytest.mark.parametrize("fmt", ["fp8_dynamic", "w8a8_int8"])
+def test_fused_wide_range_rows(cuda_device, always_fuse, fmt):
+    """Tokens whose scales take both ways of dividing (around amax = 2^-80,
+    subnormal elements, scales near the top of fp32): the fused kernel's
+    codes and scales are still the oracle's, C the two-step path's."""
+    from _lqtest import wide_range_rows
+    K, N = 1024, 256
+    x = wide_range_rows(K, seed=11).cuda()
+    M = x.shape[0]
+    w = inputs.weights(N, K, seed=12).cuda()
+    qb, sb = lq.quant_per_token(fmt, w)
+    for vd in (dict(swap_ab=1, tile_n=16, split_k=1, stages=2), dict(swap_ab=1, tile_n=16, split_k=4, stages=2)):
+        v = lq.make_variant(reduce=2, **vd)
+        C, q, s = lq.quant_scaled_mm(fmt, x, qb, sb, variant=v)
+        torch.cuda.synchronize()
+        ra, rsa = O.quant_per_token(x.float().cpu().numpy(), fmt)
+        assert np.array_equal(s.cpu().numpy(), rsa)
+        assert np.array_equal(q.cpu().numpy(), ra)
+        C2 = lq.scaled_mm(fmt, q, s, qb, sb, variant=v)
+        torch.cuda.synchronize()
+        assert torch.equal(C, C2)

@@ -8,6 +8,8 @@ import torch
 from oracle import lq_oracle as O
 from quantized_linear_gemm_b200 import inputs, lq
 
+from _lqtest import wide_range_rows
+
 pytestmark = pytest.mark.gpu
 
 PER_TOKEN_SHAPES = [(1, 16), (3, 128), (16, 2048), (32, 4096), (7, 4112), (24, 12288), (64, 25600), (300, 1024), (2, 40960), (5, 2064)]
@@ -43,6 +45,25 @@ def test_quant_per_token_special_rows(cuda_device, fmt):
     xb = x.to(torch.bfloat16)
     q, s = lq.quant_per_token(fmt, xb.to(cuda_device))
     q_ref, s_ref = O.quant_per_token(xb.float().numpy(), fmt)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+@pytest.mark.parametrize("fmt", ["fp8_dynamic", "w8a8_int8"])
+@pytest.mark.parametrize("K", [256, 4096, 12288])
+def test_quant_per_token_wide_range_rows(cuda_device, fmt, K):
+    xb = wide_range_rows(K, seed=K)
+    q, s = lq.quant_per_token(fmt, xb.to(cuda_device))
+    q_ref, s_ref = O.quant_per_token(xb.float().numpy(), fmt)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def test_quant_group128_wide_range_rows(cuda_device):
+    xb = wide_range_rows(1024, seed=3)
+    # every 128-group of a row spans a different slice of the exponent range
+    q, s = lq.quant_per_token_group128(xb.to(cuda_device))
+    q_ref, s_ref = O.quant_per_token_group128(xb.float().numpy())
     assert np.array_equal(s.cpu().numpy(), s_ref)
     assert np.array_equal(q.cpu().numpy(), q_ref)
 
