@@ -25,6 +25,15 @@
 #include "quant_common.cuh"
 
 namespace lq {
+
+// Programmatic dependent launch: every kernel here lets the next kernel on the
+// stream launch before it waits for its own predecessor.
+// The next kernel (normally the GEMM that reads these codes) can then become
+// resident and start streaming its weights while this kernel's predecessor
+// finishes; its griddepcontrol.wait still waits for this whole grid, which
+// completes only after its own predecessor did.  A dependent grid launches
+// only once every CTA of this grid has triggered, so it never takes the
+// place of a CTA of this grid that has not started.
 namespace {
 
 template <int kThreadsPerRow>
@@ -49,8 +58,8 @@ __global__ void __launch_bounds__(256) quant_per_token_reg_kernel(const __nv_bfl
                                                                    uint8_t* __restrict__ q,
                                                                    float* __restrict__ scales, int64_t K) {
   __shared__ float red[32];
+  grid_launch_dependents();   // before the wait: see the note at the top of the namespace
   grid_dependency_wait();
-  grid_launch_dependents();
   const int64_t row = blockIdx.x;
   const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
   const int nvec = static_cast<int>(K / 8);
@@ -90,8 +99,8 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const __nv_bfloat1
                                                                uint8_t* __restrict__ q, float* __restrict__ scales,
                                                                int64_t K) {
   __shared__ float red[32];
+  grid_launch_dependents();   // before the wait: see the note at the top of the namespace
   grid_dependency_wait();
-  grid_launch_dependents();
   const int64_t row = blockIdx.x;
   const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
   const int64_t nvec = K / 8;
@@ -117,8 +126,8 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const __nv_bfloat1
 __global__ void __launch_bounds__(256) quant_group128_kernel(const __nv_bfloat16* __restrict__ x,
                                                               uint8_t* __restrict__ q, float* __restrict__ scales,
                                                               int64_t M, int64_t K) {
+  grid_launch_dependents();   // before the wait: see the note at the top of the namespace
   grid_dependency_wait();
-  grid_launch_dependents();
   const int64_t KB = K / 128;
   const int64_t g = blockIdx.x * 16ll + (threadIdx.x >> 4);
   const int sub = threadIdx.x & 15;
@@ -165,8 +174,8 @@ __global__ void __launch_bounds__(256) quant_weight_block128_kernel(const __nv_b
 }
 
 __global__ void fill_zero_bf16_kernel(__nv_bfloat16* __restrict__ C, int64_t count) {
+  grid_launch_dependents();   // before the wait: see the note at the top of the namespace
   grid_dependency_wait();
-  grid_launch_dependents();
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     C[i] = __float2bfloat16_rn(0.f);

@@ -971,8 +971,8 @@ template <int FMT>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmParams p) {
   constexpr bool kInt8 = FMT == kFmtInt8;
   constexpr bool kBlocked = FMT == kFmtBlock;
+  grid_launch_dependents();   // before the wait, as the quantization kernels do
   grid_dependency_wait();
-  grid_launch_dependents();
   const int64_t MN4 = p.M * p.N / 4;
   for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < MN4;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
