@@ -240,7 +240,7 @@ lq_status lq_scaled_mm_noalloc(lq_fmt fmt, const void *A, const float *a_scales,
  *   x      : [M, K] bf16, 16-byte aligned.
  *   q      : [M, K] codes out, 8-byte aligned.
  *   scales : [M] fp32 out.  s = max(fp32(amax_row / Q), 2^-126),
- *            q = encode(fp32(x / s)) with a correctly rounded division,
+ *            q = encode(fp32(x / s)) with x / s correctly rounded,
  *            e4m3 round-to-nearest-even with saturation to +-448, int8
  *            round-half-even clamped to +-127.
  *   K % 16 == 0.  M == 0 is a no-op.
@@ -257,6 +257,48 @@ lq_status lq_quant_per_token(lq_fmt fmt, const void *x, void *q, float *scales,
  */
 lq_status lq_quant_per_token_group128(const void *x, void *q, float *scales,
                                       int64_t M, int64_t K, lq_stream_t stream);
+
+/*
+ * Producer-side fused quantizers: the kernel that computes a GEMM's input
+ * activations quantizes them in the same pass (the blog's integrated kernels
+ * rms_norm_dynamic_per_token_quant, rms_norm_per_block_quant,
+ * silu_and_mul_dynamic_per_token_quant and silu_and_mul_per_block_quant:
+ * 24-ai.news report, section "kernels integrated into vLLM").  The pages name
+ * them only; the value quantized is the bf16 output of a Qwen3-style layer,
+ * with each rounding fixed so that codes and scales are reproducible bit for
+ * bit:
+ *
+ * RMSNorm, with an optional residual added first:
+ *   h = bf16(fp32(x + residual)), written back to residual (h = x if NULL);
+ *   v = sum_k h^2 / K + eps in fp64; r = fp32(1 / sqrt(v)) (fp64 sqrt and
+ *   divide); y = bf16(fp32(bf16(fp32(h * r)) * weight)).
+ * SiLU-and-multiply of gate_up = [g | u] ([M, 2I], the fused gate/up output):
+ *   y = bf16(fp32(bf16(silu(g)) * u)), silu(g) = g / (1 + exp(-g)) rounded
+ *   once from its exact value.
+ * Then y is quantized exactly as lq_quant_per_token (per row, FP8 or INT8)
+ * or lq_quant_per_token_group128 (per 1 x 128 group, FP8) would.
+ *
+ *   x, residual, weight, gate_up : bf16, 16-byte aligned; residual may be
+ *            NULL and is otherwise read and overwritten in place.
+ *   weight : [K] bf16 RMSNorm gain.  eps: finite, >= 0.
+ *   q      : [M, K] (or [M, I]) codes out, 8-byte aligned.
+ *   scales : [M] (per token) or [M, K/128] (per block) fp32 out.
+ *   K (or I): a multiple of 16 (per token) or 128 (per block), at most
+ *            32768, else LQ_ERR_UNSUPPORTED_SHAPE (also for K = 0).
+ *   M == 0 is a no-op.  One CTA per row; the row stays in registers.
+ */
+lq_status lq_rms_norm_dynamic_per_token_quant(lq_fmt fmt, const void *x, void *residual,
+                                              const void *weight, float eps, void *q,
+                                              float *scales, int64_t M, int64_t K,
+                                              lq_stream_t stream);
+lq_status lq_rms_norm_per_block_quant(const void *x, void *residual, const void *weight,
+                                      float eps, void *q, float *scales, int64_t M,
+                                      int64_t K, lq_stream_t stream);
+lq_status lq_silu_and_mul_dynamic_per_token_quant(lq_fmt fmt, const void *gate_up, void *q,
+                                                  float *scales, int64_t M, int64_t I,
+                                                  lq_stream_t stream);
+lq_status lq_silu_and_mul_per_block_quant(const void *gate_up, void *q, float *scales,
+                                          int64_t M, int64_t I, lq_stream_t stream);
 
 /*
  * 128x128 block quantization of a Block_FP8 weight stored [N, K]: one scale

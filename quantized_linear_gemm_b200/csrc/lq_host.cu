@@ -16,6 +16,7 @@
 
 #include <atomic>
 #include <cerrno>
+#include <cfloat>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -603,6 +604,70 @@ lq_status lq_quant_per_token_group128(const void* x, void* q, float* scales, int
   if (K % 128 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
   if ((M * (K / 128) + 15) / 16 > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
   return lq::launch_quant_group128(x, q, scales, M, K, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LQ_OK
+             : LQ_ERR_CUDA;
+}
+
+namespace {
+
+lq_status check_producer(int64_t M, int64_t K, int64_t multiple, const void* in, const void* residual,
+                         const void* weight, bool need_weight, float eps, const void* q, const float* scales) {
+  if (M < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (!in || !q || !scales || (need_weight && !weight)) return LQ_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || eps > FLT_MAX) return LQ_ERR_INVALID_ARG;
+  if (!aligned(in, 16) || (residual && !aligned(residual, 16)) || (weight && !aligned(weight, 16)) ||
+      !aligned(q, 8) || !aligned(scales, 4))
+    return LQ_ERR_ALIGNMENT;
+  if (K == 0 || K % multiple != 0 || K > lq::producer_max_row() || M > 0x7FFFFFFF)
+    return LQ_ERR_UNSUPPORTED_SHAPE;
+  return LQ_OK;
+}
+
+}  // namespace
+
+lq_status lq_rms_norm_dynamic_per_token_quant(lq_fmt fmt, const void* x, void* residual, const void* weight,
+                                              float eps, void* q, float* scales, int64_t M, int64_t K,
+                                              lq_stream_t stream) {
+  if (fmt != LQ_FP8_DYNAMIC && fmt != LQ_W8A8_INT8) return LQ_ERR_INVALID_ARG;
+  if (M == 0 && K >= 0) return LQ_OK;
+  const lq_status rc = check_producer(M, K, 16, x, residual, weight, true, eps, q, scales);
+  if (rc != LQ_OK) return rc;
+  return lq::launch_rms_norm_quant(static_cast<int>(fmt), false, x, residual, weight, eps, q, scales, M, K,
+                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LQ_OK
+             : LQ_ERR_CUDA;
+}
+
+lq_status lq_rms_norm_per_block_quant(const void* x, void* residual, const void* weight, float eps, void* q,
+                                      float* scales, int64_t M, int64_t K, lq_stream_t stream) {
+  if (M == 0 && K >= 0) return LQ_OK;
+  const lq_status rc = check_producer(M, K, 128, x, residual, weight, true, eps, q, scales);
+  if (rc != LQ_OK) return rc;
+  return lq::launch_rms_norm_quant(lq::kFmtFp8, true, x, residual, weight, eps, q, scales, M, K,
+                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LQ_OK
+             : LQ_ERR_CUDA;
+}
+
+lq_status lq_silu_and_mul_dynamic_per_token_quant(lq_fmt fmt, const void* gate_up, void* q, float* scales,
+                                                  int64_t M, int64_t I, lq_stream_t stream) {
+  if (fmt != LQ_FP8_DYNAMIC && fmt != LQ_W8A8_INT8) return LQ_ERR_INVALID_ARG;
+  if (M == 0 && I >= 0) return LQ_OK;
+  const lq_status rc = check_producer(M, I, 16, gate_up, nullptr, nullptr, false, 0.f, q, scales);
+  if (rc != LQ_OK) return rc;
+  return lq::launch_silu_mul_quant(static_cast<int>(fmt), false, gate_up, q, scales, M, I,
+                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LQ_OK
+             : LQ_ERR_CUDA;
+}
+
+lq_status lq_silu_and_mul_per_block_quant(const void* gate_up, void* q, float* scales, int64_t M, int64_t I,
+                                          lq_stream_t stream) {
+  if (M == 0 && I >= 0) return LQ_OK;
+  const lq_status rc = check_producer(M, I, 128, gate_up, nullptr, nullptr, false, 0.f, q, scales);
+  if (rc != LQ_OK) return rc;
+  return lq::launch_silu_mul_quant(lq::kFmtFp8, true, gate_up, q, scales, M, I,
+                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? LQ_OK
              : LQ_ERR_CUDA;
 }

@@ -8,9 +8,9 @@
 //   s = max(fp32(amax / Q), 2^-126),   q = encode(fp32(x / s))
 //
 // with Q = 448 (e4m3, round to nearest even, saturating) or 127 (int8,
-// round half to even, clamped to +-127).  The division is the correctly
-// rounded __fdiv_rn (not a reciprocal multiply), so codes and scales are
-// reproducible bit for bit.
+// round half to even, clamped to +-127).  x / s is the correctly rounded
+// quotient (quant_common.cuh: reciprocal plus one FMA correction, or a
+// division), so codes and scales are reproducible bit for bit.
 //
 // These kernels are bandwidth / launch bound: each reads bf16 once per pass
 // with 16-byte loads and writes 8-byte code chunks.

@@ -34,7 +34,8 @@ EXPORTED = (
     "lq_quant_weight_block128", "lq_select_variant", "lq_load_dispatch_table", "lq_dispatch_table_size",
     "lq_init_device", "lq_reserve_workspace", "lq_workspace_bytes", "lq_device_status",
     "lq_status_string", "lq_version", "lq_set_trace", "lq_scaled_mm_noalloc", "lq_test_inject_stall",
-    "lq_quant_scaled_mm", "lq_set_fuse_limit",
+    "lq_quant_scaled_mm", "lq_set_fuse_limit", "lq_rms_norm_dynamic_per_token_quant",
+    "lq_rms_norm_per_block_quant", "lq_silu_and_mul_dynamic_per_token_quant", "lq_silu_and_mul_per_block_quant",
 )
 
 
@@ -104,6 +105,14 @@ def lib() -> ctypes.CDLL:
             L.lq_set_trace.restype = _i32
             L.lq_set_fuse_limit.argtypes = [ctypes.c_int64]
             L.lq_set_fuse_limit.restype = ctypes.c_int64
+            L.lq_rms_norm_dynamic_per_token_quant.argtypes = [_i32, _vp, _vp, _vp, ctypes.c_float, _vp, _vp,
+                                                              _i64, _i64, _st]
+            L.lq_rms_norm_per_block_quant.argtypes = [_vp, _vp, _vp, ctypes.c_float, _vp, _vp, _i64, _i64, _st]
+            L.lq_silu_and_mul_dynamic_per_token_quant.argtypes = [_i32, _vp, _vp, _vp, _i64, _i64, _st]
+            L.lq_silu_and_mul_per_block_quant.argtypes = [_vp, _vp, _vp, _i64, _i64, _st]
+            for name in ("lq_rms_norm_dynamic_per_token_quant", "lq_rms_norm_per_block_quant",
+                         "lq_silu_and_mul_dynamic_per_token_quant", "lq_silu_and_mul_per_block_quant"):
+                getattr(L, name).restype = _i32
             L.lq_version.argtypes = []
             L.lq_version.restype = ctypes.c_char_p
             for name in ("lq_scaled_mm", "lq_scaled_mm_i32acc", "lq_quant_per_token", "lq_quant_per_token_group128",
@@ -252,6 +261,76 @@ def quant_per_token_group128(x: torch.Tensor, q=None, scales=None, stream=None):
         scales = torch.empty((M, max(K // 128, 0)), dtype=torch.float32, device=x.device)
     rc = lib().lq_quant_per_token_group128(_ptr(x), _ptr(q), _ptr(scales), M, K, _stream(stream))
     _check("lq_quant_per_token_group128", rc)
+    return q, scales
+
+
+def _producer_out(f: int, M: int, K: int, per_block: bool, device, q, scales):
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.int8 if f == W8A8_INT8 else torch.uint8, device=device)
+    if scales is None:
+        shape = (M, max(K // 128, 0)) if per_block else (M,)
+        scales = torch.empty(shape, dtype=torch.float32, device=device)
+    return q, scales
+
+
+def rms_norm_dynamic_per_token_quant(fmt, x: torch.Tensor, weight: torch.Tensor, eps: float, residual=None,
+                                     q=None, scales=None, stream=None):
+    """(codes [M, K], scales [M]) of RMSNorm(x [+ residual]) * weight; the
+    residual, when given, is overwritten with x + residual."""
+    f = _fmt(fmt)
+    _need(x, "x", (torch.bfloat16,), 2)
+    _need(weight, "weight", (torch.bfloat16,), 1)
+    if residual is not None:
+        _need(residual, "residual", (torch.bfloat16,), 2)
+    M, K = x.shape
+    q, scales = _producer_out(f, M, K, False, x.device, q, scales)
+    rc = lib().lq_rms_norm_dynamic_per_token_quant(f, _ptr(x), _ptr(residual) if residual is not None else None,
+                                                   _ptr(weight), float(eps), _ptr(q), _ptr(scales), M, K,
+                                                   _stream(stream))
+    _check("lq_rms_norm_dynamic_per_token_quant", rc)
+    return q, scales
+
+
+def rms_norm_per_block_quant(x: torch.Tensor, weight: torch.Tensor, eps: float, residual=None, q=None,
+                             scales=None, stream=None):
+    """(e4m3 codes [M, K], scales [M, K/128]) of RMSNorm(x [+ residual]) * weight."""
+    _need(x, "x", (torch.bfloat16,), 2)
+    _need(weight, "weight", (torch.bfloat16,), 1)
+    if residual is not None:
+        _need(residual, "residual", (torch.bfloat16,), 2)
+    M, K = x.shape
+    q, scales = _producer_out(FP8_DYNAMIC, M, K, True, x.device, q, scales)
+    rc = lib().lq_rms_norm_per_block_quant(_ptr(x), _ptr(residual) if residual is not None else None, _ptr(weight),
+                                           float(eps), _ptr(q), _ptr(scales), M, K, _stream(stream))
+    _check("lq_rms_norm_per_block_quant", rc)
+    return q, scales
+
+
+def silu_and_mul_dynamic_per_token_quant(fmt, gate_up: torch.Tensor, q=None, scales=None, stream=None):
+    """(codes [M, I], scales [M]) of silu(gate_up[:, :I]) * gate_up[:, I:]."""
+    f = _fmt(fmt)
+    _need(gate_up, "gate_up", (torch.bfloat16,), 2)
+    M, two_i = gate_up.shape
+    if two_i % 2:
+        raise ValueError("gate_up must have an even number of columns ([g | u])")
+    I = two_i // 2
+    q, scales = _producer_out(f, M, I, False, gate_up.device, q, scales)
+    rc = lib().lq_silu_and_mul_dynamic_per_token_quant(f, _ptr(gate_up), _ptr(q), _ptr(scales), M, I,
+                                                       _stream(stream))
+    _check("lq_silu_and_mul_dynamic_per_token_quant", rc)
+    return q, scales
+
+
+def silu_and_mul_per_block_quant(gate_up: torch.Tensor, q=None, scales=None, stream=None):
+    """(e4m3 codes [M, I], scales [M, I/128]) of silu(g) * u."""
+    _need(gate_up, "gate_up", (torch.bfloat16,), 2)
+    M, two_i = gate_up.shape
+    if two_i % 2:
+        raise ValueError("gate_up must have an even number of columns ([g | u])")
+    I = two_i // 2
+    q, scales = _producer_out(FP8_DYNAMIC, M, I, True, gate_up.device, q, scales)
+    rc = lib().lq_silu_and_mul_per_block_quant(_ptr(gate_up), _ptr(q), _ptr(scales), M, I, _stream(stream))
+    _check("lq_silu_and_mul_per_block_quant", rc)
     return q, scales
 
 

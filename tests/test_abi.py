@@ -104,6 +104,38 @@ def test_quant_scaled_mm_argument_checks():
     assert L.lq_quant_scaled_mm(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 128, 128, None, None) == OK
 
 
+def test_producer_quant_argument_checks():
+    L = lq.lib()
+    rms = L.lq_rms_norm_dynamic_per_token_quant
+    assert rms(2, FAKE, None, FAKE, 1e-6, FAKE, FAKE, 4, 128, None) == INVALID          # block fmt
+    assert rms(0, None, None, FAKE, 1e-6, FAKE, FAKE, 4, 128, None) == INVALID
+    assert rms(0, FAKE, None, None, 1e-6, FAKE, FAKE, 4, 128, None) == INVALID          # no weight
+    assert rms(0, FAKE, None, FAKE, -1.0, FAKE, FAKE, 4, 128, None) == INVALID          # eps < 0
+    assert rms(0, FAKE, None, FAKE, float("nan"), FAKE, FAKE, 4, 128, None) == INVALID
+    assert rms(0, FAKE, None, FAKE, float("inf"), FAKE, FAKE, 4, 128, None) == INVALID
+    assert rms(0, FAKE, MISALIGNED, FAKE, 1e-6, FAKE, FAKE, 4, 128, None) == ALIGN
+    assert rms(0, FAKE, None, MISALIGNED, 1e-6, FAKE, FAKE, 4, 128, None) == ALIGN
+    assert rms(0, FAKE, None, FAKE, 1e-6, FAKE, FAKE, 4, 120, None) == SHAPE
+    assert rms(0, FAKE, None, FAKE, 1e-6, FAKE, FAKE, 4, 0, None) == SHAPE
+    assert rms(0, FAKE, None, FAKE, 1e-6, FAKE, FAKE, 4, 32768 + 16, None) == SHAPE      # longest row: 32768
+    assert rms(0, FAKE, None, FAKE, 1e-6, FAKE, FAKE, -1, 128, None) == INVALID
+    assert rms(0, FAKE, None, FAKE, 1e-6, FAKE, FAKE, 0, 128, None) == OK
+    blk = L.lq_rms_norm_per_block_quant
+    assert blk(FAKE, None, FAKE, 1e-6, FAKE, FAKE, 4, 192, None) == SHAPE
+    assert blk(FAKE, None, FAKE, 1e-6, None, FAKE, 4, 256, None) == INVALID
+    assert blk(FAKE, None, FAKE, 1e-6, FAKE, FAKE, 0, 256, None) == OK
+    silu = L.lq_silu_and_mul_dynamic_per_token_quant
+    assert silu(2, FAKE, FAKE, FAKE, 4, 128, None) == INVALID
+    assert silu(1, MISALIGNED, FAKE, FAKE, 4, 128, None) == ALIGN
+    assert silu(1, FAKE, FAKE, FAKE, 4, 24, None) == SHAPE
+    assert silu(1, FAKE, FAKE, FAKE, 4, 65536, None) == SHAPE
+    assert silu(1, FAKE, FAKE, FAKE, 0, 128, None) == OK
+    sblk = L.lq_silu_and_mul_per_block_quant
+    assert sblk(FAKE, FAKE, FAKE, 4, 64, None) == SHAPE
+    assert sblk(FAKE, FAKE, None, 4, 128, None) == INVALID
+    assert sblk(FAKE, FAKE, FAKE, 0, 128, None) == OK
+
+
 def test_stall_hook_argument_check():
     assert lq.lib().lq_test_inject_stall(-2, 0) == INVALID
     assert lq.lib().lq_test_inject_stall(-1, 0) == OK
