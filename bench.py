@@ -290,6 +290,67 @@ class Workload:
                 self.gemm(c, stream)
 
 
+def producer_bytes(op: str, M: int, K: int, residual: bool) -> int:
+    """Algorithmic HBM bytes of one producer-side fused quantizer call: bf16
+    inputs read once, codes and fp32 scales written once (plus the residual
+    read and written back, and the RMSNorm gain)."""
+    per_block = op.endswith("per_block_quant")
+    scales = 4 * M * (K // 128) if per_block else 4 * M
+    if op.startswith("rms_norm"):
+        return 2 * M * K + (4 * M * K if residual else 0) + 2 * K + M * K + scales
+    return 4 * M * K + M * K + scales
+
+
+def producer_measurements(peaks, stream) -> list:
+    """Per-call time of the four producer-side fused quantizers at the
+    Qwen3-8B sizes (hidden 4096 for RMSNorm, intermediate 12288 for
+    SiLU-and-mul): decode rows (M = 8, 32) and a prefill batch (M = 4096),
+    graph-replayed, with enough input copies that more than 2 x L2 streams
+    between two reads of one copy."""
+    out = []
+    l2 = 126 * 2 ** 20
+    K, I = 4096, 12288
+    w = torch.ones(K, dtype=torch.bfloat16, device="cuda")
+    for M in (8, 32, 4096):
+        for op in ("rms_norm_dynamic_per_token_quant", "rms_norm_per_block_quant",
+                   "silu_and_mul_dynamic_per_token_quant", "silu_and_mul_per_block_quant"):
+            rms = op.startswith("rms_norm")
+            cols = K if rms else I
+            in_bytes = M * (K * 4 if rms else 2 * I * 2)
+            copies = max(2, 2 * l2 // in_bytes + 1) if M >= 1024 else 2
+            xs = [inputs.activations(M, 2 * cols if not rms else cols, seed=inputs.stable_seed(op, M, r)).cuda()
+                  for r in range(copies)]
+            rs = [inputs.activations(M, cols, seed=inputs.stable_seed(op, "res", M, r)).cuda()
+                  for r in range(copies)] if rms else None
+            q = torch.empty((M, cols), dtype=torch.uint8, device="cuda")
+            per_block = op.endswith("per_block_quant")
+            sc = torch.empty((M, cols // 128) if per_block else (M,), dtype=torch.float32, device="cuda")
+            reps = max(copies, 8)
+
+            def run(op=op, xs=xs, rs=rs, q=q, sc=sc, reps=reps, copies=copies):
+                for r in range(reps):
+                    x = xs[r % copies]
+                    if op == "rms_norm_dynamic_per_token_quant":
+                        lq.rms_norm_dynamic_per_token_quant("fp8_dynamic", x, w, 1e-6, residual=rs[r % copies],
+                                                            q=q, scales=sc, stream=stream)
+                    elif op == "rms_norm_per_block_quant":
+                        lq.rms_norm_per_block_quant(x, w, 1e-6, residual=rs[r % copies], q=q, scales=sc,
+                                                    stream=stream)
+                    elif op == "silu_and_mul_dynamic_per_token_quant":
+                        lq.silu_and_mul_dynamic_per_token_quant("fp8_dynamic", x, q=q, scales=sc, stream=stream)
+                    else:
+                        lq.silu_and_mul_per_block_quant(x, q=q, scales=sc, stream=stream)
+            g = capture(run, stream)
+            time_replays(g, 3, stream)
+            ms = time_replays(g, 10, stream) / (10 * reps)
+            b = producer_bytes(op, M, cols, residual=rms)
+            out.append({"op": op, "M": M, "K": cols, "residual": rms, "us": round(ms * 1e3, 3),
+                        "GB/s": round(b / (ms * 1e-3) / 1e9, 1),
+                        "frac_hbm": round(b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3), "bytes": b})
+            del g, xs, rs
+    return out
+
+
 def capture(fn, stream) -> torch.cuda.CUDAGraph:
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
@@ -439,6 +500,8 @@ def main() -> None:
     ap.add_argument("--copies", type=int, default=3, help="weight copies rotated to defeat L2 reuse")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--per-shape-reps", type=int, default=30)
+    ap.add_argument("--no-producers", action="store_true",
+                    help="skip the per-call timing of the producer-side fused quantizers")
     ap.add_argument("--path", default="separate", choices=["fused", "separate"],
                     help="fused: one lq_quant_scaled_mm per linear (quantization inside the GEMM kernel); "
                          "separate: lq_quant_per_token then lq_scaled_mm")
@@ -521,6 +584,8 @@ def main() -> None:
                           "frac_hbm": round(b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
                           "variant": c["variant"].as_dict()})
         del g
+
+    producers = producer_measurements(peaks, stream) if not args.no_producers else []
 
     # End to end through the public API: every step copies its activations
     # host->device from pinned memory, runs, and copies every output back.
@@ -636,6 +701,7 @@ def main() -> None:
                 "h2d_bytes_per_step": wl.x_all.numel() * 2, "d2h_bytes_per_step": wl.c_all.numel() * 2},
         "gpu_launches": wl.launches_per_step(fused=use_fused) * args.steps,
         "per_shape": per_shape,
+        "producers": producers,
     }
     if cpu is not None:
         out["cpu_baseline"] = cpu

@@ -632,8 +632,11 @@ lq_status lq_rms_norm_dynamic_per_token_quant(lq_fmt fmt, const void* x, void* r
   if (M == 0 && K >= 0) return LQ_OK;
   const lq_status rc = check_producer(M, K, 16, x, residual, weight, true, eps, q, scales);
   if (rc != LQ_OK) return rc;
+  DeviceState* d = nullptr;
+  const lq_status ds = device_state(reinterpret_cast<cudaStream_t>(stream), &d);
+  if (ds != LQ_OK) return ds;
   return lq::launch_rms_norm_quant(static_cast<int>(fmt), false, x, residual, weight, eps, q, scales, M, K,
-                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+                                   d->status, wait_limit_ns(), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? LQ_OK
              : LQ_ERR_CUDA;
 }
@@ -643,8 +646,11 @@ lq_status lq_rms_norm_per_block_quant(const void* x, void* residual, const void*
   if (M == 0 && K >= 0) return LQ_OK;
   const lq_status rc = check_producer(M, K, 128, x, residual, weight, true, eps, q, scales);
   if (rc != LQ_OK) return rc;
-  return lq::launch_rms_norm_quant(lq::kFmtFp8, true, x, residual, weight, eps, q, scales, M, K,
-                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+  DeviceState* d = nullptr;
+  const lq_status ds = device_state(reinterpret_cast<cudaStream_t>(stream), &d);
+  if (ds != LQ_OK) return ds;
+  return lq::launch_rms_norm_quant(lq::kFmtFp8, true, x, residual, weight, eps, q, scales, M, K, d->status,
+                                   wait_limit_ns(), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? LQ_OK
              : LQ_ERR_CUDA;
 }
@@ -655,8 +661,11 @@ lq_status lq_silu_and_mul_dynamic_per_token_quant(lq_fmt fmt, const void* gate_u
   if (M == 0 && I >= 0) return LQ_OK;
   const lq_status rc = check_producer(M, I, 16, gate_up, nullptr, nullptr, false, 0.f, q, scales);
   if (rc != LQ_OK) return rc;
-  return lq::launch_silu_mul_quant(static_cast<int>(fmt), false, gate_up, q, scales, M, I,
-                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+  DeviceState* d = nullptr;
+  const lq_status ds = device_state(reinterpret_cast<cudaStream_t>(stream), &d);
+  if (ds != LQ_OK) return ds;
+  return lq::launch_silu_mul_quant(static_cast<int>(fmt), false, gate_up, q, scales, M, I, d->status,
+                                   wait_limit_ns(), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? LQ_OK
              : LQ_ERR_CUDA;
 }
@@ -666,7 +675,10 @@ lq_status lq_silu_and_mul_per_block_quant(const void* gate_up, void* q, float* s
   if (M == 0 && I >= 0) return LQ_OK;
   const lq_status rc = check_producer(M, I, 128, gate_up, nullptr, nullptr, false, 0.f, q, scales);
   if (rc != LQ_OK) return rc;
-  return lq::launch_silu_mul_quant(lq::kFmtFp8, true, gate_up, q, scales, M, I,
+  DeviceState* d = nullptr;
+  const lq_status ds = device_state(reinterpret_cast<cudaStream_t>(stream), &d);
+  if (ds != LQ_OK) return ds;
+  return lq::launch_silu_mul_quant(lq::kFmtFp8, true, gate_up, q, scales, M, I, d->status, wait_limit_ns(),
                                    reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? LQ_OK
              : LQ_ERR_CUDA;

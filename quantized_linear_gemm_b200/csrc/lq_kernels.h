@@ -75,9 +75,10 @@ cudaError_t launch_quant_group128(const void* x, void* q, float* scales, int64_t
 // producer_max_row() outputs.
 int64_t producer_max_row();
 cudaError_t launch_rms_norm_quant(int fmt, bool per_block, const void* x, void* residual, const void* weight,
-                                  float eps, void* q, float* scales, int64_t M, int64_t K, cudaStream_t stream);
+                                  float eps, void* q, float* scales, int64_t M, int64_t K, int* status,
+                                  uint64_t wait_limit_ns, cudaStream_t stream);
 cudaError_t launch_silu_mul_quant(int fmt, bool per_block, const void* gate_up, void* q, float* scales, int64_t M,
-                                  int64_t I, cudaStream_t stream);
+                                  int64_t I, int* status, uint64_t wait_limit_ns, cudaStream_t stream);
 cudaError_t launch_quant_weight_block128(const void* w, void* q, float* scales, int64_t N, int64_t K,
                                          cudaStream_t stream);
 cudaError_t launch_fill_zero_bf16(__nv_bfloat16* C, int64_t count, cudaStream_t stream);

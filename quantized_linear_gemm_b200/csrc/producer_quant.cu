@@ -17,9 +17,11 @@
 // then s = max(fp32(amax / Q), 2^-126) and q = encode(fp32(y / s)) over the
 // row or the group, as in quant_common.cuh.
 //
-// One CTA of 256 threads per row; the row stays in registers (8 values per
-// 16-byte chunk, up to 16 chunks per thread: rows of up to 32768 outputs).
-// HBM / latency bound: the row is read once and the codes written once.
+// One CTA per row; the row stays in registers (8 values per 16-byte chunk,
+// at most 32768 outputs per row).  CTAs of 256 threads for short rows when
+// there are many; with few rows (decode) or long rows 1024 threads share a
+// row, more warps per SM to hide the latency of the arithmetic.  The row is
+// read once and the codes written once.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cfloat>
@@ -32,7 +34,8 @@
 namespace lq {
 namespace {
 
-constexpr int kRowThreads = 256;
+constexpr int kMaxRow = 32768;
+constexpr int kMaxStagedSmem = 200 * 1024;   // two row buffers at most
 
 __device__ __forceinline__ float bf(uint32_t w, int hi) {
   return __uint_as_float(hi ? (w & 0xFFFF0000u) : (w << 16));
@@ -42,21 +45,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 lo, __nv_bfloat16 
   return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
 }
 
-// silu(g) rounded once to bf16.  The fp32 evaluation g / (1 + expf(-g)) is
-// within 8 fp32 units in the last place of the exact value (expf: at most 2
-// ulp; the add and the divide: half an ulp each).  Unless the fp32 result is
-// that close to a midpoint between two bf16 values (its low 16 bits within 64
-// of 0x8000), rounding it gives the rounding of the exact value (Ziv's
-// rounding test).  Otherwise, and where expf could overflow or the result
-// leave the fp32 normal range (g <= -80), the value is recomputed in fp64.
-__device__ __forceinline__ __nv_bfloat16 silu_bf16(float g) {
-  if (g > -80.f) {
-    const float s = __fdiv_rn(g, __fadd_rn(1.f, expf(-g)));
-    const uint32_t low = __float_as_uint(s) & 0xFFFFu;
-    const uint32_t dist = low > 0x8000u ? low - 0x8000u : 0x8000u - low;
-    if (dist > 64u && fabsf(s) >= 0x1p-100f) return __float2bfloat16_rn(s);
-    if (s == 0.f) return __float2bfloat16_rn(s);   // g = +-0
-  }
+// silu(g) rounded once to bf16.  The fp32 estimate g / (1 + expf(-g)) has a
+// relative error of at most about 2.25 * 2^-22: expf is within 2 ulp (2^-22
+// relative), the add within half an ulp, and __fdividef within 2 ulp for a
+// divisor in [2^-126, 2^126] (here 1 + e^-g lies in [1, e^80]).  That is at
+// most 9 ulp of the estimate.  Unless the estimate is within 32 ulp of a
+// midpoint between two bf16 values (its low 16 bits within 32 of 0x8000),
+// rounding it gives the rounding of the exact value (Ziv's rounding test).
+// Otherwise, and where the result could leave the fp32 normal range
+// (g <= -80), *ok is cleared and the caller recomputes the value with
+// silu_bf16_f64, outside its hot loop.
+__device__ __forceinline__ __nv_bfloat16 silu_bf16_fast(float g, bool* ok) {
+  const float s = __fdividef(g, __fadd_rn(1.f, expf(-g)));
+  const uint32_t low = __float_as_uint(s) & 0xFFFFu;
+  const uint32_t dist = low > 0x8000u ? low - 0x8000u : 0x8000u - low;
+  *ok = g > -80.f && ((dist > 32u && fabsf(s) >= 0x1p-100f) || s == 0.f);   // s = 0 only for g = +-0
+  return __float2bfloat16_rn(s);
+}
+
+__device__ __forceinline__ __nv_bfloat16 silu_bf16_f64(float g) {
   const double gd = static_cast<double>(g);
   return __double2bfloat16(__ddiv_rn(gd, __dadd_rn(1.0, exp(-gd))));
 }
@@ -95,35 +102,35 @@ __device__ __forceinline__ float block_max_f32(float v, float* red) {
 
 enum : int { kOpRmsNorm = 0, kOpSiluMul = 1 };
 
+template <bool kGlobal>
+__device__ __forceinline__ uint4 ld16(const uint4* p) {
+  if constexpr (kGlobal) return __ldg(p);
+  return *p;   // shared memory (staged rows)
+}
+
+// One row: y (bf16, in registers), then its quantization.  Inputs come from
+// global memory (kGlobal) or from a row staged in shared memory; `res_in`
+// (may be null) is the residual row, `res_out` (global, may be null) where h
+// goes; `wv` the RMSNorm gain chunks of this thread.
 // GROUP = 0: one scale per row (FP8 or INT8); GROUP = 128: one FP8 scale per
 // 128 outputs (16 consecutive chunks, held by 16 consecutive threads).
-template <int OP, int GROUP, bool kInt8, int VPT>
-__global__ void __launch_bounds__(kRowThreads) producer_quant_kernel(const __nv_bfloat16* __restrict__ in,
-                                                                     __nv_bfloat16* __restrict__ residual,
-                                                                     const __nv_bfloat16* __restrict__ weight,
-                                                                     float eps, uint8_t* __restrict__ q,
-                                                                     float* __restrict__ scales, int64_t Kout) {
-  static_assert(GROUP == 0 || !kInt8, "1 x 128 groups are FP8");
-  __shared__ double red_d[kRowThreads / 32];
-  __shared__ float red_f[kRowThreads / 32];
-  grid_launch_dependents();   // as the other quantization kernels: before the wait
-  grid_dependency_wait();
-  const int64_t row = blockIdx.x;
+template <int OP, int GROUP, bool kInt8, int kRowThreads, int VPT, bool kGlobal>
+__device__ __forceinline__ void quantize_row(int64_t row, const uint4* in_row, const uint4* res_in, uint4* res_out,
+                                             const uint4 (&wv)[VPT], float eps, uint8_t* __restrict__ q,
+                                             float* __restrict__ scales, int64_t Kout, double* red_d, float* red_f) {
   const int nvec = static_cast<int>(Kout / 8);
   uint4 y[VPT];
 
   if constexpr (OP == kOpRmsNorm) {
-    const uint4* xr = reinterpret_cast<const uint4*>(in + row * Kout);
-    uint4* rr = residual ? reinterpret_cast<uint4*>(residual + row * Kout) : nullptr;
     double ss = 0.0;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int idx = threadIdx.x + i * kRowThreads;
       y[i] = make_uint4(0u, 0u, 0u, 0u);
       if (idx < nvec) {
-        uint4 h = __ldg(xr + idx);
-        if (rr) {
-          const uint4 rv = rr[idx];
+        uint4 h = ld16<kGlobal>(in_row + idx);
+        if (res_in) {
+          const uint4 rv = kGlobal ? res_in[idx] : ld16<false>(res_in + idx);   // not __ldg: written below
           const uint32_t xw[4] = {h.x, h.y, h.z, h.w}, rw[4] = {rv.x, rv.y, rv.z, rv.w};
           uint32_t hw[4];
 #pragma unroll
@@ -131,7 +138,7 @@ __global__ void __launch_bounds__(kRowThreads) producer_quant_kernel(const __nv_
             hw[j] = pack_bf16x2(__float2bfloat16_rn(__fadd_rn(bf(xw[j], 0), bf(rw[j], 0))),
                                 __float2bfloat16_rn(__fadd_rn(bf(xw[j], 1), bf(rw[j], 1))));
           h = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          rr[idx] = h;
+          res_out[idx] = h;
         }
         const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
 #pragma unroll
@@ -145,13 +152,11 @@ __global__ void __launch_bounds__(kRowThreads) producer_quant_kernel(const __nv_
     const double total = block_sum_f64<kRowThreads>(ss, red_d);
     const double v = __dadd_rn(__ddiv_rn(total, static_cast<double>(Kout)), static_cast<double>(eps));
     const float r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(v)));
-    const uint4* wr = reinterpret_cast<const uint4*>(weight);
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int idx = threadIdx.x + i * kRowThreads;
       if (idx < nvec) {
-        const uint4 wv = __ldg(wr + idx);
-        const uint32_t hw[4] = {y[i].x, y[i].y, y[i].z, y[i].w}, ww[4] = {wv.x, wv.y, wv.z, wv.w};
+        const uint32_t hw[4] = {y[i].x, y[i].y, y[i].z, y[i].w}, ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
         uint32_t out[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -167,14 +172,16 @@ __global__ void __launch_bounds__(kRowThreads) producer_quant_kernel(const __nv_
       }
     }
   } else {
-    const uint4* gr = reinterpret_cast<const uint4*>(in + row * 2 * Kout);
-    const uint4* ur = gr + nvec;
+    static_assert(OP != kOpSiluMul || VPT <= 4, "one bit per element of the thread's chunks");
+    const uint4* gr = in_row;
+    const uint4* ur = in_row + nvec;
+    uint32_t redo = 0;   // bit 8 i + e: element e of chunk i needs the fp64 silu
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int idx = threadIdx.x + i * kRowThreads;
       y[i] = make_uint4(0u, 0u, 0u, 0u);
       if (idx < nvec) {
-        const uint4 gv = __ldg(gr + idx), uv = __ldg(ur + idx);
+        const uint4 gv = ld16<kGlobal>(gr + idx), uv = ld16<kGlobal>(ur + idx);
         const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
         uint32_t out[4];
 #pragma unroll
@@ -182,12 +189,38 @@ __global__ void __launch_bounds__(kRowThreads) producer_quant_kernel(const __nv_
           __nv_bfloat16 o[2];
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
-            const __nv_bfloat16 a = silu_bf16(bf(gw[j], k));
+            bool ok;
+            const __nv_bfloat16 a = silu_bf16_fast(bf(gw[j], k), &ok);
+            if (!ok) redo |= 1u << (8 * i + 2 * j + k);
             o[k] = __float2bfloat16_rn(__fmul_rn(__bfloat162float(a), bf(uw[j], k)));   // exact product
           }
           out[j] = pack_bf16x2(o[0], o[1]);
         }
         y[i] = make_uint4(out[0], out[1], out[2], out[3]);
+      }
+    }
+    // Cold pass: the few elements whose fp32 estimate could round the wrong
+    // way are recomputed from their inputs in fp64.
+    if (redo) {
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        if ((redo >> (8 * i)) & 0xFFu) {
+          const int idx = threadIdx.x + i * kRowThreads;
+          const uint4 gv = ld16<kGlobal>(gr + idx), uv = ld16<kGlobal>(ur + idx);
+          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+          uint32_t yw[4] = {y[i].x, y[i].y, y[i].z, y[i].w};
+#pragma unroll 1
+          for (int e = 0; e < 8; ++e) {
+            if ((redo >> (8 * i + e)) & 1u) {
+              const int j = e >> 1, k = e & 1;
+              const __nv_bfloat16 a = silu_bf16_f64(bf(gw[j], k));
+              const uint32_t v =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__bfloat162float(a), bf(uw[j], k))));
+              yw[j] = k ? ((yw[j] & 0x0000FFFFu) | (v << 16)) : ((yw[j] & 0xFFFF0000u) | v);
+            }
+          }
+          y[i] = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+        }
       }
     }
   }
@@ -217,10 +250,11 @@ __global__ void __launch_bounds__(kRowThreads) producer_quant_kernel(const __nv_
       }
     }
   } else {
+    static_assert(GROUP == 0 || !kInt8, "1 x 128 groups are FP8");
     const int64_t groups = Kout / 128;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-      const int idx = threadIdx.x + i * kRowThreads;   // 16 threads share idx / 16 (256 % 16 == 0)
+      const int idx = threadIdx.x + i * kRowThreads;   // 16 threads share idx / 16 (kRowThreads % 16 == 0)
       float f[8];
       bf16x8_to_f32(y[i], f);
       float a = amax8(f);
@@ -235,10 +269,114 @@ __global__ void __launch_bounds__(kRowThreads) producer_quant_kernel(const __nv_
   }
 }
 
-cudaLaunchConfig_t row_config(int64_t M, cudaStream_t stream, cudaLaunchAttribute* attr) {
+template <int kRowThreads, int VPT>
+__device__ __forceinline__ void load_gain(const __nv_bfloat16* weight, int nvec, uint4 (&wv)[VPT]) {
+  const uint4* wr = reinterpret_cast<const uint4*>(weight);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * kRowThreads;
+    wv[i] = (weight && idx < nvec) ? __ldg(wr + idx) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// One row per CTA, read straight from global memory into registers (few
+// rows, or rows too long to double-buffer in shared memory).
+template <int OP, int GROUP, bool kInt8, int kRowThreads, int VPT>
+__global__ void __launch_bounds__(kRowThreads) producer_quant_kernel(const __nv_bfloat16* __restrict__ in,
+                                                                     __nv_bfloat16* __restrict__ residual,
+                                                                     const __nv_bfloat16* __restrict__ weight,
+                                                                     float eps, uint8_t* __restrict__ q,
+                                                                     float* __restrict__ scales, int64_t Kout) {
+  static_assert(kRowThreads * VPT * 8 <= kMaxRow || VPT == 1, "row longer than the ABI allows");
+  __shared__ double red_d[kRowThreads / 32];
+  __shared__ float red_f[kRowThreads / 32];
+  grid_launch_dependents();   // as the other quantization kernels: before the wait
+  grid_dependency_wait();
+  const int64_t row = blockIdx.x;
+  const int nvec = static_cast<int>(Kout / 8);
+  uint4 wv[VPT];   // the gain, loaded with the row rather than after the reduction
+  load_gain<kRowThreads, VPT>(OP == kOpRmsNorm ? weight : nullptr, nvec, wv);
+  const int64_t in_len = OP == kOpRmsNorm ? Kout : 2 * Kout;
+  uint4* rrow = residual ? reinterpret_cast<uint4*>(residual + row * Kout) : nullptr;
+  quantize_row<OP, GROUP, kInt8, kRowThreads, VPT, true>(row, reinterpret_cast<const uint4*>(in + row * in_len),
+                                                         rrow, rrow, wv, eps, q, scales, Kout, red_d, red_f);
+}
+
+// Many rows: a persistent CTA walks rows blockIdx.x, + gridDim.x, ...; one
+// thread copies each row (and its residual) into one of two shared-memory
+// buffers with the bulk-copy engine while the CTA works on the other, so
+// the next row's load overlaps this row's arithmetic and stores.  Every
+// wait is bounded; a timeout sets bit 12 of the status word and the CTA
+// stops after waiting (bounded) for its copies still in flight.
+template <int OP, int GROUP, bool kInt8, int kRowThreads, int VPT>
+__global__ void __launch_bounds__(kRowThreads) producer_quant_staged_kernel(
+    const __nv_bfloat16* __restrict__ in, __nv_bfloat16* __restrict__ residual,
+    const __nv_bfloat16* __restrict__ weight, float eps, uint8_t* __restrict__ q, float* __restrict__ scales,
+    int64_t M, int64_t Kout, int* status, uint64_t wait_limit_ns) {
+  extern __shared__ __align__(128) uint8_t rows[];   // two buffers of row_bytes
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ double red_d[kRowThreads / 32];
+  __shared__ float red_f[kRowThreads / 32];
+  const int nvec = static_cast<int>(Kout / 8);
+  const int64_t in_len = OP == kOpRmsNorm ? Kout : 2 * Kout;    // bf16 input values per row
+  const uint32_t in_bytes = static_cast<uint32_t>(in_len * 2);
+  const uint32_t row_bytes = in_bytes + (residual ? static_cast<uint32_t>(Kout * 2) : 0u);
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  grid_launch_dependents();
+  grid_dependency_wait();
+  uint4 wv[VPT];
+  load_gain<kRowThreads, VPT>(OP == kOpRmsNorm ? weight : nullptr, nvec, wv);
+
+  auto issue = [&](int64_t r, int b) {   // thread 0 only
+    uint8_t* dst = rows + static_cast<size_t>(b) * row_bytes;
+    mbar_arrive_expect_tx(&bar[b], row_bytes);
+    bulk_copy_g2s(dst, in + r * in_len, in_bytes, &bar[b]);
+    if (residual) bulk_copy_g2s(dst + in_bytes, residual + r * Kout, static_cast<uint32_t>(Kout * 2), &bar[b]);
+  };
+  if (threadIdx.x == 0 && blockIdx.x < M) issue(blockIdx.x, 0);
+  int it = 0;
+  bool failed = false;
+  for (int64_t row = blockIdx.x; row < M; row += gridDim.x, ++it) {
+    const int b = it & 1;
+    if (threadIdx.x == 0 && row + gridDim.x < M) {
+      // buffer b ^ 1 was last read in the previous iteration, which every
+      // thread has left (barrier at its end)
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(row + gridDim.x, b ^ 1);
+    }
+    const bool landed = mbar_wait(&bar[b], static_cast<uint32_t>(it >> 1) & 1u, wait_limit_ns);
+    if (!__syncthreads_and(landed)) {
+      failed = true;
+      break;
+    }
+    const uint8_t* buf = rows + static_cast<size_t>(b) * row_bytes;
+    uint4* rout = residual ? reinterpret_cast<uint4*>(residual + row * Kout) : nullptr;
+    quantize_row<OP, GROUP, kInt8, kRowThreads, VPT, false>(
+        row, reinterpret_cast<const uint4*>(buf),
+        residual ? reinterpret_cast<const uint4*>(buf + in_bytes) : nullptr, rout, wv, eps, q, scales, Kout, red_d,
+        red_f);
+    __syncthreads();   // buffer b is free for the copy issued next iteration
+  }
+  if (failed && threadIdx.x == 0) {
+    if (status) atomicOr(status, 1 << 12);
+    // wait (bounded) for the copies this CTA may still have in flight
+    for (int k = 0; k < 2; ++k) {
+      const int jt = it + k;
+      const int64_t r = blockIdx.x + static_cast<int64_t>(jt) * gridDim.x;
+      if (r < M) mbar_wait(&bar[jt & 1], static_cast<uint32_t>(jt >> 1) & 1u, wait_limit_ns);
+    }
+  }
+}
+
+cudaLaunchConfig_t row_config(int64_t M, int threads, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(M));
-  cfg.blockDim = dim3(kRowThreads);
+  cfg.blockDim = dim3(threads);
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -247,44 +385,115 @@ cudaLaunchConfig_t row_config(int64_t M, cudaStream_t stream, cudaLaunchAttribut
   return cfg;
 }
 
+template <int OP, int GROUP, bool kInt8, int T, int V>
+cudaError_t launch_staged(const __nv_bfloat16* ip, __nv_bfloat16* rp, const __nv_bfloat16* wp, float eps,
+                          uint8_t* qp, float* scales, int64_t M, int64_t Kout, int smem, int* status,
+                          uint64_t wait_limit_ns, cudaStream_t stream) {
+  auto kern = producer_quant_staged_kernel<OP, GROUP, kInt8, T, V>;
+  static int configured = 0;   // dynamic shared memory opted in once per instantiation and process
+  if (configured < smem) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxStagedSmem);
+    if (e != cudaSuccess) return e;
+    configured = kMaxStagedSmem;
+  }
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, T, smem);
+  if (e != cudaSuccess) return e;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t ctas = M < static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1) ? M
+                                                                                 : static_cast<int64_t>(sms) * per_sm;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = row_config(ctas, T, stream, attr);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  return cudaLaunchKernelEx(&cfg, kern, ip, rp, wp, eps, qp, scales, M, Kout, status, wait_limit_ns);
+}
+
 template <int OP, int GROUP, bool kInt8>
 cudaError_t launch_rows(const void* in, void* residual, const void* weight, float eps, void* q, float* scales,
-                        int64_t M, int64_t Kout, cudaStream_t stream) {
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = row_config(M, stream, attr);
+                        int64_t M, int64_t Kout, int* status, uint64_t wait_limit_ns, cudaStream_t stream) {
   const auto* ip = static_cast<const __nv_bfloat16*>(in);
   auto* rp = static_cast<__nv_bfloat16*>(residual);
   const auto* wp = static_cast<const __nv_bfloat16*>(weight);
   auto* qp = static_cast<uint8_t*>(q);
   const int64_t nvec = Kout / 8;
-#define LQ_PROW(V) \
-  if (nvec <= kRowThreads * (V)) \
-    return cudaLaunchKernelEx(&cfg, producer_quant_kernel<OP, GROUP, kInt8, V>, ip, rp, wp, eps, qp, scales, Kout);
-  LQ_PROW(1)
-  LQ_PROW(2)
-  LQ_PROW(4)
-  LQ_PROW(8)
-  LQ_PROW(16)
+  // Many rows of at least 16 KB whose two copies fit in shared memory:
+  // persistent CTAs that double-buffer rows (256 / 512 / 1024 threads as the
+  // row grows).  Shorter rows keep more one-shot CTAs per SM in flight.
+  const int64_t row_bytes = (OP == kOpRmsNorm ? 2 * Kout : 4 * Kout) + (residual ? 2 * Kout : 0);
+  const int64_t in_row_bytes = OP == kOpRmsNorm ? 2 * Kout : 4 * Kout;
+  if (M >= 2 * 148 && in_row_bytes >= 16 * 1024 && 2 * row_bytes <= kMaxStagedSmem) {
+    const int smem = static_cast<int>(2 * row_bytes);
+#define LQ_SROW(T, V)                                                                                         \
+  if (nvec <= (T) * (V))                                                                                      \
+    return launch_staged<OP, GROUP, kInt8, T, V>(ip, rp, wp, eps, qp, scales, M, Kout, smem, status,           \
+                                                 wait_limit_ns, stream);
+    if (nvec <= 512) {
+      LQ_SROW(256, 1)
+      LQ_SROW(256, 2)
+    }
+    if (nvec <= 2048) {
+      LQ_SROW(512, 1)
+      LQ_SROW(512, 2)
+      LQ_SROW(512, 4)
+    }
+    LQ_SROW(1024, 2)
+    LQ_SROW(1024, 4)
+#undef LQ_SROW
+    return cudaErrorInvalidValue;
+  }
+  cudaLaunchAttribute attr[1];
+  // Fewer rows than two per SM, or rows longer than 8192 outputs: a row per
+  // 1024-thread CTA (more warps per SM to hide the arithmetic's latency).
+  if ((M < 2 * 148 && nvec > 256) || nvec > 1024) {
+    cudaLaunchConfig_t cfg = row_config(M, 1024, stream, attr);
+#define LQ_PROW(T, V) \
+  if (nvec <= (T) * (V)) \
+    return cudaLaunchKernelEx(&cfg, producer_quant_kernel<OP, GROUP, kInt8, T, V>, ip, rp, wp, eps, qp, scales, Kout);
+    LQ_PROW(1024, 1)
+    LQ_PROW(1024, 2)
+    LQ_PROW(1024, 4)
+    return cudaErrorInvalidValue;
+  }
+  cudaLaunchConfig_t cfg = row_config(M, 256, stream, attr);
+  LQ_PROW(256, 1)
+  LQ_PROW(256, 2)
+  LQ_PROW(256, 4)
+  if constexpr (OP == kOpRmsNorm) {   // SiLU rows this long take the 1024-thread CTAs above
+    LQ_PROW(256, 8)
+    LQ_PROW(256, 16)
+  }
 #undef LQ_PROW
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-int64_t producer_max_row() { return static_cast<int64_t>(kRowThreads) * 16 * 8; }
+int64_t producer_max_row() { return kMaxRow; }
 
 cudaError_t launch_rms_norm_quant(int fmt, bool per_block, const void* x, void* residual, const void* weight,
-                                  float eps, void* q, float* scales, int64_t M, int64_t K, cudaStream_t stream) {
-  if (per_block) return launch_rows<kOpRmsNorm, 128, false>(x, residual, weight, eps, q, scales, M, K, stream);
-  if (fmt == kFmtInt8) return launch_rows<kOpRmsNorm, 0, true>(x, residual, weight, eps, q, scales, M, K, stream);
-  return launch_rows<kOpRmsNorm, 0, false>(x, residual, weight, eps, q, scales, M, K, stream);
+                                  float eps, void* q, float* scales, int64_t M, int64_t K, int* status,
+                                  uint64_t wait_limit_ns, cudaStream_t stream) {
+  if (per_block)
+    return launch_rows<kOpRmsNorm, 128, false>(x, residual, weight, eps, q, scales, M, K, status, wait_limit_ns,
+                                               stream);
+  if (fmt == kFmtInt8)
+    return launch_rows<kOpRmsNorm, 0, true>(x, residual, weight, eps, q, scales, M, K, status, wait_limit_ns,
+                                            stream);
+  return launch_rows<kOpRmsNorm, 0, false>(x, residual, weight, eps, q, scales, M, K, status, wait_limit_ns, stream);
 }
 
 cudaError_t launch_silu_mul_quant(int fmt, bool per_block, const void* gate_up, void* q, float* scales, int64_t M,
-                                  int64_t I, cudaStream_t stream) {
-  if (per_block) return launch_rows<kOpSiluMul, 128, false>(gate_up, nullptr, nullptr, 0.f, q, scales, M, I, stream);
-  if (fmt == kFmtInt8) return launch_rows<kOpSiluMul, 0, true>(gate_up, nullptr, nullptr, 0.f, q, scales, M, I, stream);
-  return launch_rows<kOpSiluMul, 0, false>(gate_up, nullptr, nullptr, 0.f, q, scales, M, I, stream);
+                                  int64_t I, int* status, uint64_t wait_limit_ns, cudaStream_t stream) {
+  if (per_block)
+    return launch_rows<kOpSiluMul, 128, false>(gate_up, nullptr, nullptr, 0.f, q, scales, M, I, status,
+                                               wait_limit_ns, stream);
+  if (fmt == kFmtInt8)
+    return launch_rows<kOpSiluMul, 0, true>(gate_up, nullptr, nullptr, 0.f, q, scales, M, I, status, wait_limit_ns,
+                                            stream);
+  return launch_rows<kOpSiluMul, 0, false>(gate_up, nullptr, nullptr, 0.f, q, scales, M, I, status, wait_limit_ns,
+                                           stream);
 }
 
 }  // namespace lq

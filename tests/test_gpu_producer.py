@@ -19,9 +19,11 @@ pytestmark = pytest.mark.gpu
 FMTS = ["fp8_dynamic", "w8a8_int8"]
 # (M, K): decode and prefill rows of Qwen3-8B / 32B hidden sizes, a ragged
 # count of rows, a short row, and the longest row a CTA holds.
-RMS_SHAPES = [(1, 4096), (5, 5120), (32, 4096), (300, 1024), (7, 144), (2, 32768), (3, 128)]
+RMS_SHAPES = [(1, 4096), (5, 5120), (32, 4096), (300, 1024), (7, 144), (2, 32768), (3, 128),
+              (400, 5120), (296, 32768)]   # >= 296 rows: persistent CTAs with rows staged in shared memory
 # (M, I): Qwen3-8B / 32B intermediate sizes, ragged, short, longest.
-SILU_SHAPES = [(1, 12288), (8, 25600), (33, 1024), (4, 144), (2, 32768), (64, 128)]
+SILU_SHAPES = [(1, 12288), (8, 25600), (33, 1024), (4, 144), (2, 32768), (64, 128),
+               (300, 1024), (333, 25600), (296, 12288), (301, 32768)]   # staged, at the size limit, too long
 
 
 def _np(t: torch.Tensor) -> np.ndarray:
@@ -51,7 +53,7 @@ def test_rms_norm_dynamic_per_token_quant(cuda_device, fmt, M, K, with_residual)
         assert np.array_equal(_np(res_d), h_ref)
 
 
-@pytest.mark.parametrize("M,K", [(1, 4096), (5, 5120), (32, 4096), (257, 1024), (2, 32768), (3, 128)])
+@pytest.mark.parametrize("M,K", [(1, 4096), (5, 5120), (32, 4096), (257, 1024), (2, 32768), (3, 128), (310, 4096)])
 @pytest.mark.parametrize("with_residual", [False, True], ids=["plain", "residual"])
 def test_rms_norm_per_block_quant(cuda_device, M, K, with_residual):
     x = inputs.activations(M, K, seed=inputs.stable_seed("rmsb-x", M, K))
@@ -84,7 +86,8 @@ def test_silu_and_mul_dynamic_per_token_quant(cuda_device, fmt, M, I):
     assert np.array_equal(q.cpu().numpy(), q_ref)
 
 
-@pytest.mark.parametrize("M,I", [(1, 12288), (8, 25600), (33, 1024), (2, 32768), (64, 128)])
+@pytest.mark.parametrize("M,I", [(1, 12288), (8, 25600), (33, 1024), (2, 32768), (64, 128), (300, 12288),
+                                 (297, 128)])
 def test_silu_and_mul_per_block_quant(cuda_device, M, I):
     gu = _gate_up(M, I, seed=inputs.stable_seed("silub", M, I))
     q, s = lq.silu_and_mul_per_block_quant(gu.cuda())
@@ -170,3 +173,16 @@ def test_producer_empty_is_noop(cuda_device):
     assert q.shape == (0, 128) and s.shape == (0,)
     q, s = lq.silu_and_mul_per_block_quant(torch.empty((0, 256), dtype=torch.bfloat16, device=cuda_device))
     assert q.shape == (0, 128) and s.shape == (0, 1)
+
+
+def test_staged_rows_leave_the_status_word_clear(cuda_device):
+    """The persistent kernels wait (bounded) for their row copies; a normal
+    run leaves no timeout bit set."""
+    assert lq.device_status(0) == 0
+    gu = _gate_up(600, 4096, seed=41).cuda()
+    lq.silu_and_mul_dynamic_per_token_quant("fp8_dynamic", gu)
+    x = inputs.activations(600, 4096, seed=42).cuda()
+    lq.rms_norm_per_block_quant(x, torch.ones(4096, dtype=torch.bfloat16, device="cuda"), 1e-6,
+                                residual=torch.zeros_like(x))
+    torch.cuda.synchronize()
+    assert lq.device_status(0) == 0
