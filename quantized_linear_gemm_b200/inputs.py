@@ -19,6 +19,8 @@ from __future__ import annotations
 
 import hashlib
 
+import numpy as np
+
 import torch
 
 # (K, N) of the four linears of a Qwen3 decoder layer
@@ -68,3 +70,21 @@ def uniform_codes(shape, seed: int, lo: int, hi: int) -> torch.Tensor:
     """Uniform random integers in [lo, hi) as int64 (raw operand bytes for edge tests)."""
     g = torch.Generator().manual_seed(int(seed))
     return torch.randint(lo, hi, tuple(shape), generator=g, dtype=torch.int64)
+
+
+# Mixture-of-experts decode (Qwen3-30B-A3B sizes: 128 experts, 8 chosen per
+# token, hidden 2048, expert intermediate 768): (K, N) of the two expert GEMMs.
+QWEN3_30B_A3B_EXPERTS = {"gate_up": (2048, 1536), "down": (768, 2048)}
+QWEN3_30B_A3B_NUM_EXPERTS = 128
+QWEN3_30B_A3B_TOP_K = 8
+
+
+def expert_counts(tokens: int, num_experts: int, top_k: int, seed: int) -> np.ndarray:
+    """Tokens routed to each expert when each of `tokens` tokens picks
+    `top_k` distinct experts uniformly at random (a seeded stand-in for a
+    router).  int64 [num_experts]."""
+    g = np.random.default_rng(seed)
+    counts = np.zeros(num_experts, dtype=np.int64)
+    for _ in range(tokens):
+        counts[g.choice(num_experts, size=top_k, replace=False)] += 1
+    return counts
