@@ -147,6 +147,39 @@ lq_status lq_scaled_mm(lq_fmt fmt, const void *A, const float *a_scales,
                        const lq_variant *variant, lq_stream_t stream);
 
 /*
+ * Grouped (mixture-of-experts) scaled_mm: one launch for all experts, each
+ * an ordinary FP8_Dynamic / W8A8_INT8 linear layer (the pages' next target:
+ * ai-radar.it, "Helion in vLLM: il tuning dei GEMM diventa ricerca, non
+ * artigianato GPU", section "Oltre Hopper: Blackwell, AMD, TPU e il
+ * perimetro del fork": many small experts, where Split-K and Swap-AB matter
+ * more).
+ *
+ *   A        : [T, K] token codes, sorted by expert: rows
+ *              expert_offsets[e] .. expert_offsets[e+1]-1 go to expert e.
+ *   a_scales : [T] per-token scales.
+ *   B        : [E, N, K] weight codes (experts stacked), b_scales [E, N].
+ *   C        : [T, N] bf16 out; row t = token t times its expert's weights.
+ *   expert_offsets : DEVICE int32 [E + 1], offsets[0] = 0, non-decreasing,
+ *              offsets[E] = T.  Read by the kernel (no host synchronisation,
+ *              so it may come from a router kernel on the same stream).  The
+ *              kernel clamps every offset to [0, T] and uses the running max,
+ *              so a malformed table gives wrong rows, never a store outside
+ *              C.
+ *   variant  : NULL = a heuristic from T / E; else Swap-AB only (swap_ab =
+ *              1, tile_n 16/32/64), split_k <= 16 with the cluster
+ *              reduction (reduce is forced to 2).
+ * The grid has ceil(T / tile_n) + E token tiles per weight tile; CTAs past
+ * the last tile of the last expert exit at once.  K % 16 == 0, N % 8 == 0,
+ * E * N < 2^31.  Errors as lq_scaled_mm; LQ_ERR_INVALID_ARG for Block_FP8,
+ * E = 0 with T > 0, or a Standard variant.
+ */
+lq_status lq_grouped_scaled_mm(lq_fmt fmt, const void *A, const float *a_scales,
+                               const void *B, const float *b_scales, void *C,
+                               const int32_t *expert_offsets, int64_t E, int64_t T,
+                               int64_t N, int64_t K, const lq_variant *variant,
+                               lq_stream_t stream);
+
+/*
  * Test hook for W8A8_INT8: as lq_scaled_mm(LQ_W8A8_INT8, ...) and also
  * writes the exact int32 accumulator sum_k A[m,k]*B[n,k] to acc_out [M, N]
  * (device, 16-byte aligned), so that it can be compared bit for bit with an

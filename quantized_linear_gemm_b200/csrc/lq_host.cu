@@ -530,6 +530,99 @@ lq_status lq_scaled_mm(lq_fmt fmt, const void* A, const float* a_scales, const v
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
+namespace {
+
+// Variant for a grouped launch when the caller gives none: Swap-AB with the
+// token tile that fits the mean tokens per expert, Split-K until the CTAs
+// cover the SMs twice (cluster reduction, at most 16).
+lq_variant heuristic_grouped(int64_t T, int64_t E, int64_t N, int64_t K) {
+  lq_variant v{};
+  v.swap_ab = 1;
+  const int64_t per_expert = E > 0 ? (T + E - 1) / E : T;
+  v.tile_n = per_expert <= 16 ? 16 : (per_expert <= 32 ? 32 : 64);
+  const int64_t tiles = ((N + 127) / 128) * (T < E ? T : E);
+  const int64_t kt = (K + 127) / 128;
+  int S = 1;
+  while (S < 16 && tiles * S * 2 <= 2 * kNumSms && kt / (S * 2) >= 2) S *= 2;
+  v.split_k = S;
+  v.reduce = 2;
+  v.pdl = 1;
+  v.stages = max_stages_fit(v.tile_n, 2, S > 1);
+  return v;
+}
+
+}  // namespace
+
+lq_status lq_grouped_scaled_mm(lq_fmt fmt_, const void* A, const float* a_scales, const void* B,
+                               const float* b_scales, void* C, const int32_t* expert_offsets, int64_t E, int64_t T,
+                               int64_t N, int64_t K, const lq_variant* variant, lq_stream_t stream_) {
+  const int fmt = static_cast<int>(fmt_);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (fmt != lq::kFmtFp8 && fmt != lq::kFmtInt8) return LQ_ERR_INVALID_ARG;
+  if (E < 0 || T < 0 || N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (T == 0 || N == 0) return LQ_OK;
+  if (E == 0 || !C) return LQ_ERR_INVALID_ARG;
+  if (!aligned(C, 16)) return LQ_ERR_ALIGNMENT;
+  if (K == 0)
+    return lq::launch_fill_zero_bf16(static_cast<__nv_bfloat16*>(C), T * N, stream) == cudaSuccess ? LQ_OK
+                                                                                                   : LQ_ERR_CUDA;
+  if (!A || !B || !a_scales || !b_scales || !expert_offsets) return LQ_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(a_scales, 4) || !aligned(b_scales, 4) ||
+      !aligned(expert_offsets, 4))
+    return LQ_ERR_ALIGNMENT;
+  if (K % 16 != 0 || N % 8 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (T > 0x7FFFFFFF || E > 0x7FFFFFFF || E * N > 0x7FFFFFFF || K > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+  lq_variant v = variant ? *variant : heuristic_grouped(T, E, N, K);
+  if (v.swap_ab != 1) return LQ_ERR_INVALID_ARG;   // tokens on the MMA N side
+  if (v.split_k > 16) return LQ_ERR_INVALID_ARG;
+  if (v.split_k > 1) v.reduce = 2;   // the Split-K CTAs of a tile reduce in their cluster
+  lq_status rc = check_variant(fmt, v);
+  if (rc != LQ_OK) return rc;
+  const bool cluster_reduce = v.split_k > 1;
+  if (v.stages == 0) v.stages = max_stages_fit(v.tile_n, 1, cluster_reduce);
+  const int64_t gx = (N + 127) / 128;
+  const int64_t gy = (T + v.tile_n - 1) / v.tile_n + E;   // at most one partial tile per expert
+  if (gy > 65535) return LQ_ERR_UNSUPPORTED_SHAPE;
+
+  DeviceState* d = nullptr;
+  rc = device_state(stream, &d);
+  if (rc != LQ_OK) return rc;
+  GemmLaunch l;
+  std::memset(&l, 0, sizeof(l));
+  GemmParams& p = l.p;
+  p.M = T;
+  p.N = N;
+  p.K = K;
+  p.T = static_cast<int>((K + 127) / 128);
+  p.KB = static_cast<int>(K / 128);
+  p.S = v.split_k;
+  p.stages = v.stages;
+  p.reduce_mode = 2;
+  p.early_weights = v.pdl == 2 ? 1 : 0;
+  p.a_s = a_scales;
+  p.b_s = b_scales;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.status = d->status;
+  p.wait_limit_ns = wait_limit_ns();
+  p.trace = g_trace.load();
+  p.skip_stage = g_skip_stage.load();
+  p.expert_offsets = expert_offsets;
+  p.num_experts = static_cast<int>(E);
+  if (!encode_operand(&l.tmX, B, E * N, K, 128) || !encode_operand(&l.tmY, A, T, K, v.tile_n)) return LQ_ERR_CUDA;
+  l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
+  l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce);
+  l.pdl = v.pdl != 0;
+  l.cluster_z = cluster_reduce ? v.split_k : 1;
+  l.stream = stream;
+  const cudaError_t e =
+      fmt == lq::kFmtFp8 ? lq::launch_scaled_mm_fp8(l, 1, v.tile_n) : lq::launch_scaled_mm_int8(l, 1, v.tile_n);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return LQ_ERR_CUDA;
+  }
+  return LQ_OK;
+}
+
 lq_status lq_scaled_mm_i32acc(const void* A, const float* a_scales, const void* B, const float* b_scales, void* C,
                               int32_t* acc_out, int64_t M, int64_t N, int64_t K, const lq_variant* variant,
                               lq_stream_t stream) {

@@ -35,6 +35,9 @@ struct GemmParams {
   const __nv_bfloat16* x;   // bf16 activations [M, K]
   uint8_t* a_codes_out;     // [M, K] codes written by the first n-tile's CTAs
   float* a_scales_out;      // [M] per-token scales
+  // grouped (mixture-of-experts) launch, Swap-AB: M = tokens T, N = rows per expert
+  const int* expert_offsets;   // device [num_experts + 1]; null = one GEMM
+  int num_experts;
 };
 
 constexpr int kTraceSlots = 12;

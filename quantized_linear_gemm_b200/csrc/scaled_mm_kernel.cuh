@@ -197,6 +197,75 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nkb = kb_hi - kb_lo;
 
   if (threadIdx.x == 0) trace_stamp(p, 0);
+
+  // Tile origin, and the bounds / output column offset of the tile's GEMM.
+  int64_t x_row0 = static_cast<int64_t>(blockIdx.x) * kTileM;
+  int64_t y_row0 = static_cast<int64_t>(blockIdx.y) * TN;
+  int64_t m_end = p.M, n_end = p.N, c_off = 0;
+  if (p.expert_offsets) {
+    // Grouped (mixture-of-experts) launch, Swap-AB: X = the weights of all
+    // experts stacked [E N, K], Y = the tokens sorted by expert [T, K].
+    // blockIdx.y enumerates the token tiles of expert 0, then expert 1, ...;
+    // warp 0 finds this CTA's expert with a prefix sum of per-expert tile
+    // counts.  Expert e's tokens are [H(e-1), H(e)) with H(e) the running
+    // max of offsets[1..e+1] clamped to [0, T] (H(-1) = 0): for a valid
+    // table (offsets[0] = 0, non-decreasing) that is [offsets[e],
+    // offsets[e+1]); for any other no store leaves C.  A CTA past the last
+    // tile leaves at once (all CTAs of its cluster share blockIdx.y).
+    volatile int* grp = c.last_flag + 1;   // expert (-1: none), tile, first token, end token
+    if (warp == 0) {
+      const int E = p.num_experts;
+      const int want = static_cast<int>(blockIdx.y);
+      const int T = static_cast<int>(p.M);
+      int carry = 0, prev_hi = 0, found = -1, f_tile = 0, f_lo = 0, f_hi = 0;
+      for (int base = 0; base < E && found < 0; base += 32) {
+        const int e = base + lane;
+        int hi = e < E ? min(max(p.expert_offsets[e + 1], 0), T) : 0;
+        hi = max(hi, prev_hi);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {   // inclusive running max
+          const int v = __shfl_up_sync(0xffffffffu, hi, o);
+          if (lane >= o) hi = max(hi, v);
+        }
+        int lo = __shfl_up_sync(0xffffffffu, hi, 1);
+        if (lane == 0) lo = prev_hi;
+        const int tiles = e < E ? (hi - lo + TN - 1) / TN : 0;
+        int incl = tiles;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const bool mine = e < E && want >= carry + incl - tiles && want < carry + incl;
+        const unsigned who = __ballot_sync(0xffffffffu, mine);
+        if (who) {
+          const int src = __ffs(who) - 1;
+          found = base + src;
+          f_tile = __shfl_sync(0xffffffffu, want - (carry + incl - tiles), src);
+          f_lo = __shfl_sync(0xffffffffu, lo, src);
+          f_hi = __shfl_sync(0xffffffffu, hi, src);
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+        prev_hi = __shfl_sync(0xffffffffu, hi, 31);
+      }
+      if (lane == 0) {
+        grp[0] = found;
+        grp[1] = f_tile;
+        grp[2] = f_lo;
+        grp[3] = f_hi;
+      }
+    }
+    __syncthreads();
+    const int e = grp[0];
+    if (e < 0 || x_row0 >= p.N) return;   // before any barrier, TMEM or cluster work
+    y_row0 = grp[2] + static_cast<int64_t>(grp[1]) * TN;
+    m_end = grp[3];
+    c_off = static_cast<int64_t>(e) * p.N;
+    x_row0 += c_off;
+    n_end = c_off + p.N;
+    __syncthreads();   // grp is read by every thread before the control block is initialised
+  }
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&c.full[s], FUSE ? kEpiThreads / 32 : 1);   // the TMA, or the four A-producer warps
@@ -235,8 +304,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Let the next kernel on the stream start its own prologue / weight stream.
   grid_launch_dependents();
 
-  const int x_row0 = blockIdx.x * kTileM;
-  const int y_row0 = blockIdx.y * TN;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -369,7 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     // (m, n) of accumulator element (r, j): Standard (x_row0 + r, y_row0 + j),
     // Swap-AB (y_row0 + j, x_row0 + r).
-    const int64_t M = p.M, N = p.N;
+    // bounds of the tile's GEMM: tokens [.., m_end), weight rows [.., n_end)
+    const int64_t M = m_end, N = n_end;
 
     float accr[kBlocked ? TN : 1];
 #pragma unroll
@@ -648,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < CH; ++j) {
               const int64_t m = y_row0 + c0 + j;
               if (m < M) {
-                const int64_t idx = m * N + n;
+                const int64_t idx = m * p.N + (n - c_off);   // c_off: the expert's first weight row (grouped)
                 if (split_mode) {
                   const int64_t widx = (static_cast<int64_t>(split) * M + m) * N + n;
                   if (kInt8) wsi[widx] = static_cast<int32_t>(v[j]);
@@ -793,7 +861,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int S = p.S;
         const int W = TN / S;
         const int j0 = split * W;
-        const int64_t M = p.M, N = p.N;
+        const int64_t M = m_end, N = n_end;
         // partial of split s for column j0 + jj of this thread's row
         auto slot = [&](int s, int jj) -> uint32_t { return slots[(s * kTileM + r) * W + jj]; };
         if (SWAP) {
@@ -814,8 +882,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               float val;
               if (kBlocked) val = sf;
               else val = (kInt8 ? static_cast<float>(si) : sf) * colsc[j0 + jj] * bsn;
-              p.C[m * N + n] = __float2bfloat16_rn(val);
-              if (kInt8 && p.acc_out) p.acc_out[m * N + n] = si;
+              p.C[m * p.N + (n - c_off)] = __float2bfloat16_rn(val);
+              if (kInt8 && p.acc_out) p.acc_out[m * p.N + (n - c_off)] = si;
             }
           }
         } else {

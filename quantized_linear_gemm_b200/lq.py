@@ -36,6 +36,7 @@ EXPORTED = (
     "lq_status_string", "lq_version", "lq_set_trace", "lq_scaled_mm_noalloc", "lq_test_inject_stall",
     "lq_quant_scaled_mm", "lq_set_fuse_limit", "lq_rms_norm_dynamic_per_token_quant",
     "lq_rms_norm_per_block_quant", "lq_silu_and_mul_dynamic_per_token_quant", "lq_silu_and_mul_per_block_quant",
+    "lq_grouped_scaled_mm",
 )
 
 
@@ -113,6 +114,9 @@ def lib() -> ctypes.CDLL:
             for name in ("lq_rms_norm_dynamic_per_token_quant", "lq_rms_norm_per_block_quant",
                          "lq_silu_and_mul_dynamic_per_token_quant", "lq_silu_and_mul_per_block_quant"):
                 getattr(L, name).restype = _i32
+            L.lq_grouped_scaled_mm.argtypes = [_i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                               ctypes.POINTER(Variant), _st]
+            L.lq_grouped_scaled_mm.restype = _i32
             L.lq_version.argtypes = []
             L.lq_version.restype = ctypes.c_char_p
             for name in ("lq_scaled_mm", "lq_scaled_mm_i32acc", "lq_quant_per_token", "lq_quant_per_token_group128",
@@ -199,6 +203,31 @@ def quant_scaled_mm(fmt, x: torch.Tensor, B: torch.Tensor, b_scales: torch.Tenso
                                   ctypes.byref(variant) if variant is not None else None, _stream(stream))
     _check("lq_quant_scaled_mm", rc)
     return C, q, s
+
+
+def grouped_scaled_mm(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor, b_scales: torch.Tensor,
+                      expert_offsets: torch.Tensor, C: torch.Tensor | None = None, variant: Variant | None = None,
+                      stream=None) -> torch.Tensor:
+    """``lq_grouped_scaled_mm``: A [T, K] tokens sorted by expert, B [E, N, K]
+    stacked expert weights, b_scales [E, N], expert_offsets int32 [E + 1] on
+    the device.  Returns C [T, N] bf16."""
+    f = _fmt(fmt)
+    _need(A, "A", _CODE_DTYPES, 2)
+    _need(B, "B", _CODE_DTYPES, 3)
+    _need(a_scales, "a_scales", (torch.float32,), 1)
+    _need(b_scales, "b_scales", (torch.float32,), 2)
+    _need(expert_offsets, "expert_offsets", (torch.int32,), 1)
+    T, K = A.shape
+    E, N, _ = B.shape
+    if expert_offsets.numel() != E + 1:
+        raise ValueError("expert_offsets must hold E + 1 entries")
+    if C is None:
+        C = torch.empty((T, N), dtype=torch.bfloat16, device=A.device)
+    rc = lib().lq_grouped_scaled_mm(f, _ptr(A), _ptr(a_scales), _ptr(B), _ptr(b_scales), _ptr(C),
+                                    _ptr(expert_offsets), E, T, N, K,
+                                    ctypes.byref(variant) if variant is not None else None, _stream(stream))
+    _check("lq_grouped_scaled_mm", rc)
+    return C
 
 
 def scaled_mm_noalloc(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor, b_scales: torch.Tensor,

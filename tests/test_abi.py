@@ -136,6 +136,23 @@ def test_producer_quant_argument_checks():
     assert sblk(FAKE, FAKE, FAKE, 0, 128, None) == OK
 
 
+def test_grouped_argument_checks():
+    L = lq.lib()
+    g = L.lq_grouped_scaled_mm
+    v_std = lq.make_variant(swap_ab=0, tile_n=128)
+    assert g(2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 256, 128, None, None) == INVALID      # Block_FP8
+    assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 256, 128, None, None) == INVALID      # tokens, no expert
+    assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, None, 4, 64, 256, 128, None, None) == INVALID      # no offsets
+    assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 256, 128, ctypes.byref(v_std), None) == INVALID
+    assert g(0, FAKE, FAKE, FAKE, FAKE, MISALIGNED, FAKE, 4, 64, 256, 128, None, None) == ALIGN
+    assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, 4, 64, 256, 128, None, None) == ALIGN
+    assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 256, 120, None, None) == SHAPE        # K % 16
+    assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 252, 128, None, None) == SHAPE        # N % 8
+    assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 70000, 64, 256, 128, None, None) == SHAPE    # grid y
+    assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0, 256, 128, None, None) == OK
+    assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, 64, 256, 128, None, None) == INVALID
+
+
 def test_stall_hook_argument_check():
     assert lq.lib().lq_test_inject_stall(-2, 0) == INVALID
     assert lq.lib().lq_test_inject_stall(-1, 0) == OK
