@@ -40,6 +40,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from quantized_linear_gemm_b200 import inputs, lq  # noqa: E402
@@ -351,6 +352,62 @@ def producer_measurements(peaks, stream) -> list:
     return out
 
 
+def moe_measurements(peaks, stream) -> list:
+    """Per-call time of lq_grouped_scaled_mm on the Qwen3-30B-A3B expert
+    GEMMs (128 experts, 8 per token) at decode batch sizes, graph-replayed
+    over several seeded routings so that more than 2 x L2 of expert weights
+    streams between two reads of one expert; beside it, the same work as one
+    lq_scaled_mm per active expert."""
+    out = []
+    l2 = 126 * 2 ** 20
+    E, top_k = inputs.QWEN3_30B_A3B_NUM_EXPERTS, inputs.QWEN3_30B_A3B_TOP_K
+    g = torch.Generator().manual_seed(11)
+    for layer, (K, N) in inputs.QWEN3_30B_A3B_EXPERTS.items():
+        B = (torch.randint(0, 256, (E, N, K), generator=g, dtype=torch.uint8) & 0x77).cuda()   # finite e4m3 codes
+        sb = (torch.rand((E, N), generator=g) * 1e-3).cuda()
+        for tokens in (1, 8, 32, 64):
+            T = tokens * top_k
+            routes, nbytes = [], []
+            while sum(nbytes) < 2 * l2 or len(routes) < 4:
+                c = inputs.expert_counts(tokens, E, top_k, seed=inputs.stable_seed("moe-bench", layer, tokens, len(routes)))
+                off = torch.tensor(np.concatenate([[0], np.cumsum(c)]), dtype=torch.int32).cuda()
+                act = int((c > 0).sum())
+                routes.append((off, act, c))
+                nbytes.append(act * N * K + T * K + 4 * T + 4 * act * N + 2 * T * N)
+            A = (torch.randint(0, 256, (T, K), generator=g, dtype=torch.uint8) & 0x77).cuda()
+            sa = (torch.rand(T, generator=g) * 1e-2).cuda()
+            C = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+
+            def grouped(routes=routes, A=A, sa=sa, B=B, sb=sb, C=C):
+                for off, _, _ in routes:
+                    lq.grouped_scaled_mm("fp8_dynamic", A, sa, B, sb, off, C=C, stream=stream)
+
+            def per_expert(routes=routes, A=A, sa=sa, B=B, sb=sb, C=C):
+                for _, _, c in routes:
+                    lo = 0
+                    for e in range(E):
+                        n = int(c[e])
+                        if n:
+                            lq.scaled_mm("fp8_dynamic", A[lo:lo + n], sa[lo:lo + n], B[e], sb[e], C[lo:lo + n],
+                                         stream=stream)
+                        lo += n
+
+            row = {"layer": layer, "K": K, "N": N, "tokens": tokens, "T": T,
+                   "active_experts": round(sum(a for _, a, _ in routes) / len(routes), 1)}
+            for name, fn in (("grouped", grouped), ("per_expert_calls", per_expert)):
+                gr = capture(fn, stream)
+                time_replays(gr, 2, stream)
+                ms = time_replays(gr, 5, stream) / (5 * len(routes))
+                row[name + "_us"] = round(ms * 1e3, 2)
+                del gr
+            b = sum(nbytes) / len(nbytes)
+            row["GB/s"] = round(b / (row["grouped_us"] * 1e-6) / 1e9, 1)
+            row["frac_hbm"] = round(row["GB/s"] / peaks["hbm_gbs"], 3)
+            out.append(row)
+        del B
+    return out
+
+
 def capture(fn, stream) -> torch.cuda.CUDAGraph:
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
@@ -502,6 +559,7 @@ def main() -> None:
     ap.add_argument("--per-shape-reps", type=int, default=30)
     ap.add_argument("--no-producers", action="store_true",
                     help="skip the per-call timing of the producer-side fused quantizers")
+    ap.add_argument("--no-moe", action="store_true", help="skip the grouped (MoE) GEMM timing")
     ap.add_argument("--path", default="separate", choices=["fused", "separate"],
                     help="fused: one lq_quant_scaled_mm per linear (quantization inside the GEMM kernel); "
                          "separate: lq_quant_per_token then lq_scaled_mm")
@@ -586,6 +644,7 @@ def main() -> None:
         del g
 
     producers = producer_measurements(peaks, stream) if not args.no_producers else []
+    moe = moe_measurements(peaks, stream) if not args.no_moe else []
 
     # End to end through the public API: every step copies its activations
     # host->device from pinned memory, runs, and copies every output back.
@@ -702,6 +761,7 @@ def main() -> None:
         "gpu_launches": wl.launches_per_step(fused=use_fused) * args.steps,
         "per_shape": per_shape,
         "producers": producers,
+        "moe": moe,
     }
     if cpu is not None:
         out["cpu_baseline"] = cpu

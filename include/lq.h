@@ -165,11 +165,14 @@ lq_status lq_scaled_mm(lq_fmt fmt, const void *A, const float *a_scales,
  *              kernel clamps every offset to [0, T] and uses the running max,
  *              so a malformed table gives wrong rows, never a store outside
  *              C.
- *   variant  : NULL = a heuristic from T / E; else Swap-AB only (swap_ab =
- *              1, tile_n 16/32/64), split_k <= 16 with the cluster
- *              reduction (reduce is forced to 2).
- * The grid has ceil(T / tile_n) + E token tiles per weight tile; CTAs past
- * the last tile of the last expert exit at once.  K % 16 == 0, N % 8 == 0,
+ *   variant  : NULL = a rule from T, E and N (tuned on the Qwen3-30B-A3B
+ *              expert GEMMs: one split, tile_n 16, 2-4 stages); else
+ *              Swap-AB only (swap_ab = 1, tile_n 16/32/64), split_k <= 16
+ *              with the cluster reduction (reduce is forced to 2).
+ * The grid has ceil(T / tile_n) + min(E, T) token tiles per weight tile
+ * (a bound on the sum over experts of ceil(count / tile_n)); CTAs past the
+ * last tile of the last expert exit at once.  The kernel reads the table
+ * after waiting for the previous kernel on the stream.  K % 16 == 0, N % 8 == 0,
  * E * N < 2^31.  Errors as lq_scaled_mm; LQ_ERR_INVALID_ARG for Block_FP8,
  * E = 0 with T > 0, or a Standard variant.
  */

@@ -35,6 +35,7 @@ constexpr int kTileM = 128;      // MMA M (rows of X)
 constexpr int kTileK = 128;      // K elements (bytes) per pipeline stage
 constexpr int kMmaK = 32;        // K per tcgen05.mma for 8-bit operands
 constexpr int kThreads = 192;
+constexpr int kScanChunks = 8;   // grouped launch: expert offsets loaded 256 at a time
 constexpr int kEpiThreads = 128;
 constexpr int kCtlBytes = 64 * 8 + 64;     // mbarriers, TMEM address, flags
 constexpr int kScaleBytes = 1024 * 4;      // staged scales: [0,256) per column, [256,384) per row,
@@ -214,39 +215,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tile leaves at once (all CTAs of its cluster share blockIdx.y).
     volatile int* grp = c.last_flag + 1;   // expert (-1: none), tile, first token, end token
     if (warp == 0) {
+      // the table may come from the previous kernel on the stream (a router)
+      grid_dependency_wait();
       const int E = p.num_experts;
       const int want = static_cast<int>(blockIdx.y);
       const int T = static_cast<int>(p.M);
       int carry = 0, prev_hi = 0, found = -1, f_tile = 0, f_lo = 0, f_hi = 0;
-      for (int base = 0; base < E && found < 0; base += 32) {
-        const int e = base + lane;
-        int hi = e < E ? min(max(p.expert_offsets[e + 1], 0), T) : 0;
-        hi = max(hi, prev_hi);
+      for (int base0 = 0; base0 < E && found < 0; base0 += 32 * kScanChunks) {
+        int his[kScanChunks];   // all loads of this batch in flight at once
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {   // inclusive running max
-          const int v = __shfl_up_sync(0xffffffffu, hi, o);
-          if (lane >= o) hi = max(hi, v);
+        for (int k = 0; k < kScanChunks; ++k) {
+          const int e = base0 + 32 * k + lane;
+          his[k] = e < E ? p.expert_offsets[e + 1] : 0;
         }
-        int lo = __shfl_up_sync(0xffffffffu, hi, 1);
-        if (lane == 0) lo = prev_hi;
-        const int tiles = e < E ? (hi - lo + TN - 1) / TN : 0;
-        int incl = tiles;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
+        for (int k = 0; k < kScanChunks; ++k) {
+          const int base = base0 + 32 * k;
+          if (base >= E || found >= 0) break;
+          const int e = base + lane;
+          int hi = e < E ? min(max(his[k], 0), T) : 0;
+          hi = max(hi, prev_hi);
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {   // inclusive running max
+            const int v = __shfl_up_sync(0xffffffffu, hi, o);
+            if (lane >= o) hi = max(hi, v);
+          }
+          int lo = __shfl_up_sync(0xffffffffu, hi, 1);
+          if (lane == 0) lo = prev_hi;
+          const int tiles = e < E ? (hi - lo + TN - 1) / TN : 0;
+          int incl = tiles;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+          }
+          const bool mine = e < E && want >= carry + incl - tiles && want < carry + incl;
+          const unsigned who = __ballot_sync(0xffffffffu, mine);
+          if (who) {
+            const int src = __ffs(who) - 1;
+            found = base + src;
+            f_tile = __shfl_sync(0xffffffffu, want - (carry + incl - tiles), src);
+            f_lo = __shfl_sync(0xffffffffu, lo, src);
+            f_hi = __shfl_sync(0xffffffffu, hi, src);
+          }
+          carry += __shfl_sync(0xffffffffu, incl, 31);
+          prev_hi = __shfl_sync(0xffffffffu, hi, 31);
         }
-        const bool mine = e < E && want >= carry + incl - tiles && want < carry + incl;
-        const unsigned who = __ballot_sync(0xffffffffu, mine);
-        if (who) {
-          const int src = __ffs(who) - 1;
-          found = base + src;
-          f_tile = __shfl_sync(0xffffffffu, want - (carry + incl - tiles), src);
-          f_lo = __shfl_sync(0xffffffffu, lo, src);
-          f_hi = __shfl_sync(0xffffffffu, hi, src);
-        }
-        carry += __shfl_sync(0xffffffffu, incl, 31);
-        prev_hi = __shfl_sync(0xffffffffu, hi, 31);
       }
       if (lane == 0) {
         grp[0] = found;

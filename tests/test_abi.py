@@ -148,7 +148,7 @@ def test_grouped_argument_checks():
     assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, 4, 64, 256, 128, None, None) == ALIGN
     assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 256, 120, None, None) == SHAPE        # K % 16
     assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 252, 128, None, None) == SHAPE        # N % 8
-    assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 70000, 64, 256, 128, None, None) == SHAPE    # grid y
+    assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 70000, 2000000, 256, 128, None, None) == SHAPE   # grid y
     assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0, 256, 128, None, None) == OK
     assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, 64, 256, 128, None, None) == INVALID
 
