@@ -15,6 +15,10 @@
  *   LQ_W8A8_INT8   : int8 codes, the same scale granularity, int32 sums;
  *   LQ_BLOCK_FP8   : e4m3 codes, one activation scale per 1x128 K-group and
  *                    one weight scale per 128x128 (n, k) block.
+ *   LQ_BLOCK_FP8_UE8M0 : Block_FP8 whose scales are powers of two stored as
+ *                    UE8M0 bytes (value 2^(b - 127)), the scale format the
+ *                    24-ai.news report (section "実際の制限事項") says DeepGEMM
+ *                    needs on B200 and the per-group quantizer lacked.
  *
  * The algorithmic variants Standard, Split-K and Swap-AB of the same page's
  * section "Kernel Implementation" are selected per call by an lq_variant (or
@@ -57,7 +61,8 @@ typedef struct CUstream_st *lq_stream_t;
 typedef enum {
   LQ_FP8_DYNAMIC = 0,
   LQ_W8A8_INT8 = 1,
-  LQ_BLOCK_FP8 = 2
+  LQ_BLOCK_FP8 = 2,
+  LQ_BLOCK_FP8_UE8M0 = 3
 } lq_fmt;
 
 typedef enum {
@@ -122,15 +127,18 @@ typedef struct {
  * Linear Backend with Helion", sections "Helion Linear Backend > Scope"
  * (formats, scale granularity) and "Kernel Implementation" (variants).
  *
- *   fmt      : LQ_FP8_DYNAMIC, LQ_W8A8_INT8 or LQ_BLOCK_FP8.
+ *   fmt      : LQ_FP8_DYNAMIC, LQ_W8A8_INT8, LQ_BLOCK_FP8 or
+ *              LQ_BLOCK_FP8_UE8M0.
  *   A        : [M, K] codes (uint8 e4m3 or int8), 16-byte aligned.
- *   a_scales : fp32; [M] for FP8_DYNAMIC/W8A8_INT8, [M, K/128] for BLOCK_FP8.
+ *   a_scales : fp32; [M] for FP8_DYNAMIC/W8A8_INT8, [M, K/128] for BLOCK_FP8;
+ *              for BLOCK_FP8_UE8M0 [M, K/128] UE8M0 bytes (pass the byte
+ *              array's address, any alignment).
  *   B        : [N, K] codes, 16-byte aligned.
  *   b_scales : fp32; [N] for FP8_DYNAMIC/W8A8_INT8, [N/128, K/128] for
- *              BLOCK_FP8.
+ *              BLOCK_FP8; [N/128, K/128] UE8M0 bytes for BLOCK_FP8_UE8M0.
  *   C        : [M, N] bf16 output, 16-byte aligned.
  *   M, N, K  : M >= 0, N >= 0, K >= 0; K % 16 == 0 and N % 8 == 0;
- *              BLOCK_FP8 also needs K % 128 == 0 and N % 128 == 0.
+ *              the Block_FP8 formats also need K % 128 == 0, N % 128 == 0.
  *              M == 0 or N == 0 is a no-op; K == 0 writes C = 0.
  *   variant  : NULL = the dispatch table's choice for (fmt, M, N, K).
  *   stream   : CUDA stream.
@@ -335,6 +343,23 @@ lq_status lq_silu_and_mul_dynamic_per_token_quant(lq_fmt fmt, const void *gate_u
                                                   lq_stream_t stream);
 lq_status lq_silu_and_mul_per_block_quant(const void *gate_up, void *q, float *scales,
                                           int64_t M, int64_t I, lq_stream_t stream);
+
+/*
+ * Block_FP8 quantizers with UE8M0 scales: the scale of a group is the
+ * smallest power of two 2^e with amax / 2^e <= 448 (e clamped to
+ * [-127, 127]; an all-zero group gets e = -127), written as the byte e + 127;
+ * codes are e4m3(x * 2^-e), exact scaling then round to nearest even, so no
+ * code saturates.
+ *   lq_quant_per_token_group128_ue8m0: x [M, K] bf16 (16-byte aligned) ->
+ *     q [M, K] e4m3 (8-byte aligned), scales [M, K/128] bytes; K % 128 == 0.
+ *   lq_quant_weight_block128_ue8m0: w [N, K] -> q [N, K], scales
+ *     [N/128, K/128] bytes; N % 128 == 0 and K % 128 == 0.
+ * Errors as lq_quant_per_token_group128 / lq_quant_weight_block128.
+ */
+lq_status lq_quant_per_token_group128_ue8m0(const void *x, void *q, uint8_t *scales,
+                                           int64_t M, int64_t K, lq_stream_t stream);
+lq_status lq_quant_weight_block128_ue8m0(const void *w, void *q, uint8_t *scales,
+                                         int64_t N, int64_t K, lq_stream_t stream);
 
 /*
  * 128x128 block quantization of a Block_FP8 weight stored [N, K]: one scale

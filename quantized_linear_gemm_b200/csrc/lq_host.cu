@@ -280,7 +280,7 @@ lq_variant heuristic_variant(int fmt, int64_t M, int64_t N, int64_t K) {
     v.stages = per_split < 2 ? 2 : (per_split > cap ? cap : per_split);
   } else {
     v.swap_ab = 0;
-    v.tile_n = fmt == lq::kFmtBlock ? 128 : 256;
+    v.tile_n = lq::is_block_fmt(fmt) ? 128 : 256;
     const int64_t tiles = ((M + 127) / 128) * ((N + v.tile_n - 1) / v.tile_n);
     int S = 1;
     while (S < 256 && tiles * S < kNumSms && T / (S * 2) >= 4) S *= 2;
@@ -295,7 +295,9 @@ bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, lq_variant* out) {
   auto t = current_table();
   const int64_t mb = m_bucket(M);
   for (const TableEntry& e : *t) {
-    if (e.fmt == fmt && e.m_bucket == mb && e.N == N && e.K == K) {
+    // UE8M0 Block_FP8 runs the Block_FP8 kernels: it shares their entries
+    const int key = fmt == lq::kFmtBlockE8m0 ? lq::kFmtBlock : fmt;
+    if (e.fmt == key && e.m_bucket == mb && e.N == N && e.K == K) {
       *out = e.v;
       return true;
     }
@@ -317,7 +319,7 @@ lq_status check_variant(int fmt, const lq_variant& v) {
     if (v.tile_n != 16 && v.tile_n != 32 && v.tile_n != 64) return LQ_ERR_INVALID_ARG;
   } else {
     if (v.tile_n != 64 && v.tile_n != 128 && v.tile_n != 256) return LQ_ERR_INVALID_ARG;
-    if (fmt == lq::kFmtBlock && v.tile_n == 256) return LQ_ERR_INVALID_ARG;
+    if (lq::is_block_fmt(fmt) && v.tile_n == 256) return LQ_ERR_INVALID_ARG;
   }
   if (v.stages != 0 && (v.stages < 2 || v.stages > kMaxStages)) return LQ_ERR_INVALID_ARG;
   if (v.stages != 0 &&
@@ -328,7 +330,7 @@ lq_status check_variant(int fmt, const lq_variant& v) {
 
 lq_status check_gemm_args(int fmt, const void* A, const float* a_s, const void* B, const float* b_s, const void* C,
                           int64_t M, int64_t N, int64_t K) {
-  if (fmt < 0 || fmt > 2) return LQ_ERR_INVALID_ARG;
+  if (fmt < 0 || fmt > 3) return LQ_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return LQ_OK;
   if (!C) return LQ_ERR_INVALID_ARG;
@@ -336,9 +338,9 @@ lq_status check_gemm_args(int fmt, const void* A, const float* a_s, const void* 
   if (K == 0) return LQ_OK;
   if (!A || !B || !a_s || !b_s) return LQ_ERR_INVALID_ARG;
   if (!aligned(A, 16) || !aligned(B, 16)) return LQ_ERR_ALIGNMENT;
-  if (!aligned(a_s, 4) || !aligned(b_s, 4)) return LQ_ERR_ALIGNMENT;
+  if (fmt != lq::kFmtBlockE8m0 && (!aligned(a_s, 4) || !aligned(b_s, 4))) return LQ_ERR_ALIGNMENT;   // e8m0: bytes
   if (K % 16 != 0 || N % 8 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
-  if (fmt == lq::kFmtBlock && (K % 128 != 0 || N % 128 != 0)) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (lq::is_block_fmt(fmt) && (K % 128 != 0 || N % 128 != 0)) return LQ_ERR_UNSUPPORTED_SHAPE;
   if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1)
     return LQ_ERR_UNSUPPORTED_SHAPE;
   return LQ_OK;
@@ -433,6 +435,7 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   switch (fmt) {
     case lq::kFmtFp8: e = lq::launch_scaled_mm_fp8(l, v.swap_ab, v.tile_n); break;
     case lq::kFmtInt8: e = lq::launch_scaled_mm_int8(l, v.swap_ab, v.tile_n); break;
+    case lq::kFmtBlockE8m0: e = lq::launch_scaled_mm_block_e8m0(l, v.swap_ab, v.tile_n); break;
     default: e = lq::launch_scaled_mm_block(l, v.swap_ab, v.tile_n); break;
   }
   if (e != cudaSuccess) {
@@ -699,7 +702,7 @@ lq_status lq_quant_per_token_group128(const void* x, void* q, float* scales, int
   if (!aligned(x, 16) || !aligned(q, 8) || !aligned(scales, 4)) return LQ_ERR_ALIGNMENT;
   if (K % 128 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
   if ((M * (K / 128) + 15) / 16 > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
-  return lq::launch_quant_group128(x, q, scales, M, K, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+  return lq::launch_quant_group128(x, q, scales, M, K, false, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? LQ_OK
              : LQ_ERR_CUDA;
 }
@@ -787,14 +790,40 @@ lq_status lq_quant_weight_block128(const void* w, void* q, float* scales, int64_
   if (!w || !q || !scales) return LQ_ERR_INVALID_ARG;
   if (!aligned(w, 16) || !aligned(q, 8) || !aligned(scales, 4)) return LQ_ERR_ALIGNMENT;
   if (N % 128 != 0 || K % 128 != 0 || N / 128 > 65535 || K / 128 > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
-  return lq::launch_quant_weight_block128(w, q, scales, N, K, reinterpret_cast<cudaStream_t>(stream)) ==
+  return lq::launch_quant_weight_block128(w, q, scales, N, K, false, reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? LQ_OK
+             : LQ_ERR_CUDA;
+}
+
+lq_status lq_quant_per_token_group128_ue8m0(const void* x, void* q, uint8_t* scales, int64_t M, int64_t K,
+                                           lq_stream_t stream) {
+  if (M < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (M == 0 || K == 0) return LQ_OK;
+  if (!x || !q || !scales) return LQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 8)) return LQ_ERR_ALIGNMENT;
+  if (K % 128 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if ((M * (K / 128) + 15) / 16 > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+  return lq::launch_quant_group128(x, q, scales, M, K, true, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LQ_OK
+             : LQ_ERR_CUDA;
+}
+
+lq_status lq_quant_weight_block128_ue8m0(const void* w, void* q, uint8_t* scales, int64_t N, int64_t K,
+                                         lq_stream_t stream) {
+  if (N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (N == 0 || K == 0) return LQ_OK;
+  if (!w || !q || !scales) return LQ_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(q, 8)) return LQ_ERR_ALIGNMENT;
+  if (N % 128 != 0 || K % 128 != 0 || N / 128 > 65535 || K / 128 > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+  return lq::launch_quant_weight_block128(w, q, scales, N, K, true, reinterpret_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? LQ_OK
              : LQ_ERR_CUDA;
 }
 
 lq_status lq_select_variant(lq_fmt fmt, int64_t M, int64_t N, int64_t K, lq_variant* out) {
-  if (!out || fmt < 0 || fmt > 2 || M < 0 || N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (!out || fmt < 0 || fmt > 3 || M < 0 || N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
   if (!lookup_table(static_cast<int>(fmt), M, N, K, out)) *out = heuristic_variant(static_cast<int>(fmt), M, N, K);
   return LQ_OK;
 }
@@ -834,7 +863,7 @@ lq_status lq_reserve_workspace(int device, size_t bytes) {
 }
 
 size_t lq_workspace_bytes(lq_fmt fmt, int64_t M, int64_t N, int64_t K, const lq_variant* variant) {
-  if (M <= 0 || N <= 0 || K <= 0 || fmt < 0 || fmt > 2) return 0;
+  if (M <= 0 || N <= 0 || K <= 0 || fmt < 0 || fmt > 3) return 0;
   lq_variant v{};
   if (variant) v = *variant;
   else if (!lookup_table(static_cast<int>(fmt), M, N, K, &v)) v = heuristic_variant(static_cast<int>(fmt), M, N, K);
@@ -982,6 +1011,7 @@ extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const floa
   switch (fmt) {
     case lq::kFmtFp8: e = lq::launch_scaled_mm_fp8(l, v.swap_ab, v.tile_n); break;
     case lq::kFmtInt8: e = lq::launch_scaled_mm_int8(l, v.swap_ab, v.tile_n); break;
+    case lq::kFmtBlockE8m0: e = lq::launch_scaled_mm_block_e8m0(l, v.swap_ab, v.tile_n); break;
     default: e = lq::launch_scaled_mm_block(l, v.swap_ab, v.tile_n); break;
   }
   if (e == cudaSuccess && v.split_k > 1) e = lq::launch_splitk_reduce(fmt, p, v.pdl != 0, stream);

@@ -12,6 +12,8 @@ namespace lq {
 constexpr int kFmtFp8 = 0;    // LQ_FP8_DYNAMIC
 constexpr int kFmtInt8 = 1;   // LQ_W8A8_INT8
 constexpr int kFmtBlock = 2;  // LQ_BLOCK_FP8
+constexpr int kFmtBlockE8m0 = 3;  // LQ_BLOCK_FP8_UE8M0: Block_FP8 with power-of-two (e8m0 byte) scales
+__host__ __device__ constexpr bool is_block_fmt(int fmt) { return fmt == kFmtBlock || fmt == kFmtBlockE8m0; }
 
 struct GemmParams {
   int64_t M, N, K;
@@ -61,6 +63,7 @@ struct GemmLaunch {
 cudaError_t launch_scaled_mm_fp8(const GemmLaunch& l, int swap_ab, int tile_n);
 cudaError_t launch_scaled_mm_int8(const GemmLaunch& l, int swap_ab, int tile_n);
 cudaError_t launch_scaled_mm_block(const GemmLaunch& l, int swap_ab, int tile_n);
+cudaError_t launch_scaled_mm_block_e8m0(const GemmLaunch& l, int swap_ab, int tile_n);
 cudaError_t launch_splitk_reduce(int fmt, const GemmParams& p, int pdl, cudaStream_t stream);
 
 // Dynamic shared memory of the GEMM kernel for (tile_n, stages), with or
@@ -72,7 +75,7 @@ int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce, bool fuse =
 // Quantization kernels (quant_kernels.cu).
 cudaError_t launch_quant_per_token(int fmt, const void* x, void* q, float* scales, int64_t M, int64_t K,
                                    cudaStream_t stream);
-cudaError_t launch_quant_group128(const void* x, void* q, float* scales, int64_t M, int64_t K,
+cudaError_t launch_quant_group128(const void* x, void* q, void* scales, int64_t M, int64_t K, bool e8m0,
                                   cudaStream_t stream);
 // Producer-side fused quantizers (producer_quant.cu); rows of at most
 // producer_max_row() outputs.
@@ -82,7 +85,7 @@ cudaError_t launch_rms_norm_quant(int fmt, bool per_block, const void* x, void* 
                                   uint64_t wait_limit_ns, cudaStream_t stream);
 cudaError_t launch_silu_mul_quant(int fmt, bool per_block, const void* gate_up, void* q, float* scales, int64_t M,
                                   int64_t I, int* status, uint64_t wait_limit_ns, cudaStream_t stream);
-cudaError_t launch_quant_weight_block128(const void* w, void* q, float* scales, int64_t N, int64_t K,
+cudaError_t launch_quant_weight_block128(const void* w, void* q, void* scales, int64_t N, int64_t K, bool e8m0,
                                          cudaStream_t stream);
 cudaError_t launch_fill_zero_bf16(__nv_bfloat16* C, int64_t count, cudaStream_t stream);
 

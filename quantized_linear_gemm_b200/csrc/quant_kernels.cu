@@ -122,9 +122,37 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const __nv_bfloat1
   }
 }
 
+// UE8M0 scale of a group: the smallest power of two 2^e with amax <= 448 2^e,
+// e clamped to [-127, 127], decided exactly on the bits of amax (448 =
+// 1.75 2^8): for amax = m 2^E (m in [1, 2)), e = E - 8, plus one when
+// m > 1.75.  Zero and subnormal amax give e = -127 (byte 0).
+__device__ __forceinline__ int ue8m0_exponent(float amax) {
+  const uint32_t bits = __float_as_uint(amax);
+  const int biased = static_cast<int>(bits >> 23);
+  if (biased == 0) return -127;
+  const int e = (biased - 127) - 8 + ((bits & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  return e < -127 ? -127 : e;
+}
+
+// 2^-e as a float; for e in [-127, 120] (finite amax) a normal number.
+__device__ __forceinline__ float pow2_neg(int e) { return __uint_as_float(static_cast<uint32_t>(127 - e) << 23); }
+
+// 8 values times 2^-e (exact) -> 8 e4m3 bytes.
+__device__ __forceinline__ uint2 encode8_e4m3_pow2(const float (&f)[8], int e) {
+  const float r = pow2_neg(e);
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(f[2 * i], r), __fmul_rn(f[2 * i + 1], r)),
+                                                          __NV_SATFINITE, __NV_E4M3));
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
 // 16 threads per 128-element group, 8 elements each; 16 groups per CTA.
+// kE8m0: UE8M0 scale bytes (power-of-two scales) instead of fp32 scales.
+template <bool kE8m0>
 __global__ void __launch_bounds__(256) quant_group128_kernel(const __nv_bfloat16* __restrict__ x,
-                                                              uint8_t* __restrict__ q, float* __restrict__ scales,
+                                                              uint8_t* __restrict__ q, void* __restrict__ scales,
                                                               int64_t M, int64_t K) {
   grid_launch_dependents();   // before the wait: see the note at the top of the namespace
   grid_dependency_wait();
@@ -140,17 +168,26 @@ __global__ void __launch_bounds__(256) quant_group128_kernel(const __nv_bfloat16
   float a = amax8(f);
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));   // within 16 lanes
-  const float s = scale_from_amax(a, kE4m3Max);
-  if (valid) {
-    if (sub == 0) scales[row * KB + kb] = s;
-    *reinterpret_cast<uint2*>(q + off) = encode8_e4m3(f, make_divisor(a, s));
+  if constexpr (kE8m0) {
+    const int e = ue8m0_exponent(a);
+    if (valid) {
+      if (sub == 0) static_cast<uint8_t*>(scales)[row * KB + kb] = static_cast<uint8_t>(e + 127);
+      *reinterpret_cast<uint2*>(q + off) = encode8_e4m3_pow2(f, e);
+    }
+  } else {
+    const float s = scale_from_amax(a, kE4m3Max);
+    if (valid) {
+      if (sub == 0) static_cast<float*>(scales)[row * KB + kb] = s;
+      *reinterpret_cast<uint2*>(q + off) = encode8_e4m3(f, make_divisor(a, s));
+    }
   }
 }
 
 // One CTA per 128x128 block of W[N, K]; thread t covers row t/2, 64 columns.
+template <bool kE8m0>
 __global__ void __launch_bounds__(256) quant_weight_block128_kernel(const __nv_bfloat16* __restrict__ w,
                                                                      uint8_t* __restrict__ q,
-                                                                     float* __restrict__ scales, int64_t K) {
+                                                                     void* __restrict__ scales, int64_t K) {
   __shared__ float red[32];
   const int64_t KB = K / 128;
   const int64_t nb = blockIdx.y, kb = blockIdx.x;
@@ -165,12 +202,19 @@ __global__ void __launch_bounds__(256) quant_weight_block128_kernel(const __nv_b
     a = fmaxf(a, amax8(f[i]));
   }
   const float amax = block_max<256>(a, red);
-  const float s = scale_from_amax(amax, kE4m3Max);
-  const Divisor d = make_divisor(amax, s);
-  if (threadIdx.x == 0) scales[nb * KB + kb] = s;
   uint2* dst = reinterpret_cast<uint2*>(q + row * K + col);
+  if constexpr (kE8m0) {
+    const int e = ue8m0_exponent(amax);
+    if (threadIdx.x == 0) static_cast<uint8_t*>(scales)[nb * KB + kb] = static_cast<uint8_t>(e + 127);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) dst[i] = encode8_e4m3(f[i], d);
+    for (int i = 0; i < 8; ++i) dst[i] = encode8_e4m3_pow2(f[i], e);
+  } else {
+    const float s = scale_from_amax(amax, kE4m3Max);
+    const Divisor d = make_divisor(amax, s);
+    if (threadIdx.x == 0) static_cast<float*>(scales)[nb * KB + kb] = s;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = encode8_e4m3(f[i], d);
+  }
 }
 
 __global__ void fill_zero_bf16_kernel(__nv_bfloat16* __restrict__ C, int64_t count) {
@@ -217,20 +261,27 @@ cudaError_t launch_quant_per_token(int fmt, const void* x, void* q, float* scale
   return cudaLaunchKernelEx(&cfg, quant_per_token_kernel<false>, xp, qp, scales, K);
 }
 
-cudaError_t launch_quant_group128(const void* x, void* q, float* scales, int64_t M, int64_t K,
+cudaError_t launch_quant_group128(const void* x, void* q, void* scales, int64_t M, int64_t K, bool e8m0,
                                   cudaStream_t stream) {
   const int64_t groups = M * (K / 128);
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = pdl_config(dim3(static_cast<unsigned>((groups + 15) / 16)), dim3(256), stream, attr);
-  return cudaLaunchKernelEx(&cfg, quant_group128_kernel, static_cast<const __nv_bfloat16*>(x),
+  if (e8m0)
+    return cudaLaunchKernelEx(&cfg, quant_group128_kernel<true>, static_cast<const __nv_bfloat16*>(x),
+                              static_cast<uint8_t*>(q), scales, M, K);
+  return cudaLaunchKernelEx(&cfg, quant_group128_kernel<false>, static_cast<const __nv_bfloat16*>(x),
                             static_cast<uint8_t*>(q), scales, M, K);
 }
 
-cudaError_t launch_quant_weight_block128(const void* w, void* q, float* scales, int64_t N, int64_t K,
+cudaError_t launch_quant_weight_block128(const void* w, void* q, void* scales, int64_t N, int64_t K, bool e8m0,
                                          cudaStream_t stream) {
-  quant_weight_block128_kernel<<<dim3(static_cast<unsigned>(K / 128), static_cast<unsigned>(N / 128)), 256, 0,
-                                  stream>>>(static_cast<const __nv_bfloat16*>(w), static_cast<uint8_t*>(q), scales,
-                                            K);
+  const dim3 grid(static_cast<unsigned>(K / 128), static_cast<unsigned>(N / 128));
+  if (e8m0)
+    quant_weight_block128_kernel<true><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(w),
+                                                                 static_cast<uint8_t*>(q), scales, K);
+  else
+    quant_weight_block128_kernel<false><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(w),
+                                                                  static_cast<uint8_t*>(q), scales, K);
   return cudaGetLastError();
 }
 

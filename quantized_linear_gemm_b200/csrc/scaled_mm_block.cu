@@ -41,7 +41,9 @@ cudaError_t launch_splitk_reduce(int fmt, const GemmParams& p, int pdl, cudaStre
   switch (fmt) {
     case kFmtFp8: return cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<kFmtFp8>, p);
     case kFmtInt8: return cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<kFmtInt8>, p);
-    case kFmtBlock: return cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<kFmtBlock>, p);
+    case kFmtBlock:
+    case kFmtBlockE8m0:   // the partials already carry their block scales
+      return cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<kFmtBlock>, p);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -153,12 +153,12 @@ template <int FMT, bool SWAP, int TN, bool FUSE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     scaled_mm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                         const GemmParams p) {
-  static_assert(!FUSE || (SWAP && FMT != kFmtBlock && TN <= 64), "fused quantization: Swap-AB FP8/INT8 tiles");
+  static_assert(!FUSE || (SWAP && !is_block_fmt(FMT) && TN <= 64), "fused quantization: Swap-AB FP8/INT8 tiles");
   using Shape = TileShape<TN, FUSE>;
   // bytes the TMA delivers per stage (the fused path writes the activation slot itself)
   constexpr uint32_t kTmaStageBytes = FUSE ? Shape::kXBytes : Shape::kStageBytes;
   constexpr bool kInt8 = FMT == kFmtInt8;
-  constexpr bool kBlocked = FMT == kFmtBlock;
+  constexpr bool kBlocked = is_block_fmt(FMT);
   constexpr int kAccBufs = kBlocked ? 2 : 1;
   constexpr int kTmemCols = tmem_cols_for(TN * kAccBufs);
   constexpr int CH = TN < 32 ? TN : 32;   // TMEM columns per tcgen05.ld
@@ -601,13 +601,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // so the named barriers always match.
       const int nb = SWAP ? x_row0 / 128 : y_row0 / 128;
       const int64_t m_thread = x_row0 + r;   // Standard: this thread's token
+      // Block scale i of an operand: fp32, or a UE8M0 byte (2^(b - 127)).
+      auto scale_at = [&](const float* base, int64_t i) -> float {
+        if constexpr (FMT == kFmtBlockE8m0) {
+          const uint32_t b = __ldg(reinterpret_cast<const uint8_t*>(base) + i);
+          return __uint_as_float(b == 0u ? 0x00400000u : (b == 255u ? 0x7FC00000u : b << 23));
+        } else {
+          return __ldg(base + i);
+        }
+      };
       auto load_scale = [&](int kb) -> float {
-        const float sb = __ldg(p.b_s + static_cast<int64_t>(nb) * p.KB + kb);
+        const float sb = scale_at(p.b_s, static_cast<int64_t>(nb) * p.KB + kb);
         if (SWAP) {
           const int64_t m = y_row0 + r;     // column r of the tile (r < TN)
-          return (m < M ? __ldg(p.a_s + m * p.KB + kb) : 0.f) * sb;
+          return (m < M ? scale_at(p.a_s, m * p.KB + kb) : 0.f) * sb;
         }
-        return (m_thread < M ? __ldg(p.a_s + m_thread * p.KB + kb) : 0.f) * sb;
+        return (m_thread < M ? scale_at(p.a_s, m_thread * p.KB + kb) : 0.f) * sb;
       };
       const bool loader = SWAP ? (r < TN) : true;
       float cur = 0.f;   // Standard: this thread's scale product of the current block
@@ -1052,7 +1061,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int FMT>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmParams p) {
   constexpr bool kInt8 = FMT == kFmtInt8;
-  constexpr bool kBlocked = FMT == kFmtBlock;
+  constexpr bool kBlocked = is_block_fmt(FMT);
   grid_launch_dependents();   // before the wait, as the quantization kernels do
   grid_dependency_wait();
   const int64_t MN4 = p.M * p.N / 4;

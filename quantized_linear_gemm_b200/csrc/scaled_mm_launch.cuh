@@ -45,7 +45,7 @@ cudaError_t launch_tc(const GemmLaunch& l) {
 template <int FMT>
 cudaError_t launch_format(const GemmLaunch& l, int swap_ab, int tile_n) {
   if (l.fuse) {
-    if constexpr (FMT != kFmtBlock) {
+    if constexpr (!is_block_fmt(FMT)) {
       if (!swap_ab) return cudaErrorInvalidValue;
       switch (tile_n) {
         case 16: return launch_tc<FMT, true, 16, true>(l);
@@ -68,7 +68,7 @@ cudaError_t launch_format(const GemmLaunch& l, int swap_ab, int tile_n) {
     case 64: return launch_tc<FMT, false, 64>(l);
     case 128: return launch_tc<FMT, false, 128>(l);
     case 256:
-      if constexpr (FMT != kFmtBlock) return launch_tc<FMT, false, 256>(l);
+      if constexpr (!is_block_fmt(FMT)) return launch_tc<FMT, false, 256>(l);
       return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }

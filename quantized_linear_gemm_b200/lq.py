@@ -21,7 +21,9 @@ LIB_PATH = os.path.join(_PKG, "liblq.so")
 FP8_DYNAMIC = 0
 W8A8_INT8 = 1
 BLOCK_FP8 = 2
-FORMATS = {"fp8_dynamic": FP8_DYNAMIC, "w8a8_int8": W8A8_INT8, "block_fp8": BLOCK_FP8}
+BLOCK_FP8_UE8M0 = 3
+FORMATS = {"fp8_dynamic": FP8_DYNAMIC, "w8a8_int8": W8A8_INT8, "block_fp8": BLOCK_FP8,
+           "block_fp8_ue8m0": BLOCK_FP8_UE8M0}
 
 STATUS = {
     0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_ALIGNMENT", 3: "LQ_ERR_UNSUPPORTED_SHAPE",
@@ -36,7 +38,7 @@ EXPORTED = (
     "lq_status_string", "lq_version", "lq_set_trace", "lq_scaled_mm_noalloc", "lq_test_inject_stall",
     "lq_quant_scaled_mm", "lq_set_fuse_limit", "lq_rms_norm_dynamic_per_token_quant",
     "lq_rms_norm_per_block_quant", "lq_silu_and_mul_dynamic_per_token_quant", "lq_silu_and_mul_per_block_quant",
-    "lq_grouped_scaled_mm",
+    "lq_grouped_scaled_mm", "lq_quant_per_token_group128_ue8m0", "lq_quant_weight_block128_ue8m0",
 )
 
 
@@ -117,6 +119,9 @@ def lib() -> ctypes.CDLL:
             L.lq_grouped_scaled_mm.argtypes = [_i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                                ctypes.POINTER(Variant), _st]
             L.lq_grouped_scaled_mm.restype = _i32
+            for name in ("lq_quant_per_token_group128_ue8m0", "lq_quant_weight_block128_ue8m0"):
+                getattr(L, name).argtypes = [_vp, _vp, _vp, _i64, _i64, _st]
+                getattr(L, name).restype = _i32
             L.lq_version.argtypes = []
             L.lq_version.restype = ctypes.c_char_p
             for name in ("lq_scaled_mm", "lq_scaled_mm_i32acc", "lq_quant_per_token", "lq_quant_per_token_group128",
@@ -167,8 +172,10 @@ def scaled_mm(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor, b_s
     f = _fmt(fmt)
     _need(A, "A", _CODE_DTYPES, 2)
     _need(B, "B", _CODE_DTYPES, 2)
-    _need(a_scales, "a_scales", (torch.float32,), 2 if f == BLOCK_FP8 else 1)
-    _need(b_scales, "b_scales", (torch.float32,), 2 if f == BLOCK_FP8 else 1)
+    block = f in (BLOCK_FP8, BLOCK_FP8_UE8M0)
+    sdt = (torch.uint8,) if f == BLOCK_FP8_UE8M0 else (torch.float32,)
+    _need(a_scales, "a_scales", sdt, 2 if block else 1)
+    _need(b_scales, "b_scales", sdt, 2 if block else 1)
     M, K = A.shape
     N = B.shape[0]
     if B.shape[1] != K:
@@ -363,6 +370,32 @@ def silu_and_mul_per_block_quant(gate_up: torch.Tensor, q=None, scales=None, str
     return q, scales
 
 
+def quant_per_token_group128_ue8m0(x: torch.Tensor, q=None, scales=None, stream=None):
+    """(e4m3 codes [M, K], UE8M0 scale bytes [M, K/128]) of a bf16 [M, K] tensor."""
+    _need(x, "x", (torch.bfloat16,), 2)
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((M, max(K // 128, 0)), dtype=torch.uint8, device=x.device)
+    rc = lib().lq_quant_per_token_group128_ue8m0(_ptr(x), _ptr(q), _ptr(scales), M, K, _stream(stream))
+    _check("lq_quant_per_token_group128_ue8m0", rc)
+    return q, scales
+
+
+def quant_weight_block128_ue8m0(w: torch.Tensor, q=None, scales=None, stream=None):
+    """(e4m3 codes [N, K], UE8M0 scale bytes [N/128, K/128]) of a bf16 weight [N, K]."""
+    _need(w, "w", (torch.bfloat16,), 2)
+    N, K = w.shape
+    if q is None:
+        q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty((max(N // 128, 0), max(K // 128, 0)), dtype=torch.uint8, device=w.device)
+    rc = lib().lq_quant_weight_block128_ue8m0(_ptr(w), _ptr(q), _ptr(scales), N, K, _stream(stream))
+    _check("lq_quant_weight_block128_ue8m0", rc)
+    return q, scales
+
+
 def quant_weight_block128(w: torch.Tensor, q=None, scales=None, stream=None):
     """(e4m3 codes [N, K], scales [N/128, K/128]) of a bf16 weight [N, K]."""
     _need(w, "w", (torch.bfloat16,), 2)
@@ -453,8 +486,9 @@ class Problem:
     @property
     def bytes(self) -> int:
         """Algorithmic HBM bytes: weights + activations + scales + bf16 output."""
-        if self.fmt == BLOCK_FP8:
-            scales = 4 * (self.M * (self.K // 128) + (self.N // 128) * (self.K // 128))
+        if self.fmt in (BLOCK_FP8, BLOCK_FP8_UE8M0):
+            per = 1 if self.fmt == BLOCK_FP8_UE8M0 else 4   # UE8M0 scales are bytes
+            scales = per * (self.M * (self.K // 128) + (self.N // 128) * (self.K // 128))
         else:
             scales = 4 * (self.M + self.N)
         return self.N * self.K + self.M * self.K + scales + 2 * self.M * self.N

@@ -46,13 +46,14 @@ def _mm(fmt=0, A=FAKE, a_s=FAKE, B=FAKE, b_s=FAKE, C=FAKE, M=16, N=128, K=128, v
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(fmt=3), INVALID), (dict(fmt=-1), INVALID),
+    (dict(fmt=4), INVALID), (dict(fmt=-1), INVALID),
     (dict(A=None), INVALID), (dict(B=None), INVALID), (dict(C=None), INVALID),
     (dict(a_s=None), INVALID), (dict(b_s=None), INVALID),
     (dict(M=-1), INVALID), (dict(K=-16), INVALID),
     (dict(A=MISALIGNED), ALIGN), (dict(B=MISALIGNED), ALIGN), (dict(C=MISALIGNED), ALIGN),
     (dict(K=120), SHAPE), (dict(N=100), SHAPE),
     (dict(fmt=2, K=192), SHAPE), (dict(fmt=2, N=192), SHAPE),
+    (dict(fmt=3, K=192), SHAPE), (dict(fmt=3, N=192), SHAPE), (dict(fmt=3, a_s=None), INVALID),
 ])
 def test_scaled_mm_argument_checks(kw, code):
     assert _mm(**kw) == code
@@ -151,6 +152,19 @@ def test_grouped_argument_checks():
     assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 70000, 2000000, 256, 128, None, None) == SHAPE   # grid y
     assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0, 256, 128, None, None) == OK
     assert g(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, 64, 256, 128, None, None) == INVALID
+
+
+def test_ue8m0_quant_argument_checks():
+    L = lq.lib()
+    assert L.lq_quant_per_token_group128_ue8m0(FAKE, FAKE, FAKE, 4, 192, None) == SHAPE
+    assert L.lq_quant_per_token_group128_ue8m0(None, FAKE, FAKE, 4, 256, None) == INVALID
+    assert L.lq_quant_per_token_group128_ue8m0(MISALIGNED, FAKE, FAKE, 4, 256, None) == ALIGN
+    assert L.lq_quant_per_token_group128_ue8m0(FAKE, FAKE, FAKE + 1, 0, 256, None) == OK     # bytes: any alignment
+    assert L.lq_quant_weight_block128_ue8m0(FAKE, FAKE, FAKE, 192, 256, None) == SHAPE
+    assert L.lq_quant_weight_block128_ue8m0(FAKE, FAKE, None, 128, 256, None) == INVALID
+    assert L.lq_quant_weight_block128_ue8m0(FAKE, FAKE, FAKE, 0, 256, None) == OK
+    # UE8M0 scales are bytes: an odd scale address passes the checks (M = 0 stops before any launch)
+    assert _mm(fmt=3, a_s=FAKE + 1, b_s=FAKE + 3, M=0) == OK
 
 
 def test_stall_hook_argument_check():
