@@ -155,6 +155,20 @@ lq_status lq_scaled_mm(lq_fmt fmt, const void *A, const float *a_scales,
                        const lq_variant *variant, lq_stream_t stream);
 
 /*
+ * scaled_mm with a bias: C[m, n] = bf16(acc * a_s * b_s + bias[n]), the
+ * scaled accumulator and the bias added in fp32 before the one rounding to
+ * bf16.  bias: [N] bf16 (device, 2-byte aligned, not NULL).  Same formats,
+ * arguments, variants and errors as lq_scaled_mm; K == 0 is refused with
+ * LQ_ERR_UNSUPPORTED_SHAPE.  The pages have no bias (a linear layer of the
+ * served models has none); it serves layers that do, and the N-sliced
+ * multi-GPU linear, whose shards each add their slice of it.
+ */
+lq_status lq_scaled_mm_bias(lq_fmt fmt, const void *A, const float *a_scales,
+                            const void *B, const float *b_scales, const void *bias,
+                            void *C, int64_t M, int64_t N, int64_t K,
+                            const lq_variant *variant, lq_stream_t stream);
+
+/*
  * Grouped (mixture-of-experts) scaled_mm: one launch for all experts, each
  * an ordinary FP8_Dynamic / W8A8_INT8 linear layer (the pages' next target:
  * ai-radar.it, "Helion in vLLM: il tuning dei GEMM diventa ricerca, non

@@ -349,7 +349,7 @@ lq_status check_gemm_args(int fmt, const void* A, const float* a_s, const void* 
 lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B, const float* b_s, void* C,
                          int32_t* acc_out, int64_t M, int64_t N, int64_t K, const lq_variant* variant,
                          cudaStream_t stream, const void* x_fused = nullptr, void* codes_out = nullptr,
-                         float* scales_out = nullptr) {
+                         float* scales_out = nullptr, const void* bias = nullptr) {
   const bool fused = x_fused != nullptr;
   lq_status rc = fused ? LQ_OK : check_gemm_args(fmt, A, a_s, B, b_s, C, M, N, K);
   if (rc != LQ_OK) return rc;
@@ -407,6 +407,7 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   p.x = static_cast<const __nv_bfloat16*>(x_fused);
   p.a_codes_out = static_cast<uint8_t*>(codes_out);
   p.a_scales_out = scales_out;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
   if (v.split_k > 1 && v.reduce != 2) {   // the cluster reduction needs no global workspace
     const size_t need = static_cast<size_t>(v.split_k) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
     rc = ensure_workspace(d, need, stream);
@@ -627,6 +628,16 @@ lq_status lq_grouped_scaled_mm(lq_fmt fmt_, const void* A, const float* a_scales
     return LQ_ERR_CUDA;
   }
   return LQ_OK;
+}
+
+lq_status lq_scaled_mm_bias(lq_fmt fmt, const void* A, const float* a_scales, const void* B, const float* b_scales,
+                            const void* bias, void* C, int64_t M, int64_t N, int64_t K, const lq_variant* variant,
+                            lq_stream_t stream) {
+  if (bias && !aligned(bias, 2)) return LQ_ERR_ALIGNMENT;
+  if (!bias && M > 0 && N > 0) return LQ_ERR_INVALID_ARG;
+  if (K == 0 && M > 0 && N > 0) return LQ_ERR_UNSUPPORTED_SHAPE;   // C would be the bias alone: not a GEMM
+  return scaled_mm_impl(static_cast<int>(fmt), A, a_scales, B, b_scales, C, nullptr, M, N, K, variant,
+                        reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr, bias);
 }
 
 lq_status lq_scaled_mm_i32acc(const void* A, const float* a_scales, const void* B, const float* b_scales, void* C,

@@ -40,6 +40,7 @@ struct GemmParams {
   // grouped (mixture-of-experts) launch, Swap-AB: M = tokens T, N = rows per expert
   const int* expert_offsets;   // device [num_experts + 1]; null = one GEMM
   int num_experts;
+  const __nv_bfloat16* bias;   // optional bf16 [N], added before the rounding to bf16
 };
 
 constexpr int kTraceSlots = 12;

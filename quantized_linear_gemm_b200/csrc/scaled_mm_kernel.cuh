@@ -100,6 +100,12 @@ struct SmemCtl {
   volatile int* last_flag;
 };
 
+// Optional bias of output column n (bf16 [N]), added to the scaled
+// accumulator before the one rounding to bf16.
+__device__ __forceinline__ float bias_at(const GemmParams& p, int64_t n) {
+  return p.bias ? __bfloat162float(p.bias[n]) : 0.f;
+}
+
 __device__ __forceinline__ void report_timeout(const GemmParams& p, int where) {
   if (p.status) atomicOr(p.status, 1 << where);
 }
@@ -752,6 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float a = kInt8 ? static_cast<float>(static_cast<int32_t>(v[j])) : __uint_as_float(v[j]);
                     val = a * colsc[c0 + j] * bsn;
                   }
+                  val += bias_at(p, n - c_off);
                   p.C[idx] = __float2bfloat16_rn(val);
                   if (kInt8 && p.acc_out) p.acc_out[idx] = static_cast<int32_t>(v[j]);
                 }
@@ -782,6 +789,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                           kInt8 ? static_cast<float>(static_cast<int32_t>(v[j8 + e])) : __uint_as_float(v[j8 + e]);
                       f[e] = a * asm_ * colsc[c0 + j8 + e];
                     }
+                  }
+                  if (p.bias) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] += bias_at(p, n + e);
                   }
                   uint4 pk = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
                                         pack_bf16x2(f[6], f[7]));
@@ -836,6 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               float val;
               if (kBlocked) val = sf;
               else val = (kInt8 ? static_cast<float>(si) : sf) * colsc[j] * bsn;
+              val += bias_at(p, n);
               p.C[m * N + n] = __float2bfloat16_rn(val);
               if (kInt8 && p.acc_out) p.acc_out[m * N + n] = si;
             }
@@ -865,6 +877,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!kBlocked) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * colsc[j4 + e];
+              }
+              if (p.bias) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) f[e] += bias_at(p, n + e);
               }
               uint2 pk = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
               *reinterpret_cast<uint2*>(p.C + m * N + n) = pk;
@@ -905,6 +921,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               float val;
               if (kBlocked) val = sf;
               else val = (kInt8 ? static_cast<float>(si) : sf) * colsc[j0 + jj] * bsn;
+              val += bias_at(p, n - c_off);
               p.C[m * p.N + (n - c_off)] = __float2bfloat16_rn(val);
               if (kInt8 && p.acc_out) p.acc_out[m * p.N + (n - c_off)] = si;
             }
@@ -934,6 +951,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!kBlocked) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * colsc[j0 + jj + e];
+              }
+              if (p.bias) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) f[e] += bias_at(p, n + e);
               }
               *reinterpret_cast<uint2*>(p.C + m * N + n) =
                   make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
@@ -996,6 +1017,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float val;
             if (kBlocked) val = sf;
             else val = (kInt8 ? static_cast<float>(si) : sf) * colsc[j] * bsn;
+            val += bias_at(p, n);
             p.C[m * N + n] = __float2bfloat16_rn(val);
             if (kInt8 && p.acc_out) p.acc_out[m * N + n] = si;
           }
@@ -1030,6 +1052,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!kBlocked) {
 #pragma unroll
               for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * colsc[j + e];
+            }
+            if (p.bias) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) f[e] += bias_at(p, n + e);
             }
             *reinterpret_cast<uint2*>(p.C + m * N + n) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
             if (kInt8 && p.acc_out)
@@ -1092,6 +1118,10 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmParams p) 
       const float a = __ldg(p.a_s + m);
 #pragma unroll
       for (int e = 0; e < 4; ++e) f[e] = f[e] * a * __ldg(p.b_s + n + e);
+    }
+    if (p.bias) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f[e] += bias_at(p, n + e);
     }
     *reinterpret_cast<uint2*>(p.C + e0) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
     if (kInt8 && p.acc_out) *reinterpret_cast<int4*>(p.acc_out + e0) = si;

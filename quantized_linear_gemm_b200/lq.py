@@ -39,6 +39,7 @@ EXPORTED = (
     "lq_quant_scaled_mm", "lq_set_fuse_limit", "lq_rms_norm_dynamic_per_token_quant",
     "lq_rms_norm_per_block_quant", "lq_silu_and_mul_dynamic_per_token_quant", "lq_silu_and_mul_per_block_quant",
     "lq_grouped_scaled_mm", "lq_quant_per_token_group128_ue8m0", "lq_quant_weight_block128_ue8m0",
+    "lq_scaled_mm_bias",
 )
 
 
@@ -122,6 +123,9 @@ def lib() -> ctypes.CDLL:
             for name in ("lq_quant_per_token_group128_ue8m0", "lq_quant_weight_block128_ue8m0"):
                 getattr(L, name).argtypes = [_vp, _vp, _vp, _i64, _i64, _st]
                 getattr(L, name).restype = _i32
+            L.lq_scaled_mm_bias.argtypes = [_i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                            ctypes.POINTER(Variant), _st]
+            L.lq_scaled_mm_bias.restype = _i32
             L.lq_version.argtypes = []
             L.lq_version.restype = ctypes.c_char_p
             for name in ("lq_scaled_mm", "lq_scaled_mm_i32acc", "lq_quant_per_token", "lq_quant_per_token_group128",
@@ -210,6 +214,26 @@ def quant_scaled_mm(fmt, x: torch.Tensor, B: torch.Tensor, b_scales: torch.Tenso
                                   ctypes.byref(variant) if variant is not None else None, _stream(stream))
     _check("lq_quant_scaled_mm", rc)
     return C, q, s
+
+
+def scaled_mm_bias(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor, b_scales: torch.Tensor,
+                   bias: torch.Tensor, C: torch.Tensor | None = None, variant: Variant | None = None,
+                   stream=None) -> torch.Tensor:
+    """``lq_scaled_mm_bias``: scaled_mm plus a bf16 bias [N] added before the rounding."""
+    f = _fmt(fmt)
+    _need(A, "A", _CODE_DTYPES, 2)
+    _need(B, "B", _CODE_DTYPES, 2)
+    _need(bias, "bias", (torch.bfloat16,), 1)
+    M, K = A.shape
+    N = B.shape[0]
+    if bias.numel() != N:
+        raise ValueError("bias must hold N values")
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    rc = lib().lq_scaled_mm_bias(f, _ptr(A), _ptr(a_scales), _ptr(B), _ptr(b_scales), _ptr(bias), _ptr(C), M, N, K,
+                                 ctypes.byref(variant) if variant is not None else None, _stream(stream))
+    _check("lq_scaled_mm_bias", rc)
+    return C
 
 
 def grouped_scaled_mm(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor, b_scales: torch.Tensor,

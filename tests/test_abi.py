@@ -167,6 +167,16 @@ def test_ue8m0_quant_argument_checks():
     assert _mm(fmt=3, a_s=FAKE + 1, b_s=FAKE + 3, M=0) == OK
 
 
+def test_bias_argument_checks():
+    L = lq.lib()
+    b = L.lq_scaled_mm_bias
+    assert b(0, FAKE, FAKE, FAKE, FAKE, None, FAKE, 16, 128, 128, None, None) == INVALID     # no bias
+    assert b(0, FAKE, FAKE, FAKE, FAKE, FAKE + 1, FAKE, 16, 128, 128, None, None) == ALIGN  # odd bias address
+    assert b(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 128, 0, None, None) == SHAPE        # K = 0
+    assert b(4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 128, 128, None, None) == INVALID    # format
+    assert b(0, FAKE, FAKE, FAKE, FAKE, None, FAKE, 0, 128, 128, None, None) == OK          # M = 0
+
+
 def test_stall_hook_argument_check():
     assert lq.lib().lq_test_inject_stall(-2, 0) == INVALID
     assert lq.lib().lq_test_inject_stall(-1, 0) == OK
