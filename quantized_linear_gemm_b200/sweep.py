@@ -1,6 +1,7 @@
 """On-device variant selector: writes the static dispatch table.
 
-    python -m quantized_linear_gemm_b200.sweep [--configs decode,block,prefill] [--out PATH] [--inc]
+    python -m quantized_linear_gemm_b200.sweep [--configs decode,block,prefill] [--formats ...]
+        [--with-quant] [--out PATH] [--inc]
 
 For every (format, token bucket, N, K) of the Qwen3 decode / prefill shapes
 this enumerates the variant space - Swap-AB or Standard, tile_n, split_k,
@@ -95,11 +96,13 @@ class Shape:
     """Device buffers of one (fmt, M, N, K) with enough weight copies that
     more than 2x L2 is streamed between two reads of one copy."""
 
-    def __init__(self, fmt, M, N, K, device):
+    def __init__(self, fmt, M, N, K, device, with_quant=False):
         self.fmt, self.M, self.N, self.K = fmt, M, N, K
+        self.with_quant = with_quant and fmt != lq.BLOCK_FP8
         name = FMT_NAMES[fmt]
         w = inputs.weights(N, K, seed=inputs.stable_seed("sweep-W", N, K)).to(device)
         x = inputs.activations(M, K, seed=inputs.stable_seed("sweep-A", M, K)).to(device)
+        self.x = x
         if fmt == lq.BLOCK_FP8:
             qb, sb = lq.quant_weight_block128(w)
             self.qa, self.sa = lq.quant_per_token_group128(x)
@@ -126,10 +129,13 @@ class Shape:
         except lq.LQError:
             return None
         g = torch.cuda.CUDAGraph()
+        name = FMT_NAMES[self.fmt]
         with torch.cuda.stream(stream):
             with torch.cuda.graph(g, stream=stream):
                 for i in range(calls):
                     qb, sb = self.W[i % self.copies]
+                    if self.with_quant:   # as in a decode step: the activations are quantized right before
+                        lq.quant_per_token(name, self.x, self.qa, self.sa, stream=stream)
                     lq.scaled_mm(self.fmt, self.qa, self.sa, qb, sb, C=self.C, variant=v, stream=stream)
         g.replay()
         torch.cuda.synchronize()
@@ -145,13 +151,15 @@ class Shape:
         return 1e3 * e0.elapsed_time(e1) / (replays * calls)
 
 
-def sweep(groups, device, log=sys.stderr, budget_s=None):
+def sweep(groups, device, log=sys.stderr, budget_s=None, with_quant=False, formats=None):
     stream = torch.cuda.Stream(device=device)
     results = []
     t_start = time.time()
     for key in keys_for(groups):
         fmt, M, N, K = key
-        sh = Shape(fmt, M, N, K, device)
+        if formats is not None and fmt not in formats:
+            continue
+        sh = Shape(fmt, M, N, K, device, with_quant=with_quant)
         big = sh.flops > 2e11
         best = None
         tried = 0
@@ -224,6 +232,9 @@ def main():
     ap.add_argument("--inc", action="store_true", help="regenerate csrc/dispatch_table.inc from --out")
     ap.add_argument("--inc-only", action="store_true", help="only regenerate the .inc from an existing table")
     ap.add_argument("--budget-s", type=float, default=None)
+    ap.add_argument("--formats", default=None, help="comma-separated subset, e.g. fp8_dynamic")
+    ap.add_argument("--with-quant", action="store_true",
+                    help="time each candidate after lq_quant_per_token, as the decode step runs it")
     a = ap.parse_args()
     if a.inc_only:
         write_inc(a.out, TABLE_INC)
@@ -232,7 +243,8 @@ def main():
     torch.cuda.set_device(device)
     lq.init_device(0)
     lq.load_dispatch_table(None)
-    res = sweep(set(a.configs.split(",")), device, budget_s=a.budget_s)
+    fmts = None if a.formats is None else {lq.FORMATS[f] for f in a.formats.split(",")}
+    res = sweep(set(a.configs.split(",")), device, budget_s=a.budget_s, with_quant=a.with_quant, formats=fmts)
     write_table(res, a.out)
     if a.json:
         with open(a.json, "w") as f:
