@@ -620,6 +620,7 @@ lq_status lq_grouped_scaled_mm(lq_fmt fmt_, const void* A, const float* a_scales
   l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce);
   l.pdl = v.pdl != 0;
   l.cluster_z = cluster_reduce ? v.split_k : 1;
+  l.grouped = 1;
   l.stream = stream;
   const cudaError_t e =
       fmt == lq::kFmtFp8 ? lq::launch_scaled_mm_fp8(l, 1, v.tile_n) : lq::launch_scaled_mm_int8(l, 1, v.tile_n);

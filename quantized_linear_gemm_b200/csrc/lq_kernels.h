@@ -55,6 +55,7 @@ struct GemmLaunch {
   int pdl;
   int cluster_z;       // > 1: launch clusters of (1, 1, cluster_z) CTAs
   int fuse;            // fused activation quantization (Swap-AB only)
+  int grouped;         // grouped (mixture-of-experts) launch (Swap-AB only; p.expert_offsets set)
   cudaStream_t stream;
 };
 

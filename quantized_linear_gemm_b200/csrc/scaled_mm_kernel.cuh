@@ -100,10 +100,10 @@ struct SmemCtl {
   volatile int* last_flag;
 };
 
-// Optional bias of output column n (bf16 [N]), added to the scaled
-// accumulator before the one rounding to bf16.
+// Bias of output column n (bf16 [N]), added to the scaled accumulator
+// before the one rounding to bf16.
 __device__ __forceinline__ float bias_at(const GemmParams& p, int64_t n) {
-  return p.bias ? __bfloat162float(p.bias[n]) : 0.f;
+  return __bfloat162float(p.bias[n]);
 }
 
 __device__ __forceinline__ void report_timeout(const GemmParams& p, int where) {
@@ -155,11 +155,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // each K tile of them beside the weights, and the epilogue warps, idle during
 // the mainloop, quantize it per token into the ring's activation slot (see
 // the A-producer below).
-template <int FMT, bool SWAP, int TN, bool FUSE = false>
+// GROUPED (Swap-AB, FP8_Dynamic / W8A8_INT8): the grouped (mixture-of-
+// experts) launch below; a compile-time switch so that the other
+// instantiations carry none of its code.
+// BIAS: the epilogue adds p.bias (also compile-time, for the same reason).
+template <int FMT, bool SWAP, int TN, bool FUSE = false, bool GROUPED = false, bool BIAS = false>
 __global__ void __launch_bounds__(kThreads, 1)
     scaled_mm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                         const GemmParams p) {
   static_assert(!FUSE || (SWAP && !is_block_fmt(FMT) && TN <= 64), "fused quantization: Swap-AB FP8/INT8 tiles");
+  static_assert(!GROUPED || (SWAP && !is_block_fmt(FMT) && !FUSE && TN <= 64), "grouped launch: Swap-AB FP8/INT8 tiles");
   using Shape = TileShape<TN, FUSE>;
   // bytes the TMA delivers per stage (the fused path writes the activation slot itself)
   constexpr uint32_t kTmaStageBytes = FUSE ? Shape::kXBytes : Shape::kStageBytes;
@@ -209,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int64_t x_row0 = static_cast<int64_t>(blockIdx.x) * kTileM;
   int64_t y_row0 = static_cast<int64_t>(blockIdx.y) * TN;
   int64_t m_end = p.M, n_end = p.N, c_off = 0;
-  if (p.expert_offsets) {
+  if constexpr (GROUPED) {
     // Grouped (mixture-of-experts) launch, Swap-AB: X = the weights of all
     // experts stacked [E N, K], Y = the tokens sorted by expert [T, K].
     // blockIdx.y enumerates the token tiles of expert 0, then expert 1, ...;
@@ -758,7 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float a = kInt8 ? static_cast<float>(static_cast<int32_t>(v[j])) : __uint_as_float(v[j]);
                     val = a * colsc[c0 + j] * bsn;
                   }
-                  val += bias_at(p, n - c_off);
+                  if constexpr (BIAS) val += bias_at(p, n - c_off);
                   p.C[idx] = __float2bfloat16_rn(val);
                   if (kInt8 && p.acc_out) p.acc_out[idx] = static_cast<int32_t>(v[j]);
                 }
@@ -790,7 +795,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       f[e] = a * asm_ * colsc[c0 + j8 + e];
                     }
                   }
-                  if (p.bias) {
+                  if constexpr (BIAS) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) f[e] += bias_at(p, n + e);
                   }
@@ -847,7 +852,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               float val;
               if (kBlocked) val = sf;
               else val = (kInt8 ? static_cast<float>(si) : sf) * colsc[j] * bsn;
-              val += bias_at(p, n);
+              if constexpr (BIAS) val += bias_at(p, n);
               p.C[m * N + n] = __float2bfloat16_rn(val);
               if (kInt8 && p.acc_out) p.acc_out[m * N + n] = si;
             }
@@ -878,7 +883,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * colsc[j4 + e];
               }
-              if (p.bias) {
+              if constexpr (BIAS) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) f[e] += bias_at(p, n + e);
               }
@@ -921,7 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               float val;
               if (kBlocked) val = sf;
               else val = (kInt8 ? static_cast<float>(si) : sf) * colsc[j0 + jj] * bsn;
-              val += bias_at(p, n - c_off);
+              if constexpr (BIAS) val += bias_at(p, n - c_off);
               p.C[m * p.N + (n - c_off)] = __float2bfloat16_rn(val);
               if (kInt8 && p.acc_out) p.acc_out[m * p.N + (n - c_off)] = si;
             }
@@ -952,7 +957,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * colsc[j0 + jj + e];
               }
-              if (p.bias) {
+              if constexpr (BIAS) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) f[e] += bias_at(p, n + e);
               }
@@ -1017,7 +1022,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float val;
             if (kBlocked) val = sf;
             else val = (kInt8 ? static_cast<float>(si) : sf) * colsc[j] * bsn;
-            val += bias_at(p, n);
+            if constexpr (BIAS) val += bias_at(p, n);
             p.C[m * N + n] = __float2bfloat16_rn(val);
             if (kInt8 && p.acc_out) p.acc_out[m * N + n] = si;
           }
@@ -1053,7 +1058,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int e = 0; e < 4; ++e) f[e] = f[e] * asm_ * colsc[j + e];
             }
-            if (p.bias) {
+            if constexpr (BIAS) {
 #pragma unroll
               for (int e = 0; e < 4; ++e) f[e] += bias_at(p, n + e);
             }
@@ -1119,7 +1124,7 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmParams p) 
 #pragma unroll
       for (int e = 0; e < 4; ++e) f[e] = f[e] * a * __ldg(p.b_s + n + e);
     }
-    if (p.bias) {
+    if (p.bias) {   // a separate pass: a runtime test costs nothing here
 #pragma unroll
       for (int e = 0; e < 4; ++e) f[e] += bias_at(p, n + e);
     }

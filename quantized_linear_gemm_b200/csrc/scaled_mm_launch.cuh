@@ -5,9 +5,9 @@
 
 namespace lq {
 
-template <int FMT, bool SWAP, int TN, bool FUSE = false>
+template <int FMT, bool SWAP, int TN, bool FUSE = false, bool GROUPED = false, bool BIAS = false>
 cudaError_t launch_tc(const GemmLaunch& l) {
-  auto kern = scaled_mm_tc_kernel<FMT, SWAP, TN, FUSE>;
+  auto kern = scaled_mm_tc_kernel<FMT, SWAP, TN, FUSE, GROUPED, BIAS>;
   static int configured = 0;   // max dynamic smem set once per instantiation and process
   if (configured < l.smem_bytes) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
@@ -42,8 +42,41 @@ cudaError_t launch_tc(const GemmLaunch& l) {
   return cudaLaunchKernelEx(&cfg, kern, l.tmX, l.tmY, l.p);
 }
 
+// The plain GEMM instantiations, with or without the bias epilogue.
+template <int FMT, bool BIAS>
+cudaError_t launch_dense(const GemmLaunch& l, int swap_ab, int tile_n) {
+  if (swap_ab) {
+    switch (tile_n) {
+      case 16: return launch_tc<FMT, true, 16, false, false, BIAS>(l);
+      case 32: return launch_tc<FMT, true, 32, false, false, BIAS>(l);
+      case 64: return launch_tc<FMT, true, 64, false, false, BIAS>(l);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  switch (tile_n) {
+    case 64: return launch_tc<FMT, false, 64, false, false, BIAS>(l);
+    case 128: return launch_tc<FMT, false, 128, false, false, BIAS>(l);
+    case 256:
+      if constexpr (!is_block_fmt(FMT)) return launch_tc<FMT, false, 256, false, false, BIAS>(l);
+      return cudaErrorInvalidValue;
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 template <int FMT>
 cudaError_t launch_format(const GemmLaunch& l, int swap_ab, int tile_n) {
+  if (l.grouped) {
+    if constexpr (!is_block_fmt(FMT)) {
+      if (!swap_ab) return cudaErrorInvalidValue;
+      switch (tile_n) {
+        case 16: return launch_tc<FMT, true, 16, false, true>(l);
+        case 32: return launch_tc<FMT, true, 32, false, true>(l);
+        case 64: return launch_tc<FMT, true, 64, false, true>(l);
+        default: return cudaErrorInvalidValue;
+      }
+    }
+    return cudaErrorInvalidValue;
+  }
   if (l.fuse) {
     if constexpr (!is_block_fmt(FMT)) {
       if (!swap_ab) return cudaErrorInvalidValue;
@@ -56,22 +89,7 @@ cudaError_t launch_format(const GemmLaunch& l, int swap_ab, int tile_n) {
     }
     return cudaErrorInvalidValue;
   }
-  if (swap_ab) {
-    switch (tile_n) {
-      case 16: return launch_tc<FMT, true, 16>(l);
-      case 32: return launch_tc<FMT, true, 32>(l);
-      case 64: return launch_tc<FMT, true, 64>(l);
-      default: return cudaErrorInvalidValue;
-    }
-  }
-  switch (tile_n) {
-    case 64: return launch_tc<FMT, false, 64>(l);
-    case 128: return launch_tc<FMT, false, 128>(l);
-    case 256:
-      if constexpr (!is_block_fmt(FMT)) return launch_tc<FMT, false, 256>(l);
-      return cudaErrorInvalidValue;
-    default: return cudaErrorInvalidValue;
-  }
+  return l.p.bias ? launch_dense<FMT, true>(l, swap_ab, tile_n) : launch_dense<FMT, false>(l, swap_ab, tile_n);
 }
 
 }  // namespace lq
