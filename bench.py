@@ -626,6 +626,8 @@ def main() -> None:
     gemm_gbs = wl.gemm_bytes / (ms_gemm * 1e-3) / 1e9
 
     # per-shape breakdown: R calls of one shape per graph, rotating weight copies
+    compute_bound = min(wl.ms) >= 256        # prefill configs: tensor-bound
+    tensor_peak = 2.0 * peaks["bf16_tflops_sustained"]
     per_shape = []
     for c in wl.calls:
         reps = max(args.per_shape_reps, len(wl.weights[c["layer"]]))
@@ -640,6 +642,7 @@ def main() -> None:
         per_shape.append({"layer": c["layer"], "M": c["M"], "N": c["N"], "K": c["K"], "us": round(ms * 1e3, 3),
                           "GB/s": round(b / (ms * 1e-3) / 1e9, 1), "TFLOP/s": round(2 * c["M"] * c["N"] * c["K"] / (ms * 1e-3) / 1e12, 2),
                           "frac_hbm": round(b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+                          "frac_tensor": round(2 * c["M"] * c["N"] * c["K"] / (ms * 1e-3) / 1e12 / tensor_peak, 3),
                           "variant": c["variant"].as_dict()})
         del g
 
@@ -720,6 +723,18 @@ def main() -> None:
                     "traffic_unit": "DRAM bytes per step of the fused launches (ncu)",
                     "algorithmic_bytes_per_step": step_bytes, "launches_per_step": wl.launches_per_step(fused=True),
                     "us_per_step": round(ms_step * 1e3, 2), "peak_source": peaks["source"]}
+    elif compute_bound:
+        # prefill: 2MNK flops against the 8-bit tensor-core peak (a kernel timed inside a long step:
+        # the sustained bf16 measurement times the nominal 8-bit / bf16 ratio of 2)
+        gemm_tflops = wl.flops / (ms_gemm * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": "scaled_mm (all launches of one step)",
+                    "achieved": round(gemm_tflops, 1), "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(gemm_tflops / tensor_peak, 4),
+                    "traffic": recorded_traffic(args.config, "scaled_mm"),
+                    "traffic_unit": "DRAM bytes per step of scaled_mm launches (ncu)",
+                    "algorithmic_flops_per_step": wl.flops, "launches_per_step": wl.launches_per_step(quant=False),
+                    "us_per_step": round(ms_gemm * 1e3, 2),
+                    "peak_source": f"{peaks['source']} bf16 sustained x 2 (nominal 8-bit : bf16 tensor ratio)"}
     else:
         roofline = {"bound": "hbm", "kernel": "scaled_mm (all launches of one step)",
                     "achieved": round(gemm_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
