@@ -193,6 +193,60 @@ def test_deterministic_and_graph_replay(cuda_device, fmt):
     assert lq.device_status(0) == 0
 
 
+def _random_operands(fmt, M, N, K, seed):
+    """Random finite codes and positive scales, generated on the device (a
+    run-to-run invariant needs no reference values)."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+
+    def codes(rows):
+        if fmt == lq.W8A8_INT8:
+            return torch.randint(-127, 128, (rows, K), generator=g, device="cuda", dtype=torch.int8)
+        q = torch.randint(0, 256, (rows, K), generator=g, device="cuda", dtype=torch.uint8)
+        return torch.where((q & 0x7F) == 0x7F, torch.zeros_like(q), q)   # no NaN codes
+
+    def scales(shape):
+        return torch.rand(shape, generator=g, device="cuda") * 1e-3 + 1e-5
+
+    block = fmt == lq.BLOCK_FP8
+    A, B = codes(M), codes(N)
+    sa = scales((M, K // 128) if block else (M,))
+    sb = scales((N // 128, K // 128) if block else (N,))
+    return A, sa, B, sb
+
+
+DEEP_K = [  # (M, N, K, variant): Qwen3-32B down (K = 25600, 200 K tiles) in prefill and decode tiles
+    (2048, 1024, 25600, dict(swap_ab=0, tile_n=128, split_k=1, stages=4, reduce=2, pdl=2)),
+    (2048, 1024, 25600, dict(swap_ab=0, tile_n=64, split_k=1, stages=3, reduce=2, pdl=2)),
+    (256, 1024, 25600, dict(swap_ab=0, tile_n=128, split_k=4, stages=3, reduce=2, pdl=2)),
+    (8, 5120, 25600, dict(swap_ab=1, tile_n=16, split_k=8, stages=4, reduce=2, pdl=2)),
+    (8, 5120, 25600, dict(swap_ab=1, tile_n=16, split_k=8, stages=4, reduce=0, pdl=2)),
+    (8, 5120, 25600, None),
+]
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
+@pytest.mark.parametrize("M,N,K,vd", DEEP_K, ids=lambda x: None if not isinstance(x, (dict, type(None))) else
+                         ("table" if x is None else _vid(x)))
+def test_deep_k_bitwise_reproducible(cuda_device, fmt, M, N, K, vd):
+    """Run to run the same bits at the deepest K of the workloads: every
+    variant sums its partial products and its splits in one fixed order, so
+    repeated calls (eager, back to back on one stream) must agree bit for bit."""
+    A, sa, B, sb = _random_operands(fmt, M, N, K, seed=M + N)
+    v = None if vd is None else lq.make_variant(**vd)
+    if v is not None:
+        lq.reserve_workspace(0, lq.workspace_bytes(fmt, M, N, K, v))
+    C0 = lq.scaled_mm(fmt, A, sa, B, sb, variant=v).clone()
+    out = torch.empty_like(C0)
+    for _ in range(3):
+        out.zero_()
+        lq.scaled_mm(fmt, A, sa, B, sb, C=out, variant=v)
+        torch.cuda.synchronize()
+        assert torch.equal(out, C0)
+    assert torch.isfinite(C0.float()).all()
+    assert lq.device_status(0) == 0
+
+
 def test_default_variant_selection_runs(cuda_device):
     """variant = NULL takes the table / heuristic choice."""
     for fmt in FMTS:
