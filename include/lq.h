@@ -147,7 +147,13 @@ typedef struct {
  * before any launch; LQ_ERR_WORKSPACE when split_k > 1 needs a larger
  * workspace while `stream` is capturing; LQ_ERR_CUDA when a launch fails.
  * A Split-K call with reduce 0 or 1 uses the library's per-device workspace:
- * such calls on different streams of one device must not overlap in time.
+ * such calls on different streams of one device must not overlap in time,
+ * and must not be issued from several host threads at once: a call that
+ * grows the workspace frees the old one, which a call being issued at the
+ * same moment by another thread may still be about to use.  Call
+ * lq_reserve_workspace with the largest size first to rule growth out.
+ * Calls with split_k == 1 or reduce 2 (the dispatch table's choices) use no
+ * workspace and have neither restriction.
  */
 lq_status lq_scaled_mm(lq_fmt fmt, const void *A, const float *a_scales,
                        const void *B, const float *b_scales, void *C,
