@@ -31,8 +31,9 @@
  *    pointer of the current CUDA device, owned by the caller.  Arrays are
  *    dense and row-major with the shapes given below.
  *  - A is [M, K], one row per token.  B is stored [N, K] (one row per output
- *    channel, K contiguous), i.e. the pages' logical b[k, n] transposed, as a
- *    linear layer stores its weight.  C is [M, N] bf16.
+ *    channel, K contiguous), as a linear layer stores its weight: the
+ *    logical b[k, n] of the techfeed.io summary's code sample (section
+ *    "何が面白いのか"), transposed.  C is [M, N] bf16.
  *  - e4m3 codes are OCP E4M3 "fn" bytes; int8 codes are two's complement.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream) and never synchronise.  They may be captured into a
@@ -165,7 +166,7 @@ lq_status lq_scaled_mm(lq_fmt fmt, const void *A, const float *a_scales,
  * scaled accumulator and the bias added in fp32 before the one rounding to
  * bf16.  bias: [N] bf16 (device, 2-byte aligned, not NULL).  Same formats,
  * arguments, variants and errors as lq_scaled_mm; K == 0 is refused with
- * LQ_ERR_UNSUPPORTED_SHAPE.  The pages have no bias (a linear layer of the
+ * LQ_ERR_UNSUPPORTED_SHAPE.  The blog has no bias (a linear layer of the
  * served models has none); it serves layers that do, and the N-sliced
  * multi-GPU linear, whose shards each add their slice of it.
  */
@@ -176,7 +177,7 @@ lq_status lq_scaled_mm_bias(lq_fmt fmt, const void *A, const float *a_scales,
 
 /*
  * Grouped (mixture-of-experts) scaled_mm: one launch for all experts, each
- * an ordinary FP8_Dynamic / W8A8_INT8 linear layer (the pages' next target:
+ * an ordinary FP8_Dynamic / W8A8_INT8 linear layer (a next target named by
  * ai-radar.it, "Helion in vLLM: il tuning dei GEMM diventa ricerca, non
  * artigianato GPU", section "Oltre Hopper: Blackwell, AMD, TPU e il
  * perimetro del fork": many small experts, where Split-K and Swap-AB matter
@@ -224,7 +225,7 @@ lq_status lq_scaled_mm_i32acc(const void *A, const float *a_scales,
 /*
  * Quantize the activations and multiply, in one kernel where possible: the
  * per-token dynamic quantization of lq_quant_per_token fused with
- * lq_scaled_mm (the in-GEMM activation quantization that the pages' fused
+ * lq_scaled_mm (the in-GEMM activation quantization that the report's fused
  * quantization kernels motivate; 24-ai.news report, section "kernels
  * integrated into vLLM", and the blog's aim of fewer kernel calls per
  * forward pass).
@@ -270,7 +271,7 @@ int64_t lq_set_fuse_limit(int64_t max_slice_bytes);
  * latency-critical services that must not allocate or synchronise after
  * start-up.  lq_scaled_mm may allocate its per-device state and Split-K
  * workspace on first use; this entry point never calls cudaMalloc, cudaFree
- * or any allocating routine.  The pages have no counterpart: it is an
+ * or any allocating routine.  The blog has no counterpart: it is an
  * interface of this library only.
  *
  * Same arguments, layouts and results as lq_scaled_mm.  Differences:
@@ -327,7 +328,7 @@ lq_status lq_quant_per_token_group128(const void *x, void *q, float *scales,
  * activations quantizes them in the same pass (the blog's integrated kernels
  * rms_norm_dynamic_per_token_quant, rms_norm_per_block_quant,
  * silu_and_mul_dynamic_per_token_quant and silu_and_mul_per_block_quant:
- * 24-ai.news report, section "kernels integrated into vLLM").  The pages name
+ * 24-ai.news report, section "kernels integrated into vLLM").  The report names
  * them only; the value quantized is the bf16 output of a Qwen3-style layer,
  * with each rounding fixed so that codes and scales are reproducible bit for
  * bit:

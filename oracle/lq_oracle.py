@@ -24,7 +24,7 @@ Split-K and Swap-AB variants as rewrites of the *same* product, so the oracle
 has one definition of C and only uses split / transposed loop orders as
 self-checks (``acc_split_k``, ``acc_swap_ab``).
 
-The pages leave the numeric details open.  Readings adopted here (each listed
+The blog and its re-reports leave the numeric details open.  Readings adopted here (each listed
 in the design notes of the repository):
 
 * FP8 means OCP e4m3fn (finite max 448, no infinities, NaN = S.1111.111).
@@ -33,8 +33,9 @@ in the design notes of the repository):
 * A quantization scale is s = max(fp32(amax / Q), 2^-126) with Q = 448 (e4m3)
   or 127 (int8), amax the largest magnitude over the scale's group, and the
   code is enc(fp32(x / s)) with a correctly rounded fp32 division.
-* Weights are stored [N, K] (output channel major, K contiguous); the pages'
-  logical operand is b[k, n].
+* Weights are stored [N, K] (output channel major, K contiguous); the code
+  sample of the techfeed.io summary (section "何が面白いのか") indexes the
+  logical operand as b[k, n].
 * Output C is the exact product rounded once; the oracle returns it in fp64.
 
 Exactness.  Every finite e4m3 value is an integer multiple of 2^-9 whose

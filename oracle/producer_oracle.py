@@ -13,7 +13,7 @@ The 24-ai.news report "HelionがvLLMに統合：PyTorchネイティブDSLがCUDA
 lists, among the nine kernels of the FP8 forward pass,
 ``rms_norm_dynamic_per_token_quant``, ``silu_and_mul_dynamic_per_token_quant``,
 ``rms_norm_per_block_quant`` and ``silu_and_mul_per_block_quant``; section
-"個別カーネルレベルのパフォーマンス" gives their speed-ups.  The pages name the
+"個別カーネルレベルのパフォーマンス" gives their speed-ups.  The report names the
 kernels and nothing more.  The readings below are the plain ones, in the
 precision of a bf16 Qwen3 forward pass, and each intermediate rounding is
 written out so that the kernels can match the codes bit for bit:

@@ -9,7 +9,7 @@ Where it comes from
 The 24-ai.news report "HelionがvLLMに統合：PyTorchネイティブDSLがCUDAカーネルを
 代替し、Qwen3モデルのFP8推論を高速化", section "実際の制限事項", notes that the
 per-group quantization kernel is not yet compatible with the UE8M0 scale format
-that DeepGEMM requires on B200.  The pages do not define UE8M0.  Reading used
+that DeepGEMM requires on B200.  The report does not define UE8M0.  Reading used
 here (the OCP microscaling E8M0 scale type): an unsigned byte b holding a
 power of two, value 2^(b - 127) for b in 0..254 (255 is NaN and never
 produced).  A UE8M0 scale is the smallest power of two s with amax / s <= Q

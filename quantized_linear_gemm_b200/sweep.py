@@ -7,9 +7,10 @@ For every (format, token bucket, N, K) of the Qwen3 decode / prefill shapes
 this enumerates the variant space - Swap-AB or Standard, tile_n, split_k,
 the reduction mode, ring depth and launch mode - times each candidate under
 CUDA-graph replay with weight copies rotated so that every call reads its
-weights from HBM, and keeps the fastest.  It replaces the pages' offline
-autotuner (an LLM-seeded tree search) by exhaustive search: the space is
-small and discrete.
+weights from HBM, and keeps the fastest.  It replaces the offline autotuner
+of the techfeed.io summary of the Helion blog (section "オートチューニングの仕組み":
+an LLM-seeded tree search) by exhaustive search: the space is small and
+discrete.
 
 The result is a text table (one line per key, the format that
 lq_load_dispatch_table reads) and, with --inc, the compiled-in table

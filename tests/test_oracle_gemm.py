@@ -1,6 +1,6 @@
 """Pins of the oracle's scaled_mm: hand cases, exact-rational brute force with
 an independent decoder, the exactness bound, and the invariants that the
-variants of the pages must satisfy (Split-K and Swap-AB compute the same C;
+blog's variants must satisfy (Split-K and Swap-AB compute the same C;
 doubling a scale doubles C; identity weights give back dequant(A))."""
 
 import json
