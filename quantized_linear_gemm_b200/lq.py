@@ -1,8 +1,9 @@
 """Python binding of liblq (ctypes).  Argument marshalling only.
 
-Every function here checks tensor devices / dtypes / contiguity, then calls
-the C function of the same name in ``liblq.so`` on torch's current CUDA
-stream.  All arithmetic runs in the library's CUDA kernels; there is no
+Every function here checks its tensors (dtype, rank, contiguity, the exact
+shape the C function reads or writes, and one device: the current CUDA
+device), then calls the C function of the same name in ``liblq.so`` on
+torch's current CUDA stream.  All arithmetic runs in the library's CUDA kernels; there is no
 fallback.  If ``liblq.so`` is missing the first call raises.
 """
 
@@ -156,39 +157,88 @@ def _ptr(t: torch.Tensor | None) -> int | None:
     return None if t is None else t.data_ptr()
 
 
-def _need(t: torch.Tensor, name: str, dtypes, ndim: int) -> None:
+_DEVICE_TYPE = "cuda"   # the only device type the library runs on
+
+_CODE_DTYPES = (torch.uint8, torch.int8, torch.float8_e4m3fn)   # one byte per code
+
+
+def _need(t: torch.Tensor, name: str, dtypes, ndim: int, shape=None) -> None:
+    """t is a contiguous ndim-d tensor of one of `dtypes` on the GPU, of
+    exactly `shape` when given (the C ABI reads that many elements)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a tensor")
-    if t.device.type != "cuda":
+    if t.device.type != _DEVICE_TYPE:
         raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype not in dtypes:
         raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
     if t.dim() != ndim or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
-_CODE_DTYPES = (torch.uint8, torch.int8, torch.float8_e4m3fn)
+def _one_device(*ts) -> None:
+    """All tensors on one device, the current CUDA device (the library
+    launches on the current device and dereferences every pointer there)."""
+    ts = [t for t in ts if t is not None]
+    dev = ts[0].device
+    for t in ts[1:]:
+        if t.device != dev:
+            raise ValueError(f"tensors on different devices: {dev} and {t.device}")
+    if dev.type == "cuda" and dev.index != torch.cuda.current_device():
+        raise ValueError(f"tensors are on {dev} but the current CUDA device is cuda:{torch.cuda.current_device()}")
+
+
+def _scales_spec(f: int, M: int, N: int, K: int):
+    """dtype and shapes of (a_scales, b_scales) for format f: per token and
+    per output channel, or per 1 x 128 group and per 128 x 128 block."""
+    if f in (BLOCK_FP8, BLOCK_FP8_UE8M0):
+        dt = (torch.uint8,) if f == BLOCK_FP8_UE8M0 else (torch.float32,)
+        return dt, (M, K // 128), (N // 128, K // 128)
+    return (torch.float32,), (M,), (N,)
+
+
+def _gemm_operands(f: int, A, a_scales, B, b_scales, C):
+    """Check the operands of one [M, K] x [N, K]^T product; returns (M, N, K)."""
+    _need(A, "A", _CODE_DTYPES, 2)
+    _need(B, "B", _CODE_DTYPES, 2)
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] != K:
+        raise ValueError("A and B disagree on K")
+    dt, sa, sb = _scales_spec(f, M, N, K)
+    _need(a_scales, "a_scales", dt, len(sa), sa)
+    _need(b_scales, "b_scales", dt, len(sb), sb)
+    if C is not None:
+        _need(C, "C", (torch.bfloat16,), 2, (M, N))
+    _one_device(A, a_scales, B, b_scales, C)
+    return M, N, K
+
+
+def _outputs(device, q, q_shape, q_dtype, scales, s_shape, s_dtype=torch.float32):
+    """Allocate the codes / scales outputs, or check the caller's."""
+    if q is None:
+        q = torch.empty(q_shape, dtype=q_dtype, device=device)
+    else:
+        _need(q, "q", _CODE_DTYPES, len(q_shape), q_shape)
+    if scales is None:
+        scales = torch.empty(s_shape, dtype=s_dtype, device=device)
+    else:
+        _need(scales, "scales", (s_dtype,), len(s_shape), s_shape)
+    return q, scales
+
+
+def _code_dtype(f: int):
+    return torch.int8 if f == W8A8_INT8 else torch.uint8
 
 
 def scaled_mm(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor, b_scales: torch.Tensor,
               C: torch.Tensor | None = None, variant: Variant | None = None, stream=None) -> torch.Tensor:
     """C[M, N] (bf16) = dequant(A[M, K]) @ dequant(B[N, K])^T through ``lq_scaled_mm``."""
     f = _fmt(fmt)
-    _need(A, "A", _CODE_DTYPES, 2)
-    _need(B, "B", _CODE_DTYPES, 2)
-    block = f in (BLOCK_FP8, BLOCK_FP8_UE8M0)
-    sdt = (torch.uint8,) if f == BLOCK_FP8_UE8M0 else (torch.float32,)
-    _need(a_scales, "a_scales", sdt, 2 if block else 1)
-    _need(b_scales, "b_scales", sdt, 2 if block else 1)
-    M, K = A.shape
-    N = B.shape[0]
-    if B.shape[1] != K:
-        raise ValueError("A and B disagree on K")
+    M, N, K = _gemm_operands(f, A, a_scales, B, b_scales, C)
     if C is None:
         C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
-    _need(C, "C", (torch.bfloat16,), 2)
-    if tuple(C.shape) != (M, N):
-        raise ValueError("C has the wrong shape")
     rc = lib().lq_scaled_mm(f, _ptr(A), _ptr(a_scales), _ptr(B), _ptr(b_scales), _ptr(C), M, N, K,
                             ctypes.byref(variant) if variant is not None else None, _stream(stream))
     _check("lq_scaled_mm", rc)
@@ -204,12 +254,14 @@ def quant_scaled_mm(fmt, x: torch.Tensor, B: torch.Tensor, b_scales: torch.Tenso
     _need(B, "B", _CODE_DTYPES, 2)
     M, K = x.shape
     N = B.shape[0]
+    if B.shape[1] != K:
+        raise ValueError("x and B disagree on K")
+    _need(b_scales, "b_scales", (torch.float32,), 1, (N,))
     if C is None:
         C = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    if q is None:
-        q = torch.empty((M, K), dtype=torch.int8 if f == W8A8_INT8 else torch.uint8, device=x.device)
-    if s is None:
-        s = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _need(C, "C", (torch.bfloat16,), 2, (M, N))
+    q, s = _outputs(x.device, q, (M, K), _code_dtype(f), s, (M,))
+    _one_device(x, B, b_scales, C, q, s)
     rc = lib().lq_quant_scaled_mm(f, _ptr(x), _ptr(B), _ptr(b_scales), _ptr(C), _ptr(q), _ptr(s), M, N, K,
                                   ctypes.byref(variant) if variant is not None else None, _stream(stream))
     _check("lq_quant_scaled_mm", rc)
@@ -221,13 +273,9 @@ def scaled_mm_bias(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Tensor
                    stream=None) -> torch.Tensor:
     """``lq_scaled_mm_bias``: scaled_mm plus a bf16 bias [N] added before the rounding."""
     f = _fmt(fmt)
-    _need(A, "A", _CODE_DTYPES, 2)
-    _need(B, "B", _CODE_DTYPES, 2)
-    _need(bias, "bias", (torch.bfloat16,), 1)
-    M, K = A.shape
-    N = B.shape[0]
-    if bias.numel() != N:
-        raise ValueError("bias must hold N values")
+    M, N, K = _gemm_operands(f, A, a_scales, B, b_scales, C)
+    _need(bias, "bias", (torch.bfloat16,), 1, (N,))
+    _one_device(A, bias)
     if C is None:
         C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     rc = lib().lq_scaled_mm_bias(f, _ptr(A), _ptr(a_scales), _ptr(B), _ptr(b_scales), _ptr(bias), _ptr(C), M, N, K,
@@ -245,15 +293,17 @@ def grouped_scaled_mm(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Ten
     f = _fmt(fmt)
     _need(A, "A", _CODE_DTYPES, 2)
     _need(B, "B", _CODE_DTYPES, 3)
-    _need(a_scales, "a_scales", (torch.float32,), 1)
-    _need(b_scales, "b_scales", (torch.float32,), 2)
-    _need(expert_offsets, "expert_offsets", (torch.int32,), 1)
     T, K = A.shape
-    E, N, _ = B.shape
-    if expert_offsets.numel() != E + 1:
-        raise ValueError("expert_offsets must hold E + 1 entries")
+    E, N, KB = B.shape
+    if KB != K:
+        raise ValueError("A and B disagree on K")
+    _need(a_scales, "a_scales", (torch.float32,), 1, (T,))
+    _need(b_scales, "b_scales", (torch.float32,), 2, (E, N))
+    _need(expert_offsets, "expert_offsets", (torch.int32,), 1, (E + 1,))
     if C is None:
         C = torch.empty((T, N), dtype=torch.bfloat16, device=A.device)
+    _need(C, "C", (torch.bfloat16,), 2, (T, N))
+    _one_device(A, a_scales, B, b_scales, expert_offsets, C)
     rc = lib().lq_grouped_scaled_mm(f, _ptr(A), _ptr(a_scales), _ptr(B), _ptr(b_scales), _ptr(C),
                                     _ptr(expert_offsets), E, T, N, K,
                                     ctypes.byref(variant) if variant is not None else None, _stream(stream))
@@ -266,13 +316,9 @@ def scaled_mm_noalloc(fmt, A: torch.Tensor, a_scales: torch.Tensor, B: torch.Ten
     """``lq_scaled_mm_noalloc``: scaled_mm whose Split-K partials use the library's
     fixed device array instead of allocated workspace (see include/lq.h)."""
     f = _fmt(fmt)
-    _need(A, "A", _CODE_DTYPES, 2)
-    _need(B, "B", _CODE_DTYPES, 2)
-    M, K = A.shape
-    N = B.shape[0]
+    M, N, K = _gemm_operands(f, A, a_scales, B, b_scales, C)
     if C is None:
         C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
-    _need(C, "C", (torch.bfloat16,), 2)
     rc = lib().lq_scaled_mm_noalloc(f, _ptr(A), _ptr(a_scales), _ptr(B), _ptr(b_scales), _ptr(C), M, N, K,
                                     ctypes.byref(variant) if variant is not None else None, _stream(stream))
     _check("lq_scaled_mm_noalloc", rc)
@@ -283,13 +329,13 @@ def scaled_mm_i32acc(A, a_scales, B, b_scales, C=None, acc=None, variant: Varian
     """W8A8_INT8 scaled_mm that also returns the exact int32 accumulators."""
     _need(A, "A", (torch.int8,), 2)
     _need(B, "B", (torch.int8,), 2)
-    M, K = A.shape
-    N = B.shape[0]
+    M, N, K = _gemm_operands(W8A8_INT8, A, a_scales, B, b_scales, C)
     if C is None:
         C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     if acc is None:
         acc = torch.empty((M, N), dtype=torch.int32, device=A.device)
-    _need(acc, "acc", (torch.int32,), 2)
+    _need(acc, "acc", (torch.int32,), 2, (M, N))
+    _one_device(A, acc)
     rc = lib().lq_scaled_mm_i32acc(_ptr(A), _ptr(a_scales), _ptr(B), _ptr(b_scales), _ptr(C), _ptr(acc), M, N, K,
                                    ctypes.byref(variant) if variant is not None else None, _stream(stream))
     _check("lq_scaled_mm_i32acc", rc)
@@ -302,10 +348,8 @@ def quant_per_token(fmt, x: torch.Tensor, q: torch.Tensor | None = None, scales:
     f = _fmt(fmt)
     _need(x, "x", (torch.bfloat16,), 2)
     M, K = x.shape
-    if q is None:
-        q = torch.empty((M, K), dtype=torch.int8 if f == W8A8_INT8 else torch.uint8, device=x.device)
-    if scales is None:
-        scales = torch.empty((M,), dtype=torch.float32, device=x.device)
+    q, scales = _outputs(x.device, q, (M, K), _code_dtype(f), scales, (M,))
+    _one_device(x, q, scales)
     rc = lib().lq_quant_per_token(f, _ptr(x), _ptr(q), _ptr(scales), M, K, _stream(stream))
     _check("lq_quant_per_token", rc)
     return q, scales
@@ -315,22 +359,24 @@ def quant_per_token_group128(x: torch.Tensor, q=None, scales=None, stream=None):
     """(e4m3 codes [M, K], scales [M, K/128]) of a bf16 [M, K] tensor."""
     _need(x, "x", (torch.bfloat16,), 2)
     M, K = x.shape
-    if q is None:
-        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
-    if scales is None:
-        scales = torch.empty((M, max(K // 128, 0)), dtype=torch.float32, device=x.device)
+    q, scales = _outputs(x.device, q, (M, K), torch.uint8, scales, (M, max(K // 128, 0)))
+    _one_device(x, q, scales)
     rc = lib().lq_quant_per_token_group128(_ptr(x), _ptr(q), _ptr(scales), M, K, _stream(stream))
     _check("lq_quant_per_token_group128", rc)
     return q, scales
 
 
 def _producer_out(f: int, M: int, K: int, per_block: bool, device, q, scales):
-    if q is None:
-        q = torch.empty((M, K), dtype=torch.int8 if f == W8A8_INT8 else torch.uint8, device=device)
-    if scales is None:
-        shape = (M, max(K // 128, 0)) if per_block else (M,)
-        scales = torch.empty(shape, dtype=torch.float32, device=device)
-    return q, scales
+    return _outputs(device, q, (M, K), _code_dtype(f), scales, (M, max(K // 128, 0)) if per_block else (M,))
+
+
+def _rms_inputs(x, weight, residual):
+    _need(x, "x", (torch.bfloat16,), 2)
+    M, K = x.shape
+    _need(weight, "weight", (torch.bfloat16,), 1, (K,))
+    if residual is not None:
+        _need(residual, "residual", (torch.bfloat16,), 2, (M, K))
+    return M, K
 
 
 def rms_norm_dynamic_per_token_quant(fmt, x: torch.Tensor, weight: torch.Tensor, eps: float, residual=None,
@@ -338,12 +384,9 @@ def rms_norm_dynamic_per_token_quant(fmt, x: torch.Tensor, weight: torch.Tensor,
     """(codes [M, K], scales [M]) of RMSNorm(x [+ residual]) * weight; the
     residual, when given, is overwritten with x + residual."""
     f = _fmt(fmt)
-    _need(x, "x", (torch.bfloat16,), 2)
-    _need(weight, "weight", (torch.bfloat16,), 1)
-    if residual is not None:
-        _need(residual, "residual", (torch.bfloat16,), 2)
-    M, K = x.shape
+    M, K = _rms_inputs(x, weight, residual)
     q, scales = _producer_out(f, M, K, False, x.device, q, scales)
+    _one_device(x, weight, residual, q, scales)
     rc = lib().lq_rms_norm_dynamic_per_token_quant(f, _ptr(x), _ptr(residual) if residual is not None else None,
                                                    _ptr(weight), float(eps), _ptr(q), _ptr(scales), M, K,
                                                    _stream(stream))
@@ -354,27 +397,29 @@ def rms_norm_dynamic_per_token_quant(fmt, x: torch.Tensor, weight: torch.Tensor,
 def rms_norm_per_block_quant(x: torch.Tensor, weight: torch.Tensor, eps: float, residual=None, q=None,
                              scales=None, stream=None):
     """(e4m3 codes [M, K], scales [M, K/128]) of RMSNorm(x [+ residual]) * weight."""
-    _need(x, "x", (torch.bfloat16,), 2)
-    _need(weight, "weight", (torch.bfloat16,), 1)
-    if residual is not None:
-        _need(residual, "residual", (torch.bfloat16,), 2)
-    M, K = x.shape
+    M, K = _rms_inputs(x, weight, residual)
     q, scales = _producer_out(FP8_DYNAMIC, M, K, True, x.device, q, scales)
+    _one_device(x, weight, residual, q, scales)
     rc = lib().lq_rms_norm_per_block_quant(_ptr(x), _ptr(residual) if residual is not None else None, _ptr(weight),
                                            float(eps), _ptr(q), _ptr(scales), M, K, _stream(stream))
     _check("lq_rms_norm_per_block_quant", rc)
     return q, scales
 
 
-def silu_and_mul_dynamic_per_token_quant(fmt, gate_up: torch.Tensor, q=None, scales=None, stream=None):
-    """(codes [M, I], scales [M]) of silu(gate_up[:, :I]) * gate_up[:, I:]."""
-    f = _fmt(fmt)
+def _gate_up_width(gate_up) -> tuple[int, int]:
     _need(gate_up, "gate_up", (torch.bfloat16,), 2)
     M, two_i = gate_up.shape
     if two_i % 2:
         raise ValueError("gate_up must have an even number of columns ([g | u])")
-    I = two_i // 2
+    return M, two_i // 2
+
+
+def silu_and_mul_dynamic_per_token_quant(fmt, gate_up: torch.Tensor, q=None, scales=None, stream=None):
+    """(codes [M, I], scales [M]) of silu(gate_up[:, :I]) * gate_up[:, I:]."""
+    f = _fmt(fmt)
+    M, I = _gate_up_width(gate_up)
     q, scales = _producer_out(f, M, I, False, gate_up.device, q, scales)
+    _one_device(gate_up, q, scales)
     rc = lib().lq_silu_and_mul_dynamic_per_token_quant(f, _ptr(gate_up), _ptr(q), _ptr(scales), M, I,
                                                        _stream(stream))
     _check("lq_silu_and_mul_dynamic_per_token_quant", rc)
@@ -383,12 +428,9 @@ def silu_and_mul_dynamic_per_token_quant(fmt, gate_up: torch.Tensor, q=None, sca
 
 def silu_and_mul_per_block_quant(gate_up: torch.Tensor, q=None, scales=None, stream=None):
     """(e4m3 codes [M, I], scales [M, I/128]) of silu(g) * u."""
-    _need(gate_up, "gate_up", (torch.bfloat16,), 2)
-    M, two_i = gate_up.shape
-    if two_i % 2:
-        raise ValueError("gate_up must have an even number of columns ([g | u])")
-    I = two_i // 2
+    M, I = _gate_up_width(gate_up)
     q, scales = _producer_out(FP8_DYNAMIC, M, I, True, gate_up.device, q, scales)
+    _one_device(gate_up, q, scales)
     rc = lib().lq_silu_and_mul_per_block_quant(_ptr(gate_up), _ptr(q), _ptr(scales), M, I, _stream(stream))
     _check("lq_silu_and_mul_per_block_quant", rc)
     return q, scales
@@ -398,10 +440,8 @@ def quant_per_token_group128_ue8m0(x: torch.Tensor, q=None, scales=None, stream=
     """(e4m3 codes [M, K], UE8M0 scale bytes [M, K/128]) of a bf16 [M, K] tensor."""
     _need(x, "x", (torch.bfloat16,), 2)
     M, K = x.shape
-    if q is None:
-        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
-    if scales is None:
-        scales = torch.empty((M, max(K // 128, 0)), dtype=torch.uint8, device=x.device)
+    q, scales = _outputs(x.device, q, (M, K), torch.uint8, scales, (M, max(K // 128, 0)), torch.uint8)
+    _one_device(x, q, scales)
     rc = lib().lq_quant_per_token_group128_ue8m0(_ptr(x), _ptr(q), _ptr(scales), M, K, _stream(stream))
     _check("lq_quant_per_token_group128_ue8m0", rc)
     return q, scales
@@ -411,10 +451,9 @@ def quant_weight_block128_ue8m0(w: torch.Tensor, q=None, scales=None, stream=Non
     """(e4m3 codes [N, K], UE8M0 scale bytes [N/128, K/128]) of a bf16 weight [N, K]."""
     _need(w, "w", (torch.bfloat16,), 2)
     N, K = w.shape
-    if q is None:
-        q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
-    if scales is None:
-        scales = torch.empty((max(N // 128, 0), max(K // 128, 0)), dtype=torch.uint8, device=w.device)
+    q, scales = _outputs(w.device, q, (N, K), torch.uint8, scales, (max(N // 128, 0), max(K // 128, 0)),
+                         torch.uint8)
+    _one_device(w, q, scales)
     rc = lib().lq_quant_weight_block128_ue8m0(_ptr(w), _ptr(q), _ptr(scales), N, K, _stream(stream))
     _check("lq_quant_weight_block128_ue8m0", rc)
     return q, scales
@@ -424,10 +463,8 @@ def quant_weight_block128(w: torch.Tensor, q=None, scales=None, stream=None):
     """(e4m3 codes [N, K], scales [N/128, K/128]) of a bf16 weight [N, K]."""
     _need(w, "w", (torch.bfloat16,), 2)
     N, K = w.shape
-    if q is None:
-        q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
-    if scales is None:
-        scales = torch.empty((max(N // 128, 0), max(K // 128, 0)), dtype=torch.float32, device=w.device)
+    q, scales = _outputs(w.device, q, (N, K), torch.uint8, scales, (max(N // 128, 0), max(K // 128, 0)))
+    _one_device(w, q, scales)
     rc = lib().lq_quant_weight_block128(_ptr(w), _ptr(q), _ptr(scales), N, K, _stream(stream))
     _check("lq_quant_weight_block128", rc)
     return q, scales
