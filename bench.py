@@ -531,8 +531,9 @@ def run_reference(args) -> None:
         secs += dt
         nbytes += b
     value = nbytes / secs / 1e9
+    lo, hi = min(cols.values()), max(cols.values())
     sample = (f"{cfg}: per step one linear (cycling {','.join(names)}) at M={M}, exact product for the first "
-              f"{min(cols.values())}-{max(cols.values())} output channels; numpy int64 matmul, single thread")
+              f"{lo if lo == hi else f'{lo}-{hi}'} output channels; numpy int64 matmul, single thread")
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE[fmt],
