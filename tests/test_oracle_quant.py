@@ -1,5 +1,7 @@
 """Pins of the oracle's quantizers: hand-worked rows, the scale floor, the
-amax element, and the dequantization error bound that the rounding implies."""
+amax element, the dequantization error bound that the rounding implies, and
+rows where only the correctly rounded quotient x / s (not x * (1 / s)) gives
+the right code, checked in exact rational arithmetic."""
 
 import json
 import os
@@ -131,3 +133,115 @@ def test_per_channel_weight_is_per_row():
     assert s.shape == (5,)
     for n in range(5):
         assert s[n] == np.float32(np.float32(np.max(np.abs(w[n]))) / np.float32(127.0))
+
+
+# ---------------------------------------------------------------------------
+# The code is enc(RN32(x / s)), the correctly rounded quotient, not
+# x * RN32(1 / s).  The two differ in the last fp32 bit for some x, and the
+# code differs when that bit straddles a rounding boundary of the code grid.
+# The hand rows above use power-of-two scales, where both agree; these rows
+# are found by a search over bf16 values and checked in exact rational
+# arithmetic (an fp32 rounding and both encoders written out here, apart from
+# the oracle's).
+
+from fractions import Fraction  # noqa: E402
+
+import torch  # noqa: E402
+
+
+def _rn32(f: Fraction) -> Fraction:
+    """Nearest fp32 value of a rational (ties to even; normal and subnormal range)."""
+    if f == 0:
+        return Fraction(0)
+    sign, a = (-1, -f) if f < 0 else (1, f)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    quantum = Fraction(2) ** (max(e, -126) - 23)
+    n, rem = divmod(a / quantum, 1)
+    n = int(n)
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2):
+        n += 1
+    return sign * n * quantum
+
+
+def _e4m3_exact(y: Fraction) -> Fraction:
+    """Value of the e4m3 code of y: round to nearest even on the 3-bit
+    significand (subnormal quantum 2^-9), saturating at +-448."""
+    if y == 0:
+        return Fraction(0)
+    sign, a = (-1, -y) if y < 0 else (1, y)
+    if a >= 448:
+        return sign * Fraction(448)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    quantum = Fraction(2) ** (max(e, -6) - 3)
+    n, rem = divmod(a / quantum, 1)
+    n = int(n)
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2):
+        n += 1
+    return sign * min(Fraction(448), n * quantum)
+
+
+def _int8_exact(y: Fraction) -> int:
+    return max(-127, min(127, round(y)))   # Fraction rounds half to even
+
+
+def _bf16_grid():
+    bits = np.arange(0x0080, 0x7F80, dtype=np.uint32)   # every positive normal bf16
+    return (bits << 16).view(np.float32)
+
+
+def _straddling_rows(fmt, limit=16):
+    """(amax, x) bf16 pairs, |x| <= amax, whose codes under x / s and under
+    x * (1 / s) differ (found with numpy fp32 arithmetic and torch's cast)."""
+    Q = np.float32(448.0 if fmt == O.FMT_FP8_DYNAMIC else 127.0)
+    vals = _bf16_grid()
+    rows = []
+    for amax in vals[(vals >= 1) & (vals < 4)]:
+        s = np.float32(amax) / Q
+        xs = vals[(vals <= amax) & (vals >= amax / 256)]
+        yd, yr = xs / s, xs * (np.float32(1) / s)
+        if fmt == O.FMT_FP8_DYNAMIC:
+            cd = torch.from_numpy(yd).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            cr = torch.from_numpy(yr).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        else:
+            cd, cr = np.rint(yd), np.rint(yr)
+        rows += [(float(amax), float(xs[i])) for i in np.nonzero(cd != cr)[0][:1]]
+        if len(rows) >= limit:
+            break
+    return rows
+
+
+@pytest.mark.parametrize("fmt", [O.FMT_FP8_DYNAMIC, O.FMT_W8A8_INT8])
+def test_codes_use_the_correctly_rounded_quotient(fmt):
+    Q = 448 if fmt == O.FMT_FP8_DYNAMIC else 127
+    rows = _straddling_rows(fmt)
+    assert len(rows) >= 8   # the check below can tell the two quotients apart
+    for amax, x in rows:
+        q, s = O.quant_per_token(np.array([[amax, x]], dtype=np.float32), fmt)
+        s_exact = _rn32(Fraction(amax) / Q)
+        assert Fraction(float(s[0])) == s_exact
+        y_div = _rn32(Fraction(x) / s_exact)
+        y_rcp = _rn32(Fraction(x) * _rn32(1 / s_exact))
+        if fmt == O.FMT_FP8_DYNAMIC:
+            got = Fraction(float(torch.from_numpy(q[0].copy()).view(torch.float8_e4m3fn)[1].to(torch.float64)))
+            want, wrong = _e4m3_exact(y_div), _e4m3_exact(y_rcp)
+        else:
+            got, want, wrong = int(q[0, 1]), _int8_exact(y_div), _int8_exact(y_rcp)
+        assert want != wrong, (amax, x)
+        assert got == want, (amax, x, got, want)
+
+
+def test_exact_helpers_on_known_values():
+    """The rational helpers of the check above, on values fixed by hand."""
+    assert _rn32(Fraction(1, 3)) == Fraction(11184811, 2 ** 25)     # 0x3EAAAAAB
+    assert _rn32(Fraction(2 ** 24 + 1)) == 2 ** 24                   # tie to even
+    assert _rn32(Fraction(2 ** 24 + 3)) == 2 ** 24 + 4               # tie to even, upwards
+    assert _rn32(Fraction(1, 2 ** 149)) == Fraction(1, 2 ** 149)     # smallest subnormal
+    assert _e4m3_exact(Fraction(17, 16)) == 1                        # 1.0625: tie, to even (1.0)
+    assert _e4m3_exact(Fraction(19, 16)) == Fraction(5, 4)           # 1.1875: tie, to even (1.25)
+    assert _e4m3_exact(Fraction(460)) == 448 and _e4m3_exact(Fraction(-1000)) == -448
+    assert _e4m3_exact(Fraction(3, 2 ** 10)) == Fraction(2, 2 ** 9)  # subnormal tie 1.5 quanta -> 2
+    assert _int8_exact(Fraction(5, 2)) == 2 and _int8_exact(Fraction(-7, 2)) == -4
