@@ -2,7 +2,6 @@
 is the slowest rank's, the throughput aggregates every rank's work, and the
 reference arm runs on rank 0 only."""
 
-import json
 import os
 import subprocess
 import sys

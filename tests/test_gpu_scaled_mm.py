@@ -9,7 +9,7 @@ import torch
 from oracle import lq_oracle as O
 from quantized_linear_gemm_b200 import inputs, lq
 
-from _lqtest import assert_close, bf16_to_f64, make_problem
+from _lqtest import assert_close, make_problem
 
 pytestmark = pytest.mark.gpu
 

@@ -6,7 +6,6 @@ of the codes, and an exact rational brute-force product.  CPU only."""
 from fractions import Fraction
 
 import numpy as np
-import pytest
 import torch
 
 from oracle import lq_oracle as O
