@@ -270,10 +270,10 @@ class Workload:
         else:
             lq.quant_per_token(self.fmt, c["x"], c["q"], c["s"], stream=stream)
 
-    def gemm(self, c, stream, copy=None):
+    def gemm(self, c, stream, copy=None, variant=None):
         reps = self.weights[c["layer"]]
         qb, sb = reps[c["copy"] if copy is None else copy % len(reps)]
-        lq.scaled_mm(self.fmt, c["q"], c["s"], qb, sb, C=c["C"], variant=c["variant"], stream=stream)
+        lq.scaled_mm(self.fmt, c["q"], c["s"], qb, sb, C=c["C"], variant=variant or c["variant"], stream=stream)
 
     def fused(self, c, stream):
         qb, sb = self.weights[c["layer"]][c["copy"]]
@@ -417,6 +417,20 @@ def capture(fn, stream) -> torch.cuda.CUDAGraph:
             fn()
     torch.cuda.synchronize()
     return g
+
+
+def time_cycle(graphs, n: int, stream) -> float:
+    """Total ms of n graph launches cycling through `graphs`, CUDA events on `stream`."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(n):
+            graphs[i % len(graphs)].replay()
+        end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end)
 
 
 def time_replays(g: torch.cuda.CUDAGraph, n: int, stream, pre=None, post=None) -> float:
@@ -639,13 +653,31 @@ def main() -> None:
         g = capture(one, stream)
         time_replays(g, 3, stream)
         ms = time_replays(g, 10, stream) / (10 * reps)
+        del g
+        # the same calls without programmatic dependent launch
+        v_off = lq.make_variant(**{**c["variant"].as_dict(), "pdl": 0})
+
+        def one_off(c=c, reps=reps, v_off=v_off):
+            for r in range(reps):
+                wl.gemm(c, stream, copy=r, variant=v_off)
+        g = capture(one_off, stream)
+        time_replays(g, 3, stream)
+        ms_off = time_replays(g, 10, stream) / (10 * reps)
+        del g
+        # launch floor: every call its own graph launch (R = 1), weight copies still rotated
+        n_copies = len(wl.weights[c["layer"]])
+        singles = [capture(lambda c=c, r=r: wl.gemm(c, stream, copy=r), stream) for r in range(n_copies)]
+        time_cycle(singles, 2 * n_copies, stream)
+        n_single = max(30, 2 * n_copies)
+        ms_single = time_cycle(singles, n_single, stream) / n_single
+        del singles
         b = gemm_bytes(wl.fmt, c["M"], c["N"], c["K"])
         per_shape.append({"layer": c["layer"], "M": c["M"], "N": c["N"], "K": c["K"], "us": round(ms * 1e3, 3),
                           "GB/s": round(b / (ms * 1e-3) / 1e9, 1), "TFLOP/s": round(2 * c["M"] * c["N"] * c["K"] / (ms * 1e-3) / 1e12, 2),
                           "frac_hbm": round(b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
                           "frac_tensor": round(2 * c["M"] * c["N"] * c["K"] / (ms * 1e-3) / 1e12 / tensor_peak, 3),
+                          "us_pdl_off": round(ms_off * 1e3, 3), "us_single_graph": round(ms_single * 1e3, 3),
                           "variant": c["variant"].as_dict()})
-        del g
 
     producers = producer_measurements(peaks, stream) if not args.no_producers else []
     moe = moe_measurements(peaks, stream) if not args.no_moe else []
