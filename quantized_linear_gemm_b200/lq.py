@@ -503,7 +503,12 @@ def device_status(device: int = 0) -> int:
 
 def set_trace(buf: torch.Tensor | None) -> None:
     """Record 12 globaltimer stamps per CTA of the following scaled_mm launches
-    into ``buf`` (int64 CUDA tensor with 12 entries per CTA), or stop (None)."""
+    into ``buf`` (a contiguous 1-d int64 CUDA tensor), or stop (None).  The
+    library cannot know the grids to come: ``buf`` must hold 12 entries for
+    every CTA of the largest launch made while tracing is on."""
+    if buf is not None:
+        _need(buf, "buf", (torch.int64,), 1)
+        _one_device(buf)
     lib().lq_set_trace(None if buf is None else buf.data_ptr())
 
 

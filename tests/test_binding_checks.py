@@ -158,6 +158,16 @@ def test_quantizer_output_checks(rec):
                                          "lq_rms_norm_dynamic_per_token_quant"]
 
 
+def test_trace_buffer_checks(rec):
+    lq.set_trace(torch.zeros(12 * 4, dtype=torch.int64))
+    lq.set_trace(None)
+    with pytest.raises(TypeError):
+        lq.set_trace(torch.zeros(48, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        lq.set_trace(torch.zeros((4, 12), dtype=torch.int64))
+    assert [c[0] for c in rec.calls] == ["lq_set_trace", "lq_set_trace"]
+
+
 def test_tensors_must_share_one_device():
     a = torch.zeros(4)
     with pytest.raises(ValueError):
