@@ -19,7 +19,7 @@ the three formats:
   scale per 128x128 block.
 
 The same page, section "Kernel Implementation", and the techfeed.io summary of
-it (section "one kernel covers several algorithmic variants") define the
+it (section "何が面白いのか") define the
 Split-K and Swap-AB variants as rewrites of the *same* product, so the oracle
 has one definition of C and only uses split / transposed loop orders as
 self-checks (``acc_split_k``, ``acc_swap_ab``).
@@ -70,6 +70,9 @@ def e4m3_decode(codes) -> np.ndarray:
 
     exponent field e (4 bits), mantissa field m (3 bits):
     e == 0 -> (-1)^s * m * 2^-9 ; otherwise (-1)^s * (8 + m) * 2^(e - 10).
+
+    Source: "FP8" of the PyTorch blog "Building a High-Performance and Portable vLLM Linear Backend
+    with Helion", section "Helion Linear Backend > Scope", read as the OCP FP8 E4M3 ("fn") format.
     """
     c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
     s = (c >> 7) & 1
@@ -82,7 +85,10 @@ def e4m3_decode(codes) -> np.ndarray:
 
 
 def e4m3_decode_int(codes) -> np.ndarray:
-    """e4m3fn value times 2^9, as an exact int64 (NaN codes are rejected)."""
+    """e4m3fn value times 2^9, as an exact int64 (NaN codes are rejected).
+
+    Source: as e4m3_decode; the integer form makes the accumulation below exact.
+    """
     c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
     s = (c >> 7) & 1
     e = (c >> 3) & 0xF
@@ -100,6 +106,10 @@ def e4m3_encode(v) -> np.ndarray:
     Works in float64, where every fp32 input and every scaling by a power of
     two below is exact.  The sign of the input is kept (so -0.0 and negative
     values that round to zero give 0x80).
+
+    Source: "FP8" of the PyTorch blog "Building a High-Performance and Portable vLLM Linear Backend
+    with Helion", section "Helion Linear Backend > Scope"; the rounding (nearest even, saturating) is
+    this oracle's reading.
     """
     x = np.asarray(v, dtype=np.float32)
     if not np.all(np.isfinite(x)):
@@ -122,7 +132,12 @@ def e4m3_encode(v) -> np.ndarray:
 
 
 def int8_encode(v) -> np.ndarray:
-    """Symmetric int8 code: clamp(round_half_even(v), -127, 127)."""
+    """Symmetric int8 code: clamp(round_half_even(v), -127, 127).
+
+    Source: W8A8_INT8 of the PyTorch blog "Building a High-Performance and Portable vLLM Linear Backend
+    with Helion", section "Helion Linear Backend > Scope"; the symmetric half-even code is this
+    oracle's reading.
+    """
     x = np.asarray(v, dtype=np.float32)
     if not np.all(np.isfinite(x)):
         raise ValueError("non-finite value given to the int8 encoder")
@@ -142,7 +157,12 @@ def _encode(fmt: str, y) -> np.ndarray:
 
 
 def scale_from_amax(amax, qmax: float) -> np.ndarray:
-    """s = max(fp32(amax / qmax), 2^-126), one correctly rounded fp32 division."""
+    """s = max(fp32(amax / qmax), 2^-126), one correctly rounded fp32 division.
+
+    Source: the per-token / per-channel / per-group scales of the PyTorch blog "Building a
+    High-Performance and Portable vLLM Linear Backend with Helion", section "Helion Linear Backend >
+    Scope"; the division and the 2^-126 floor are this oracle's reading.
+    """
     a = np.asarray(amax, dtype=np.float32)
     s = a / np.float32(qmax)
     return np.maximum(s, FP32_MIN_NORMAL).astype(np.float32)
@@ -153,6 +173,10 @@ def quantize_groups(x, fmt: str, axis_len: int):
 
     x: float32 array [..., L] with L % axis_len == 0.
     Returns (codes [..., L], scales [..., L // axis_len] float32).
+
+    Source: the step shared by the three scale granularities of the PyTorch blog "Building a
+    High-Performance and Portable vLLM Linear Backend with Helion", section "Helion Linear Backend >
+    Scope".
     """
     x = np.asarray(x, dtype=np.float32)
     L = x.shape[-1]
@@ -180,7 +204,12 @@ def quant_per_token(x, fmt: str):
 
 
 def quant_per_channel(w, fmt: str):
-    """Per-output-channel weight quantization of W stored [N, K]: one scale per n."""
+    """Per-output-channel weight quantization of W stored [N, K]: one scale per n.
+
+    Source: FP8_Dynamic / W8A8_INT8 weights, one scale per output channel (PyTorch blog "Building a
+    High-Performance and Portable vLLM Linear Backend with Helion", section "Helion Linear Backend >
+    Scope").
+    """
     return quant_per_token(w, fmt)
 
 
@@ -188,6 +217,10 @@ def quant_per_token_group128(x):
     """1x128 group activation quantization of Block_FP8 (``per_token_group_fp8_quant``).
 
     x: [M, K], K % 128 == 0.  Returns (codes [M, K], scales [M, K/128]).
+
+    Source: Block_FP8 activations (PyTorch blog "Building a High-Performance and Portable vLLM Linear
+    Backend with Helion", section "Helion Linear Backend > Scope"); the kernel is named in the
+    24-ai.news report, section "vLLMに統合されたカーネル".
     """
     return quantize_groups(np.asarray(x, dtype=np.float32), FMT_BLOCK_FP8, BLOCK)
 
@@ -197,6 +230,9 @@ def quant_weight_block128(w):
 
     One scale per (n-block, k-block) from the amax over the whole block.
     Returns (codes [N, K] uint8, scales [N/128, K/128] float32).
+
+    Source: Block_FP8 weights, one scale per 128 x 128 block (PyTorch blog "Building a High-Performance
+    and Portable vLLM Linear Backend with Helion", section "Helion Linear Backend > Scope").
     """
     w = np.asarray(w, dtype=np.float32)
     N, K = w.shape
@@ -216,7 +252,12 @@ def quant_weight_block128(w):
 # ---------------------------------------------------------------------------
 
 def operand_int(fmt: str, codes) -> np.ndarray:
-    """Operand codes as exact int64: e4m3 value * 2^9, or the int8 value."""
+    """Operand codes as exact int64: e4m3 value * 2^9, or the int8 value.
+
+    Source: the operands of the PyTorch blog "Building a High-Performance and Portable vLLM Linear
+    Backend with Helion", section "Helion Linear Backend > Scope" in the exact integer form acc_exact
+    sums.
+    """
     if fmt == FMT_W8A8_INT8:
         return np.asarray(codes, dtype=np.int8).astype(np.int64)
     return e4m3_decode_int(codes)
@@ -234,7 +275,11 @@ def acc_exact(fmt: str, a_codes, b_codes) -> np.ndarray:
 
 
 def acc_exact_blocks(a_codes, b_codes) -> list:
-    """Per-128-K-block exact e4m3 accumulators (list over kb of int64 [M, N])."""
+    """Per-128-K-block exact e4m3 accumulators (list over kb of int64 [M, N]).
+
+    Source: Block_FP8's per-128-K partial products (PyTorch blog "Building a High-Performance and
+    Portable vLLM Linear Backend with Helion", section "Helion Linear Backend > Scope").
+    """
     A = e4m3_decode_int(a_codes)
     B = e4m3_decode_int(b_codes)
     K = A.shape[1]
@@ -289,7 +334,11 @@ def split_ranges(num_k_tiles: int, split_k: int):
 
 
 def acc_split_k(fmt: str, a_codes, b_codes, split_k: int) -> np.ndarray:
-    """Split-K order: one exact partial per K range, summed in order s = 0..S-1."""
+    """Split-K order: one exact partial per K range, summed in order s = 0..S-1.
+
+    Source: the Split-K variant (PyTorch blog "Building a High-Performance and Portable vLLM Linear
+    Backend with Helion", section "Kernel Implementation"); a self-check, not a second definition.
+    """
     A = operand_int(fmt, a_codes)
     B = operand_int(fmt, b_codes)
     K = A.shape[1]
@@ -307,6 +356,10 @@ def acc_swap_ab(fmt: str, a_codes, b_codes) -> np.ndarray:
 
     The accumulator is built as D[n, m] = sum_k B[n, k] * A[m, k] by an explicit
     loop over K (not via ``acc_exact``) and transposed at the end.
+
+    Source: the Swap-AB variant (PyTorch blog "Building a High-Performance and Portable vLLM Linear
+    Backend with Helion", section "Kernel Implementation"; its formula is garbled in the extracted text
+    and read as (B^T A^T)^T).
     """
     A = operand_int(fmt, a_codes)
     B = operand_int(fmt, b_codes)
@@ -321,7 +374,10 @@ def acc_swap_ab(fmt: str, a_codes, b_codes) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 def bf16_tolerance(C_ref) -> np.ndarray:
-    """Per-element bound 2^-7 * |C_ref| + 1e-3 * rms(C_ref) for a bf16 result."""
+    """Per-element bound 2^-7 * |C_ref| + 1e-3 * rms(C_ref) for a bf16 result.
+
+    Source: none in the blog or its re-reports; the acceptance bound adopted for bf16 outputs.
+    """
     C_ref = np.asarray(C_ref, dtype=np.float64)
     rms = float(np.sqrt(np.mean(C_ref * C_ref))) if C_ref.size else 0.0
     return 2.0 ** -7 * np.abs(C_ref) + 1e-3 * rms
@@ -329,7 +385,10 @@ def bf16_tolerance(C_ref) -> np.ndarray:
 
 def within_tolerance(C, C_ref, rms_of=None):
     """(ok, worst ratio |C - C_ref| / bound).  ``rms_of`` overrides the rms source
-    (the full reference when C_ref is only a sample of it)."""
+    (the full reference when C_ref is only a sample of it).
+
+    Source: as bf16_tolerance.
+    """
     C = np.asarray(C, dtype=np.float64)
     C_ref = np.asarray(C_ref, dtype=np.float64)
     src = C_ref if rms_of is None else np.asarray(rms_of, dtype=np.float64)

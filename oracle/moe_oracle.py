@@ -30,6 +30,14 @@ from oracle import lq_oracle as O
 
 
 def check_offsets(offsets, T: int, E: int) -> np.ndarray:
+    """The expert offsets [E + 1] as int64: expert e's tokens are the rows
+    [offsets[e], offsets[e + 1]) of A, so the table starts at 0, never
+    decreases and ends at T (anything else is refused).
+
+    Source: the routing table of the grouped GEMM (MoE is named as the next
+    target by ai-radar.it, section "Oltre Hopper: Blackwell, AMD, TPU e il
+    perimetro del fork"; the layout is this oracle's reading).
+    """
     off = np.asarray(offsets, dtype=np.int64)
     if off.shape != (E + 1,) or off[0] != 0 or off[-1] != T or np.any(np.diff(off) < 0):
         raise ValueError("offsets must be non-decreasing, start at 0 and end at T")

@@ -54,7 +54,10 @@ _BF16_MIN_QUANTUM = 2.0 ** -133   # spacing of bf16 subnormals
 def bf16_round(v) -> np.ndarray:
     """Round float64 values to the nearest bfloat16 value, ties to even, with
     one rounding (no detour through fp32).  Returned as float64.  Values at or
-    beyond BF16_MAX + half a unit in the last place become +-inf."""
+    beyond BF16_MAX + half a unit in the last place become +-inf.
+
+    Source: the bf16 rounding of a bf16 decoder layer's intermediates (reading; see the module notes).
+    """
     v = np.asarray(v, dtype=np.float64)
     out = np.array(v, copy=True)
     finite = np.isfinite(v) & (v != 0)
@@ -71,14 +74,21 @@ def bf16_round(v) -> np.ndarray:
 
 
 def f32(v) -> np.ndarray:
-    """Round float64 values to fp32 (nearest, ties to even) and back."""
+    """Round float64 values to fp32 (nearest, ties to even) and back.
+
+    Source: the fp32 roundings of the same computation (reading; see the module notes).
+    """
     return np.asarray(v, dtype=np.float64).astype(np.float32).astype(np.float64)
 
 
 def rms_norm_ref(x, weight, eps: float, residual=None):
     """(y, h): the normalised and weighted bf16 row values y [M, K] and the
     (new) residual h [M, K], both as float64 holding bf16 values.  x, weight
-    and residual hold bf16 values (float arrays)."""
+    and residual hold bf16 values (float arrays).
+
+    Source: the RMSNorm of ``rms_norm_*_quant``, named in the 24-ai.news report, section
+    "vLLMに統合されたカーネル".
+    """
     x = np.asarray(x, dtype=np.float64)
     w = np.asarray(weight, dtype=np.float64)
     M, K = x.shape
@@ -98,7 +108,11 @@ def rms_norm_ref(x, weight, eps: float, residual=None):
 
 def silu_and_mul_ref(gu):
     """y [M, I] as float64 holding bf16 values, from gu = [g | u] of shape
-    [M, 2I] holding bf16 values."""
+    [M, 2I] holding bf16 values.
+
+    Source: the SiLU-and-multiply of ``silu_and_mul_*_quant``, named in the 24-ai.news report, section
+    "vLLMに統合されたカーネル".
+    """
     gu = np.asarray(gu, dtype=np.float64)
     M, two_i = gu.shape
     assert two_i % 2 == 0
@@ -111,24 +125,36 @@ def silu_and_mul_ref(gu):
 
 
 def rms_norm_dynamic_per_token_quant(x, weight, eps: float, fmt: str, residual=None):
-    """(codes, scales [M], h): RMSNorm, then per-token quantization."""
+    """(codes, scales [M], h): RMSNorm, then per-token quantization.
+
+    Source: 24-ai.news report, section "vLLMに統合されたカーネル".
+    """
     y, h = rms_norm_ref(x, weight, eps, residual)
     q, s = O.quant_per_token(y, fmt)
     return q, s, h
 
 
 def rms_norm_per_block_quant(x, weight, eps: float, residual=None):
-    """(codes, scales [M, K/128], h): RMSNorm, then 1 x 128 FP8 quantization."""
+    """(codes, scales [M, K/128], h): RMSNorm, then 1 x 128 FP8 quantization.
+
+    Source: 24-ai.news report, section "vLLMに統合されたカーネル".
+    """
     y, h = rms_norm_ref(x, weight, eps, residual)
     q, s = O.quant_per_token_group128(y)
     return q, s, h
 
 
 def silu_and_mul_dynamic_per_token_quant(gu, fmt: str):
-    """(codes [M, I], scales [M])."""
+    """(codes [M, I], scales [M]).
+
+    Source: 24-ai.news report, section "vLLMに統合されたカーネル".
+    """
     return O.quant_per_token(silu_and_mul_ref(gu), fmt)
 
 
 def silu_and_mul_per_block_quant(gu):
-    """(codes [M, I], scales [M, I/128])."""
+    """(codes [M, I], scales [M, I/128]).
+
+    Source: 24-ai.news report, section "vLLMに統合されたカーネル".
+    """
     return O.quant_per_token_group128(silu_and_mul_ref(gu))

@@ -34,7 +34,11 @@ E8M0_BIAS = 127
 
 
 def e8m0_decode(b) -> np.ndarray:
-    """Scale bytes -> float64 values 2^(b - 127) (255 -> NaN)."""
+    """Scale bytes -> float64 values 2^(b - 127) (255 -> NaN).
+
+    Source: 24-ai.news report, section "実際の制限事項" (UE8M0 scales on B200), read as the OCP microscaling
+    E8M0 scale.
+    """
     b = np.asarray(b, dtype=np.int64)
     v = np.exp2((b - E8M0_BIAS).astype(np.float64))
     return np.where(b == 255, np.nan, v)
@@ -43,7 +47,11 @@ def e8m0_decode(b) -> np.ndarray:
 def ue8m0_exponent(amax) -> np.ndarray:
     """Smallest integer e with amax <= 448 * 2^e, clamped to [-127, 127];
     amax = 0 gives -127.  Exact: 448 = 7 * 2^6, so the test is
-    amax * 2^-e <= 448 decided on the float64 significand and exponent."""
+    amax * 2^-e <= 448 decided on the float64 significand and exponent.
+
+    Source: 24-ai.news report, section "実際の制限事項" (UE8M0 scales on B200), read as the OCP microscaling
+    E8M0 scale.
+    """
     a = np.asarray(amax, dtype=np.float64)
     m, ex = np.frexp(a)                 # a = m * 2^ex, m in [0.5, 1)
     # 448 * 2^e = 0.875 * 2^(e + 9): amax <= it  <=>  ex < e + 9, or ex == e + 9 and m <= 0.875
@@ -53,7 +61,11 @@ def ue8m0_exponent(amax) -> np.ndarray:
 
 
 def quantize_groups_ue8m0(x, axis_len: int):
-    """Codes [..., L] and scale bytes [..., L / axis_len] of contiguous groups."""
+    """Codes [..., L] and scale bytes [..., L / axis_len] of contiguous groups.
+
+    Source: 24-ai.news report, section "実際の制限事項" (UE8M0 scales on B200), read as the OCP microscaling
+    E8M0 scale.
+    """
     x = np.asarray(x, dtype=np.float32)
     L = x.shape[-1]
     if L % axis_len:
@@ -66,12 +78,20 @@ def quantize_groups_ue8m0(x, axis_len: int):
 
 
 def quant_per_token_group128_ue8m0(x):
-    """1 x 128 activation groups: (codes [M, K], scale bytes [M, K/128])."""
+    """1 x 128 activation groups: (codes [M, K], scale bytes [M, K/128]).
+
+    Source: 24-ai.news report, section "実際の制限事項" (UE8M0 scales on B200), read as the OCP microscaling
+    E8M0 scale.
+    """
     return quantize_groups_ue8m0(x, O.BLOCK)
 
 
 def quant_weight_block128_ue8m0(w):
-    """128 x 128 weight blocks of W [N, K]: (codes [N, K], scale bytes [N/128, K/128])."""
+    """128 x 128 weight blocks of W [N, K]: (codes [N, K], scale bytes [N/128, K/128]).
+
+    Source: 24-ai.news report, section "実際の制限事項" (UE8M0 scales on B200), read as the OCP microscaling
+    E8M0 scale.
+    """
     w = np.asarray(w, dtype=np.float32)
     N, K = w.shape
     if N % O.BLOCK or K % O.BLOCK:
@@ -85,5 +105,9 @@ def quant_weight_block128_ue8m0(w):
 
 
 def blockwise_ue8m0_ref(a_codes, a_bytes, b_codes, b_bytes) -> np.ndarray:
-    """C [M, N] in fp64: the Block_FP8 product with the decoded power-of-two scales."""
+    """C [M, N] in fp64: the Block_FP8 product with the decoded power-of-two scales.
+
+    Source: 24-ai.news report, section "実際の制限事項" (UE8M0 scales on B200), read as the OCP microscaling
+    E8M0 scale.
+    """
     return O.blockwise_ref(a_codes, e8m0_decode(a_bytes), b_codes, e8m0_decode(b_bytes))
