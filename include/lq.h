@@ -216,6 +216,9 @@ lq_status lq_grouped_scaled_mm(lq_fmt fmt, const void *A, const float *a_scales,
  * writes the exact int32 accumulator sum_k A[m,k]*B[n,k] to acc_out [M, N]
  * (device, 16-byte aligned), so that it can be compared bit for bit with an
  * exact integer reference.  Same arguments and errors as lq_scaled_mm.
+ * Source: W8A8_INT8 (int8 operands, int32 accumulation) of the PyTorch blog "Building a High-Performance and Portable vLLM Linear
+ * Backend with Helion", section "Helion Linear Backend > Scope";
+ * the accumulator output is a test interface of this library.
  */
 lq_status lq_scaled_mm_i32acc(const void *A, const float *a_scales,
                               const void *B, const float *b_scales, void *C,
@@ -259,7 +262,7 @@ lq_status lq_quant_scaled_mm(lq_fmt fmt, const void *x, const void *B,
  * which lq_quant_scaled_mm uses its one-kernel path; 0 = never fuse, a
  * negative value restores the default (0, or LQ_FUSE_MAX_SLICE_BYTES).
  * Returns the limit in force before the call.  A tuning and test hook: it
- * changes which kernels run, never the results.
+ * changes which kernels run, never the results.  No page defines it.
  */
 int64_t lq_set_fuse_limit(int64_t max_slice_bytes);
 
@@ -376,6 +379,8 @@ lq_status lq_silu_and_mul_per_block_quant(const void *gate_up, void *q, float *s
  *   lq_quant_weight_block128_ue8m0: w [N, K] -> q [N, K], scales
  *     [N/128, K/128] bytes; N % 128 == 0 and K % 128 == 0.
  * Errors as lq_quant_per_token_group128 / lq_quant_weight_block128.
+ * Source: 24-ai.news report, section "実際の制限事項" (the UE8M0 scale format
+ * needed on B200), read as the OCP microscaling E8M0 scale.
  */
 lq_status lq_quant_per_token_group128_ue8m0(const void *x, void *q, uint8_t *scales,
                                            int64_t M, int64_t K, lq_stream_t stream);
@@ -387,6 +392,8 @@ lq_status lq_quant_weight_block128_ue8m0(const void *w, void *q, uint8_t *scales
  * per (n-block, k-block) from the amax over the whole block.
  *   w [N, K] bf16 (16-byte aligned) -> q [N, K] e4m3, scales [N/128, K/128].
  *   N % 128 == 0 and K % 128 == 0.
+ * Source: the Block_FP8 weight scales of the PyTorch blog "Building a High-Performance and Portable vLLM Linear
+ * Backend with Helion", section "Helion Linear Backend > Scope".
  */
 lq_status lq_quant_weight_block128(const void *w, void *q, float *scales,
                                    int64_t N, int64_t K, lq_stream_t stream);
@@ -396,6 +403,9 @@ lq_status lq_quant_weight_block128(const void *w, void *q, float *scales,
  * the dispatch-table entry for the token bucket of M (the next of
  * 1,2,4,8,16,24,32, then powers of two), else a built-in heuristic.
  * Host-only; writes *out.  Errors: LQ_ERR_INVALID_ARG.
+ * Source: the per-shape tuned configurations and the dispatch by token count
+ * of the techfeed.io summary of the blog, sections "オートチューニングの仕組み"
+ * and "ハイブリッドディスパッチ：Helionの弱点を補う設計" (Fig. 2).
  */
 lq_status lq_select_variant(lq_fmt fmt, int64_t M, int64_t N, int64_t K,
                             lq_variant *out);
@@ -406,18 +416,21 @@ lq_status lq_select_variant(lq_fmt fmt, int64_t M, int64_t N, int64_t K,
  * starts a comment).  path == NULL restores the compiled-in table.  At
  * start-up the environment variable LQ_DISPATCH_TABLE, when set, names a
  * file that replaces the compiled-in table.  On error
- * the current table is kept and LQ_ERR_TABLE is returned.  Not thread-safe
- * with concurrent lq_scaled_mm calls that pass variant == NULL.
+ * the current table is kept and LQ_ERR_TABLE is returned.  Safe while other
+ * threads call lq_scaled_mm: each call uses the table in force when it looked
+ * up its variant.  Source: as lq_select_variant.
  */
 lq_status lq_load_dispatch_table(const char *path);
 
-/* Number of entries in the current dispatch table. */
+/* Number of entries in the current dispatch table (as lq_select_variant). */
 int64_t lq_dispatch_table_size(void);
 
 /*
  * Create the per-device state of `device` (status word, Split-K arrival
  * counters) if it does not exist yet.  Call it before capturing a CUDA graph
- * that contains lq calls.  Errors: LQ_ERR_CUDA.
+ * that contains lq calls.  Errors: LQ_ERR_CUDA.  Library infrastructure: no
+ * page defines it (likewise the workspace, status, trace, version and status
+ * string entry points below).
  */
 lq_status lq_init_device(int device);
 
