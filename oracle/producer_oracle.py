@@ -30,7 +30,10 @@ RMSNorm (optionally with the residual added first, the decoder layer's
 SiLU-and-multiply on the fused gate/up projection output gu = [g | u],
 [M, 2I]:
 
-* a_k = bf16(g_k / (1 + exp(-g_k)))       evaluated in fp64, rounded once;
+* a_k = bf16(g_k / (1 + exp(-g_k)))       rounded once from the exact value:
+  evaluated in fp64, and wherever the fp64 value is too close to a
+  midpoint between two bf16 values for its own error to decide the
+  rounding, evaluated again with 60 significant decimal digits;
 * y_k = bf16(fp32(a_k * u_k))             (the product is exact in fp32).
 
 Then y is quantized with the per-token dynamic rule (FP8 e4m3 or INT8, one
@@ -42,6 +45,8 @@ group), exactly as ``lq_oracle.quant_per_token`` and
 from __future__ import annotations
 
 import math
+from decimal import Context, Decimal
+from fractions import Fraction
 
 import numpy as np
 
@@ -106,6 +111,63 @@ def rms_norm_ref(x, weight, eps: float, residual=None):
     return y, h
 
 
+def _silu_decimal(g: float, ctx: Context) -> Decimal:
+    """silu(g) = g / (1 + e^-g) with 60 significant digits (g exact)."""
+    d = Decimal(g)
+    return ctx.divide(d, ctx.add(Decimal(1), ctx.exp(ctx.minus(d))))
+
+
+def _nearest_bf16_to(exact: Decimal, guess: float) -> float:
+    """The bf16 value nearest to `exact` among `guess` and its two bf16
+    neighbours (ties to the even significand), compared in exact rational
+    arithmetic; `guess` is a bf16 value within one unit of the answer."""
+    g32 = np.array([guess], dtype=np.float32)
+    bits = int(g32.view(np.uint32)[0]) >> 16
+    cands = []
+    for b in (bits - 1, bits, bits + 1):
+        if b < 0:   # below +0: the negative side, -2^-133
+            b = 0x8001
+        v = float(np.array([b << 16], dtype=np.uint32).view(np.float32)[0])
+        if math.isfinite(v):
+            cands.append((v, b))
+    if guess == 0.0:   # +-0: the neighbours on both sides
+        cands += [(2.0 ** -133, 1), (-(2.0 ** -133), 0x8001)]
+    x = Fraction(exact)   # the 60-digit value, exactly
+    best = min(cands, key=lambda c: (abs(x - Fraction(c[0])), c[1] & 1))
+    return best[0]
+
+
+def silu_bf16(g) -> np.ndarray:
+    """bf16(silu(g)) for bf16 values g (float64 array), rounded once from the
+    exact value of g / (1 + e^-g).
+
+    The fp64 evaluation is within a few units of 2^-52 (relative) of the
+    exact value, so its bf16 rounding is the rounding of the exact value
+    unless the fp64 value lies within 2^-40 (relative) of a midpoint between
+    two bf16 values; those elements are evaluated again with 60 significant
+    decimal digits and rounded by exact comparison.  (For |g| < 2^-125 the
+    fp64 value is exactly g / 2, a midpoint, while the exact value lies above
+    g / 2 since sigma(g) > 1/2 for g > 0 and < 1/2 for g < 0.)
+
+    Source: the SiLU of ``silu_and_mul_*_quant``, named in the 24-ai.news report, section
+    "vLLMに統合されたカーネル" (the rounding is a reading: once, from the exact value).
+    """
+    g = np.asarray(g, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        s = g / (1.0 + np.exp(-g))
+    a = bf16_round(s)
+    lo = bf16_round(s * (1.0 - 2.0 ** -40))
+    hi = bf16_round(s * (1.0 + 2.0 ** -40))
+    unsure = np.flatnonzero((lo != a) | (hi != a))
+    if unsure.size:
+        ctx = Context(prec=60, Emin=-10 ** 9, Emax=10 ** 9)
+        flat = a.reshape(-1)
+        gf = g.reshape(-1)
+        for i in unsure:
+            flat[i] = _nearest_bf16_to(_silu_decimal(float(gf[i]), ctx), float(flat[i]))
+    return a
+
+
 def silu_and_mul_ref(gu):
     """y [M, I] as float64 holding bf16 values, from gu = [g | u] of shape
     [M, 2I] holding bf16 values.
@@ -118,9 +180,7 @@ def silu_and_mul_ref(gu):
     assert two_i % 2 == 0
     I = two_i // 2
     g, u = gu[:, :I], gu[:, I:]
-    with np.errstate(over="ignore"):
-        silu = g / (1.0 + np.exp(-g))
-    a = bf16_round(silu)
+    a = silu_bf16(g)
     return bf16_round(f32(a * u))
 
 

@@ -3,6 +3,10 @@ dynamic quantization) against things other than itself: torch's own bf16
 cast and fp64 rms_norm / silu, closed forms, exact special cases and
 composition invariants.  CPU only."""
 
+import math
+from decimal import Context, Decimal
+from fractions import Fraction
+
 import numpy as np
 import pytest
 import torch
@@ -162,15 +166,71 @@ def test_silu_and_mul_power_of_two_up_scales_exactly():
         assert np.array_equal(y, a * 2.0 ** k)
 
 
-def test_silu_rounds_once_from_fp64():
-    """a = bf16(silu(g)) straight from fp64: compare with an fp32 detour on
-    many g and require the fp64 path to be the nearest bf16 to the fp64 silu."""
-    g = _rows(4, 4096, seed=10) * 3
-    y = P.silu_and_mul_ref(np.concatenate([g, np.ones_like(g)], axis=1))
-    s = g / (1 + np.exp(-g))
-    err = np.abs(y - s)
-    ulp = _ulp_bf16(s)
-    assert np.all(err <= ulp / 2 * (1 + 1e-12))
+def _round_rational_to_bf16(x: Fraction) -> Fraction:
+    """Nearest bf16 value to the rational x, ties to the even significand
+    (8 significant bits, subnormal spacing 2^-133), in integer arithmetic."""
+    if x == 0:
+        return Fraction(0)
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()   # 2^e <= a < 2^(e+2)
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    q = Fraction(2) ** max(e - 7, -133)
+    n, rem = divmod(a, q)
+    if rem * 2 > q or (rem * 2 == q and n % 2 == 1):
+        n += 1
+    r = n * q
+    return r if x > 0 else -r
+
+
+def test_silu_is_correctly_rounded_for_every_bf16_gate():
+    """Every finite bf16 g: bf16(silu(g)) is the bf16 value nearest to the
+    exact silu(g), found here from a 50-digit decimal evaluation and an exact
+    rational rounding written out in this test (for g >= 100 the answer is g,
+    for g <= -100 it is -0)."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    g = (bits << 16).view(np.float32)
+    g = g[np.isfinite(g)].astype(np.float64)
+    got = P.silu_bf16(g)
+    ctx = Context(prec=50, Emin=-10 ** 6, Emax=10 ** 6)
+    for gi, yi in zip(g.tolist(), got.tolist()):
+        if gi >= 100:
+            want = Fraction(gi)
+        elif gi <= -100:
+            assert yi == 0.0 and math.copysign(1.0, yi) < 0, gi
+            continue
+        else:
+            d = Decimal(gi)
+            exact = Fraction(ctx.divide(d, ctx.add(Decimal(1), ctx.exp(-d))))
+            want = _round_rational_to_bf16(exact)
+        assert Fraction(yi) == want, (gi, yi, float(want))
+    # through silu_and_mul_ref with u = 1 as well
+    y = P.silu_and_mul_ref(np.concatenate([g[None, :], np.ones((1, g.size))], axis=1))
+    assert np.array_equal(y[0], got)
+
+
+def test_silu_ties_of_tiny_gates_round_towards_plus_infinity():
+    """For 0 < |g| < 2^-125 the fp64 value of g / (1 + e^-g) is exactly g / 2.
+    silu(g) - g / 2 = g (sigma(g) - 1/2) > 0 for every g != 0, so where g / 2
+    lies halfway between two bf16 values the answer is the upper one (for
+    g < 0: the one nearer zero); elsewhere it is g / 2 itself."""
+    q = 2.0 ** -133
+    ks = np.arange(1, 256)                       # |g| = k 2^-133 (subnormal) ...
+    mags = np.concatenate([ks * q, (128 + np.arange(128)) * 2.0 ** -133])   # ... and the lowest normal binade
+    mags = np.unique(mags[mags < 2.0 ** -125])
+    for sign in (1.0, -1.0):
+        g = sign * mags
+        got = P.silu_bf16(g)
+        half = g / 2                              # exact
+        n = half / q                              # integer or integer + 1/2
+        want = np.where(n == np.floor(n), half, np.ceil(n) * q)   # up at ties (towards +inf)
+        assert np.array_equal(got, want), sign
+    n = mags / q / 2
+    ties = n != np.floor(n)
+    assert ties.sum() == 128                                   # odd multiples of 2^-133 on each side
+    assert (ties & (np.floor(n) % 2 == 0)).sum() == 64         # of which ties-to-even would go down
 
 
 # ----------------------------------------------------------------- composition
