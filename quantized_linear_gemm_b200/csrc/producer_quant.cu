@@ -63,8 +63,17 @@ __device__ __forceinline__ __nv_bfloat16 silu_bf16_fast(float g, bool* ok) {
   return __float2bfloat16_rn(s);
 }
 
+// silu(g) from fp64, rounded once to bf16.  Over all bf16 inputs the fp64
+// quotient (within a few units of 2^-52 of the exact value) decides the
+// rounding, except where it is exactly g / 2: for 0 < |g| < 2^-125, where
+// 1 + e^-g rounds to 2.  For half of those gates g / 2 is a midpoint between
+// two bf16 values, and the exact value lies above it (silu(g) - g / 2 =
+// g (sigma(g) - 1/2) > 0 for every g != 0).  There g / 2 is rounded with a
+// positive excess of |g| 2^-20, far below half a bf16 unit: the rounding of
+// a value just above g / 2, like the exact one.
 __device__ __forceinline__ __nv_bfloat16 silu_bf16_f64(float g) {
   const double gd = static_cast<double>(g);
+  if (gd != 0.0 && fabs(gd) < 0x1p-60) return __double2bfloat16(fma(fabs(gd), 0x1p-20, gd * 0.5));
   return __double2bfloat16(__ddiv_rn(gd, __dadd_rn(1.0, exp(-gd))));
 }
 

@@ -122,6 +122,32 @@ def test_silu_rounding_paths(cuda_device):
         assert np.array_equal(q.cpu().numpy(), q_ref), uval
 
 
+def test_silu_ties_of_tiny_gates(cuda_device):
+    """Gates 0 < |g| < 2^-125 where g / 2 lies halfway between two bf16
+    values (odd multiples of 2^-133, both signs), alone in a row so that the
+    scale floor 2^-126 makes their codes depend on the silu's last bit: the
+    silu goes towards +inf at those ties (silu(g) > g / 2), codes bit-exact
+    against the oracle.  u = 3.984375 makes 40 of the FP8 codes differ from
+    those of a silu rounded ties-to-even."""
+    k = torch.arange(1, 256, 2, dtype=torch.float64)
+    mag = k * 2.0 ** -133
+    g = torch.cat([mag, -mag]).to(torch.float32).to(torch.bfloat16)[None, :]   # 256 gates, exact in bf16
+    assert torch.equal(g.double()[0, :128], mag)
+    for uval in (1.0, 3.984375):
+        gu = torch.cat([g, torch.full_like(g, uval)], dim=1)
+        for fmt in FMTS:
+            q, s = lq.silu_and_mul_dynamic_per_token_quant(fmt, gu.cuda())
+            torch.cuda.synchronize()
+            q_ref, s_ref = P.silu_and_mul_dynamic_per_token_quant(_np(gu), fmt)
+            assert np.array_equal(s.cpu().numpy(), s_ref), (fmt, uval)
+            assert np.array_equal(q.cpu().numpy(), q_ref), (fmt, uval)
+        q, s = lq.silu_and_mul_per_block_quant(gu.cuda())
+        torch.cuda.synchronize()
+        q_ref, s_ref = P.silu_and_mul_per_block_quant(_np(gu))
+        assert np.array_equal(s.cpu().numpy(), s_ref), uval
+        assert np.array_equal(q.cpu().numpy(), q_ref), uval
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_rms_norm_wide_range_rows(cuda_device, fmt):
     """Rows spanning 230 binades, subnormal entries, amax around 2^-80 (both
