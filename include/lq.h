@@ -44,7 +44,15 @@
  *    this interface.
  *  - The library allocates device memory only in lq_init_device,
  *    lq_reserve_workspace and, outside stream capture, when a Split-K call
- *    needs more workspace than it holds.
+ *    needs more workspace than it holds.  It never frees device memory that
+ *    a call may have used: a workspace that is replaced by a larger one is
+ *    kept until the process exits, so a CUDA graph captured earlier stays
+ *    valid.
+ *  - variant == NULL: the dispatch table's (or the heuristic's) variant,
+ *    with pdl lowered from 2 to 1 unless lq_declare_static_weights(1) has
+ *    been called, so that a call never reads B before the kernels ahead of
+ *    it on the stream have finished (a weight quantized on the same stream
+ *    just before is safe).
  */
 #ifndef LQ_H_
 #define LQ_H_
@@ -110,7 +118,8 @@ typedef enum {
  *            that wait.  With 2 the caller guarantees that B and b_scales
  *            are not being written by any kernel that may still be running
  *            when the call is launched (true of model weights, which are
- *            written once before inference).
+ *            written once before inference).  A NULL variant uses 2 only
+ *            after lq_declare_static_weights(1).
  */
 typedef struct {
   int32_t swap_ab;
@@ -139,22 +148,27 @@ typedef struct {
  *              BLOCK_FP8; [N/128, K/128] UE8M0 bytes for BLOCK_FP8_UE8M0.
  *   C        : [M, N] bf16 output, 16-byte aligned.
  *   M, N, K  : M >= 0, N >= 0, K >= 0; K % 16 == 0 and N % 8 == 0;
- *              the Block_FP8 formats also need K % 128 == 0, N % 128 == 0.
- *              M == 0 or N == 0 is a no-op; K == 0 writes C = 0.
- *   variant  : NULL = the dispatch table's choice for (fmt, M, N, K).
+ *              the Block_FP8 formats also need K % 128 == 0, N % 128 == 0;
+ *              W8A8_INT8 needs K <= 131071 (so that no int32 sum of int8
+ *              products can wrap).  M == 0 or N == 0 is a no-op; K == 0
+ *              writes C = 0.
+ *   variant  : NULL = the dispatch table's choice for (fmt, M, N, K), which
+ *              reads B only after the previous kernels on the stream have
+ *              finished unless lq_declare_static_weights(1) was called.
  *   stream   : CUDA stream.
  *
  * Errors: LQ_ERR_INVALID_ARG / LQ_ERR_ALIGNMENT / LQ_ERR_UNSUPPORTED_SHAPE
  * before any launch; LQ_ERR_WORKSPACE when split_k > 1 needs a larger
  * workspace while `stream` is capturing; LQ_ERR_CUDA when a launch fails.
  * A Split-K call with reduce 0 or 1 uses the library's per-device workspace:
- * such calls on different streams of one device must not overlap in time,
- * and must not be issued from several host threads at once: a call that
- * grows the workspace frees the old one, which a call being issued at the
- * same moment by another thread may still be about to use.  Call
- * lq_reserve_workspace with the largest size first to rule growth out.
- * Calls with split_k == 1 or reduce 2 (the dispatch table's choices) use no
- * workspace and have neither restriction.
+ * such calls on different streams of one device must not overlap in time on
+ * the GPU (they share the workspace and the arrival counters).  The
+ * workspace only grows (a replaced one is kept until exit), so a graph
+ * captured before a later call grew it stays valid; capturing such a call
+ * needs the workspace reserved first (lq_reserve_workspace with the largest
+ * split_k * M * N * 4), since growth is refused during capture.  Calls with
+ * split_k == 1 or reduce 2 (the dispatch table's choices) use no workspace
+ * and have neither restriction.
  */
 lq_status lq_scaled_mm(lq_fmt fmt, const void *A, const float *a_scales,
                        const void *B, const float *b_scales, void *C,
@@ -238,7 +252,8 @@ lq_status lq_scaled_mm_i32acc(const void *A, const float *a_scales,
  *   B, b_scales, C, M, N, K : as lq_scaled_mm.
  *   a_codes  : [M, K] out, the activation codes (16-byte aligned).
  *   a_scales : [M] out, the per-token scales.
- *   variant  : NULL = the dispatch table's choice for (fmt, M, N, K).
+ *   variant  : NULL = the dispatch table's choice for (fmt, M, N, K), with
+ *              pdl as for lq_scaled_mm.
  * a_codes, a_scales and C equal, bit for bit, those of lq_quant_per_token
  * followed by lq_scaled_mm with the same variant.  By default the two
  * kernels run (lq_quant_per_token, then lq_scaled_mm).  With a Swap-AB
@@ -249,8 +264,11 @@ lq_status lq_scaled_mm_i32acc(const void *A, const float *a_scales,
  * read once), one kernel does both: the TMA stages each bf16 activation tile
  * beside the weight tile, the CTA's idle epilogue warps quantize it into the
  * tensor core's operand slot, and the Split-K CTAs form a cluster (reduce is
- * forced to 2) that exchanges the per-token amax.  Errors as lq_scaled_mm;
- * LQ_ERR_INVALID_ARG for Block_FP8.
+ * forced to 2) that exchanges the per-token amax; a variant that is not
+ * valid with that cluster takes the two-kernel path.  The two-kernel path
+ * runs lq_scaled_mm with the caller's variant unchanged.  Errors as
+ * lq_scaled_mm, all found before the first launch; LQ_ERR_INVALID_ARG for
+ * Block_FP8.
  */
 lq_status lq_quant_scaled_mm(lq_fmt fmt, const void *x, const void *B,
                              const float *b_scales, void *C, void *a_codes,
@@ -436,8 +454,9 @@ lq_status lq_init_device(int device);
 
 /*
  * Make sure the per-device Split-K workspace holds at least `bytes` bytes
- * (a Split-K call needs split_k * M * N * 4).  Synchronises the device when
- * it has to replace a smaller workspace.  Call it before stream capture.
+ * (a Split-K call needs split_k * M * N * 4).  A smaller workspace that it
+ * replaces is kept until exit (graphs captured with it stay valid); growth
+ * is at least twofold.  Call it before stream capture.
  */
 lq_status lq_reserve_workspace(int device, size_t bytes);
 
@@ -452,6 +471,21 @@ size_t lq_workspace_bytes(lq_fmt fmt, int64_t M, int64_t N, int64_t K,
  * bounded wait (its output is then undefined).  Synchronises the device.
  */
 lq_status lq_device_status(int device);
+
+/*
+ * Declare (static_weights != 0) that the weights B and b_scales of every
+ * later call are never written by a kernel that may still be running when a
+ * GEMM reading them is launched (model weights, written once before
+ * inference).  Then a NULL variant may stream the first weight tiles before
+ * waiting for the previous kernel on the stream (the table's pdl 2), which
+ * hides their latency behind that kernel's tail.  Without the declaration
+ * (the default) a NULL variant waits first (pdl 1), which is safe when a
+ * weight is quantized or updated on the same stream just before.  Explicit
+ * variants are used as given.  Process-wide; a captured CUDA graph keeps the
+ * variants chosen at capture time.  Returns the previous setting (0 or 1).
+ * Library infrastructure: no page defines it.
+ */
+int lq_declare_static_weights(int static_weights);
 
 /*
  * Diagnostics: while `device_buffer` is non-NULL, every scaled_mm kernel

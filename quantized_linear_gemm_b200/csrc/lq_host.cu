@@ -39,7 +39,10 @@ constexpr int kMaxDevices = 64;
 constexpr int kMaxSmemPerCta = 227 * 1024;
 constexpr size_t kCounterCapacity = size_t(1) << 20;   // Split-K arrival counters per device
 constexpr int kNumSms = 148;
-constexpr int kMaxStages = 14;   // the kernel's control block holds 4 x stages + 7 mbarriers (64 at most)
+constexpr int kMaxStages = 14;
+// W8A8_INT8 sums products of int8 codes in int32: |a b| <= 128 * 128, so K
+// up to 131071 can never wrap the accumulator (131071 * 2^14 < 2^31).
+constexpr int64_t kInt8MaxK = 131071;   // the kernel's control block holds 4 x stages + 7 mbarriers (64 at most)
 // 0: lq_quant_scaled_mm runs the quantization kernel and the GEMM unless a
 // caller raises the limit.  Measured on B200 (Qwen3-8B decode shapes, FP8):
 // the one-kernel path saves up to 1.2 us per call at M = 1 on the down
@@ -55,6 +58,7 @@ struct DeviceState {
   int* counters = nullptr;     // kCounterCapacity ints, zero between calls
   void* ws = nullptr;          // Split-K partials
   size_t ws_bytes = 0;
+  std::vector<void*> retired;  // smaller workspaces replaced by ws, kept until exit
 };
 
 std::mutex g_dev_mutex;
@@ -62,6 +66,15 @@ DeviceState g_dev[kMaxDevices];
 std::atomic<uint64_t*> g_trace{nullptr};   // diagnostics: per-CTA stamps of the next launches
 std::atomic<int> g_skip_stage{-1};          // test hook: K tile the producer never fills
 std::atomic<uint64_t> g_wait_limit_override{0};
+// Whether the caller has declared that weight operands are never written
+// while a GEMM that reads them may run (lq_declare_static_weights).  Until
+// then a variant taken from the dispatch table or the heuristic never
+// streams weights before its dependency wait (pdl 2 is lowered to 1).
+std::atomic<int> g_static_weights{0};
+
+// The variant for a call that passed none: the table's entry for the token
+// bucket, else the heuristic, with pdl 2 allowed only for static weights.
+lq_variant default_variant(int fmt, int64_t M, int64_t N, int64_t K);
 
 // Largest per-CTA activation slice (tokens x K range x 2 bytes) for which
 // lq_quant_scaled_mm uses the fused kernel; LQ_FUSE_MAX_SLICE_BYTES overrides.
@@ -139,20 +152,23 @@ lq_status device_state(cudaStream_t stream, DeviceState** out) {
   return LQ_OK;
 }
 
+// The Split-K workspace only grows.  A replaced buffer is never freed: a CUDA
+// graph captured earlier keeps its address, and so may a call that another
+// host thread is issuing at the same moment.  It is kept until the process
+// exits; growth is at least twofold, so at most about log2(largest / 2 MiB)
+// buffers are ever kept.
 lq_status ensure_workspace(DeviceState* d, size_t bytes, cudaStream_t stream) {
   if (bytes <= d->ws_bytes) return LQ_OK;
   if (stream_capturing(stream)) return LQ_ERR_WORKSPACE;
-  if (d->ws) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return LQ_ERR_CUDA;
-    cudaFree(d->ws);
-    d->ws = nullptr;
-    d->ws_bytes = 0;
-  }
-  const size_t rounded = (bytes + (size_t(1) << 21) - 1) & ~((size_t(1) << 21) - 1);
-  if (cudaMalloc(&d->ws, rounded) != cudaSuccess) {
+  size_t want = bytes > 2 * d->ws_bytes ? bytes : 2 * d->ws_bytes;
+  const size_t rounded = (want + (size_t(1) << 21) - 1) & ~((size_t(1) << 21) - 1);
+  void* fresh = nullptr;
+  if (cudaMalloc(&fresh, rounded) != cudaSuccess) {
     cudaGetLastError();
     return LQ_ERR_WORKSPACE;
   }
+  if (d->ws) d->retired.push_back(d->ws);
+  d->ws = fresh;
   d->ws_bytes = rounded;
   return LQ_OK;
 }
@@ -280,7 +296,7 @@ lq_variant heuristic_variant(int fmt, int64_t M, int64_t N, int64_t K) {
     v.stages = per_split < 2 ? 2 : (per_split > cap ? cap : per_split);
   } else {
     v.swap_ab = 0;
-    v.tile_n = lq::is_block_fmt(fmt) ? 128 : 256;
+    v.tile_n = fmt == lq::kFmtBlock ? 128 : 256;
     const int64_t tiles = ((M + 127) / 128) * ((N + v.tile_n - 1) / v.tile_n);
     int S = 1;
     while (S < 256 && tiles * S < kNumSms && T / (S * 2) >= 4) S *= 2;
@@ -291,17 +307,27 @@ lq_variant heuristic_variant(int fmt, int64_t M, int64_t N, int64_t K) {
   return v;
 }
 
+bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, lq_variant* out);
+
+lq_variant default_variant(int fmt, int64_t M, int64_t N, int64_t K) {
+  lq_variant v{};
+  if (!lookup_table(fmt, M, N, K, &v)) v = heuristic_variant(fmt, M, N, K);
+  if (v.pdl == 2 && !g_static_weights.load()) v.pdl = 1;
+  return v;
+}
+
 bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, lq_variant* out) {
   auto t = current_table();
   const int64_t mb = m_bucket(M);
   for (const TableEntry& e : *t) {
-    // UE8M0 Block_FP8 runs the Block_FP8 kernels: it shares their entries
-    const int key = fmt == lq::kFmtBlockE8m0 ? lq::kFmtBlock : fmt;
-    if (e.fmt == key && e.m_bucket == mb && e.N == N && e.K == K) {
+    if (e.fmt == fmt && e.m_bucket == mb && e.N == N && e.K == K) {
       *out = e.v;
       return true;
     }
   }
+  // UE8M0 Block_FP8 without entries of its own: the Block_FP8 entries (every
+  // Block_FP8 variant is valid for it)
+  if (fmt == lq::kFmtBlockE8m0) return lookup_table(lq::kFmtBlock, M, N, K, out);
   return false;
 }
 
@@ -319,7 +345,7 @@ lq_status check_variant(int fmt, const lq_variant& v) {
     if (v.tile_n != 16 && v.tile_n != 32 && v.tile_n != 64) return LQ_ERR_INVALID_ARG;
   } else {
     if (v.tile_n != 64 && v.tile_n != 128 && v.tile_n != 256) return LQ_ERR_INVALID_ARG;
-    if (lq::is_block_fmt(fmt) && v.tile_n == 256) return LQ_ERR_INVALID_ARG;
+    if (fmt == lq::kFmtBlock && v.tile_n == 256) return LQ_ERR_INVALID_ARG;   // promotion in registers
   }
   if (v.stages != 0 && (v.stages < 2 || v.stages > kMaxStages)) return LQ_ERR_INVALID_ARG;
   if (v.stages != 0 &&
@@ -341,6 +367,7 @@ lq_status check_gemm_args(int fmt, const void* A, const float* a_s, const void* 
   if (fmt != lq::kFmtBlockE8m0 && (!aligned(a_s, 4) || !aligned(b_s, 4))) return LQ_ERR_ALIGNMENT;   // e8m0: bytes
   if (K % 16 != 0 || N % 8 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
   if (lq::is_block_fmt(fmt) && (K % 128 != 0 || N % 128 != 0)) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (fmt == lq::kFmtInt8 && K > kInt8MaxK) return LQ_ERR_UNSUPPORTED_SHAPE;
   if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1)
     return LQ_ERR_UNSUPPORTED_SHAPE;
   return LQ_OK;
@@ -361,12 +388,7 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
     return lq::launch_fill_zero_bf16(static_cast<__nv_bfloat16*>(C), M * N, stream) == cudaSuccess ? LQ_OK
                                                                                                   : LQ_ERR_CUDA;
   }
-  lq_variant v{};
-  if (variant) {
-    v = *variant;
-  } else if (!lookup_table(fmt, M, N, K, &v)) {
-    v = heuristic_variant(fmt, M, N, K);
-  }
+  lq_variant v = variant ? *variant : default_variant(fmt, M, N, K);
   rc = check_variant(fmt, v);
   if (rc != LQ_OK) return rc;
   const bool cluster_reduce = v.split_k > 1 && v.reduce == 2;
@@ -472,6 +494,7 @@ bool parse_table_file(const char* path, std::vector<TableEntry>* out, std::strin
     if (fmt_s == "fp8_dynamic" || fmt_s == "0") e.fmt = 0;
     else if (fmt_s == "w8a8_int8" || fmt_s == "1") e.fmt = 1;
     else if (fmt_s == "block_fp8" || fmt_s == "2") e.fmt = 2;
+    else if (fmt_s == "block_fp8_ue8m0" || fmt_s == "3") e.fmt = 3;
     else {
       *err = "bad format at line " + std::to_string(lineno);
       return false;
@@ -521,6 +544,10 @@ lq_status lq_test_inject_stall(int k_tile, uint64_t wait_limit_ns) {
   g_skip_stage.store(k_tile);
   g_wait_limit_override.store(wait_limit_ns);
   return LQ_OK;
+}
+
+int lq_declare_static_weights(int static_weights) {
+  return g_static_weights.exchange(static_weights ? 1 : 0);
 }
 
 lq_status lq_set_trace(uint64_t* device_buffer) {
@@ -577,6 +604,7 @@ lq_status lq_grouped_scaled_mm(lq_fmt fmt_, const void* A, const float* a_scales
     return LQ_ERR_ALIGNMENT;
   if (K % 16 != 0 || N % 8 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
   if (T > 0x7FFFFFFF || E > 0x7FFFFFFF || E * N > 0x7FFFFFFF || K > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (fmt == lq::kFmtInt8 && K > kInt8MaxK) return LQ_ERR_UNSUPPORTED_SHAPE;
   lq_variant v = variant ? *variant : heuristic_grouped(T, E, N, K);
   if (v.swap_ab != 1) return LQ_ERR_INVALID_ARG;   // tokens on the MMA N side
   if (v.split_k > 16) return LQ_ERR_INVALID_ARG;
@@ -663,27 +691,30 @@ lq_status lq_quant_scaled_mm(lq_fmt fmt_, const void* x, const void* B, const fl
     return LQ_ERR_ALIGNMENT;
   if (K % 16 != 0 || N % 8 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
   if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
-  lq_variant v{};
-  if (variant) v = *variant;
-  else if (!lookup_table(fmt, M, N, K, &v)) v = heuristic_variant(fmt, M, N, K);
-  if (v.split_k > 1) v.reduce = 2;   // the per-token amax is exchanged inside the Split-K cluster
+  if (fmt == lq::kFmtInt8 && K > kInt8MaxK) return LQ_ERR_UNSUPPORTED_SHAPE;
+  const lq_variant v = variant ? *variant : default_variant(fmt, M, N, K);
   // Each CTA of the fused kernel reads its tokens' slice of x once more to
   // find the per-token amax before any code exists; that read sits on the
   // critical path, so the kernel is used only while the slice is small.
   const int64_t T = (K + 127) / 128;
   const int64_t slice_bytes = (M < v.tile_n ? M : v.tile_n) * ((T + v.split_k - 1) / v.split_k) * 128 * 2;
+  lq_variant vf = v;
+  if (vf.split_k > 1) vf.reduce = 2;   // the per-token amax is exchanged inside the Split-K cluster
   const bool fusable = K > 0 && v.swap_ab == 1 && v.split_k <= 16 && v.split_k * v.tile_n <= 512 &&
-                       slice_bytes <= fuse_max_slice_bytes();
+                       slice_bytes <= fuse_max_slice_bytes() && check_variant(fmt, vf) == LQ_OK;
   if (!fusable) {
-    // quantize, then scaled_mm (same codes, scales and result as the fused kernel)
-    if (M > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED_SHAPE;
+    // quantize, then scaled_mm (same codes, scales and result as the fused kernel);
+    // the variant is checked before the first launch
+    const lq_status vrc = check_variant(fmt, v);
+    if (vrc != LQ_OK) return vrc;
     if (lq::launch_quant_per_token(fmt, x, a_codes, a_scales, M, K, stream) != cudaSuccess) {
       cudaGetLastError();
       return LQ_ERR_CUDA;
     }
-    return scaled_mm_impl(fmt, a_codes, a_scales, B, b_scales, C, nullptr, M, N, K, variant ? &v : nullptr, stream);
+    return scaled_mm_impl(fmt, a_codes, a_scales, B, b_scales, C, nullptr, M, N, K, &v, stream);
   }
-  return scaled_mm_impl(fmt, a_codes, a_scales, B, b_scales, C, nullptr, M, N, K, &v, stream, x, a_codes, a_scales);
+  return scaled_mm_impl(fmt, a_codes, a_scales, B, b_scales, C, nullptr, M, N, K, &vf, stream, x, a_codes,
+                        a_scales);
 }
 
 int64_t lq_set_fuse_limit(int64_t max_slice_bytes) {
@@ -836,7 +867,7 @@ lq_status lq_quant_weight_block128_ue8m0(const void* w, void* q, uint8_t* scales
 
 lq_status lq_select_variant(lq_fmt fmt, int64_t M, int64_t N, int64_t K, lq_variant* out) {
   if (!out || fmt < 0 || fmt > 3 || M < 0 || N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
-  if (!lookup_table(static_cast<int>(fmt), M, N, K, out)) *out = heuristic_variant(static_cast<int>(fmt), M, N, K);
+  *out = default_variant(static_cast<int>(fmt), M, N, K);
   return LQ_OK;
 }
 
@@ -876,9 +907,7 @@ lq_status lq_reserve_workspace(int device, size_t bytes) {
 
 size_t lq_workspace_bytes(lq_fmt fmt, int64_t M, int64_t N, int64_t K, const lq_variant* variant) {
   if (M <= 0 || N <= 0 || K <= 0 || fmt < 0 || fmt > 3) return 0;
-  lq_variant v{};
-  if (variant) v = *variant;
-  else if (!lookup_table(static_cast<int>(fmt), M, N, K, &v)) v = heuristic_variant(static_cast<int>(fmt), M, N, K);
+  const lq_variant v = variant ? *variant : default_variant(static_cast<int>(fmt), M, N, K);
   if (v.split_k <= 1 || v.reduce == 2) return 0;
   return static_cast<size_t>(v.split_k) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
 }
@@ -961,12 +990,7 @@ extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const floa
   if (K == 0)
     return lq::launch_fill_zero_bf16(static_cast<__nv_bfloat16*>(C), M * N, stream) == cudaSuccess ? LQ_OK
                                                                                                   : LQ_ERR_CUDA;
-  lq_variant v{};
-  if (variant) {
-    v = *variant;
-  } else if (!lookup_table(fmt, M, N, K, &v)) {
-    v = heuristic_variant(fmt, M, N, K);
-  }
+  lq_variant v = variant ? *variant : default_variant(fmt, M, N, K);
   // Split-K partials always go through the scratch array and the separate
   // fixed-order reduction kernel (no arrival counters, nothing to re-arm).
   if (v.split_k > 1) v.reduce = 0;

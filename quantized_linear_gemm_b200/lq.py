@@ -40,7 +40,7 @@ EXPORTED = (
     "lq_quant_scaled_mm", "lq_set_fuse_limit", "lq_rms_norm_dynamic_per_token_quant",
     "lq_rms_norm_per_block_quant", "lq_silu_and_mul_dynamic_per_token_quant", "lq_silu_and_mul_per_block_quant",
     "lq_grouped_scaled_mm", "lq_quant_per_token_group128_ue8m0", "lq_quant_weight_block128_ue8m0",
-    "lq_scaled_mm_bias",
+    "lq_scaled_mm_bias", "lq_declare_static_weights",
 )
 
 
@@ -108,6 +108,8 @@ def lib() -> ctypes.CDLL:
             L.lq_test_inject_stall.restype = _i32
             L.lq_set_trace.argtypes = [_vp]
             L.lq_set_trace.restype = _i32
+            L.lq_declare_static_weights.argtypes = [_i32]
+            L.lq_declare_static_weights.restype = _i32
             L.lq_set_fuse_limit.argtypes = [ctypes.c_int64]
             L.lq_set_fuse_limit.restype = ctypes.c_int64
             L.lq_rms_norm_dynamic_per_token_quant.argtypes = [_i32, _vp, _vp, _vp, ctypes.c_float, _vp, _vp,
@@ -510,6 +512,13 @@ def set_trace(buf: torch.Tensor | None) -> None:
         _need(buf, "buf", (torch.int64,), 1)
         _one_device(buf)
     lib().lq_set_trace(None if buf is None else buf.data_ptr())
+
+
+def declare_static_weights(static: bool = True) -> bool:
+    """Declare that weights are never written while a GEMM reading them may
+    run, so that a default (None) variant may stream weight tiles before the
+    previous kernel finishes; returns the previous setting."""
+    return bool(lib().lq_declare_static_weights(1 if static else 0))
 
 
 def set_fuse_limit(max_slice_bytes: int) -> int:

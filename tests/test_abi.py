@@ -59,6 +59,47 @@ def test_scaled_mm_argument_checks(kw, code):
     assert _mm(**kw) == code
 
 
+def test_int8_depth_bound():
+    """W8A8_INT8 sums int8 products in int32: K up to 131071 cannot wrap
+    (131071 * 128 * 128 < 2^31); deeper K is refused before any launch."""
+    assert _mm(fmt=1, K=131072) == SHAPE
+    assert _mm(fmt=1, K=131072 + 16) == SHAPE
+    assert 131071 * 128 * 128 < 2 ** 31 <= 131072 * 128 * 128
+    # the other formats accumulate in fp32 and take any K
+    assert _mm(fmt=0, K=131072, M=0) == OK
+    v = lq.make_variant(swap_ab=1, split_k=2, tile_n=32)
+    rc = lq.lib().lq_grouped_scaled_mm(1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 16, 128, 131072,
+                                       ctypes.byref(v), None)
+    assert rc == SHAPE
+    rc = lq.lib().lq_quant_scaled_mm(1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 128, 131072, None, None)
+    assert rc == SHAPE
+
+
+def test_default_variant_waits_before_reading_weights():
+    """A NULL variant lowers the table's pdl 2 (weights streamed before the
+    dependency wait) to 1 until the caller declares static weights."""
+    prev = lq.declare_static_weights(False)
+    try:
+        shapes = [(1, 6144, 4096), (8, 4096, 4096), (32, 24576, 4096), (16, 4096, 12288)]
+        for fmt in (0, 1, 2):
+            for M, N, K in shapes:
+                assert lq.select_variant(fmt, M, N, K).pdl <= 1
+        assert lq.declare_static_weights(True) is False
+        assert any(lq.select_variant(0, M, N, K).pdl == 2 for M, N, K in shapes)
+        assert lq.declare_static_weights(False) is True
+        assert all(lq.select_variant(0, M, N, K).pdl <= 1 for M, N, K in shapes)
+    finally:
+        lq.declare_static_weights(prev)
+
+
+def test_quant_scaled_mm_checks_the_variant_before_launching():
+    """The two-kernel path checks the caller's variant before it launches the
+    quantization kernel: an invalid one launches nothing."""
+    v = lq.make_variant(swap_ab=1, split_k=3, tile_n=16)
+    assert lq.lib().lq_quant_scaled_mm(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 128, 1024,
+                                       ctypes.byref(v), None) == INVALID
+
+
 def test_empty_problem_is_a_noop():
     # M == 0 or N == 0: nothing to do, no pointer is needed
     assert _mm(M=0, A=None, B=None, C=None, a_s=None, b_s=None) == OK
