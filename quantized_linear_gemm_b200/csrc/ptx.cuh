@@ -142,6 +142,22 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_
       : "memory");
 }
 
+// D(tmem) (+)= (A . 2^(sfa - 127)) * (B . 2^(sfb - 127))^T, e4m3 x e4m3 -> f32,
+// with the tensor core's own block scaling: one UE8M0 scale factor per row
+// of A and per row of B for the instruction's 32 K elements, read from
+// tensor memory at sfa_tmem / sfb_tmem (the byte of each 32-bit column picked
+// by the scale-factor ids of the instruction descriptor).
+__device__ __forceinline__ void mma_mxf8f6f4_block_scale(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // Arrive (once) on `bar` when all tcgen05 operations issued so far by this
 // thread have completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -177,6 +193,19 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Warp-collective store of 32 lanes x 4 (x 8) consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // -------------------------------------------------- descriptors (tcgen05)
 // Shared-memory matrix descriptor of a K-major operand tile stored with the
 // 128-byte swizzle: rows of 128 bytes, 8-row core groups 1024 bytes apart.
@@ -200,6 +229,20 @@ template <bool kInt8>
 __host__ __device__ constexpr uint32_t make_idesc(int m, int n) {
   return (kInt8 ? (2u << 4) : (1u << 4)) | (kInt8 ? (1u << 7) : 0u) | (kInt8 ? (1u << 10) : 0u) |
          (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// Instruction descriptor of tcgen05.mma kind::mxf8f6f4 with block scaling,
+// e4m3 x e4m3 with UE8M0 scale factors, K-major A and B:
+//   b_sf_id [4,6): byte of B's scale-factor column; a_format [7,10) and
+//   b_format [10,13): e4m3 = 0; a_major bit 15, b_major bit 16: 0 = K-major;
+//   n_dim [17,23) = N >> 3; scale type bit 23: 1 = UE8M0; m_dim [24,29) =
+//   M >> 4; a_sf_id [29,31): byte of A's scale-factor column.  (No
+//   accumulator-format field: the accumulator is f32.)
+__host__ __device__ constexpr uint32_t make_idesc_mx(int m, int n) {
+  return (static_cast<uint32_t>(n >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_with_sf_ids(uint32_t idesc, uint32_t a_id, uint32_t b_id) {
+  return idesc | (b_id << 4) | (a_id << 29);
 }
 
 // ------------------------------------------------ grid dependency control

@@ -55,6 +55,22 @@ __host__ __device__ constexpr int tmem_cols_for(int cols) {
   return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
 }
 
+// Tensor-memory columns of the UE8M0 scale factors of the block-scaled MMA
+// (after the accumulator's TN columns).  Two slots, each the scale factors of
+// four consecutive 128-K blocks: one 32-bit column per 32 rows of an operand
+// tile, the byte of block t (0..3) of the group in bits [8t, 8t+8), row e of
+// the tile at lane e % 32 and column e / 32 of the operand's part of the
+// slot, the same in all four lane quarters.  X (128 rows) takes 4 columns, Y
+// (TN rows) max(4, TN / 32); slots start on 8-column boundaries.
+template <int TN>
+struct MxSf {
+  static constexpr int kBase = TN < 32 ? 32 : TN;
+  static constexpr int kXCols = 4;
+  static constexpr int kYCols = TN > 128 ? TN / 32 : 4;
+  static constexpr int kSlotCols = (kXCols + kYCols + 7) / 8 * 8;
+  static constexpr int kEnd = kBase + 2 * kSlotCols;
+};
+
 // Cluster Split-K reduction.  Tiles up to 64 wide push: every CTA sends its
 // partial columns, from registers, into slots in the shared memory of the
 // CTA that owns those columns (st.async, completion counted in bytes on the
@@ -160,7 +176,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // instantiations carry none of its code.
 // BIAS: the epilogue adds p.bias (also compile-time, for the same reason).
 template <int FMT, bool SWAP, int TN, bool FUSE = false, bool GROUPED = false, bool BIAS = false>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, SWAP ? 2 : 1)   // Swap-AB: two CTAs per SM
     scaled_mm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                         const GemmParams p) {
   static_assert(!FUSE || (SWAP && !is_block_fmt(FMT) && TN <= 64), "fused quantization: Swap-AB FP8/INT8 tiles");
@@ -169,9 +185,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // bytes the TMA delivers per stage (the fused path writes the activation slot itself)
   constexpr uint32_t kTmaStageBytes = FUSE ? Shape::kXBytes : Shape::kStageBytes;
   constexpr bool kInt8 = FMT == kFmtInt8;
-  constexpr bool kBlocked = is_block_fmt(FMT);
-  constexpr int kAccBufs = kBlocked ? 2 : 1;
-  constexpr int kTmemCols = tmem_cols_for(TN * kAccBufs);
+  constexpr bool kBlocked = is_block_fmt(FMT);        // scales per 128-K block: partials carry them
+  // UE8M0 Block_FP8: the tensor core applies the power-of-two block scales
+  // itself (kind::mxf8f6f4 block scaling, scale factors in tensor memory),
+  // so one accumulator runs over the whole K range.  fp32-scale Block_FP8
+  // promotes a per-block accumulator into registers instead.
+  constexpr bool kMX = FMT == kFmtBlockE8m0;
+  constexpr bool kPromote = kBlocked && !kMX;
+  constexpr int kAccBufs = kPromote ? 2 : 1;
+  constexpr int kTmemCols = kMX ? tmem_cols_for(MxSf<TN>::kEnd) : tmem_cols_for(TN * kAccBufs);
   constexpr int CH = TN < 32 ? TN : 32;   // TMEM columns per tcgen05.ld
 
   extern __shared__ uint8_t smem_raw[];
@@ -295,7 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < stages; ++s) {
       mbar_init(&c.full[s], FUSE ? kEpiThreads / 32 : 1);   // the TMA, or the four A-producer warps
       mbar_init(&c.empty[s], 1);
-      mbar_init(&c.xfull[s], 1);
+      // block-scaled MMA: xfull[0..1] = scale-factor slot written (the four
+      // epilogue warps), wfull[0..1] = slot read by the tensor core (commit)
+      mbar_init(&c.xfull[s], (kMX && s < 2) ? kEpiThreads / 32 : 1);
       mbar_init(&c.wfull[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -413,13 +437,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- MMA issuer
     grid_dependency_wait();
     if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc<kInt8>(kTileM, TN);
+      constexpr uint32_t idesc = kMX ? make_idesc_mx(kTileM, TN) : make_idesc<kInt8>(kTileM, TN);
       bool issued_any = false;
       for (int i = 0; i < nkb; ++i) {
         const int s = i % stages;
         const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
         uint32_t d_tmem = tmem_base;
-        if (kBlocked) {
+        if (kMX && (i & 3) == 0) {   // the scale factors of blocks i .. i+3 are in tensor memory
+          const int g = i >> 2;
+          if (!wait_bar(&c.xfull[g & 1], static_cast<uint32_t>(g >> 1) & 1u, p, c, 13)) break;
+        }
+        if (kPromote) {
           const int buf = i & 1;
           const uint32_t use = static_cast<uint32_t>(i >> 1);
           if (!wait_bar(&c.tempty[buf], (use & 1u) ^ 1u, p, c, 1)) break;
@@ -435,18 +463,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kTileK / kMmaK; ++kk) {
           // +32 bytes along K inside the 128-byte swizzle row = +2 in the 16-byte address field
-          const uint32_t acc = kBlocked ? (kk > 0) : (i > 0 || kk > 0);
-          if (kInt8)
+          const uint32_t acc = kPromote ? (kk > 0) : (i > 0 || kk > 0);
+          if constexpr (kMX) {
+            const uint32_t t = static_cast<uint32_t>(i & 3);   // this block's byte in the slot
+            const uint32_t sf = tmem_base + static_cast<uint32_t>(MxSf<TN>::kBase + ((i >> 2) & 1) * MxSf<TN>::kSlotCols);
+            mma_mxf8f6f4_block_scale(d_tmem, xd + 2 * kk, yd + 2 * kk, idesc_with_sf_ids(idesc, t, t), sf,
+                                     sf + MxSf<TN>::kXCols, acc);
+          } else if (kInt8) {
             mma_i8(d_tmem, xd + 2 * kk, yd + 2 * kk, idesc, acc);
-          else
+          } else {
             mma_f8f6f4(d_tmem, xd + 2 * kk, yd + 2 * kk, idesc, acc);
+          }
         }
         issued_any = true;
         mma_commit(&c.empty[s]);
-        if (kBlocked) mma_commit(&c.tfull[i & 1]);
+        if (kPromote) mma_commit(&c.tfull[i & 1]);
+        if (kMX && ((i & 3) == 3 || i == nkb - 1)) mma_commit(&c.wfull[(i >> 2) & 1]);   // slot read
       }
       trace_stamp(p, 4);
-      if (!kBlocked && nkb > 0 && !*c.abort_flag) mma_commit(&c.tfull[0]);
+      if (!kPromote && nkb > 0 && !*c.abort_flag) mma_commit(&c.tfull[0]);
       if (issued_any) {
         // All MMAs must be complete before TMEM is released at teardown.
         mma_commit(c.mma_done);
@@ -464,9 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // bounds of the tile's GEMM: tokens [.., m_end), weight rows [.., n_end)
     const int64_t M = m_end, N = n_end;
 
-    float accr[kBlocked ? TN : 1];
+    float accr[kPromote ? TN : 1];
 #pragma unroll
-    for (int j = 0; j < (kBlocked ? TN : 1); ++j) accr[j] = 0.f;
+    for (int j = 0; j < (kPromote ? TN : 1); ++j) accr[j] = 0.f;
 
     if (!kBlocked) {
       // Scales do not depend on the accumulator: load them while the mainloop
@@ -604,12 +639,91 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     bool ok = true;
-    if (kBlocked) {
+    if constexpr (kMX) {
+      // ------------------------------------- scale factors (block-scaled MMA)
+      // For each group of four K blocks of this CTA's range: gather the UE8M0
+      // bytes of the X tile's 128 rows and the Y tile's TN rows, pack four
+      // blocks per 32-bit column, write them to the group's slot in tensor
+      // memory (each warp its own lane quarter: the layout is the same in all
+      // four) and tell the MMA warp.  A slot is rewritten only after the
+      // tensor core has read it (wfull, committed by the MMA warp).  The
+      // bytes of the next group are loaded while the current one is used.
+      using Sf = MxSf<TN>;
+      const uint8_t* a_b = reinterpret_cast<const uint8_t*>(p.a_s);   // [M, KB]
+      const uint8_t* b_b = reinterpret_cast<const uint8_t*>(p.b_s);   // [N / 128, KB]
+      // byte of row e (< 128) of X, or of row e (< TN) of Y, for this CTA's block i
+      auto x_byte = [&](int e, int i) -> uint32_t {
+        if (i >= nkb) return 127u;
+        const int64_t kb = kb_lo + i;
+        if (SWAP) {
+          const int64_t n = x_row0 + e;
+          return n < N ? b_b[(n >> 7) * p.KB + kb] : 127u;
+        }
+        const int64_t m = x_row0 + e;
+        return m < M ? a_b[m * p.KB + kb] : 127u;
+      };
+      auto y_byte = [&](int e, int i) -> uint32_t {
+        if (i >= nkb || e >= TN) return 127u;
+        const int64_t kb = kb_lo + i;
+        if (SWAP) {
+          const int64_t m = y_row0 + e;
+          return m < M ? a_b[m * p.KB + kb] : 127u;
+        }
+        const int64_t n = y_row0 + e;
+        return n < N ? b_b[(n >> 7) * p.KB + kb] : 127u;
+      };
+      uint32_t wx[Sf::kXCols], wy[Sf::kYCols];
+      auto gather = [&](int g) {
+#pragma unroll
+        for (int col = 0; col < Sf::kXCols; ++col) {
+          uint32_t w = 0;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) w |= x_byte(col * 32 + lane, 4 * g + t) << (8 * t);
+          wx[col] = w;
+        }
+#pragma unroll
+        for (int col = 0; col < Sf::kYCols; ++col) {
+          uint32_t w = 0;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) w |= y_byte(col * 32 + lane, 4 * g + t) << (8 * t);
+          wy[col] = w;
+        }
+      };
+      const int groups = (nkb + 3) / 4;
+      if (groups > 0) gather(0);
+      for (int g = 0; g < groups && ok; ++g) {
+        const int slot = g & 1;
+        if (g >= 2) ok = __all_sync(0xffffffffu, wait_bar(&c.wfull[slot], static_cast<uint32_t>((g - 2) >> 1) & 1u, p, c, 14));
+        if (!ok) break;
+        tc_fence_after_sync();
+        const uint32_t col0 = t_row + static_cast<uint32_t>(Sf::kBase + slot * Sf::kSlotCols);
+        tmem_st_32x32b_x4(col0, wx);
+        if constexpr (Sf::kYCols == 8)
+          tmem_st_32x32b_x8(col0 + Sf::kXCols, wy);
+        else
+          tmem_st_32x32b_x4(col0 + Sf::kXCols, wy);
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.xfull[slot]);
+        if (g + 1 < groups) gather(g + 1);
+      }
+      if (ok && nkb > 0) {
+        ok = wait_bar(&c.tfull[0], 0, p, c, 5);
+        tc_fence_after_sync();
+      }
+    } else if (kPromote) {
       // Per-128-K-block promotion: acc += D_kb * a_s[m, kb] * b_s[nb, kb].
-      // The scale products of block kb+1 are loaded while block kb is
-      // waited for and promoted (double buffer blksc, one named barrier per
-      // block).  Every thread runs every iteration (also after a timeout),
-      // so the named barriers always match.
+      // The scale products are loaded kPre blocks at a time, a group ahead:
+      // the loads of group g + 1 are issued as group g starts, so their
+      // latency (an L2 round trip while the operand stream keeps L2 busy)
+      // hides behind kPre blocks of promotion.  (Loaded one block ahead, the
+      // register copy that carries the value into the next iteration waited
+      // for the load every block.)  Swap-AB stages each block's products in
+      // shared memory (double buffer blksc, one named barrier per block).
+      // Every thread runs every iteration (also after a timeout), so the
+      // named barriers always match.
+      constexpr int kPre = SWAP ? 4 : 8;   // Swap-AB: fewer registers (two CTAs per SM at tile_n 64)
       const int nb = SWAP ? x_row0 / 128 : y_row0 / 128;
       const int64_t m_thread = x_row0 + r;   // Standard: this thread's token
       // Block scale i of an operand: fp32, or a UE8M0 byte (2^(b - 127)).
@@ -621,7 +735,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           return __ldg(base + i);
         }
       };
-      auto load_scale = [&](int kb) -> float {
+      const bool loader = SWAP ? (r < TN) : true;
+      auto load_scale = [&](int i) -> float {   // product of the CTA's i-th block (0 past the range)
+        if (!loader || i >= nkb) return 0.f;
+        const int kb = kb_lo + i;
         const float sb = scale_at(p.b_s, static_cast<int64_t>(nb) * p.KB + kb);
         if (SWAP) {
           const int64_t m = y_row0 + r;     // column r of the tile (r < TN)
@@ -629,43 +746,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return (m_thread < M ? scale_at(p.a_s, m_thread * p.KB + kb) : 0.f) * sb;
       };
-      const bool loader = SWAP ? (r < TN) : true;
-      float cur = 0.f;   // Standard: this thread's scale product of the current block
-      if (nkb > 0 && loader) {
-        cur = load_scale(kb_lo);
-        if (SWAP) blksc[r] = cur;
+      float cur[kPre], nxt[kPre];
+#pragma unroll
+      for (int j = 0; j < kPre; ++j) cur[j] = load_scale(j);
+      if (SWAP) {
+        if (loader) blksc[r] = cur[0];
+        named_barrier_sync(2, kEpiThreads);
       }
-      if (SWAP) named_barrier_sync(2, kEpiThreads);
-      for (int i = 0; i < nkb; ++i) {
-        const int buf = i & 1;
-        const uint32_t use = static_cast<uint32_t>(i >> 1);
-        const float nxt = (loader && i + 1 < nkb) ? load_scale(kb_lo + i + 1) : 0.f;
-        // warp-uniform decision: the tcgen05.ld below is .sync.aligned
-        if (ok) ok = __all_sync(0xffffffffu, wait_bar(&c.tfull[buf], use & 1u, p, c, 4));
-        if (ok) {
-          tc_fence_after_sync();
-          const float* bs = blksc + (i & 1) * 256;
+      for (int i0 = 0; i0 < nkb; i0 += kPre) {
 #pragma unroll
-          for (int c0 = 0; c0 < TN; c0 += CH) {
-            uint32_t v[CH];
-            if constexpr (CH == 32)
-              tmem_ld_32x32b_x32(t_row + buf * TN + c0, v);
-            else
-              tmem_ld_32x32b_x16(t_row + buf * TN + c0, v);
-            tmem_ld_wait();
+        for (int j = 0; j < kPre; ++j) nxt[j] = load_scale(i0 + kPre + j);
 #pragma unroll
-            for (int j = 0; j < CH; ++j)
-              accr[c0 + j] = fmaf(__uint_as_float(v[j]), SWAP ? bs[c0 + j] : cur, accr[c0 + j]);
+        for (int j = 0; j < kPre; ++j) {
+          const int i = i0 + j;
+          if (i < nkb) {   // the same for every epilogue thread
+            const int buf = i & 1;
+            const uint32_t use = static_cast<uint32_t>(i >> 1);
+            // warp-uniform decision: the tcgen05.ld below is .sync.aligned
+            if (ok) ok = __all_sync(0xffffffffu, wait_bar(&c.tfull[buf], use & 1u, p, c, 4));
+            if (ok) {
+              tc_fence_after_sync();
+              const float* bs = blksc + (i & 1) * 256;
+#pragma unroll
+              for (int c0 = 0; c0 < TN; c0 += CH) {
+                uint32_t v[CH];
+                if constexpr (CH == 32)
+                  tmem_ld_32x32b_x32(t_row + buf * TN + c0, v);
+                else
+                  tmem_ld_32x32b_x16(t_row + buf * TN + c0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int jj = 0; jj < CH; ++jj)
+                  accr[c0 + jj] = fmaf(__uint_as_float(v[jj]), SWAP ? bs[c0 + jj] : cur[j], accr[c0 + jj]);
+              }
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&c.tempty[buf]);
+            }
+            if (SWAP) {
+              if (loader && i + 1 < nkb) blksc[((i + 1) & 1) * 256 + r] = j + 1 < kPre ? cur[j + 1] : nxt[0];
+              named_barrier_sync(2, kEpiThreads);
+            }
           }
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&c.tempty[buf]);
         }
-        cur = nxt;
-        if (SWAP) {
-          if (loader && i + 1 < nkb) blksc[((i + 1) & 1) * 256 + r] = nxt;
-          named_barrier_sync(2, kEpiThreads);
-        }
+#pragma unroll
+        for (int j = 0; j < kPre; ++j) cur[j] = nxt[j];
       }
     } else if (nkb > 0) {
       ok = wait_bar(&c.tfull[0], 0, p, c, 5);
@@ -693,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c0 = 0; c0 < TN; c0 += CH) {
         uint32_t v[CH];
-        if (kBlocked) {
+        if (kPromote) {
 #pragma unroll
           for (int j = 0; j < CH; ++j) v[j] = __float_as_uint(accr[c0 + j]);
         } else if (nkb > 0) {

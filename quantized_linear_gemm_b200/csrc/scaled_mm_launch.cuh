@@ -56,8 +56,8 @@ cudaError_t launch_dense(const GemmLaunch& l, int swap_ab, int tile_n) {
   switch (tile_n) {
     case 64: return launch_tc<FMT, false, 64, false, false, BIAS>(l);
     case 128: return launch_tc<FMT, false, 128, false, false, BIAS>(l);
-    case 256:
-      if constexpr (!is_block_fmt(FMT)) return launch_tc<FMT, false, 256, false, false, BIAS>(l);
+    case 256:   // fp32-scale Block_FP8 promotes in registers: its tiles stop at 128
+      if constexpr (FMT != kFmtBlock) return launch_tc<FMT, false, 256, false, false, BIAS>(l);
       return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }

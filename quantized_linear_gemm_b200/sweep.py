@@ -35,7 +35,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 TABLE_TXT = os.path.join(PKG, "dispatch_table.txt")
 TABLE_INC = os.path.join(PKG, "csrc", "dispatch_table.inc")
 L2_BYTES = 126 * 2 ** 20
-FMT_NAMES = {lq.FP8_DYNAMIC: "fp8_dynamic", lq.W8A8_INT8: "w8a8_int8", lq.BLOCK_FP8: "block_fp8"}
+FMT_NAMES = {lq.FP8_DYNAMIC: "fp8_dynamic", lq.W8A8_INT8: "w8a8_int8", lq.BLOCK_FP8: "block_fp8",
+             lq.BLOCK_FP8_UE8M0: "block_fp8_ue8m0"}
 
 
 def keys_for(groups):
@@ -55,6 +56,15 @@ def keys_for(groups):
                 K, N = inputs.QWEN3_32B[layer]
                 for M in inputs.PREFILL_M:
                     keys.append((fmt, M, N, K))
+    if "ue8m0" in groups:   # Block_FP8 with UE8M0 scales (the tensor core's block-scaled MMA)
+        for (K, N) in inputs.QWEN3_32B.values():
+            for M in inputs.DECODE_M:
+                keys.append((lq.BLOCK_FP8_UE8M0, M, N, K))
+    if "ue8m0-prefill" in groups:
+        for layer in ("gate_up", "down"):
+            K, N = inputs.QWEN3_32B[layer]
+            for M in inputs.PREFILL_M:
+                keys.append((lq.BLOCK_FP8_UE8M0, M, N, K))
     return keys
 
 
@@ -82,7 +92,7 @@ def candidates(fmt, M, N, K):
                     add(swap_ab=1, tile_n=tn, split_k=S, stages=2, reduce=1, pdl=2)
                     add(swap_ab=1, tile_n=tn, split_k=S, stages=2, reduce=0, pdl=2)
     if M >= 16:
-        tns = (64, 128) if fmt == lq.BLOCK_FP8 else (64, 128, 256)
+        tns = (64, 128) if fmt == lq.BLOCK_FP8 else (64, 128, 256)   # fp32-scale Block_FP8: up to 128
         for tn in tns:
             for S in (1, 2, 4, 8):
                 if S > T:
@@ -99,7 +109,7 @@ class Shape:
 
     def __init__(self, fmt, M, N, K, device, with_quant=False):
         self.fmt, self.M, self.N, self.K = fmt, M, N, K
-        self.with_quant = with_quant and fmt != lq.BLOCK_FP8
+        self.with_quant = with_quant and fmt not in (lq.BLOCK_FP8, lq.BLOCK_FP8_UE8M0)
         name = FMT_NAMES[fmt]
         w = inputs.weights(N, K, seed=inputs.stable_seed("sweep-W", N, K)).to(device)
         x = inputs.activations(M, K, seed=inputs.stable_seed("sweep-A", M, K)).to(device)
@@ -107,6 +117,9 @@ class Shape:
         if fmt == lq.BLOCK_FP8:
             qb, sb = lq.quant_weight_block128(w)
             self.qa, self.sa = lq.quant_per_token_group128(x)
+        elif fmt == lq.BLOCK_FP8_UE8M0:
+            qb, sb = lq.quant_weight_block128_ue8m0(w)
+            self.qa, self.sa = lq.quant_per_token_group128_ue8m0(x)
         else:
             qb, sb = lq.quant_per_token(name, w)
             self.qa, self.sa = lq.quant_per_token(name, x)
@@ -206,8 +219,26 @@ def write_table(results, path):
         f.write("\n".join(lines) + "\n")
 
 
+def merge_table(base_path, new_path, out_path):
+    """The entries of base_path with those of new_path added; an entry of
+    new_path replaces the base entry of the same (fmt, m_bucket, N, K)."""
+    def entries(path):
+        out = []
+        for line in open(path):
+            body = line.split("#")[0].split()
+            if body:
+                out.append((tuple(body[:4]), line.rstrip("\n")))
+        return out
+    new = entries(new_path)
+    keys = {k for k, _ in new}
+    kept = [ln for k, ln in entries(base_path) if k not in keys]
+    head = [ln.rstrip("\n") for ln in open(base_path) if ln.startswith("#")]
+    with open(out_path, "w") as f:
+        f.write("\n".join(head + kept + [ln for _, ln in new]) + "\n")
+
+
 def write_inc(txt_path, inc_path):
-    fmt_id = {"fp8_dynamic": 0, "w8a8_int8": 1, "block_fp8": 2}
+    fmt_id = {"fp8_dynamic": 0, "w8a8_int8": 1, "block_fp8": 2, "block_fp8_ue8m0": 3}
     rows = []
     for line in open(txt_path):
         line = line.split("#")[0].split()
@@ -234,6 +265,8 @@ def main():
     ap.add_argument("--inc-only", action="store_true", help="only regenerate the .inc from an existing table")
     ap.add_argument("--budget-s", type=float, default=None)
     ap.add_argument("--formats", default=None, help="comma-separated subset, e.g. fp8_dynamic")
+    ap.add_argument("--merge", default=None, metavar="TABLE",
+                    help="merge the measured entries into TABLE (same key: replaced) and write the result to --out")
     ap.add_argument("--with-quant", action="store_true",
                     help="time each candidate after lq_quant_per_token, as the decode step runs it")
     a = ap.parse_args()
@@ -246,7 +279,13 @@ def main():
     lq.load_dispatch_table(None)
     fmts = None if a.formats is None else {lq.FORMATS[f] for f in a.formats.split(",")}
     res = sweep(set(a.configs.split(",")), device, budget_s=a.budget_s, with_quant=a.with_quant, formats=fmts)
-    write_table(res, a.out)
+    if a.merge:
+        tmp = a.out + ".new"
+        write_table(res, tmp)
+        merge_table(a.merge, tmp, a.out)
+        os.remove(tmp)
+    else:
+        write_table(res, a.out)
     if a.json:
         with open(a.json, "w") as f:
             for r in res:
