@@ -53,7 +53,12 @@ CONFIGS = {
     "qwen3-32b-fp8-prefill": ("fp8_dynamic", {k: inputs.QWEN3_32B[k] for k in ("gate_up", "down")}, inputs.PREFILL_M),
     "qwen3-32b-int8-prefill": ("w8a8_int8", {k: inputs.QWEN3_32B[k] for k in ("gate_up", "down")}, inputs.PREFILL_M),
     "qwen3-32b-block-prefill": ("block_fp8", {k: inputs.QWEN3_32B[k] for k in ("gate_up", "down")}, inputs.PREFILL_M),
+    # Block_FP8 with power-of-two (UE8M0) scales: the tensor core's block-scaled MMA
+    "qwen3-32b-ue8m0-decode": ("block_fp8_ue8m0", inputs.QWEN3_32B, inputs.DECODE_M),
+    "qwen3-32b-ue8m0-prefill": ("block_fp8_ue8m0", {k: inputs.QWEN3_32B[k] for k in ("gate_up", "down")},
+                                inputs.PREFILL_M),
 }
+BLOCK_FMTS = ("block_fp8", "block_fp8_ue8m0")
 DEFAULT_CONFIG = "qwen3-8b-fp8-decode"
 L2_BYTES = 126 * 2 ** 20
 
@@ -66,6 +71,22 @@ def load_peaks() -> dict:
                 "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
                 "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def tensor_peak_8bit(fmt: str, peaks: dict) -> tuple[float, str]:
+    """(TFLOP/s, source) of the dense 8-bit tensor-core peak for a kernel timed
+    inside a long step: the sustained figure measured on this machine with a
+    library GEMM (profiles/tensor_peaks_8bit.json, written by
+    ``python -m quantized_linear_gemm_b200.peaks``), e4m3 for the FP8 formats
+    and int8 for W8A8_INT8; without that file, twice the measured bf16
+    sustained figure (the nominal 8-bit : bf16 ratio)."""
+    p = os.path.join(ROOT, "profiles", "tensor_peaks_8bit.json")
+    key = "int8" if fmt == "w8a8_int8" else "e4m3"
+    if os.path.exists(p):
+        d = json.load(open(p)).get(key, {})
+        if "tflops_sustained" in d:
+            return float(d["tflops_sustained"]), f"measured {key} sustained ({d.get('call', 'library GEMM')})"
+    return 2.0 * peaks["bf16_tflops_sustained"], f"{peaks['source']} bf16 sustained x 2 (nominal 8-bit : bf16 ratio)"
 
 
 def kernel_sources_digest() -> str:
@@ -119,7 +140,7 @@ def gemm_bytes(fmt: str, M: int, N: int, K: int) -> int:
 
 def quant_bytes(fmt: str, M: int, K: int) -> int:
     """bf16 read + codes written + scales written."""
-    scales = 4 * M * (K // 128) if fmt == "block_fp8" else 4 * M
+    scales = {"block_fp8": 4 * M * (K // 128), "block_fp8_ue8m0": M * (K // 128)}.get(fmt, 4 * M)
     return 2 * M * K + M * K + scales
 
 
@@ -182,9 +203,13 @@ class Workload:
     """Device buffers of one configuration: rotated weight copies, bf16
     activations, codes, scales and outputs of every (M, layer) call."""
 
-    def __init__(self, config: str, device: torch.device, copies: int = 3, seed: int = 0):
+    def __init__(self, config: str, device: torch.device, copies: int = 3, seed: int = 0, ms=None, layers=None):
         self.config = config
         self.fmt, self.layers, self.ms = CONFIGS[config]
+        if ms:   # a subset of the configuration's token counts (profiling of one shape)
+            self.ms = [m for m in self.ms if m in ms]
+        if layers:
+            self.layers = {k: v for k, v in self.layers.items() if k in layers}
         self.device = device
         self.copies = copies
         f = self.fmt
@@ -193,6 +218,8 @@ class Workload:
             w = inputs.weights(N, K, seed=inputs.stable_seed(config, "W", layer, seed)).to(device)
             if f == "block_fp8":
                 q, s = lq.quant_weight_block128(w)
+            elif f == "block_fp8_ue8m0":
+                q, s = lq.quant_weight_block128_ue8m0(w)
             else:
                 q, s = lq.quant_per_token(f, w)
             # enough copies that more than 2x L2 is streamed between two reads of one copy
@@ -220,7 +247,10 @@ class Workload:
             c["x"].copy_(x)
             c["C"] = self.c_all[c["c_off"]:c["c_off"] + M * N].view(M, N)
             c["q"] = torch.empty((M, K), dtype=code_dt, device=device)
-            c["s"] = torch.empty((M, K // 128) if f == "block_fp8" else (M,), dtype=torch.float32, device=device)
+            if f == "block_fp8_ue8m0":
+                c["s"] = torch.empty((M, K // 128), dtype=torch.uint8, device=device)
+            else:
+                c["s"] = torch.empty((M, K // 128) if f == "block_fp8" else (M,), dtype=torch.float32, device=device)
             c["copy"] = self.ms.index(M) % len(self.weights[c["layer"]])
             c["variant"] = lq.select_variant(f, M, N, K)
         self.x_host = torch.empty(self.x_all.shape, dtype=torch.bfloat16, pin_memory=True)
@@ -267,6 +297,8 @@ class Workload:
     def quant(self, c, stream):
         if self.fmt == "block_fp8":
             lq.quant_per_token_group128(c["x"], c["q"], c["s"], stream=stream)
+        elif self.fmt == "block_fp8_ue8m0":
+            lq.quant_per_token_group128_ue8m0(c["x"], c["q"], c["s"], stream=stream)
         else:
             lq.quant_per_token(self.fmt, c["x"], c["q"], c["s"], stream=stream)
 
@@ -452,42 +484,69 @@ def time_replays(g: torch.cuda.CUDAGraph, n: int, stream, pre=None, post=None) -
 
 
 # ----------------------------------------------------------- CPU leg
+def _oracle_quant_weight(fmt: str, w):
+    from oracle import lq_oracle as O
+    from oracle import ue8m0_oracle as U
+    if fmt == "block_fp8":
+        return O.quant_weight_block128(w)
+    if fmt == "block_fp8_ue8m0":
+        return U.quant_weight_block128_ue8m0(w)
+    return O.quant_per_channel(w, fmt)
+
+
+def _oracle_step(fmt: str, x, qb, sb) -> None:
+    """Quantize activations and compute the exact product, with the oracle."""
+    from oracle import lq_oracle as O
+    from oracle import ue8m0_oracle as U
+    if fmt == "block_fp8":
+        qa, sa = O.quant_per_token_group128(x)
+        O.blockwise_ref(qa, sa, qb, sb)
+    elif fmt == "block_fp8_ue8m0":
+        qa, sa = U.quant_per_token_group128_ue8m0(x)
+        U.blockwise_ue8m0_ref(qa, sa, qb, sb)
+    else:
+        qa, sa = O.quant_per_token(x, fmt)
+        O.scaled_mm_ref(fmt, qa, sa, qb, sb)
+
+
 def cpu_baseline(config: str, budget_s: float = 20.0) -> dict:
     """The oracle, as it stands, on a bounded sample of the same workload:
     every linear at the middle decode size (activation quantization plus the
-    exact product), repeated until about `budget_s` seconds have passed."""
-    import numpy as np
-    from oracle import lq_oracle as O
+    exact product), repeated until about `budget_s` seconds have passed, once
+    on one core and once on every host core (output columns split over
+    worker processes).  `value` and `cores` are the all-core figures."""
+    from oracle import parallel_runner
 
     fmt, layers, ms = CONFIGS[config]
     M = ms[len(ms) // 2]
     prepared = []
     for layer, (K, N) in layers.items():
         w = inputs.weights(N, K, seed=inputs.stable_seed(config, "W", layer, 0)).float().numpy()
-        if fmt == "block_fp8":
-            qb, sb = O.quant_weight_block128(w)
-        else:
-            qb, sb = O.quant_per_channel(w, fmt)
+        qb, sb = _oracle_quant_weight(fmt, w)
         x = inputs.activations(M, K, seed=inputs.stable_seed(config, "A", layer, M, 0)).float().numpy()
         prepared.append((M, N, K, x, qb, sb))
-    nbytes = 0
+    round_bytes = sum(gemm_bytes(fmt, M_, N, K) + quant_bytes(fmt, M_, K) for (M_, N, K, _, _, _) in prepared)
     t0 = time.perf_counter()
     rounds = 0
     while True:
-        for (M_, N, K, x, qb, sb) in prepared:
-            if fmt == "block_fp8":
-                qa, sa = O.quant_per_token_group128(x)
-            else:
-                qa, sa = O.quant_per_token(x, fmt)
-            O.scaled_mm_ref(fmt, qa, sa, qb, sb)
-            nbytes += gemm_bytes(fmt, M_, N, K) + quant_bytes(fmt, M_, K)
+        for (_, _, _, x, qb, sb) in prepared:
+            _oracle_step(fmt, x, qb, sb)
         rounds += 1
-        if time.perf_counter() - t0 > budget_s or rounds >= 50:
+        if time.perf_counter() - t0 > budget_s / 2 or rounds >= 50:
             break
-    dt = time.perf_counter() - t0
-    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{config}: all {len(layers)} linears at M={M}, quantize + exact product, {rounds} round(s), "
-                      f"{dt:.1f} s (numpy int64 matmul, single thread)"}
+    dt1 = time.perf_counter() - t0
+    single = rounds * round_bytes / dt1 / 1e9
+    box_cores = os.cpu_count() or 1
+    par = parallel_runner.time_all_cores(fmt, [(x, qb, sb) for (_, _, _, x, qb, sb) in prepared], budget_s / 2)
+    value = par["rounds"] * round_bytes / par["seconds"] / 1e9
+    return {"value": value, "unit": "GB/s", "cores": par["workers"], "kind": "oracle",
+            "single_core": {"value": single, "unit": "GB/s", "cores": 1, "rounds": rounds,
+                            "seconds": round(dt1, 2)},
+            "box_cores": box_cores,
+            "sample": f"{config}: all {len(layers)} linears at M={M}, quantize + exact product; all-core: "
+                      f"{par['rounds']} round(s) in {par['seconds']:.1f} s, output columns split into "
+                      f"{par['tasks_per_round']} slices over {par['workers']} worker processes (numpy int64 "
+                      f"matmul is single-threaded); single core: {rounds} round(s) in {dt1:.1f} s"}
 
 
 def run_reference(args) -> None:
@@ -514,19 +573,15 @@ def run_reference(args) -> None:
         n_max = min(N, 2048)   # weights are pre-quantized (not part of a step)
         w = inputs.weights(n_max, K, seed=inputs.stable_seed(cfg, "W", layer, 0)).float().numpy()
         x = inputs.activations(M, K, seed=inputs.stable_seed(cfg, "A", layer, M, 0)).float().numpy()
-        qw = O.quant_weight_block128(w) if fmt == "block_fp8" else O.quant_per_channel(w, fmt)
+        qw = _oracle_quant_weight(fmt, w)
         prepared[layer] = (K, N, x, qw, n_max)
 
     def one(layer, n_cols):
         K, N, x, (qw, sw), _ = prepared[layer]
         qb = qw[:n_cols]
-        sb = sw[:n_cols // 128] if fmt == "block_fp8" else sw[:n_cols]
+        sb = sw[:n_cols // 128] if fmt in BLOCK_FMTS else sw[:n_cols]
         t0 = time.perf_counter()
-        if fmt == "block_fp8":
-            qa, sa = O.quant_per_token_group128(x)
-        else:
-            qa, sa = O.quant_per_token(x, fmt)
-        O.scaled_mm_ref(fmt, qa, sa, qb, sb)
+        _oracle_step(fmt, x, qb, sb)
         return time.perf_counter() - t0, gemm_bytes(fmt, M, n_cols, K) + quant_bytes(fmt, M, K)
 
     # calibrate columns per second on each layer, then size every step to the budget
@@ -558,7 +613,8 @@ def run_reference(args) -> None:
 
 
 METRIC = "scaled_mm HBM GB/s (algorithmic bytes) at M=1..32 on Qwen3 linear shapes"
-DTYPE = {"fp8_dynamic": "e4m3 x e4m3 -> f32", "w8a8_int8": "s8 x s8 -> s32", "block_fp8": "e4m3 x e4m3 -> f32"}
+DTYPE = {"fp8_dynamic": "e4m3 x e4m3 -> f32", "w8a8_int8": "s8 x s8 -> s32", "block_fp8": "e4m3 x e4m3 -> f32",
+         "block_fp8_ue8m0": "e4m3 x e4m3 (UE8M0 block scales) -> f32"}
 
 
 # ---------------------------------------------------------------- main
@@ -575,6 +631,9 @@ def main() -> None:
     ap.add_argument("--no-producers", action="store_true",
                     help="skip the per-call timing of the producer-side fused quantizers")
     ap.add_argument("--no-moe", action="store_true", help="skip the grouped (MoE) GEMM timing")
+    ap.add_argument("--ms", default=None,
+                    help="comma-separated subset of the configuration's token counts (e.g. to profile one shape)")
+    ap.add_argument("--layers", default=None, help="comma-separated subset of the configuration's linears")
     ap.add_argument("--path", default="separate", choices=["fused", "separate"],
                     help="fused: one lq_quant_scaled_mm per linear (quantization inside the GEMM kernel); "
                          "separate: lq_quant_per_token then lq_scaled_mm")
@@ -596,14 +655,20 @@ def main() -> None:
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     lq.init_device(local)
+    # the weights are quantized once, before any timed work, and never written afterwards
+    lq.declare_static_weights(True)
     peaks = load_peaks()
 
-    wl = Workload(args.config, device, copies=args.copies)
+    wl = Workload(args.config, device, copies=args.copies,
+                  ms=[int(m) for m in args.ms.split(",")] if args.ms else None,
+                  layers=args.layers.split(",") if args.layers else None)
+    if not wl.calls:
+        raise SystemExit("--ms / --layers leave no call of the configuration")
     stream = torch.cuda.Stream(device=device)
     stream.wait_stream(torch.cuda.current_stream())
 
     # one CUDA graph per step (quant + GEMM of every call), and GEMM-only / quant-only graphs
-    use_fused = args.path == "fused" and wl.fmt != "block_fp8"
+    use_fused = args.path == "fused" and wl.fmt not in BLOCK_FMTS
     if use_fused:
         lq.set_fuse_limit(1 << 40)   # every fusable call takes the one-kernel path
     g_step = capture(lambda: wl.step(stream, fused=use_fused), stream)
@@ -642,7 +707,7 @@ def main() -> None:
 
     # per-shape breakdown: R calls of one shape per graph, rotating weight copies
     compute_bound = min(wl.ms) >= 256        # prefill configs: tensor-bound
-    tensor_peak = 2.0 * peaks["bf16_tflops_sustained"]
+    tensor_peak, tensor_peak_source = tensor_peak_8bit(wl.fmt, peaks)
     per_shape = []
     for c in wl.calls:
         reps = max(args.per_shape_reps, len(wl.weights[c["layer"]]))
@@ -767,7 +832,7 @@ def main() -> None:
                     "traffic_unit": "DRAM bytes per step of scaled_mm launches (ncu)",
                     "algorithmic_flops_per_step": wl.flops, "launches_per_step": wl.launches_per_step(quant=False),
                     "us_per_step": round(ms_gemm * 1e3, 2),
-                    "peak_source": f"{peaks['source']} bf16 sustained x 2 (nominal 8-bit : bf16 tensor ratio)"}
+                    "peak_source": tensor_peak_source}
     else:
         roofline = {"bound": "hbm", "kernel": "scaled_mm (all launches of one step)",
                     "achieved": round(gemm_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -789,7 +854,8 @@ def main() -> None:
         "vs_baseline": None,
         "dtype": DTYPE[wl.fmt],
         "data": "synthetic",
-        "config": {"workload": args.config, "format": wl.fmt, "layers": layers, "M": list(wl.ms),
+        "config": {"workload": args.config + ("" if not (args.ms or args.layers) else " (subset)"),
+                   "format": wl.fmt, "layers": layers, "M": list(wl.ms),
                    "calls_per_step": len(wl.calls), "parallelism": f"replicas x{world}",
                    "l2": "weight copies rotated so that > 2x L2 is streamed between two reads of one copy",
                    "graph": "one CUDA graph per step",
@@ -800,7 +866,7 @@ def main() -> None:
         "roofline": roofline,
         "scaled_mm_only": {"GB/s": round(gemm_gbs, 1), "frac": round(gemm_gbs / peaks["hbm_gbs"], 4),
                            "us_per_step": round(ms_gemm * 1e3, 2), "algorithmic_bytes_per_step": wl.gemm_bytes,
-                           "what": "the step's 28 lq_scaled_mm calls alone (codes already quantized)"},
+                           "what": f"the step's {len(wl.calls)} lq_scaled_mm calls alone (codes already quantized)"},
         "quant_us_per_step": round(ms_quant * 1e3, 2),
         "clocks": clocks,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "ms_per_step": round(ms_e2e, 5),
