@@ -110,6 +110,12 @@ typedef enum {
  *            through distributed shared memory, each finishing a slice of the
  *            tile (split_k <= 16, no workspace).  All three sum the partials
  *            in the order s = 0..split_k-1 and give identical results.
+ *  persistent : 0 = one output tile per CTA; 1 = persistent CTAs (Standard
+ *            orientation, split_k 1, FP8_DYNAMIC / W8A8_INT8; tile_n 64, 128
+ *            or 256): one CTA per SM loops over the output tiles, its
+ *            shared-memory ring runs on across tiles, and the accumulator is
+ *            double-buffered in tensor memory so that a tile's epilogue
+ *            overlaps the next tile's mainloop.  Same results bit for bit.
  *  pdl     : 0 = plain launch;
  *            1 = programmatic dependent launch: the kernel's set-up overlaps
  *            the tail of the previous kernel on the stream, and all of its
@@ -128,6 +134,7 @@ typedef struct {
   int32_t stages;
   int32_t reduce;
   int32_t pdl;
+  int32_t persistent;
 } lq_variant;
 
 /*
@@ -430,8 +437,9 @@ lq_status lq_select_variant(lq_fmt fmt, int64_t M, int64_t N, int64_t K,
 
 /*
  * Replace the dispatch table by the entries of a text file (one entry per
- * line: "fmt m_bucket N K swap_ab split_k tile_n stages reduce pdl", '#'
- * starts a comment).  path == NULL restores the compiled-in table.  At
+ * line: "fmt m_bucket N K swap_ab split_k tile_n stages reduce pdl
+ * [persistent]", '#' starts a comment; fmt is fp8_dynamic, w8a8_int8,
+ * block_fp8, block_fp8_ue8m0 or 0..3).  path == NULL restores the compiled-in table.  At
  * start-up the environment variable LQ_DISPATCH_TABLE, when set, names a
  * file that replaces the compiled-in table.  On error
  * the current table is kept and LQ_ERR_TABLE is returned.  Safe while other

@@ -278,6 +278,30 @@ int max_stages_fit(int tile_n, int ctas_per_sm, bool cluster_reduce, bool fuse =
   return best;
 }
 
+// Deepest ring of the persistent kernel (one CTA per SM).
+int max_persistent_stages(int tile_n) {
+  int best = 2;
+  for (int s = 2; s <= kMaxStages; ++s)
+    if (lq::persistent_smem_bytes_for(tile_n, s) <= kMaxSmemPerCta) best = s;
+  return best;
+}
+
+// Streaming multiprocessors of the current device (148 on B200).
+int sm_count() {
+  static int cached[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return kNumSms;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = kNumSms;
+    }
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 lq_variant heuristic_variant(int fmt, int64_t M, int64_t N, int64_t K) {
   lq_variant v{};
   const int64_t T = (K + 127) / 128;
@@ -303,6 +327,11 @@ lq_variant heuristic_variant(int fmt, int64_t M, int64_t N, int64_t K) {
     v.split_k = S;
     v.reduce = S <= 16 ? 2 : 1;
     v.stages = max_stages_fit(v.tile_n, 1, S > 1 && v.reduce == 2);
+    // many waves of tiles: persistent CTAs overlap each tile's epilogue with the next mainloop
+    if (S == 1 && (fmt == lq::kFmtFp8 || fmt == lq::kFmtInt8) && tiles >= 2 * kNumSms) {
+      v.persistent = 1;
+      v.stages = max_persistent_stages(v.tile_n);
+    }
   }
   return v;
 }
@@ -348,6 +377,13 @@ lq_status check_variant(int fmt, const lq_variant& v) {
     if (fmt == lq::kFmtBlock && v.tile_n == 256) return LQ_ERR_INVALID_ARG;   // promotion in registers
   }
   if (v.stages != 0 && (v.stages < 2 || v.stages > kMaxStages)) return LQ_ERR_INVALID_ARG;
+  if (v.persistent != 0 && v.persistent != 1) return LQ_ERR_INVALID_ARG;
+  if (v.persistent) {
+    // Standard orientation, one split, FP8_Dynamic / W8A8_INT8
+    if (v.swap_ab || v.split_k != 1 || (fmt != lq::kFmtFp8 && fmt != lq::kFmtInt8)) return LQ_ERR_INVALID_ARG;
+    if (v.stages != 0 && lq::persistent_smem_bytes_for(v.tile_n, v.stages) > kMaxSmemPerCta) return LQ_ERR_INVALID_ARG;
+    return LQ_OK;
+  }
   if (v.stages != 0 &&
       lq::gemm_smem_bytes_for(v.tile_n, v.stages, v.split_k > 1 && v.reduce == 2) > kMaxSmemPerCta)
     return LQ_ERR_INVALID_ARG;
@@ -392,7 +428,7 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   rc = check_variant(fmt, v);
   if (rc != LQ_OK) return rc;
   const bool cluster_reduce = v.split_k > 1 && v.reduce == 2;
-  if (v.stages == 0) v.stages = max_stages_fit(v.tile_n, 1, cluster_reduce, fused);
+  if (v.stages == 0) v.stages = v.persistent ? max_persistent_stages(v.tile_n) : max_stages_fit(v.tile_n, 1, cluster_reduce, fused);
   if (fused && lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce, true) > kMaxSmemPerCta)
     v.stages = max_stages_fit(v.tile_n, 1, cluster_reduce, true);
 
@@ -450,6 +486,13 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   l.fuse = fused ? 1 : 0;
   l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
   l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce, fused);
+  if (v.persistent) {   // one CTA per SM (at most one per tile), each looping over tiles
+    const int64_t tiles = gx * gy;
+    const int64_t ctas = tiles < sm_count() ? tiles : sm_count();
+    l.grid = dim3(static_cast<unsigned>(ctas), 1, 1);
+    l.smem_bytes = lq::persistent_smem_bytes_for(v.tile_n, v.stages);
+    l.persistent = 1;
+  }
   l.pdl = v.pdl != 0;
   l.cluster_z = (v.split_k > 1 && v.reduce == 2) ? v.split_k : 1;
   l.stream = stream;
@@ -508,7 +551,9 @@ bool parse_table_file(const char* path, std::vector<TableEntry>* out, std::strin
     e.m_bucket = mb;
     e.N = n;
     e.K = k;
-    e.v = lq_variant{sw, sk, tn, st, rd, pdl};
+    int persistent = 0;   // optional 11th column
+    if (!(is >> persistent)) persistent = 0;
+    e.v = lq_variant{sw, sk, tn, st, rd, pdl, persistent};
     if (check_variant(e.fmt, e.v) != LQ_OK) {
       *err = "invalid variant at line " + std::to_string(lineno);
       return false;
@@ -1000,7 +1045,7 @@ extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const floa
                                           static_cast<size_t>(N) * 4u
                                     : 0;
   if (need > kNoAllocScratchBytes) return LQ_ERR_WORKSPACE;
-  if (v.stages == 0) v.stages = max_stages_fit(v.tile_n, 1, false);
+  if (v.stages == 0) v.stages = v.persistent ? max_persistent_stages(v.tile_n) : max_stages_fit(v.tile_n, 1, false);
 
   const int64_t x_rows = v.swap_ab ? N : M;
   const int64_t y_rows = v.swap_ab ? M : N;
@@ -1040,6 +1085,13 @@ extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const floa
     return LQ_ERR_CUDA;
   l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
   l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, false);
+  if (v.persistent) {   // split_k 1: no scratch; one CTA per SM looping over tiles
+    const int64_t tiles = gx * gy;
+    const int64_t ctas = tiles < sm_count() ? tiles : sm_count();
+    l.grid = dim3(static_cast<unsigned>(ctas), 1, 1);
+    l.smem_bytes = lq::persistent_smem_bytes_for(v.tile_n, v.stages);
+    l.persistent = 1;
+  }
   l.pdl = v.pdl != 0;
   l.cluster_z = 1;
   l.stream = stream;

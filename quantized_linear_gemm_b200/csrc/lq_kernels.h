@@ -56,6 +56,7 @@ struct GemmLaunch {
   int cluster_z;       // > 1: launch clusters of (1, 1, cluster_z) CTAs
   int fuse;            // fused activation quantization (Swap-AB only)
   int grouped;         // grouped (mixture-of-experts) launch (Swap-AB only; p.expert_offsets set)
+  int persistent;      // persistent CTAs looping over output tiles (Standard, split_k 1, FP8 / INT8)
   cudaStream_t stream;
 };
 
@@ -73,6 +74,8 @@ cudaError_t launch_splitk_reduce(int fmt, const GemmParams& p, int pdl, cudaStre
 // Dynamic shared memory of the GEMM kernel; `fuse`: the fused-quantization
 // instantiation (each ring slot also stages a bf16 activation tile).
 int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce, bool fuse = false);
+// Dynamic shared memory of the persistent kernel for (tile_n, stages).
+int persistent_smem_bytes_for(int tile_n, int stages);
 
 // Quantization kernels (quant_kernels.cu).
 cudaError_t launch_quant_per_token(int fmt, const void* x, void* q, float* scales, int64_t M, int64_t K,

@@ -24,6 +24,15 @@ int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce, bool fuse) 
   }
 }
 
+int persistent_smem_bytes_for(int tile_n, int stages) {
+  switch (tile_n) {
+    case 64: return persistent_smem_bytes<64>(stages);
+    case 128: return persistent_smem_bytes<128>(stages);
+    case 256: return persistent_smem_bytes<256>(stages);
+    default: return -1;
+  }
+}
+
 cudaError_t launch_splitk_reduce(int fmt, const GemmParams& p, int pdl, cudaStream_t stream) {
   const int64_t work = p.M * p.N / 4;
   int64_t blocks = (work + 255) / 256;

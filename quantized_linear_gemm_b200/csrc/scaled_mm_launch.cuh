@@ -2,6 +2,7 @@
 #pragma once
 
 #include "scaled_mm_kernel.cuh"
+#include "scaled_mm_persistent.cuh"
 
 namespace lq {
 
@@ -88,6 +89,10 @@ cudaError_t launch_format(const GemmLaunch& l, int swap_ab, int tile_n) {
       }
     }
     return cudaErrorInvalidValue;
+  }
+  if (l.persistent) {
+    if (swap_ab) return cudaErrorInvalidValue;
+    return l.p.bias ? launch_persistent<FMT, true>(l, tile_n) : launch_persistent<FMT, false>(l, tile_n);
   }
   return l.p.bias ? launch_dense<FMT, true>(l, swap_ab, tile_n) : launch_dense<FMT, false>(l, swap_ab, tile_n);
 }

@@ -52,16 +52,17 @@ class LQError(RuntimeError):
 
 class Variant(ctypes.Structure):
     _fields_ = [("swap_ab", ctypes.c_int32), ("split_k", ctypes.c_int32), ("tile_n", ctypes.c_int32),
-                ("stages", ctypes.c_int32), ("reduce", ctypes.c_int32), ("pdl", ctypes.c_int32)]
+                ("stages", ctypes.c_int32), ("reduce", ctypes.c_int32), ("pdl", ctypes.c_int32),
+                ("persistent", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {f: int(getattr(self, f)) for f, _ in self._fields_}
 
 
-def make_variant(swap_ab=0, split_k=1, tile_n=None, stages=0, reduce=1, pdl=1) -> Variant:
+def make_variant(swap_ab=0, split_k=1, tile_n=None, stages=0, reduce=1, pdl=1, persistent=0) -> Variant:
     if tile_n is None:
         tile_n = 32 if swap_ab else 128
-    return Variant(int(swap_ab), int(split_k), int(tile_n), int(stages), int(reduce), int(pdl))
+    return Variant(int(swap_ab), int(split_k), int(tile_n), int(stages), int(reduce), int(pdl), int(persistent))
 
 
 _lib = None

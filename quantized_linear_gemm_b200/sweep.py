@@ -100,6 +100,10 @@ def candidates(fmt, M, N, K):
                 for st in (3, 4, 6, 0):
                     for pdl in (1, 2):
                         add(swap_ab=0, tile_n=tn, split_k=S, stages=st, reduce=2, pdl=pdl)
+            if fmt in (lq.FP8_DYNAMIC, lq.W8A8_INT8):   # persistent CTAs (one split)
+                for st in (3, 4, 0):
+                    for pdl in (1, 2):
+                        add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=1)
     return out
 
 
@@ -214,7 +218,8 @@ def write_table(results, path):
     for r in results:
         v = r["variant"]
         lines.append(f"{r['fmt']} {m_bucket(r['M'])} {r['N']} {r['K']} {v['swap_ab']} {v['split_k']} {v['tile_n']} "
-                     f"{v['stages']} {v['reduce']} {v['pdl']}   # {r['us']} {r['gbs']} {r['tflops']}")
+                     f"{v['stages']} {v['reduce']} {v['pdl']} {v.get('persistent', 0)}   "
+                     f"# {r['us']} {r['gbs']} {r['tflops']}")
     with open(path, "w") as f:
         f.write("\n".join(lines) + "\n")
 
@@ -244,14 +249,15 @@ def write_inc(txt_path, inc_path):
         line = line.split("#")[0].split()
         if not line:
             continue
-        f, mb, n, k, sw, sk, tn, st, rd, pdl = line
-        rows.append(f"    {{{fmt_id[f]}, {mb}, {n}, {k}, {{{sw}, {sk}, {tn}, {st}, {rd}, {pdl}}}}},")
-    body = "\n".join(rows) if rows else "    {-1, 0, 0, 0, {0, 1, 64, 2, 1, 1}},   // placeholder (never matches)"
+        f, mb, n, k, sw, sk, tn, st, rd, pdl = line[:10]
+        pers = line[10] if len(line) > 10 else "0"
+        rows.append(f"    {{{fmt_id[f]}, {mb}, {n}, {k}, {{{sw}, {sk}, {tn}, {st}, {rd}, {pdl}, {pers}}}}},")
+    body = "\n".join(rows) if rows else "    {-1, 0, 0, 0, {0, 1, 64, 2, 1, 1, 0}},   // placeholder (never matches)"
     with open(inc_path, "w") as f:
         f.write("// Compiled-in dispatch table: (format, token bucket, N, K) -> variant.\n"
                 "// Generated by quantized_linear_gemm_b200/sweep.py from dispatch_table.txt\n"
                 "// (measured best variants on B200).  Keys not listed use the heuristic.\n"
-                "// fields: fmt, m_bucket, N, K, {swap_ab, split_k, tile_n, stages, reduce, pdl}\n"
+                "// fields: fmt, m_bucket, N, K, {swap_ab, split_k, tile_n, stages, reduce, pdl, persistent}\n"
                 "static const TableEntry kDefaultTable[] = {\n" + body + "\n};\n"
                 f"static const size_t kDefaultTableSize = {len(rows)};\n")
 

@@ -10,6 +10,7 @@ import numpy as np
 import torch
 
 from oracle import lq_oracle as O
+from oracle import ue8m0_oracle as U
 from quantized_linear_gemm_b200 import inputs, lq
 
 FMT_NAME = {lq.FP8_DYNAMIC: O.FMT_FP8_DYNAMIC, lq.W8A8_INT8: O.FMT_W8A8_INT8, lq.BLOCK_FP8: O.FMT_BLOCK_FP8}
@@ -30,21 +31,27 @@ class Problem:
         """(A, a_scales, B, b_scales) on the GPU: uint8 e4m3 codes or int8 codes, fp32 scales."""
         A = torch.from_numpy(np.ascontiguousarray(self.qa)).to(dev)
         B = torch.from_numpy(np.ascontiguousarray(self.qb)).to(dev)
-        sa = torch.from_numpy(np.ascontiguousarray(self.sa, dtype=np.float32)).to(dev)
-        sb = torch.from_numpy(np.ascontiguousarray(self.sb, dtype=np.float32)).to(dev)
+        sdt = np.uint8 if self.fmt == lq.BLOCK_FP8_UE8M0 else np.float32   # UE8M0 scales are bytes
+        sa = torch.from_numpy(np.ascontiguousarray(self.sa, dtype=sdt)).to(dev)
+        sb = torch.from_numpy(np.ascontiguousarray(self.sb, dtype=sdt)).to(dev)
         return A, sa, B, sb
 
     def reference(self, rows=None, cols=None):
         qa, sa, qb, sb = self.qa, self.sa, self.qb, self.sb
+        if self.fmt == lq.BLOCK_FP8_UE8M0:   # the decoded power-of-two scales, then as Block_FP8
+            sa, sb = U.e8m0_decode(sa), U.e8m0_decode(sb)
         if rows is not None:
             qa, sa = qa[rows], sa[rows]
+        block = self.fmt in (lq.BLOCK_FP8, lq.BLOCK_FP8_UE8M0)
         if cols is not None:
             qb = qb[cols]
-            if self.fmt != lq.BLOCK_FP8:
+            if not block:
                 sb = sb[cols]
-        if self.fmt == lq.BLOCK_FP8 and cols is not None:
+        if block and cols is not None:
             # keep the n-block scale of each sampled column: expand to per-column blocks
             return _block_ref_cols(qa, sa, qb, sb, np.asarray(cols))
+        if block:
+            return O.blockwise_ref(qa, sa, qb, sb)
         return O.scaled_mm_ref(FMT_NAME[self.fmt], qa, sa, qb, sb)
 
 
@@ -60,6 +67,10 @@ def _block_ref_cols(qa, sa, qb_cols, sb, cols):
 def make_problem(fmt: int, M: int, N: int, K: int, seed: int, outliers: bool = True) -> Problem:
     x = inputs.activations(M, K, seed=inputs.stable_seed("A", fmt, M, N, K, seed), outliers=outliers).float().numpy()
     w = inputs.weights(N, K, seed=inputs.stable_seed("B", fmt, M, N, K, seed)).float().numpy()
+    if fmt == lq.BLOCK_FP8_UE8M0:
+        qa, sa = U.quant_per_token_group128_ue8m0(x)
+        qb, sb = U.quant_weight_block128_ue8m0(w)
+        return Problem(fmt, M, N, K, qa, sa, qb, sb)
     name = FMT_NAME[fmt]
     if fmt == lq.BLOCK_FP8:
         qa, sa = O.quant_per_token_group128(x)

@@ -116,6 +116,17 @@ def test_variant_checks(field, value):
     assert _mm(variant=v) == INVALID
 
 
+def test_persistent_variant_rules():
+    """persistent = 1 needs the Standard orientation, one split and FP8 / INT8."""
+    ok = lq.make_variant(swap_ab=0, tile_n=256, split_k=1, persistent=1)
+    assert _mm(variant=ok, C=MISALIGNED) == ALIGN        # accepted up to the pointer checks
+    for bad in (dict(swap_ab=1, tile_n=16, persistent=1), dict(swap_ab=0, tile_n=128, split_k=2, persistent=1),
+                dict(swap_ab=0, tile_n=128, persistent=2), dict(swap_ab=0, tile_n=256, stages=5, persistent=1)):
+        assert _mm(variant=lq.make_variant(**bad)) == INVALID, bad
+    for fmt in (2, 3):
+        assert _mm(fmt=fmt, K=256, N=256, variant=lq.make_variant(swap_ab=0, tile_n=128, persistent=1)) == INVALID
+
+
 def test_variant_tile_rules():
     assert _mm(variant=lq.make_variant(swap_ab=1, tile_n=128)) == INVALID      # swap tiles are 16/32/64
     assert _mm(variant=lq.make_variant(swap_ab=0, tile_n=16)) == INVALID       # standard tiles are 64/128/256
@@ -257,14 +268,17 @@ def test_dispatch_table_file(tmp_path):
     p = tmp_path / "table.txt"
     p.write_text("# fmt m_bucket N K swap split tile stages reduce pdl\n"
                  "fp8_dynamic 8 4096 4096 1 8 16 4 0 1\n"
-                 "w8a8_int8 32 6144 4096 0 2 64 6 1 0   # trailing comment\n")
+                 "w8a8_int8 32 6144 4096 0 2 64 6 1 0   # trailing comment\n"
+                 "fp8_dynamic 2048 51200 5120 0 1 256 4 1 2 1   # 11th column: persistent\n")
     try:
         lq.load_dispatch_table(str(p))
-        assert lq.dispatch_table_size() == 2
+        assert lq.dispatch_table_size() == 3
         v = lq.select_variant("fp8_dynamic", 5, 4096, 4096)      # M=5 -> bucket 8
-        assert v.as_dict() == dict(swap_ab=1, split_k=8, tile_n=16, stages=4, reduce=0, pdl=1)
+        assert v.as_dict() == dict(swap_ab=1, split_k=8, tile_n=16, stages=4, reduce=0, pdl=1, persistent=0)
         v = lq.select_variant("w8a8_int8", 32, 6144, 4096)
-        assert v.as_dict() == dict(swap_ab=0, split_k=2, tile_n=64, stages=6, reduce=1, pdl=0)
+        assert v.as_dict() == dict(swap_ab=0, split_k=2, tile_n=64, stages=6, reduce=1, pdl=0, persistent=0)
+        v = lq.select_variant("fp8_dynamic", 2048, 51200, 5120)
+        assert v.as_dict() == dict(swap_ab=0, split_k=1, tile_n=256, stages=4, reduce=1, pdl=1, persistent=1)
         # workspace need follows the selected variant
         assert lq.workspace_bytes("fp8_dynamic", 5, 4096, 4096) == 8 * 5 * 4096 * 4
         bad = tmp_path / "bad.txt"
@@ -272,7 +286,7 @@ def test_dispatch_table_file(tmp_path):
         with pytest.raises(lq.LQError) as e:
             lq.load_dispatch_table(str(bad))
         assert e.value.code == TABLE
-        assert lq.dispatch_table_size() == 2                       # the table in force is kept
+        assert lq.dispatch_table_size() == 3                       # the table in force is kept
         with pytest.raises(lq.LQError):
             lq.load_dispatch_table(str(tmp_path / "missing.txt"))
     finally:

@@ -21,6 +21,8 @@ CASES = [
     (lq.W8A8_INT8, dict(swap_ab=1, tile_n=16, split_k=4, stages=2, reduce=2)),      # cluster, push
     (lq.FP8_DYNAMIC, dict(swap_ab=0, tile_n=128, split_k=2, stages=3, reduce=2)),   # cluster, pull
     (lq.BLOCK_FP8, dict(swap_ab=1, tile_n=16, split_k=2, stages=2, reduce=2)),
+    (lq.FP8_DYNAMIC, dict(swap_ab=0, tile_n=64, split_k=1, stages=3, persistent=1)),   # persistent CTAs
+    (lq.BLOCK_FP8_UE8M0, dict(swap_ab=0, tile_n=128, split_k=1, stages=3)),            # block-scaled MMA
 ]
 
 

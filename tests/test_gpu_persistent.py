@@ -1,0 +1,136 @@
+"""GPU parity of the persistent scaled_mm (one CTA per SM looping over output
+tiles, two tensor-memory accumulators), through the C ABI: the same bits as
+the one-tile-per-CTA kernel with the same tile, within tolerance of the
+oracle, exact INT8 accumulators, bias, ragged tails, several tiles per CTA,
+and graph replay."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import lq_oracle as O
+from quantized_linear_gemm_b200 import inputs, lq
+
+from _lqtest import assert_close, make_problem
+
+pytestmark = pytest.mark.gpu
+
+FMTS = [lq.FP8_DYNAMIC, lq.W8A8_INT8]
+FMT_IDS = ["fp8", "int8"]
+
+
+def _pair(prob, tn, stages=0, pdl=1, bias=None):
+    """(persistent C, one-tile-per-CTA C) for the same tile."""
+    A, sa, B, sb = prob.device()
+    outs = []
+    for pers in (1, 0):
+        v = lq.make_variant(swap_ab=0, tile_n=tn, split_k=1, stages=stages, pdl=pdl, persistent=pers)
+        if bias is None:
+            outs.append(lq.scaled_mm(prob.fmt, A, sa, B, sb, variant=v))
+        else:
+            outs.append(lq.scaled_mm_bias(prob.fmt, A, sa, B, sb, bias, variant=v))
+    torch.cuda.synchronize()
+    assert lq.device_status(0) == 0
+    return outs
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
+@pytest.mark.parametrize("tn", [64, 128, 256])
+@pytest.mark.parametrize("stages", [2, 3, 0])
+def test_persistent_small_ragged(cuda_device, fmt, tn, stages):
+    """M = 300 (a ragged m-block), N = 1000 (ragged n-block), K = 1040 (a
+    16-wide last K tile): fewer tiles than SMs, one tile per CTA."""
+    prob = make_problem(fmt, 300, 1000, 1040, seed=401)
+    Cp, Cs = _pair(prob, tn, stages)
+    assert torch.equal(Cp, Cs)
+    assert_close(Cp, prob.reference(), f"persistent tn={tn} stages={stages}")
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
+@pytest.mark.parametrize("tn", [64, 128, 256])
+@pytest.mark.parametrize("pdl", [0, 1, 2])
+def test_persistent_many_tiles_per_cta(cuda_device, fmt, tn, pdl):
+    """M = 1100, N = 4096: 9 x (64 .. 16) tiles, up to four per CTA, both
+    accumulator buffers reused; equal to the one-tile kernel bit for bit and
+    to the oracle on sampled rows and columns (every m-block, both ends)."""
+    M, N, K = 1100, 4096, 1024
+    prob = make_problem(fmt, M, N, K, seed=402 + tn, outliers=False)
+    Cp, Cs = _pair(prob, tn, pdl=pdl)
+    assert torch.equal(Cp, Cs)
+    rows = np.array([0, 127, 128, 500, 1023, 1024, 1099])
+    cols = np.array([0, 7, 255, 256, 2047, 4088, 4095])
+    ref = O.scaled_mm_ref({lq.FP8_DYNAMIC: O.FMT_FP8_DYNAMIC, lq.W8A8_INT8: O.FMT_W8A8_INT8}[fmt],
+                          prob.qa[rows], prob.sa[rows], prob.qb[cols], prob.sb[cols])
+    got = Cp.float().cpu().numpy().astype(np.float64)[np.ix_(rows, cols)]
+    ok, worst = O.within_tolerance(got, ref)
+    assert ok, worst
+
+
+def test_persistent_int8_accumulators_exact(cuda_device):
+    prob = make_problem(lq.W8A8_INT8, 300, 768, 1152, seed=403)
+    A, sa, B, sb = prob.device()
+    v = lq.make_variant(swap_ab=0, tile_n=256, split_k=1, persistent=1)
+    C, acc = lq.scaled_mm_i32acc(A, sa, B, sb, variant=v)
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.acc_exact(O.FMT_W8A8_INT8, prob.qa, prob.qb))
+    assert_close(C, prob.reference(), "int8 persistent C")
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
+def test_persistent_bias(cuda_device, fmt):
+    prob = make_problem(fmt, 260, 512, 1024, seed=404)
+    g = torch.Generator().manual_seed(405)
+    bias = (torch.randn(512, generator=g) * 0.5).to(torch.bfloat16)
+    Cp, Cs = _pair(prob, 128, bias=bias.cuda())
+    assert torch.equal(Cp, Cs)
+    ref = prob.reference() + bias.double().numpy()[None, :]
+    assert_close(Cp, ref, "persistent bias")
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
+def test_persistent_graph_replay_and_default(cuda_device, fmt):
+    """Bitwise reproducible under CUDA-graph replay; the default variant for a
+    many-tile Standard shape outside the table (at least two tiles per SM) is
+    the persistent one."""
+    M, N, K = 2048, 8192, 512
+    prob = make_problem(fmt, M, N, K, seed=406, outliers=False)
+    A, sa, B, sb = prob.device()
+    v = lq.select_variant(fmt, M, N, K)
+    assert v.persistent == 1 and v.swap_ab == 0 and v.split_k == 1
+    C0 = lq.scaled_mm(fmt, A, sa, B, sb).clone()
+    out = torch.empty_like(C0)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(2):
+                lq.scaled_mm(fmt, A, sa, B, sb, C=out, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, C0)
+    del g
+    rows = np.arange(0, M, 97)
+    cols = np.arange(0, N, 331)
+    name = {lq.FP8_DYNAMIC: O.FMT_FP8_DYNAMIC, lq.W8A8_INT8: O.FMT_W8A8_INT8}[fmt]
+    ref = O.scaled_mm_ref(name, prob.qa[rows], prob.sa[rows], prob.qb[cols], prob.sb[cols])
+    ok, worst = O.within_tolerance(C0.float().cpu().numpy().astype(np.float64)[np.ix_(rows, cols)], ref)
+    assert ok, worst
+    assert lq.device_status(0) == 0
+
+
+def test_persistent_refuses_what_it_does_not_do(cuda_device):
+    prob = make_problem(lq.FP8_DYNAMIC, 64, 256, 512, seed=407)
+    A, sa, B, sb = prob.device()
+    for bad in (dict(swap_ab=1, tile_n=16, persistent=1), dict(swap_ab=0, tile_n=128, split_k=2, persistent=1),
+                dict(swap_ab=0, tile_n=128, persistent=2)):
+        with pytest.raises(lq.LQError):
+            lq.scaled_mm(lq.FP8_DYNAMIC, A, sa, B, sb, variant=lq.make_variant(**bad))
+    qa = torch.zeros((64, 512), dtype=torch.uint8, device="cuda")
+    with pytest.raises(lq.LQError):
+        lq.scaled_mm("block_fp8", qa, torch.ones((64, 4), device="cuda"), torch.zeros((256, 512), dtype=torch.uint8,
+                     device="cuda"), torch.ones((2, 4), device="cuda"),
+                     variant=lq.make_variant(swap_ab=0, tile_n=128, persistent=1))
