@@ -231,7 +231,8 @@ DEEP_K = [  # (M, N, K, variant): Qwen3-32B down (K = 25600, 200 K tiles) in pre
 def test_deep_k_bitwise_reproducible(cuda_device, fmt, M, N, K, vd):
     """Run to run the same bits at the deepest K of the workloads: every
     variant sums its partial products and its splits in one fixed order, so
-    repeated calls (eager, back to back on one stream) must agree bit for bit."""
+    repeated calls (eager, back to back on one stream) must agree bit for bit;
+    and sampled outputs within tolerance of the oracle."""
     A, sa, B, sb = _random_operands(fmt, M, N, K, seed=M + N)
     v = None if vd is None else lq.make_variant(**vd)
     if v is not None:
@@ -244,6 +245,21 @@ def test_deep_k_bitwise_reproducible(cuda_device, fmt, M, N, K, vd):
         torch.cuda.synchronize()
         assert torch.equal(out, C0)
     assert torch.isfinite(C0.float()).all()
+    # and the oracle on sampled outputs (exact products of the random codes)
+    qa, qb = A.cpu().numpy(), B.cpu().numpy()
+    san, sbn = sa.cpu().numpy().astype(np.float64), sb.cpu().numpy().astype(np.float64)
+    rng = np.random.default_rng(M + N + K)
+    rows = np.sort(rng.choice(M, size=min(M, 6), replace=False))
+    cols = np.sort(rng.choice(N, size=12, replace=False))
+    if fmt == lq.BLOCK_FP8:
+        ref = np.stack([O.blockwise_ref(qa[rows], san[rows], qb[n:n + 1], sbn[n // 128:n // 128 + 1])[:, 0]
+                        for n in cols], axis=1)
+    else:
+        name = O.FMT_FP8_DYNAMIC if fmt == lq.FP8_DYNAMIC else O.FMT_W8A8_INT8
+        ref = O.scaled_mm_ref(name, qa[rows], san[rows], qb[cols], sbn[cols])
+    got = C0.float().cpu().numpy().astype(np.float64)[np.ix_(rows, cols)]
+    ok, worst = O.within_tolerance(got, ref)
+    assert ok, worst
     assert lq.device_status(0) == 0
 
 
