@@ -115,7 +115,11 @@ typedef enum {
  *            or 256): one CTA per SM loops over the output tiles, its
  *            shared-memory ring runs on across tiles, and the accumulator is
  *            double-buffered in tensor memory so that a tile's epilogue
- *            overlaps the next tile's mainloop.  Same results bit for bit.
+ *            overlaps the next tile's mainloop; 2 = the same on CTA pairs
+ *            (clusters of two, one MMA of 256 rows over both SMs with
+ *            tcgen05 cta_group::2; each CTA loads 128 rows of A and half of
+ *            the tile's tile_n (128 or 256) weight rows).  Same results bit
+ *            for bit.
  *  pdl     : 0 = plain launch;
  *            1 = programmatic dependent launch: the kernel's set-up overlaps
  *            the tail of the previous kernel on the stream, and all of its

@@ -14,6 +14,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <array>
 #include <atomic>
 #include <cerrno>
 #include <cfloat>
@@ -278,11 +279,14 @@ int max_stages_fit(int tile_n, int ctas_per_sm, bool cluster_reduce, bool fuse =
   return best;
 }
 
-// Deepest ring of the persistent kernel (one CTA per SM).
-int max_persistent_stages(int tile_n) {
+// Deepest ring of the persistent kernels (one CTA per SM): persistent 1
+// (one-SM tiles) or 2 (CTA pairs).
+int max_persistent_stages(int tile_n, int persistent = 1) {
   int best = 2;
-  for (int s = 2; s <= kMaxStages; ++s)
-    if (lq::persistent_smem_bytes_for(tile_n, s) <= kMaxSmemPerCta) best = s;
+  for (int s = 2; s <= kMaxStages; ++s) {
+    const int bytes = persistent == 2 ? lq::pair_smem_bytes_for(tile_n, s) : lq::persistent_smem_bytes_for(tile_n, s);
+    if (bytes > 0 && bytes <= kMaxSmemPerCta) best = s;
+  }
   return best;
 }
 
@@ -300,6 +304,23 @@ int sm_count() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+// Co-resident CTA pairs of the pair kernel for (fmt, tile_n, bias, smem),
+// cached per device (0 if the query fails).
+int pair_capacity(int fmt, int tile_n, bool bias, int smem_bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<std::array<int, 5>, int>> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const std::array<int, 5> key{dev, fmt, tile_n, bias ? 1 : 0, smem_bytes};
+  std::lock_guard<std::mutex> lk(mu);
+  for (const auto& e : cache)
+    if (e.first == key) return e.second;
+  const int n = fmt == lq::kFmtFp8 ? lq::pair_capacity_fp8(tile_n, bias, smem_bytes)
+                                   : lq::pair_capacity_int8(tile_n, bias, smem_bytes);
+  cache.emplace_back(key, n);
+  return n;
 }
 
 lq_variant heuristic_variant(int fmt, int64_t M, int64_t N, int64_t K) {
@@ -377,11 +398,14 @@ lq_status check_variant(int fmt, const lq_variant& v) {
     if (fmt == lq::kFmtBlock && v.tile_n == 256) return LQ_ERR_INVALID_ARG;   // promotion in registers
   }
   if (v.stages != 0 && (v.stages < 2 || v.stages > kMaxStages)) return LQ_ERR_INVALID_ARG;
-  if (v.persistent != 0 && v.persistent != 1) return LQ_ERR_INVALID_ARG;
+  if (v.persistent < 0 || v.persistent > 2) return LQ_ERR_INVALID_ARG;
   if (v.persistent) {
-    // Standard orientation, one split, FP8_Dynamic / W8A8_INT8
+    // Standard orientation, one split, FP8_Dynamic / W8A8_INT8 (CTA pairs: tile_n 128 or 256)
     if (v.swap_ab || v.split_k != 1 || (fmt != lq::kFmtFp8 && fmt != lq::kFmtInt8)) return LQ_ERR_INVALID_ARG;
-    if (v.stages != 0 && lq::persistent_smem_bytes_for(v.tile_n, v.stages) > kMaxSmemPerCta) return LQ_ERR_INVALID_ARG;
+    if (v.persistent == 2 && v.tile_n == 64) return LQ_ERR_INVALID_ARG;
+    const int bytes = v.persistent == 2 ? lq::pair_smem_bytes_for(v.tile_n, v.stages ? v.stages : 2)
+                                        : lq::persistent_smem_bytes_for(v.tile_n, v.stages ? v.stages : 2);
+    if (bytes > kMaxSmemPerCta) return LQ_ERR_INVALID_ARG;
     return LQ_OK;
   }
   if (v.stages != 0 &&
@@ -428,7 +452,9 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   rc = check_variant(fmt, v);
   if (rc != LQ_OK) return rc;
   const bool cluster_reduce = v.split_k > 1 && v.reduce == 2;
-  if (v.stages == 0) v.stages = v.persistent ? max_persistent_stages(v.tile_n) : max_stages_fit(v.tile_n, 1, cluster_reduce, fused);
+  if (v.stages == 0)
+    v.stages = v.persistent ? max_persistent_stages(v.tile_n, v.persistent)
+                            : max_stages_fit(v.tile_n, 1, cluster_reduce, fused);
   if (fused && lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce, true) > kMaxSmemPerCta)
     v.stages = max_stages_fit(v.tile_n, 1, cluster_reduce, true);
 
@@ -477,7 +503,10 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   const void* x_ptr = v.swap_ab ? B : A;
   const void* y_ptr = v.swap_ab ? A : B;
   if (!encode_operand(&l.tmX, x_ptr, x_rows, K, 128)) return LQ_ERR_CUDA;
-  if (fused) {
+  if (v.persistent == 2) {
+    // CTA pairs: each CTA loads half of the tile's weight rows
+    if (!encode_operand(&l.tmY, y_ptr, y_rows, K, v.tile_n / 2)) return LQ_ERR_CUDA;
+  } else if (fused) {
     // the kernel stages the bf16 activations and quantizes them itself
     if (!encode_bf16_rows(&l.tmY, x_fused, M, K, v.tile_n)) return LQ_ERR_CUDA;
   } else if (!encode_operand(&l.tmY, y_ptr, y_rows, K, v.tile_n)) {
@@ -486,12 +515,20 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   l.fuse = fused ? 1 : 0;
   l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
   l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce, fused);
-  if (v.persistent) {   // one CTA per SM (at most one per tile), each looping over tiles
+  if (v.persistent == 1) {   // one CTA per SM (at most one per tile), each looping over tiles
     const int64_t tiles = gx * gy;
     const int64_t ctas = tiles < sm_count() ? tiles : sm_count();
     l.grid = dim3(static_cast<unsigned>(ctas), 1, 1);
     l.smem_bytes = lq::persistent_smem_bytes_for(v.tile_n, v.stages);
     l.persistent = 1;
+  } else if (v.persistent == 2) {   // clusters of two CTAs, 256-row tiles, each pair looping over tiles
+    l.smem_bytes = lq::pair_smem_bytes_for(v.tile_n, v.stages);
+    const int64_t tiles = ((M + 255) / 256) * gy;
+    int cap = pair_capacity(fmt, v.tile_n, bias != nullptr, l.smem_bytes);
+    if (cap <= 0) cap = sm_count() / 2;
+    const int64_t pairs = tiles < cap ? tiles : cap;
+    l.grid = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+    l.persistent = 2;
   }
   l.pdl = v.pdl != 0;
   l.cluster_z = (v.split_k > 1 && v.reduce == 2) ? v.split_k : 1;
@@ -1045,7 +1082,8 @@ extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const floa
                                           static_cast<size_t>(N) * 4u
                                     : 0;
   if (need > kNoAllocScratchBytes) return LQ_ERR_WORKSPACE;
-  if (v.stages == 0) v.stages = v.persistent ? max_persistent_stages(v.tile_n) : max_stages_fit(v.tile_n, 1, false);
+  if (v.stages == 0)
+    v.stages = v.persistent ? max_persistent_stages(v.tile_n, v.persistent) : max_stages_fit(v.tile_n, 1, false);
 
   const int64_t x_rows = v.swap_ab ? N : M;
   const int64_t y_rows = v.swap_ab ? M : N;
@@ -1081,16 +1119,25 @@ extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const floa
   p.skip_stage = -1;
   const void* x_ptr = v.swap_ab ? B : A;
   const void* y_ptr = v.swap_ab ? A : B;
-  if (!encode_operand(&l.tmX, x_ptr, x_rows, K, 128) || !encode_operand(&l.tmY, y_ptr, y_rows, K, v.tile_n))
+  if (!encode_operand(&l.tmX, x_ptr, x_rows, K, 128) ||
+      !encode_operand(&l.tmY, y_ptr, y_rows, K, v.persistent == 2 ? v.tile_n / 2 : v.tile_n))
     return LQ_ERR_CUDA;
   l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
   l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, false);
-  if (v.persistent) {   // split_k 1: no scratch; one CTA per SM looping over tiles
+  if (v.persistent == 1) {   // split_k 1: no scratch; one CTA per SM looping over tiles
     const int64_t tiles = gx * gy;
     const int64_t ctas = tiles < sm_count() ? tiles : sm_count();
     l.grid = dim3(static_cast<unsigned>(ctas), 1, 1);
     l.smem_bytes = lq::persistent_smem_bytes_for(v.tile_n, v.stages);
     l.persistent = 1;
+  } else if (v.persistent == 2) {   // clusters of two CTAs, 256-row tiles, each pair looping over tiles
+    l.smem_bytes = lq::pair_smem_bytes_for(v.tile_n, v.stages);
+    const int64_t tiles = ((M + 255) / 256) * gy;
+    int cap = pair_capacity(fmt, v.tile_n, false, l.smem_bytes);
+    if (cap <= 0) cap = sm_count() / 2;
+    const int64_t pairs = tiles < cap ? tiles : cap;
+    l.grid = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+    l.persistent = 2;
   }
   l.pdl = v.pdl != 0;
   l.cluster_z = 1;

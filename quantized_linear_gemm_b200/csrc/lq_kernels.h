@@ -56,7 +56,8 @@ struct GemmLaunch {
   int cluster_z;       // > 1: launch clusters of (1, 1, cluster_z) CTAs
   int fuse;            // fused activation quantization (Swap-AB only)
   int grouped;         // grouped (mixture-of-experts) launch (Swap-AB only; p.expert_offsets set)
-  int persistent;      // persistent CTAs looping over output tiles (Standard, split_k 1, FP8 / INT8)
+  int persistent;      // 1: persistent CTAs looping over output tiles (Standard, split_k 1, FP8 / INT8);
+                       // 2: the same on CTA pairs (cta_group::2, 256-row tiles, clusters of two)
   cudaStream_t stream;
 };
 
@@ -76,6 +77,11 @@ cudaError_t launch_splitk_reduce(int fmt, const GemmParams& p, int pdl, cudaStre
 int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce, bool fuse = false);
 // Dynamic shared memory of the persistent kernel for (tile_n, stages).
 int persistent_smem_bytes_for(int tile_n, int stages);
+// ... and of the CTA-pair kernel (tile_n 128 or 256; -1 otherwise).
+int pair_smem_bytes_for(int tile_n, int stages);
+// Largest number of co-resident CTA pairs of the pair kernel (0 if unknown).
+int pair_capacity_fp8(int tile_n, bool bias, int smem_bytes);
+int pair_capacity_int8(int tile_n, bool bias, int smem_bytes);
 
 // Quantization kernels (quant_kernels.cu).
 cudaError_t launch_quant_per_token(int fmt, const void* x, void* q, float* scales, int64_t M, int64_t K,

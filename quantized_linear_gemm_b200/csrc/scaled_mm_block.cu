@@ -24,6 +24,14 @@ int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce, bool fuse) 
   }
 }
 
+int pair_smem_bytes_for(int tile_n, int stages) {
+  switch (tile_n) {
+    case 128: return pair_smem_bytes<128>(stages);
+    case 256: return pair_smem_bytes<256>(stages);
+    default: return -1;
+  }
+}
+
 int persistent_smem_bytes_for(int tile_n, int stages) {
   switch (tile_n) {
     case 64: return persistent_smem_bytes<64>(stages);

@@ -3,6 +3,7 @@
 
 #include "scaled_mm_kernel.cuh"
 #include "scaled_mm_persistent.cuh"
+#include "scaled_mm_pair.cuh"
 
 namespace lq {
 
@@ -90,11 +91,27 @@ cudaError_t launch_format(const GemmLaunch& l, int swap_ab, int tile_n) {
     }
     return cudaErrorInvalidValue;
   }
+  if (l.persistent == 2) {
+    if (swap_ab) return cudaErrorInvalidValue;
+    return l.p.bias ? launch_pair<FMT, true>(l, tile_n) : launch_pair<FMT, false>(l, tile_n);
+  }
   if (l.persistent) {
     if (swap_ab) return cudaErrorInvalidValue;
     return l.p.bias ? launch_persistent<FMT, true>(l, tile_n) : launch_persistent<FMT, false>(l, tile_n);
   }
   return l.p.bias ? launch_dense<FMT, true>(l, swap_ab, tile_n) : launch_dense<FMT, false>(l, swap_ab, tile_n);
+}
+
+template <int FMT>
+int pair_capacity(int tile_n, bool bias, int smem_bytes) {
+  if constexpr (FMT == kFmtFp8 || FMT == kFmtInt8) {
+    switch (tile_n) {
+      case 128: return bias ? max_pairs<FMT, 128, true>(smem_bytes) : max_pairs<FMT, 128, false>(smem_bytes);
+      case 256: return bias ? max_pairs<FMT, 256, true>(smem_bytes) : max_pairs<FMT, 256, false>(smem_bytes);
+      default: return 0;
+    }
+  }
+  return 0;
 }
 
 }  // namespace lq

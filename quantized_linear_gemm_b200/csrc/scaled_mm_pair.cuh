@@ -1,0 +1,353 @@
+// Persistent scaled_mm on CTA pairs (tcgen05 cta_group::2) for large M:
+// Standard orientation, split_k 1, FP8_Dynamic and W8A8_INT8.
+//
+// A cluster of two CTAs (two SMs) computes 256 x TN output tiles with one
+// MMA of M = 256: each CTA loads its own 128 rows of A and half (TN / 2 rows)
+// of B into its shared memory, the pair's first CTA issues the MMAs with
+// descriptors of its own tiles (the tensor cores take the other CTA's tiles
+// from the same offsets), and each CTA's tensor memory receives its 128 rows
+// of the accumulator.  Per SM that is half of B's shared-memory traffic of a
+// one-SM 128 x TN tile for the same work, which is what bounds the one-SM
+// kernel.  As in the one-SM persistent kernel, the pair loops over tiles,
+// its rings run on across tiles and the accumulator is double-buffered
+// (2 x TN columns in each CTA), so each tile's epilogue overlaps the next
+// tile's MMAs.  Synchronisation:
+//   full[s]   first CTA only: both CTAs' TMA loads of slot s count their
+//             bytes here (the first CTA announces the pair's total);
+//   empty[s]  both CTAs: slot s read by the tensor core (commit multicast);
+//   tfull[b]  both CTAs: accumulator buffer b complete (commit multicast);
+//   tempty[b] first CTA only: both CTAs' epilogue warps have read buffer b;
+//   mma_done  both CTAs: every MMA of the pair finished (before teardown).
+// Every wait is bounded; the CTAs pass two cluster barriers (after set-up,
+// before teardown) on every path.  Results equal the one-SM kernels' up to
+// the tensor core's order of accumulation within an MMA of twice the rows:
+// per output the same MMA sequence over K, so the same bits.
+#pragma once
+
+#include "scaled_mm_persistent.cuh"
+
+namespace lq {
+
+constexpr int kPairTileM = 256;
+
+template <int TN>
+struct PairShape {
+  static constexpr int kABytes = kTileM * kTileK;              // this CTA's 128 rows of A
+  static constexpr int kBBytes = (TN / 2) * kTileK;            // this CTA's half of B
+  static constexpr int kStageBytes = kABytes + kBBytes;
+};
+
+template <int TN>
+__host__ __device__ constexpr int pair_smem_bytes(int stages) {
+  return 1024 + stages * PairShape<TN>::kStageBytes + kCtlBytes + kPersistentScaleBytes;
+}
+
+template <int FMT, int TN, bool BIAS>
+__global__ void __launch_bounds__(kThreads, 1)
+    scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const GemmParams p) {
+  static_assert(FMT == kFmtFp8 || FMT == kFmtInt8, "pair kernel: FP8_Dynamic / W8A8_INT8");
+  static_assert(TN == 128 || TN == 256, "pair tiles: 256 x 128 or 256 x 256");
+  using Shape = PairShape<TN>;
+  constexpr bool kInt8 = FMT == kFmtInt8;
+  constexpr int kTmemCols = 2 * TN;
+  constexpr int CH = 32;
+  constexpr uint16_t kPairMask = 0x3;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+  const int stages = p.stages;
+  uint8_t* ring = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + stages * Shape::kStageBytes);
+  SmemCtl c;
+  c.full = bars;
+  c.empty = bars + stages;
+  c.tfull = bars + 2 * stages;
+  c.tempty = c.tfull + 2;
+  c.mma_done = c.tempty + 2;
+  c.tmem_slot = reinterpret_cast<uint32_t*>(c.mma_done + 1);
+  c.abort_flag = reinterpret_cast<volatile int*>(c.tmem_slot + 1);
+  c.last_flag = c.abort_flag + 1;
+  float* colsc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kCtlBytes);   // [2][256]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();                // 0: issues the MMAs
+  const bool leader = rank == 0;
+  const int64_t gx = (p.M + kPairTileM - 1) / kPairTileM;   // 256-row blocks
+  const int64_t gy = (p.N + TN - 1) / TN;
+  const int64_t tiles = gx * gy;
+  const int64_t pair = blockIdx.x >> 1;
+  const int64_t npairs = gridDim.x >> 1;
+  const int64_t my_tiles = tiles > pair ? (tiles - pair + npairs - 1) / npairs : 0;
+  const int T = p.T;
+  auto tile_origin = [&](int64_t j, int64_t* m0, int64_t* n0) {
+    const int64_t t = pair + j * npairs;
+    *m0 = (t % gx) * kPairTileM;
+    *n0 = (t / gx) * TN;
+  };
+
+  if (threadIdx.x == 0) trace_stamp(p, 0);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&c.full[s], 1);
+      mbar_init(&c.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&c.tfull[b], 1);
+      mbar_init(&c.tempty[b], 2 * kEpiThreads / 32);
+    }
+    mbar_init(c.mma_done, 1);
+    *c.abort_flag = 0;
+    *c.last_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensor_map(&tmA);
+    prefetch_tensor_map(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(c.tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  __syncwarp();
+  tc_fence_before_sync();
+  cluster_sync_all();   // both CTAs' barriers exist and the pair's tensor memory is allocated
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *c.tmem_slot;
+  if (threadIdx.x == 0) trace_stamp(p, 1);
+  grid_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_a = policy_evict_last();
+      const uint32_t full0 = dsmem_map(smem_addr(c.full), 0);   // the first CTA's full[0]
+      int64_t it = 0;
+      int64_t issued = 0;
+      bool go = true;
+      grid_dependency_wait();   // the activations come from the previous kernel
+      trace_stamp(p, 2);
+      for (int64_t j = 0; j < my_tiles && go; ++j) {
+        int64_t m0, n0;
+        tile_origin(j, &m0, &n0);
+        const int32_t a_row = static_cast<int32_t>(m0 + rank * kTileM);
+        const int32_t b_row = static_cast<int32_t>(n0 + rank * (TN / 2));
+        for (int kb = 0; kb < T; ++kb, ++it) {
+          const int s = static_cast<int>(it % stages);
+          const uint32_t ph = static_cast<uint32_t>(it / stages) & 1u;
+          if (!wait_bar(&c.empty[s], ph ^ 1u, p, c, 0)) {
+            go = false;
+            break;
+          }
+          uint8_t* st = ring + s * Shape::kStageBytes;
+          const uint32_t fbar = full0 + static_cast<uint32_t>(s * 8);
+          if (leader) mbar_arrive_expect_tx(&c.full[s], 2 * Shape::kStageBytes);   // both CTAs' bytes
+          tma_load_2d_pair(&tmA, fbar, st, kb * kTileK, a_row, pol_a);
+          tma_load_2d_pair(&tmB, fbar, st + Shape::kABytes, kb * kTileK, b_row, pol_w);
+          issued = it + 1;
+        }
+      }
+      if (*c.abort_flag && leader) {
+        // Drain: wait (bounded) until the pair's copies still in flight have
+        // landed (each slot's barrier counts both CTAs' bytes).
+        const int64_t first = issued > stages ? issued - stages : 0;
+        for (int64_t q = first; q < issued; ++q) {
+          const uint32_t par = static_cast<uint32_t>(q / stages) & 1u;
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&c.full[q % stages], par) && global_timer_ns() - t0 < p.wait_limit_ns) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (first CTA)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = make_idesc<kInt8>(kPairTileM, TN);
+      bool issued_any = false;
+      bool go = true;
+      int64_t it = 0;
+      for (int64_t j = 0; j < my_tiles && go; ++j) {
+        const int b = static_cast<int>(j & 1);
+        const uint32_t use = static_cast<uint32_t>(j >> 1);
+        // both CTAs' epilogues have read tile j - 2 (arrivals of both CTAs: cluster scope)
+        if (!wait_bar<true>(&c.tempty[b], (use & 1u) ^ 1u, p, c, 1)) break;
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * TN);
+        for (int kb = 0; kb < T; ++kb, ++it) {
+          const int s = static_cast<int>(it % stages);
+          const uint32_t ph = static_cast<uint32_t>(it / stages) & 1u;
+          if (!wait_bar(&c.full[s], ph, p, c, 2)) {
+            go = false;
+            break;
+          }
+          tc_fence_after_sync();
+          if (it == 0) trace_stamp(p, 3);
+          uint8_t* st = ring + s * Shape::kStageBytes;
+          const uint64_t ad = smem_desc_k_sw128(st);
+          const uint64_t bd = smem_desc_k_sw128(st + Shape::kABytes);
+#pragma unroll
+          for (int kk = 0; kk < kTileK / kMmaK; ++kk) {
+            const uint32_t acc = (kb > 0 || kk > 0);
+            if (kInt8)
+              mma_i8_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+            else
+              mma_f8f6f4_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+          }
+          issued_any = true;
+          mma_commit_pair_multicast(&c.empty[s], kPairMask);
+        }
+        if (go) mma_commit_pair_multicast(&c.tfull[b], kPairMask);
+      }
+      trace_stamp(p, 4);
+      (void)issued_any;
+      // arrives once every MMA issued so far has finished (at once if none was)
+      if (my_tiles > 0) mma_commit_pair_multicast(c.mma_done, kPairMask);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    grid_dependency_wait();   // the scales may come from the previous kernel
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t tempty0 = dsmem_map(smem_addr(c.tempty), 0);   // the first CTA's tempty[0]
+    bool ok = true;
+    for (int64_t j = 0; j < my_tiles; ++j) {
+      const int b = static_cast<int>(j & 1);
+      const uint32_t use = static_cast<uint32_t>(j >> 1);
+      int64_t m0, n0;
+      tile_origin(j, &m0, &n0);
+      float* cs = colsc + b * 256;
+      for (int col = r; col < TN; col += kEpiThreads) cs[col] = n0 + col < p.N ? __ldg(p.b_s + n0 + col) : 0.f;
+      const int64_t m = m0 + rank * kTileM + r;
+      const float as_r = m < p.M ? __ldg(p.a_s + m) : 0.f;
+      named_barrier_sync(2, kEpiThreads);
+      if (ok) ok = __all_sync(0xffffffffu, wait_bar(&c.tfull[b], use & 1u, p, c, 5) && !*c.abort_flag);
+      if (!ok) continue;
+      tc_fence_after_sync();
+      const uint32_t t_buf = t_row + static_cast<uint32_t>(b * TN);
+#pragma unroll
+      for (int c0 = 0; c0 < TN; c0 += CH) {
+        uint32_t v[CH];
+        tmem_ld_32x32b_x32(t_buf + c0, v);
+        tmem_ld_wait();
+        if (c0 + CH == TN) {
+          // the buffer's last columns are in registers: the pair's MMA may refill it
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty0 + static_cast<uint32_t>(b * 8));
+        }
+        if (m < p.M) {
+#pragma unroll
+          for (int j8 = 0; j8 < CH; j8 += 8) {
+            const int64_t n = n0 + c0 + j8;
+            if (n < p.N) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float a = kInt8 ? static_cast<float>(static_cast<int32_t>(v[j8 + e])) : __uint_as_float(v[j8 + e]);
+                f[e] = a * as_r * cs[c0 + j8 + e];
+              }
+              if constexpr (BIAS) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] += bias_at(p, n + e);
+              }
+              *reinterpret_cast<uint4*>(p.C + m * p.N + n) =
+                  make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                             pack_bf16x2(f[6], f[7]));
+              if (kInt8 && p.acc_out) {
+                uint4* ao = reinterpret_cast<uint4*>(p.acc_out + m * p.N + n);
+                ao[0] = make_uint4(v[j8 + 0], v[j8 + 1], v[j8 + 2], v[j8 + 3]);
+                ao[1] = make_uint4(v[j8 + 4], v[j8 + 5], v[j8 + 6], v[j8 + 7]);
+              }
+            }
+          }
+        }
+      }
+    }
+    if (warp == 2 && lane == 0) trace_stamp(p, 6);
+  }
+
+  // -------------------------------------------------------------- teardown
+  // Every MMA of the pair must be finished before either CTA leaves (they
+  // read both CTAs' shared memory and write both tensor memories).
+  if (warp == 1 && lane == 0 && my_tiles > 0) wait_bar(c.mma_done, 0, p, c, 3);
+  __syncwarp();
+  tc_fence_before_sync();
+  cluster_sync_all();
+  if (threadIdx.x == 0) trace_stamp(p, 7);
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+template <int FMT, int TN, bool BIAS>
+cudaError_t launch_pair_tc(const GemmLaunch& l) {
+  auto kern = scaled_mm_pair_kernel<FMT, TN, BIAS>;
+  static int configured = 0;
+  if (configured < l.smem_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    configured = 227 * 1024;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = l.grid;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(l.smem_bytes);
+  cfg.stream = l.stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = 2;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = 1;
+  ++na;
+  if (l.pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, l.tmX, l.tmY, l.p);
+}
+
+// Largest number of co-resident pairs for (FMT, TN, BIAS) with `smem_bytes`.
+template <int FMT, int TN, bool BIAS>
+int max_pairs(int smem_bytes) {
+  auto kern = scaled_mm_pair_kernel<FMT, TN, BIAS>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+template <int FMT, bool BIAS>
+cudaError_t launch_pair(const GemmLaunch& l, int tile_n) {
+  if constexpr (FMT == kFmtFp8 || FMT == kFmtInt8) {
+    switch (tile_n) {
+      case 128: return launch_pair_tc<FMT, 128, BIAS>(l);
+      case 256: return launch_pair_tc<FMT, 256, BIAS>(l);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lq

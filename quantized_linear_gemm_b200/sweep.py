@@ -100,10 +100,12 @@ def candidates(fmt, M, N, K):
                 for st in (3, 4, 6, 0):
                     for pdl in (1, 2):
                         add(swap_ab=0, tile_n=tn, split_k=S, stages=st, reduce=2, pdl=pdl)
-            if fmt in (lq.FP8_DYNAMIC, lq.W8A8_INT8):   # persistent CTAs (one split)
+            if fmt in (lq.FP8_DYNAMIC, lq.W8A8_INT8):   # persistent CTAs and CTA pairs (one split)
                 for st in (3, 4, 0):
                     for pdl in (1, 2):
                         add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=1)
+                        if tn >= 128:
+                            add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=2)
     return out
 
 

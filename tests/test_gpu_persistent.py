@@ -126,7 +126,7 @@ def test_persistent_refuses_what_it_does_not_do(cuda_device):
     prob = make_problem(lq.FP8_DYNAMIC, 64, 256, 512, seed=407)
     A, sa, B, sb = prob.device()
     for bad in (dict(swap_ab=1, tile_n=16, persistent=1), dict(swap_ab=0, tile_n=128, split_k=2, persistent=1),
-                dict(swap_ab=0, tile_n=128, persistent=2)):
+                dict(swap_ab=0, tile_n=128, persistent=3)):
         with pytest.raises(lq.LQError):
             lq.scaled_mm(lq.FP8_DYNAMIC, A, sa, B, sb, variant=lq.make_variant(**bad))
     qa = torch.zeros((64, 512), dtype=torch.uint8, device="cuda")
@@ -134,3 +134,74 @@ def test_persistent_refuses_what_it_does_not_do(cuda_device):
         lq.scaled_mm("block_fp8", qa, torch.ones((64, 4), device="cuda"), torch.zeros((256, 512), dtype=torch.uint8,
                      device="cuda"), torch.ones((2, 4), device="cuda"),
                      variant=lq.make_variant(swap_ab=0, tile_n=128, persistent=1))
+
+
+# ----------------------------------------------------------- CTA pairs (persistent = 2)
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
+@pytest.mark.parametrize("tn", [128, 256])
+def test_pair_small_ragged(cuda_device, fmt, tn):
+    """CTA pairs (tcgen05 cta_group::2, 256-row tiles): M = 300 (the second
+    CTA's rows partly past M), N = 1000 (ragged), K = 1040 (ragged K tile):
+    within tolerance of the oracle and bitwise reproducible."""
+    prob = make_problem(fmt, 300, 1000, 1040, seed=411)
+    A, sa, B, sb = prob.device()
+    v = lq.make_variant(swap_ab=0, tile_n=tn, split_k=1, persistent=2)
+    C0 = lq.scaled_mm(prob.fmt, A, sa, B, sb, variant=v).clone()
+    C1 = lq.scaled_mm(prob.fmt, A, sa, B, sb, variant=v)
+    torch.cuda.synchronize()
+    assert lq.device_status(0) == 0
+    assert torch.equal(C0, C1)
+    assert_close(C0, prob.reference(), f"pair tn={tn}")
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
+@pytest.mark.parametrize("tn", [128, 256])
+def test_pair_many_tiles_equals_one_sm(cuda_device, fmt, tn):
+    """M = 1100, N = 4096: several 256-row tiles per pair, both accumulator
+    buffers of both CTAs reused; the same bits as the one-SM persistent kernel
+    (each SM's tensor core computes its 128 rows with the same MMA sequence)
+    and the oracle on sampled outputs."""
+    M, N, K = 1100, 4096, 1024
+    prob = make_problem(fmt, M, N, K, seed=412 + tn, outliers=False)
+    A, sa, B, sb = prob.device()
+    Cp = lq.scaled_mm(prob.fmt, A, sa, B, sb, variant=lq.make_variant(swap_ab=0, tile_n=tn, persistent=2))
+    C1 = lq.scaled_mm(prob.fmt, A, sa, B, sb, variant=lq.make_variant(swap_ab=0, tile_n=tn, persistent=1))
+    torch.cuda.synchronize()
+    assert lq.device_status(0) == 0
+    assert torch.equal(Cp, C1)
+    rows = np.array([0, 127, 128, 255, 256, 700, 1023, 1024, 1099])
+    cols = np.array([0, 7, 127, 128, 255, 256, 2047, 4095])
+    name = {lq.FP8_DYNAMIC: O.FMT_FP8_DYNAMIC, lq.W8A8_INT8: O.FMT_W8A8_INT8}[fmt]
+    ref = O.scaled_mm_ref(name, prob.qa[rows], prob.sa[rows], prob.qb[cols], prob.sb[cols])
+    ok, worst = O.within_tolerance(Cp.float().cpu().numpy().astype(np.float64)[np.ix_(rows, cols)], ref)
+    assert ok, worst
+
+
+def test_pair_int8_exact_bias_and_graph(cuda_device):
+    prob = make_problem(lq.W8A8_INT8, 520, 768, 1152, seed=413)
+    A, sa, B, sb = prob.device()
+    v = lq.make_variant(swap_ab=0, tile_n=256, persistent=2)
+    C, acc = lq.scaled_mm_i32acc(A, sa, B, sb, variant=v)
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.acc_exact(O.FMT_W8A8_INT8, prob.qa, prob.qb))
+    assert_close(C, prob.reference(), "pair int8")
+    g = torch.Generator().manual_seed(414)
+    bias = (torch.randn(768, generator=g) * 0.5).to(torch.bfloat16).cuda()
+    Cb = lq.scaled_mm_bias(lq.W8A8_INT8, A, sa, B, sb, bias, variant=v)
+    torch.cuda.synchronize()
+    assert_close(Cb, prob.reference() + bias.double().cpu().numpy()[None, :], "pair bias")
+    out = torch.empty_like(C)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(gr, stream=s):
+            lq.scaled_mm(lq.W8A8_INT8, A, sa, B, sb, C=out, variant=v, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(2):
+        out.zero_()
+        gr.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, C)
+    del gr
+    assert lq.device_status(0) == 0
