@@ -119,7 +119,16 @@ typedef enum {
  *            (clusters of two, one MMA of 256 rows over both SMs with
  *            tcgen05 cta_group::2; each CTA loads 128 rows of A and half of
  *            the tile's tile_n (128 or 256) weight rows).  Same results bit
- *            for bit.
+ *            for bit; 3 = stream-K (tile_n 128 or 256): one CTA per SM,
+ *            each taking an equal contiguous share of all tiles' K blocks;
+ *            a tile split between CTAs is finished by the CTA holding its
+ *            last K block, which adds the others' partial sums (kept in the
+ *            library's workspace: the restrictions of Split-K with reduce
+ *            0 / 1 apply) in K order.  Bitwise reproducible, but FP8 results
+ *            are not bit-identical to the other schedules (its fp32 partial
+ *            sums are grouped differently; INT8 is exact in every schedule).
+ *            For shapes with few output tiles.  lq_scaled_mm_noalloc runs it
+ *            as 1.
  *  pdl     : 0 = plain launch;
  *            1 = programmatic dependent launch: the kernel's set-up overlaps
  *            the tail of the previous kernel on the stream, and all of its

@@ -39,6 +39,7 @@ using lq::GemmParams;
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSmemPerCta = 227 * 1024;
 constexpr size_t kCounterCapacity = size_t(1) << 20;   // Split-K arrival counters per device
+constexpr int kMaxStreamKCtas = 1024;                   // stream-K partial-ready flags per device
 constexpr int kNumSms = 148;
 constexpr int kMaxStages = 14;
 // W8A8_INT8 sums products of int8 codes in int32: |a b| <= 128 * 128, so K
@@ -57,6 +58,7 @@ struct DeviceState {
   bool ready = false;
   int* status = nullptr;       // one int, bit i set when wait site i timed out
   int* counters = nullptr;     // kCounterCapacity ints, zero between calls
+  int* sk_flags = nullptr;     // kMaxStreamKCtas ints: stream-K partial ready (zero between calls)
   void* ws = nullptr;          // Split-K partials
   size_t ws_bytes = 0;
   std::vector<void*> retired;  // smaller workspaces replaced by ws, kept until exit
@@ -126,8 +128,10 @@ lq_status init_device_locked(int dev) {
   lq_status rc = LQ_OK;
   if (cudaMalloc(&d.status, sizeof(int)) != cudaSuccess ||
       cudaMalloc(&d.counters, kCounterCapacity * sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&d.sk_flags, kMaxStreamKCtas * sizeof(int)) != cudaSuccess ||
       cudaMemset(d.status, 0, sizeof(int)) != cudaSuccess ||
       cudaMemset(d.counters, 0, kCounterCapacity * sizeof(int)) != cudaSuccess ||
+      cudaMemset(d.sk_flags, 0, kMaxStreamKCtas * sizeof(int)) != cudaSuccess ||
       cudaDeviceSynchronize() != cudaSuccess) {
     rc = LQ_ERR_CUDA;
   } else {
@@ -284,7 +288,7 @@ int max_stages_fit(int tile_n, int ctas_per_sm, bool cluster_reduce, bool fuse =
 int max_persistent_stages(int tile_n, int persistent = 1) {
   int best = 2;
   for (int s = 2; s <= kMaxStages; ++s) {
-    const int bytes = persistent == 2 ? lq::pair_smem_bytes_for(tile_n, s) : lq::persistent_smem_bytes_for(tile_n, s);
+    const int bytes = persistent == 2 ? lq::pair_smem_bytes_for(tile_n, s) : lq::persistent_smem_bytes_for(tile_n, s);   // 1, 3
     if (bytes > 0 && bytes <= kMaxSmemPerCta) best = s;
   }
   return best;
@@ -398,11 +402,11 @@ lq_status check_variant(int fmt, const lq_variant& v) {
     if (fmt == lq::kFmtBlock && v.tile_n == 256) return LQ_ERR_INVALID_ARG;   // promotion in registers
   }
   if (v.stages != 0 && (v.stages < 2 || v.stages > kMaxStages)) return LQ_ERR_INVALID_ARG;
-  if (v.persistent < 0 || v.persistent > 2) return LQ_ERR_INVALID_ARG;
+  if (v.persistent < 0 || v.persistent > 3) return LQ_ERR_INVALID_ARG;
   if (v.persistent) {
-    // Standard orientation, one split, FP8_Dynamic / W8A8_INT8 (CTA pairs: tile_n 128 or 256)
+    // Standard orientation, one split, FP8_Dynamic / W8A8_INT8 (CTA pairs and stream-K: tile_n 128 or 256)
     if (v.swap_ab || v.split_k != 1 || (fmt != lq::kFmtFp8 && fmt != lq::kFmtInt8)) return LQ_ERR_INVALID_ARG;
-    if (v.persistent == 2 && v.tile_n == 64) return LQ_ERR_INVALID_ARG;
+    if (v.persistent >= 2 && v.tile_n == 64) return LQ_ERR_INVALID_ARG;
     const int bytes = v.persistent == 2 ? lq::pair_smem_bytes_for(v.tile_n, v.stages ? v.stages : 2)
                                         : lq::persistent_smem_bytes_for(v.tile_n, v.stages ? v.stages : 2);
     if (bytes > kMaxSmemPerCta) return LQ_ERR_INVALID_ARG;
@@ -492,6 +496,15 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   p.a_codes_out = static_cast<uint8_t*>(codes_out);
   p.a_scales_out = scales_out;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
+  if (v.persistent == 3) {   // stream-K: one partial slot [128 x tile_n] per CTA, and the ready flags
+    const int64_t iters = ((M + 127) / 128) * gy * p.T;
+    const int64_t ctas = iters < sm_count() ? iters : sm_count();
+    if (ctas > kMaxStreamKCtas) return LQ_ERR_UNSUPPORTED_SHAPE;
+    rc = ensure_workspace(d, static_cast<size_t>(ctas) * 128u * static_cast<size_t>(v.tile_n) * 4u, stream);
+    if (rc != LQ_OK) return rc;
+    p.ws = d->ws;
+    p.counters = d->sk_flags;
+  }
   if (v.split_k > 1 && v.reduce != 2) {   // the cluster reduction needs no global workspace
     const size_t need = static_cast<size_t>(v.split_k) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
     rc = ensure_workspace(d, need, stream);
@@ -521,6 +534,12 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
     l.grid = dim3(static_cast<unsigned>(ctas), 1, 1);
     l.smem_bytes = lq::persistent_smem_bytes_for(v.tile_n, v.stages);
     l.persistent = 1;
+  } else if (v.persistent == 3) {   // stream-K: one CTA per SM splitting tiles x K blocks
+    const int64_t iters = ((M + 127) / 128) * gy * p.T;
+    const int64_t ctas = iters < sm_count() ? iters : sm_count();
+    l.grid = dim3(static_cast<unsigned>(ctas), 1, 1);
+    l.smem_bytes = lq::persistent_smem_bytes_for(v.tile_n, v.stages);
+    l.persistent = 3;
   } else if (v.persistent == 2) {   // clusters of two CTAs, 256-row tiles, each pair looping over tiles
     l.smem_bytes = lq::pair_smem_bytes_for(v.tile_n, v.stages);
     const int64_t tiles = ((M + 255) / 256) * gy;
@@ -990,6 +1009,11 @@ lq_status lq_reserve_workspace(int device, size_t bytes) {
 size_t lq_workspace_bytes(lq_fmt fmt, int64_t M, int64_t N, int64_t K, const lq_variant* variant) {
   if (M <= 0 || N <= 0 || K <= 0 || fmt < 0 || fmt > 3) return 0;
   const lq_variant v = variant ? *variant : default_variant(static_cast<int>(fmt), M, N, K);
+  if (v.persistent == 3 && !v.swap_ab && v.tile_n > 0) {   // stream-K partial slots
+    const int64_t iters = ((M + 127) / 128) * ((N + v.tile_n - 1) / v.tile_n) * ((K + 127) / 128);
+    const int64_t ctas = iters < sm_count() ? iters : sm_count();
+    return static_cast<size_t>(ctas) * 128u * static_cast<size_t>(v.tile_n) * 4u;
+  }
   if (v.split_k <= 1 || v.reduce == 2) return 0;
   return static_cast<size_t>(v.split_k) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
 }
@@ -1011,6 +1035,7 @@ lq_status lq_device_status(int device) {
     // A CTA that gave up did not count itself: clear the Split-K arrival
     // counters so that later calls start from zero.
     cudaMemset(d.counters, 0, kCounterCapacity * sizeof(int));
+    cudaMemset(d.sk_flags, 0, kMaxStreamKCtas * sizeof(int));
     cudaDeviceSynchronize();
     rc = LQ_ERR_DEVICE_TIMEOUT;
   }
@@ -1074,8 +1099,10 @@ extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const floa
                                                                                                   : LQ_ERR_CUDA;
   lq_variant v = variant ? *variant : default_variant(fmt, M, N, K);
   // Split-K partials always go through the scratch array and the separate
-  // fixed-order reduction kernel (no arrival counters, nothing to re-arm).
+  // fixed-order reduction kernel (no arrival counters, nothing to re-arm);
+  // stream-K, whose partials need a workspace, runs as persistent CTAs.
   if (v.split_k > 1) v.reduce = 0;
+  if (v.persistent == 3) v.persistent = 1;
   rc = check_variant(fmt, v);
   if (rc != LQ_OK) return rc;
   const size_t need = v.split_k > 1 ? static_cast<size_t>(v.split_k) * static_cast<size_t>(M) *

@@ -57,7 +57,8 @@ struct GemmLaunch {
   int fuse;            // fused activation quantization (Swap-AB only)
   int grouped;         // grouped (mixture-of-experts) launch (Swap-AB only; p.expert_offsets set)
   int persistent;      // 1: persistent CTAs looping over output tiles (Standard, split_k 1, FP8 / INT8);
-                       // 2: the same on CTA pairs (cta_group::2, 256-row tiles, clusters of two)
+                       // 2: the same on CTA pairs (cta_group::2, 256-row tiles, clusters of two);
+                       // 3: stream-K (equal shares of tiles x K blocks; p.ws slots, p.counters flags)
   cudaStream_t stream;
 };
 

@@ -56,8 +56,9 @@ __host__ __device__ constexpr int tmem_cols_for(int cols) {
 }
 
 // Tensor-memory columns of the UE8M0 scale factors of the block-scaled MMA
-// (after the accumulator's TN columns).  Two slots, each the scale factors of
-// four consecutive 128-K blocks: one 32-bit column per 32 rows of an operand
+// (after the accumulator's TN columns).  Up to four slots (as many as ring
+// stages, at least two), each the scale factors of four consecutive 128-K
+// blocks: one 32-bit column per 32 rows of an operand
 // tile, the byte of block t (0..3) of the group in bits [8t, 8t+8), row e of
 // the tile at lane e % 32 and column e / 32 of the operand's part of the
 // slot, the same in all four lane quarters.  X (128 rows) takes 4 columns, Y
@@ -68,8 +69,13 @@ struct MxSf {
   static constexpr int kXCols = 4;
   static constexpr int kYCols = TN > 128 ? TN / 32 : 4;
   static constexpr int kSlotCols = (kXCols + kYCols + 7) / 8 * 8;
-  static constexpr int kEnd = kBase + 2 * kSlotCols;
+  static constexpr int kMaxSlots = 4;
+  static constexpr int kEnd = kBase + kMaxSlots * kSlotCols;
 };
+
+// Scale-factor slots of a launch with `stages` ring slots (their mbarriers
+// are the ring's xfull / wfull entries).
+__device__ __forceinline__ int mx_slots(int stages) { return stages < 4 ? stages : 4; }
 
 // Cluster Split-K reduction.  Tiles up to 64 wide push: every CTA sends its
 // partial columns, from registers, into slots in the shared memory of the
@@ -317,9 +323,9 @@ __global__ void __launch_bounds__(kThreads, SWAP ? 2 : 1)   // Swap-AB: two CTAs
     for (int s = 0; s < stages; ++s) {
       mbar_init(&c.full[s], FUSE ? kEpiThreads / 32 : 1);   // the TMA, or the four A-producer warps
       mbar_init(&c.empty[s], 1);
-      // block-scaled MMA: xfull[0..1] = scale-factor slot written (the four
-      // epilogue warps), wfull[0..1] = slot read by the tensor core (commit)
-      mbar_init(&c.xfull[s], (kMX && s < 2) ? kEpiThreads / 32 : 1);
+      // block-scaled MMA: xfull[slot] = scale-factor slot written (the four
+      // epilogue warps), wfull[slot] = slot read by the tensor core (commit)
+      mbar_init(&c.xfull[s], (kMX && s < mx_slots(stages)) ? kEpiThreads / 32 : 1);
       mbar_init(&c.wfull[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -439,13 +445,23 @@ __global__ void __launch_bounds__(kThreads, SWAP ? 2 : 1)   // Swap-AB: two CTAs
     if (lane == 0) {
       constexpr uint32_t idesc = kMX ? make_idesc_mx(kTileM, TN) : make_idesc<kInt8>(kTileM, TN);
       bool issued_any = false;
+      // block-scaled MMA: the scale-factor slot of the current group of four
+      // blocks, its phase, and its tensor-memory address (advanced per group)
+      const int mx_ns = kMX ? mx_slots(stages) : 1;
+      int mx_slot = 0;
+      uint32_t mx_phase = 0;
+      uint32_t mx_sf = tmem_base + static_cast<uint32_t>(MxSf<TN>::kBase);
       for (int i = 0; i < nkb; ++i) {
         const int s = i % stages;
         const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
         uint32_t d_tmem = tmem_base;
         if (kMX && (i & 3) == 0) {   // the scale factors of blocks i .. i+3 are in tensor memory
-          const int g = i >> 2;
-          if (!wait_bar(&c.xfull[g & 1], static_cast<uint32_t>(g >> 1) & 1u, p, c, 13)) break;
+          if (i > 0 && ++mx_slot == mx_ns) {
+            mx_slot = 0;
+            mx_phase ^= 1u;
+          }
+          mx_sf = tmem_base + static_cast<uint32_t>(MxSf<TN>::kBase + mx_slot * MxSf<TN>::kSlotCols);
+          if (!wait_bar(&c.xfull[mx_slot], mx_phase, p, c, 13)) break;
         }
         if (kPromote) {
           const int buf = i & 1;
@@ -466,9 +482,8 @@ __global__ void __launch_bounds__(kThreads, SWAP ? 2 : 1)   // Swap-AB: two CTAs
           const uint32_t acc = kPromote ? (kk > 0) : (i > 0 || kk > 0);
           if constexpr (kMX) {
             const uint32_t t = static_cast<uint32_t>(i & 3);   // this block's byte in the slot
-            const uint32_t sf = tmem_base + static_cast<uint32_t>(MxSf<TN>::kBase + ((i >> 2) & 1) * MxSf<TN>::kSlotCols);
-            mma_mxf8f6f4_block_scale(d_tmem, xd + 2 * kk, yd + 2 * kk, idesc_with_sf_ids(idesc, t, t), sf,
-                                     sf + MxSf<TN>::kXCols, acc);
+            mma_mxf8f6f4_block_scale(d_tmem, xd + 2 * kk, yd + 2 * kk, idesc_with_sf_ids(idesc, t, t), mx_sf,
+                                     mx_sf + MxSf<TN>::kXCols, acc);
           } else if (kInt8) {
             mma_i8(d_tmem, xd + 2 * kk, yd + 2 * kk, idesc, acc);
           } else {
@@ -478,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, SWAP ? 2 : 1)   // Swap-AB: two CTAs
         issued_any = true;
         mma_commit(&c.empty[s]);
         if (kPromote) mma_commit(&c.tfull[i & 1]);
-        if (kMX && ((i & 3) == 3 || i == nkb - 1)) mma_commit(&c.wfull[(i >> 2) & 1]);   // slot read
+        if (kMX && ((i & 3) == 3 || i == nkb - 1)) mma_commit(&c.wfull[mx_slot]);   // slot read
       }
       trace_stamp(p, 4);
       if (!kPromote && nkb > 0 && !*c.abort_flag) mma_commit(&c.tfull[0]);
@@ -690,10 +705,16 @@ __global__ void __launch_bounds__(kThreads, SWAP ? 2 : 1)   // Swap-AB: two CTAs
         }
       };
       const int groups = (nkb + 3) / 4;
+      const int ns = mx_slots(stages);
       if (groups > 0) gather(0);
+      int slot = 0;
+      uint32_t reuse_phase = 0;   // phase of wfull[slot] that frees it for this group
       for (int g = 0; g < groups && ok; ++g) {
-        const int slot = g & 1;
-        if (g >= 2) ok = __all_sync(0xffffffffu, wait_bar(&c.wfull[slot], static_cast<uint32_t>((g - 2) >> 1) & 1u, p, c, 14));
+        if (g > 0 && ++slot == ns) {
+          slot = 0;
+          if (g > ns) reuse_phase ^= 1u;
+        }
+        if (g >= ns) ok = __all_sync(0xffffffffu, wait_bar(&c.wfull[slot], reuse_phase, p, c, 14));
         if (!ok) break;
         tc_fence_after_sync();
         const uint32_t col0 = t_row + static_cast<uint32_t>(Sf::kBase + slot * Sf::kSlotCols);

@@ -4,6 +4,7 @@
 #include "scaled_mm_kernel.cuh"
 #include "scaled_mm_persistent.cuh"
 #include "scaled_mm_pair.cuh"
+#include "scaled_mm_streamk.cuh"
 
 namespace lq {
 
@@ -90,6 +91,10 @@ cudaError_t launch_format(const GemmLaunch& l, int swap_ab, int tile_n) {
       }
     }
     return cudaErrorInvalidValue;
+  }
+  if (l.persistent == 3) {
+    if (swap_ab) return cudaErrorInvalidValue;
+    return l.p.bias ? launch_streamk<FMT, true>(l, tile_n) : launch_streamk<FMT, false>(l, tile_n);
   }
   if (l.persistent == 2) {
     if (swap_ab) return cudaErrorInvalidValue;

@@ -106,6 +106,7 @@ def candidates(fmt, M, N, K):
                         add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=1)
                         if tn >= 128:
                             add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=2)
+                            add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=3)
     return out
 
 

@@ -117,14 +117,15 @@ def test_variant_checks(field, value):
 
 
 def test_persistent_variant_rules():
-    """persistent = 1 (one-SM tiles) and 2 (CTA pairs, tile_n 128 / 256) need
-    the Standard orientation, one split and FP8 / INT8."""
-    for pers in (1, 2):
+    """persistent = 1 (one-SM tiles), 2 (CTA pairs) and 3 (stream-K; both
+    tile_n 128 / 256) need the Standard orientation, one split and FP8 / INT8."""
+    for pers in (1, 2, 3):
         ok = lq.make_variant(swap_ab=0, tile_n=256, split_k=1, persistent=pers)
         assert _mm(variant=ok, C=MISALIGNED) == ALIGN    # accepted up to the pointer checks
     for bad in (dict(swap_ab=1, tile_n=16, persistent=1), dict(swap_ab=0, tile_n=128, split_k=2, persistent=1),
-                dict(swap_ab=0, tile_n=128, persistent=3), dict(swap_ab=0, tile_n=256, stages=5, persistent=1),
-                dict(swap_ab=0, tile_n=64, persistent=2), dict(swap_ab=1, tile_n=32, persistent=2)):
+                dict(swap_ab=0, tile_n=128, persistent=4), dict(swap_ab=0, tile_n=256, stages=5, persistent=1),
+                dict(swap_ab=0, tile_n=64, persistent=2), dict(swap_ab=1, tile_n=32, persistent=2),
+                dict(swap_ab=0, tile_n=64, persistent=3), dict(swap_ab=0, tile_n=256, split_k=2, persistent=3)):
         assert _mm(variant=lq.make_variant(**bad)) == INVALID, bad
     for fmt in (2, 3):
         assert _mm(fmt=fmt, K=256, N=256, variant=lq.make_variant(swap_ab=0, tile_n=128, persistent=1)) == INVALID

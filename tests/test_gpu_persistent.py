@@ -126,7 +126,7 @@ def test_persistent_refuses_what_it_does_not_do(cuda_device):
     prob = make_problem(lq.FP8_DYNAMIC, 64, 256, 512, seed=407)
     A, sa, B, sb = prob.device()
     for bad in (dict(swap_ab=1, tile_n=16, persistent=1), dict(swap_ab=0, tile_n=128, split_k=2, persistent=1),
-                dict(swap_ab=0, tile_n=128, persistent=3)):
+                dict(swap_ab=0, tile_n=128, persistent=4)):
         with pytest.raises(lq.LQError):
             lq.scaled_mm(lq.FP8_DYNAMIC, A, sa, B, sb, variant=lq.make_variant(**bad))
     qa = torch.zeros((64, 512), dtype=torch.uint8, device="cuda")
@@ -205,3 +205,65 @@ def test_pair_int8_exact_bias_and_graph(cuda_device):
         assert torch.equal(out, C)
     del gr
     assert lq.device_status(0) == 0
+
+
+# --------------------------------------------------------------- stream-K (persistent = 3)
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
+@pytest.mark.parametrize("tn", [128, 256])
+@pytest.mark.parametrize("M,N,K", [(300, 1000, 1040),      # fewer iterations than SMs: one K block per CTA
+                                   (256, 1024, 25600)])    # 8 or 16 tiles of 200 K blocks over 148 CTAs
+def test_streamk(cuda_device, fmt, tn, M, N, K):
+    """Every tile finished by the CTA holding its last K block after adding
+    the partials of up to ~20 earlier CTAs: within tolerance of the oracle
+    (sampled at the deep size), INT8 accumulators exact, bitwise
+    reproducible, also under graph replay (the ready flags return to zero)."""
+    prob = make_problem(fmt, M, N, K, seed=421 + tn + M, outliers=False)
+    A, sa, B, sb = prob.device()
+    v = lq.make_variant(swap_ab=0, tile_n=tn, persistent=3)
+    lq.reserve_workspace(0, lq.workspace_bytes(fmt, M, N, K, v))
+    if fmt == lq.W8A8_INT8:
+        C0, acc = lq.scaled_mm_i32acc(A, sa, B, sb, variant=v)
+    else:
+        C0 = lq.scaled_mm(fmt, A, sa, B, sb, variant=v)
+    C0 = C0.clone()
+    torch.cuda.synchronize()
+    assert lq.device_status(0) == 0
+    if K > 4096:
+        rows = np.array([0, 1, 127, 128, 200, 255])
+        cols = np.array([0, 5, 255, 256, 511, 512, 1000, 1023])
+    else:
+        rows, cols = np.arange(M), np.arange(N)
+    name = {lq.FP8_DYNAMIC: O.FMT_FP8_DYNAMIC, lq.W8A8_INT8: O.FMT_W8A8_INT8}[fmt]
+    ref = O.scaled_mm_ref(name, prob.qa[rows], prob.sa[rows], prob.qb[cols], prob.sb[cols])
+    ok, worst = O.within_tolerance(C0.float().cpu().numpy().astype(np.float64)[np.ix_(rows, cols)], ref)
+    assert ok, worst
+    if fmt == lq.W8A8_INT8:
+        exact = O.acc_exact(O.FMT_W8A8_INT8, prob.qa[rows], prob.qb[cols])
+        assert np.array_equal(acc.cpu().numpy().astype(np.int64)[np.ix_(rows, cols)], exact)
+    out = torch.empty_like(C0)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            lq.scaled_mm(fmt, A, sa, B, sb, C=out, variant=v, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, C0)
+    del g
+    assert lq.device_status(0) == 0
+
+
+def test_streamk_bias(cuda_device):
+    prob = make_problem(lq.FP8_DYNAMIC, 256, 512, 8192, seed=431)
+    A, sa, B, sb = prob.device()
+    g = torch.Generator().manual_seed(432)
+    bias = (torch.randn(512, generator=g) * 0.5).to(torch.bfloat16).cuda()
+    v = lq.make_variant(swap_ab=0, tile_n=256, persistent=3)
+    lq.reserve_workspace(0, lq.workspace_bytes("fp8_dynamic", 256, 512, 8192, v))
+    C = lq.scaled_mm_bias(lq.FP8_DYNAMIC, A, sa, B, sb, bias, variant=v)
+    torch.cuda.synchronize()
+    assert_close(C, prob.reference() + bias.double().cpu().numpy()[None, :], "stream-K bias")
