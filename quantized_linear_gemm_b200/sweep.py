@@ -82,7 +82,7 @@ def candidates(fmt, M, N, K):
                 if S > T:
                     continue
                 per = -(-T // S)
-                for st in sorted({2, min(per, 4), min(per, 6), min(per, 8), min(per, 12)}):
+                for st in sorted({2, min(per, 3), min(per, 4), min(per, 5), min(per, 6), min(per, 8), min(per, 12)}):
                     if st < 2:
                         continue
                     for pdl in (1, 2):
