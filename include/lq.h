@@ -95,7 +95,8 @@ typedef enum {
  *            1 = Swap-AB: C^T = B . A^T is computed, 128 weight rows on the M
  *            side and tile_n tokens on the N side; the epilogue transposes
  *            back on store.
- *  split_k : 1, 2, 4, ..., 256.  Split s owns the 128-wide K tiles
+ *  split_k : 1, 2, 4, ..., 256 (CTA pairs with reduce 0: any of 1..256).
+ *            Split s owns the 128-wide K tiles
  *            [floor(s*T/S), floor((s+1)*T/S)), T = ceil(K/128); a split may
  *            be empty.  Partials are summed in the fixed order s = 0..S-1,
  *            so results are reproducible bit for bit.
@@ -119,7 +120,10 @@ typedef enum {
  *            (clusters of two, one MMA of 256 rows over both SMs with
  *            tcgen05 cta_group::2; each CTA loads 128 rows of A and half of
  *            the tile's tile_n (128 or 256) weight rows).  Same results bit
- *            for bit; 3 = stream-K (tile_n 128 or 256): one CTA per SM,
+ *            for bit.  Pairs also take split_k > 1 with reduce 0: the units
+ *            (256-row tile, split) are spread over the pairs and the
+ *            separate reduction sums the workspace partials, as for the
+ *            one-SM tiles; 3 = stream-K (tile_n 128 or 256): one CTA per SM,
  *            each taking an equal contiguous share of all tiles' K blocks;
  *            a tile split between CTAs is finished by the CTA holding its
  *            last K block, which adds the others' partial sums (kept in the

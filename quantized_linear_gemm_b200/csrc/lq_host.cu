@@ -321,8 +321,10 @@ int pair_capacity(int fmt, int tile_n, bool bias, int smem_bytes) {
   std::lock_guard<std::mutex> lk(mu);
   for (const auto& e : cache)
     if (e.first == key) return e.second;
-  const int n = fmt == lq::kFmtFp8 ? lq::pair_capacity_fp8(tile_n, bias, smem_bytes)
-                                   : lq::pair_capacity_int8(tile_n, bias, smem_bytes);
+  const int n = fmt == lq::kFmtFp8    ? lq::pair_capacity_fp8(tile_n, bias, smem_bytes)
+                : fmt == lq::kFmtInt8  ? lq::pair_capacity_int8(tile_n, bias, smem_bytes)
+                : fmt == lq::kFmtBlock ? lq::pair_capacity_block(tile_n, bias, smem_bytes)
+                                       : 0;
   cache.emplace_back(key, n);
   return n;
 }
@@ -389,9 +391,31 @@ bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, lq_variant* out) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
 
+// Dynamic shared memory of a CTA-pair launch.  A pair kernel that takes all
+// 512 tensor-memory columns (tile_n 256, or the four Block_FP8 buffers)
+// asks for at least 116 KB, so that two of its CTAs never share an SM and
+// never wait for each other's columns.
+int pair_launch_smem(int fmt, int tile_n, int stages) {
+  const int bytes = lq::pair_smem_bytes_for(tile_n, stages);
+  const bool all_columns = tile_n == 256 || fmt == lq::kFmtBlock;
+  return all_columns && bytes < 116 * 1024 ? 116 * 1024 : bytes;
+}
+
+// Grid of a CTA-pair launch: one pair per (256-row tile, split) unit, at most
+// as many pairs as fit on the device at once (each pair loops over units).
+dim3 pair_grid(int fmt, int64_t M, int64_t gy, int split_k, int tile_n, bool bias, int smem_bytes) {
+  const int64_t units = ((M + 255) / 256) * gy * split_k;
+  int cap = pair_capacity(fmt, tile_n, bias, smem_bytes);
+  if (cap <= 0) cap = sm_count() / 2;
+  const int64_t pairs = units < cap ? units : cap;
+  return dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+}
+
 lq_status check_variant(int fmt, const lq_variant& v) {
   if (v.swap_ab != 0 && v.swap_ab != 1) return LQ_ERR_INVALID_ARG;
-  if (!is_pow2(v.split_k) || v.split_k > 256) return LQ_ERR_INVALID_ARG;
+  if (v.split_k < 1 || v.split_k > 256) return LQ_ERR_INVALID_ARG;
+  // any split count for CTA pairs with the separate reduction; powers of two elsewhere
+  if (!is_pow2(v.split_k) && !(v.persistent == 2 && v.reduce == 0)) return LQ_ERR_INVALID_ARG;
   if (v.reduce < 0 || v.reduce > 2) return LQ_ERR_INVALID_ARG;
   if (v.reduce == 2 && v.split_k > 16) return LQ_ERR_INVALID_ARG;   // a cluster holds at most 16 CTAs
   if (v.pdl < 0 || v.pdl > 2) return LQ_ERR_INVALID_ARG;
@@ -404,8 +428,12 @@ lq_status check_variant(int fmt, const lq_variant& v) {
   if (v.stages != 0 && (v.stages < 2 || v.stages > kMaxStages)) return LQ_ERR_INVALID_ARG;
   if (v.persistent < 0 || v.persistent > 3) return LQ_ERR_INVALID_ARG;
   if (v.persistent) {
-    // Standard orientation, one split, FP8_Dynamic / W8A8_INT8 (CTA pairs and stream-K: tile_n 128 or 256)
-    if (v.swap_ab || v.split_k != 1 || (fmt != lq::kFmtFp8 && fmt != lq::kFmtInt8)) return LQ_ERR_INVALID_ARG;
+    // Standard orientation, FP8_Dynamic / W8A8_INT8 (CTA pairs and stream-K: tile_n 128 or 256), and
+    // fp32-scale Block_FP8 on CTA pairs with tile_n 128; one split, except CTA pairs, which take Split-K
+    // with the separate reduction
+    const bool block_pair = fmt == lq::kFmtBlock && v.persistent == 2 && v.tile_n == 128;
+    if (v.swap_ab || (fmt != lq::kFmtFp8 && fmt != lq::kFmtInt8 && !block_pair)) return LQ_ERR_INVALID_ARG;
+    if (v.split_k != 1 && !(v.persistent == 2 && v.reduce == 0)) return LQ_ERR_INVALID_ARG;
     if (v.persistent >= 2 && v.tile_n == 64) return LQ_ERR_INVALID_ARG;
     const int bytes = v.persistent == 2 ? lq::pair_smem_bytes_for(v.tile_n, v.stages ? v.stages : 2)
                                         : lq::persistent_smem_bytes_for(v.tile_n, v.stages ? v.stages : 2);
@@ -540,13 +568,9 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
     l.grid = dim3(static_cast<unsigned>(ctas), 1, 1);
     l.smem_bytes = lq::persistent_smem_bytes_for(v.tile_n, v.stages);
     l.persistent = 3;
-  } else if (v.persistent == 2) {   // clusters of two CTAs, 256-row tiles, each pair looping over tiles
-    l.smem_bytes = lq::pair_smem_bytes_for(v.tile_n, v.stages);
-    const int64_t tiles = ((M + 255) / 256) * gy;
-    int cap = pair_capacity(fmt, v.tile_n, bias != nullptr, l.smem_bytes);
-    if (cap <= 0) cap = sm_count() / 2;
-    const int64_t pairs = tiles < cap ? tiles : cap;
-    l.grid = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  } else if (v.persistent == 2) {   // clusters of two CTAs, 256-row tiles, each pair looping over units
+    l.smem_bytes = pair_launch_smem(fmt, v.tile_n, v.stages);
+    l.grid = pair_grid(fmt, M, gy, v.split_k, v.tile_n, bias != nullptr, l.smem_bytes);
     l.persistent = 2;
   }
   l.pdl = v.pdl != 0;
@@ -1157,13 +1181,9 @@ extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const floa
     l.grid = dim3(static_cast<unsigned>(ctas), 1, 1);
     l.smem_bytes = lq::persistent_smem_bytes_for(v.tile_n, v.stages);
     l.persistent = 1;
-  } else if (v.persistent == 2) {   // clusters of two CTAs, 256-row tiles, each pair looping over tiles
-    l.smem_bytes = lq::pair_smem_bytes_for(v.tile_n, v.stages);
-    const int64_t tiles = ((M + 255) / 256) * gy;
-    int cap = pair_capacity(fmt, v.tile_n, false, l.smem_bytes);
-    if (cap <= 0) cap = sm_count() / 2;
-    const int64_t pairs = tiles < cap ? tiles : cap;
-    l.grid = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  } else if (v.persistent == 2) {   // clusters of two CTAs, 256-row tiles, each pair looping over units
+    l.smem_bytes = pair_launch_smem(fmt, v.tile_n, v.stages);
+    l.grid = pair_grid(fmt, M, gy, v.split_k, v.tile_n, false, l.smem_bytes);
     l.persistent = 2;
   }
   l.pdl = v.pdl != 0;

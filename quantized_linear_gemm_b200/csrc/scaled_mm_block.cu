@@ -4,6 +4,9 @@ namespace lq {
 cudaError_t launch_scaled_mm_block(const GemmLaunch& l, int swap_ab, int tile_n) {
   return launch_format<kFmtBlock>(l, swap_ab, tile_n);
 }
+int pair_capacity_block(int tile_n, bool bias, int smem_bytes) {
+  return pair_capacity<kFmtBlock>(tile_n, bias, smem_bytes);
+}
 
 int gemm_smem_bytes_for(int tile_n, int stages, bool cluster_reduce, bool fuse) {
   if (fuse) {

@@ -1,5 +1,6 @@
 // Persistent scaled_mm on CTA pairs (tcgen05 cta_group::2) for large M:
-// Standard orientation, split_k 1, FP8_Dynamic and W8A8_INT8.
+// Standard orientation, FP8_Dynamic, W8A8_INT8 and Block_FP8 with fp32
+// scales, one split or Split-K with the separate fixed-order reduction.
 //
 // A cluster of two CTAs (two SMs) computes 256 x TN output tiles with one
 // MMA of M = 256: each CTA loads its own 128 rows of A and half (TN / 2 rows)
@@ -11,11 +12,24 @@
 // kernel.  As in the one-SM persistent kernel, the pair loops over tiles,
 // its rings run on across tiles and the accumulator is double-buffered
 // (2 x TN columns in each CTA), so each tile's epilogue overlaps the next
-// tile's MMAs.  Synchronisation:
+// tile's MMAs.  With split_k S > 1 the work units are (tile, split) pairs,
+// split s covering the K blocks [s T / S, (s + 1) T / S) as in the one-SM
+// kernel, and the epilogue writes the raw accumulators to the workspace
+// ws[s][M][N] for splitk_reduce_kernel; that fills the SMs when a few
+// 256-row tiles have a deep K (M = 256, K = 25600).
+//
+// Block_FP8 (fp32 block scales, 256 x 128 tiles): every 128-K block's MMA
+// goes to one of four 128-column tensor-memory buffers (the MMA may run up
+// to four blocks ahead), and each CTA's epilogue warps add their 128 rows of
+// it, times a_s[m, kb] * b_s[n / 128, kb], into fp32 registers (fmaf in K
+// order, as the one-SM kernel does: the same bits).  Per SM a 128-K block
+// then moves 24 KB of operands from L2 instead of the one-SM 128 x 128
+// tile's 32 KB, which is what bounds that tile.  Synchronisation:
 //   full[s]   first CTA only: both CTAs' TMA loads of slot s count their
 //             bytes here (the first CTA announces the pair's total);
 //   empty[s]  both CTAs: slot s read by the tensor core (commit multicast);
-//   tfull[b]  both CTAs: accumulator buffer b complete (commit multicast);
+//   tfull[b]  both CTAs: accumulator buffer b complete (commit multicast;
+//             per tile, or per K block for Block_FP8);
 //   tempty[b] first CTA only: both CTAs' epilogue warps have read buffer b;
 //   mma_done  both CTAs: every MMA of the pair finished (before teardown).
 // Every wait is bounded; the CTAs pass two cluster barriers (after set-up,
@@ -46,11 +60,14 @@ template <int FMT, int TN, bool BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
     scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const GemmParams p) {
-  static_assert(FMT == kFmtFp8 || FMT == kFmtInt8, "pair kernel: FP8_Dynamic / W8A8_INT8");
+  static_assert(FMT == kFmtFp8 || FMT == kFmtInt8 || FMT == kFmtBlock, "pair kernel: FP8, INT8, Block_FP8");
   static_assert(TN == 128 || TN == 256, "pair tiles: 256 x 128 or 256 x 256");
+  constexpr bool kPromote = FMT == kFmtBlock;
+  static_assert(!kPromote || TN == 128, "Block_FP8 pairs: 256 x 128 tiles (TN fp32 accumulators per thread)");
   using Shape = PairShape<TN>;
   constexpr bool kInt8 = FMT == kFmtInt8;
-  constexpr int kTmemCols = 2 * TN;
+  constexpr int kNBuf = kPromote ? 4 : 2;     // tensor-memory accumulator buffers
+  constexpr int kTmemCols = kNBuf * TN;
   constexpr int CH = 32;
   constexpr uint16_t kPairMask = 0x3;
 
@@ -63,8 +80,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   c.full = bars;
   c.empty = bars + stages;
   c.tfull = bars + 2 * stages;
-  c.tempty = c.tfull + 2;
-  c.mma_done = c.tempty + 2;
+  c.tempty = c.tfull + kNBuf;
+  c.mma_done = c.tempty + kNBuf;
   c.tmem_slot = reinterpret_cast<uint32_t*>(c.mma_done + 1);
   c.abort_flag = reinterpret_cast<volatile int*>(c.tmem_slot + 1);
   c.last_flag = c.abort_flag + 1;
@@ -77,15 +94,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t gx = (p.M + kPairTileM - 1) / kPairTileM;   // 256-row blocks
   const int64_t gy = (p.N + TN - 1) / TN;
   const int64_t tiles = gx * gy;
+  const int S = p.S;
+  const int64_t units = tiles * S;   // unit u: tile u mod tiles, split u / tiles
   const int64_t pair = blockIdx.x >> 1;
   const int64_t npairs = gridDim.x >> 1;
-  const int64_t my_tiles = tiles > pair ? (tiles - pair + npairs - 1) / npairs : 0;
+  const int64_t my_tiles = units > pair ? (units - pair + npairs - 1) / npairs : 0;
   const int T = p.T;
+  const bool split_mode = S > 1;
   auto tile_origin = [&](int64_t j, int64_t* m0, int64_t* n0) {
-    const int64_t t = pair + j * npairs;
+    const int64_t t = (pair + j * npairs) % tiles;
     *m0 = (t % gx) * kPairTileM;
     *n0 = (t / gx) * TN;
   };
+  auto split_of = [&](int64_t j) { return static_cast<int>((pair + j * npairs) / tiles); };
+  auto kb_begin = [&](int s) { return static_cast<int>((static_cast<int64_t>(s) * T) / S); };
 
   if (threadIdx.x == 0) trace_stamp(p, 0);
   if (threadIdx.x == 0) {
@@ -93,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&c.full[s], 1);
       mbar_init(&c.empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kNBuf; ++b) {
       mbar_init(&c.tfull[b], 1);
       mbar_init(&c.tempty[b], 2 * kEpiThreads / 32);
     }
@@ -134,7 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tile_origin(j, &m0, &n0);
         const int32_t a_row = static_cast<int32_t>(m0 + rank * kTileM);
         const int32_t b_row = static_cast<int32_t>(n0 + rank * (TN / 2));
-        for (int kb = 0; kb < T; ++kb, ++it) {
+        const int sp = split_of(j);
+        const int kb_hi = kb_begin(sp + 1);
+        for (int kb = kb_begin(sp); kb < kb_hi; ++kb, ++it) {
           const int s = static_cast<int>(it % stages);
           const uint32_t ph = static_cast<uint32_t>(it / stages) & 1u;
           if (!wait_bar(&c.empty[s], ph ^ 1u, p, c, 0)) {
@@ -168,14 +192,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool issued_any = false;
       bool go = true;
       int64_t it = 0;
-      for (int64_t j = 0; j < my_tiles && go; ++j) {
+      if constexpr (kPromote) {
+        // one accumulator buffer per 128-K block, buffers in turn across units
+        for (int64_t j = 0; j < my_tiles && go; ++j) {
+          const int sp = split_of(j);
+          const int kb_hi = kb_begin(sp + 1);
+          for (int kb = kb_begin(sp); kb < kb_hi; ++kb, ++it) {
+            const int b = static_cast<int>(it % kNBuf);
+            const uint32_t use = static_cast<uint32_t>(it / kNBuf);
+            if (!wait_bar<true>(&c.tempty[b], (use & 1u) ^ 1u, p, c, 1)) {
+              go = false;
+              break;
+            }
+            const int s = static_cast<int>(it % stages);
+            const uint32_t ph = static_cast<uint32_t>(it / stages) & 1u;
+            if (!wait_bar(&c.full[s], ph, p, c, 2)) {
+              go = false;
+              break;
+            }
+            tc_fence_after_sync();
+            if (it == 0) trace_stamp(p, 3);
+            uint8_t* st = ring + s * Shape::kStageBytes;
+            const uint64_t ad = smem_desc_k_sw128(st);
+            const uint64_t bd = smem_desc_k_sw128(st + Shape::kABytes);
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * TN);
+#pragma unroll
+            for (int kk = 0; kk < kTileK / kMmaK; ++kk)
+              mma_f8f6f4_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+            issued_any = true;
+            mma_commit_pair_multicast(&c.empty[s], kPairMask);
+            mma_commit_pair_multicast(&c.tfull[b], kPairMask);
+          }
+        }
+      }
+      for (int64_t j = 0; j < my_tiles && go && !kPromote; ++j) {
         const int b = static_cast<int>(j & 1);
         const uint32_t use = static_cast<uint32_t>(j >> 1);
         // both CTAs' epilogues have read tile j - 2 (arrivals of both CTAs: cluster scope)
         if (!wait_bar<true>(&c.tempty[b], (use & 1u) ^ 1u, p, c, 1)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * TN);
-        for (int kb = 0; kb < T; ++kb, ++it) {
+        const int sp = split_of(j);
+        const int kb_lo = kb_begin(sp);
+        const int kb_hi = kb_begin(sp + 1);
+        for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
           const int s = static_cast<int>(it % stages);
           const uint32_t ph = static_cast<uint32_t>(it / stages) & 1u;
           if (!wait_bar(&c.full[s], ph, p, c, 2)) {
@@ -189,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = smem_desc_k_sw128(st + Shape::kABytes);
 #pragma unroll
           for (int kk = 0; kk < kTileK / kMmaK; ++kk) {
-            const uint32_t acc = (kb > 0 || kk > 0);
+            const uint32_t acc = (kb > kb_lo || kk > 0);
             if (kInt8)
               mma_i8_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, acc);
             else
@@ -198,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           issued_any = true;
           mma_commit_pair_multicast(&c.empty[s], kPairMask);
         }
+        // (a unit with no K blocks commits at once; its epilogue stores zeros)
         if (go) mma_commit_pair_multicast(&c.tfull[b], kPairMask);
       }
       trace_stamp(p, 4);
@@ -213,15 +274,108 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t tempty0 = dsmem_map(smem_addr(c.tempty), 0);   // the first CTA's tempty[0]
     bool ok = true;
-    for (int64_t j = 0; j < my_tiles; ++j) {
+    if constexpr (kPromote) {
+      // Block scale products of this thread's row, a group of kPre K blocks
+      // ahead (the loads' latency hides behind a group of promotions).
+      constexpr int kPre = 8;
+      int64_t g = 0;   // running K block over all units: buffer g mod kNBuf
+      for (int64_t j = 0; j < my_tiles; ++j) {
+        int64_t m0, n0;
+        tile_origin(j, &m0, &n0);
+        const int sp = split_of(j);
+        const int kb_lo = kb_begin(sp);
+        const int nkb = kb_begin(sp + 1) - kb_lo;
+        const int64_t m = m0 + rank * kTileM + r;
+        const int64_t nb = n0 / 128;
+        auto load_scale = [&](int i) -> float {   // 0 past the unit's blocks
+          if (i >= nkb) return 0.f;
+          const int64_t kb = kb_lo + i;
+          const float sb = __ldg(p.b_s + nb * p.KB + kb);
+          return (m < p.M ? __ldg(p.a_s + m * p.KB + kb) : 0.f) * sb;
+        };
+        float accr[TN];
+#pragma unroll
+        for (int e = 0; e < TN; ++e) accr[e] = 0.f;
+        float cur[kPre], nxt[kPre];
+#pragma unroll
+        for (int e = 0; e < kPre; ++e) cur[e] = load_scale(e);
+        for (int i0 = 0; i0 < nkb; i0 += kPre) {
+#pragma unroll
+          for (int e = 0; e < kPre; ++e) nxt[e] = load_scale(i0 + kPre + e);
+#pragma unroll
+          for (int e = 0; e < kPre; ++e) {
+            if (i0 + e < nkb) {   // the same for every epilogue thread
+              const int b = static_cast<int>(g % kNBuf);
+              const uint32_t use = static_cast<uint32_t>(g / kNBuf);
+              ++g;
+              // warp-uniform decision: the tcgen05.ld below is .sync.aligned
+              if (ok) ok = __all_sync(0xffffffffu, wait_bar(&c.tfull[b], use & 1u, p, c, 4) && !*c.abort_flag);
+              if (ok) {
+                tc_fence_after_sync();
+                const uint32_t t_buf = t_row + static_cast<uint32_t>(b * TN);
+                // two loads in flight per wait (a round trip is most of a load's cost)
+#pragma unroll
+                for (int c0 = 0; c0 < TN; c0 += 2 * CH) {
+                  uint32_t v0[CH], v1[CH];
+                  tmem_ld_32x32b_x32(t_buf + c0, v0);
+                  tmem_ld_32x32b_x32(t_buf + c0 + CH, v1);
+                  tmem_ld_wait();
+#pragma unroll
+                  for (int jj = 0; jj < CH; ++jj) {
+                    accr[c0 + jj] = fmaf(__uint_as_float(v0[jj]), cur[e], accr[c0 + jj]);
+                    accr[c0 + CH + jj] = fmaf(__uint_as_float(v1[jj]), cur[e], accr[c0 + CH + jj]);
+                  }
+                }
+                // The block's partial is in registers: the pair's MMA may refill the
+                // buffer.  The arrive publishes no memory writes, so it needs no
+                // release fence (one per block and warp cost hundreds of cycles).
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + static_cast<uint32_t>(b * 8));
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < kPre; ++e) cur[e] = nxt[e];
+        }
+        if (!ok || m >= p.M) continue;
+#pragma unroll
+        for (int j8 = 0; j8 < TN; j8 += 8) {
+          const int64_t n = n0 + j8;
+          if (n >= p.N) break;
+          if (split_mode) {   // the unit's promoted partial; the reduction adds the splits in order
+            uint4* wo = reinterpret_cast<uint4*>(static_cast<float*>(p.ws) + (sp * p.M + m) * p.N + n);
+            wo[0] = make_uint4(__float_as_uint(accr[j8 + 0]), __float_as_uint(accr[j8 + 1]),
+                               __float_as_uint(accr[j8 + 2]), __float_as_uint(accr[j8 + 3]));
+            wo[1] = make_uint4(__float_as_uint(accr[j8 + 4]), __float_as_uint(accr[j8 + 5]),
+                               __float_as_uint(accr[j8 + 6]), __float_as_uint(accr[j8 + 7]));
+          } else {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = accr[j8 + e];
+            if constexpr (BIAS) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] += bias_at(p, n + e);
+            }
+            *reinterpret_cast<uint4*>(p.C + m * p.N + n) =
+                make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                           pack_bf16x2(f[6], f[7]));
+          }
+        }
+      }
+    }
+    for (int64_t j = 0; j < my_tiles && !kPromote; ++j) {
       const int b = static_cast<int>(j & 1);
       const uint32_t use = static_cast<uint32_t>(j >> 1);
       int64_t m0, n0;
       tile_origin(j, &m0, &n0);
+      const int sp = split_of(j);
+      const bool empty_unit = kb_begin(sp + 1) == kb_begin(sp);
       float* cs = colsc + b * 256;
-      for (int col = r; col < TN; col += kEpiThreads) cs[col] = n0 + col < p.N ? __ldg(p.b_s + n0 + col) : 0.f;
+      if (!split_mode)
+        for (int col = r; col < TN; col += kEpiThreads) cs[col] = n0 + col < p.N ? __ldg(p.b_s + n0 + col) : 0.f;
       const int64_t m = m0 + rank * kTileM + r;
-      const float as_r = m < p.M ? __ldg(p.a_s + m) : 0.f;
+      const float as_r = (m < p.M && !split_mode) ? __ldg(p.a_s + m) : 0.f;
       named_barrier_sync(2, kEpiThreads);
       if (ok) ok = __all_sync(0xffffffffu, wait_bar(&c.tfull[b], use & 1u, p, c, 5) && !*c.abort_flag);
       if (!ok) continue;
@@ -230,8 +384,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c0 = 0; c0 < TN; c0 += CH) {
         uint32_t v[CH];
-        tmem_ld_32x32b_x32(t_buf + c0, v);
-        tmem_ld_wait();
+        if (!empty_unit) {
+          tmem_ld_32x32b_x32(t_buf + c0, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < CH; ++e) v[e] = 0u;   // a split with no K blocks: zero partial
+        }
         if (c0 + CH == TN) {
           // the buffer's last columns are in registers: the pair's MMA may refill it
           tc_fence_before_sync();
@@ -242,7 +401,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j8 = 0; j8 < CH; j8 += 8) {
             const int64_t n = n0 + c0 + j8;
-            if (n < p.N) {
+            if (n < p.N && split_mode) {
+              // raw accumulators (fp32 or int32 bits); the reduction scales them
+              uint4* wo = reinterpret_cast<uint4*>(static_cast<uint32_t*>(p.ws) + (sp * p.M + m) * p.N + n);
+              wo[0] = make_uint4(v[j8 + 0], v[j8 + 1], v[j8 + 2], v[j8 + 3]);
+              wo[1] = make_uint4(v[j8 + 4], v[j8 + 5], v[j8 + 6], v[j8 + 7]);
+            } else if (n < p.N) {
               float f[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
@@ -346,6 +510,9 @@ cudaError_t launch_pair(const GemmLaunch& l, int tile_n) {
       case 256: return launch_pair_tc<FMT, 256, BIAS>(l);
       default: return cudaErrorInvalidValue;
     }
+  }
+  if constexpr (FMT == kFmtBlock) {
+    if (tile_n == 128) return launch_pair_tc<FMT, 128, BIAS>(l);
   }
   return cudaErrorInvalidValue;
 }

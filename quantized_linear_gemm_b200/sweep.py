@@ -68,6 +68,9 @@ def keys_for(groups):
     return keys
 
 
+PAIRS = 74   # CTA pairs resident at once on a B200 (148 SMs)
+
+
 def candidates(fmt, M, N, K):
     T = -(-K // 128)
     out = []
@@ -100,6 +103,10 @@ def candidates(fmt, M, N, K):
                 for st in (3, 4, 6, 0):
                     for pdl in (1, 2):
                         add(swap_ab=0, tile_n=tn, split_k=S, stages=st, reduce=2, pdl=pdl)
+            if fmt == lq.BLOCK_FP8 and tn == 128:   # fp32-scale Block_FP8 on CTA pairs (256 x 128 tiles)
+                for st in (4, 6, 0):
+                    for pdl in (1, 2):
+                        add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=2)
             if fmt in (lq.FP8_DYNAMIC, lq.W8A8_INT8):   # persistent CTAs and CTA pairs (one split)
                 for st in (3, 4, 0):
                     for pdl in (1, 2):
@@ -107,6 +114,14 @@ def candidates(fmt, M, N, K):
                         if tn >= 128:
                             add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=2)
                             add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=3)
+            # CTA pairs with Split-K where the 256-row tiles alone leave pairs idle
+            pair_ok = tn == 128 if fmt == lq.BLOCK_FP8 else (tn >= 128 and fmt != lq.BLOCK_FP8_UE8M0)
+            tiles = -(-M // 256) * -(-N // tn)
+            if pair_ok and tiles < PAIRS:
+                for S in range(2, 9):
+                    if S <= T and tiles * S <= 3 * PAIRS:
+                        for st in (3, 4, 0):
+                            add(swap_ab=0, tile_n=tn, split_k=S, stages=st, reduce=0, pdl=2, persistent=2)
     return out
 
 
@@ -172,7 +187,7 @@ class Shape:
         return 1e3 * e0.elapsed_time(e1) / (replays * calls)
 
 
-def sweep(groups, device, log=sys.stderr, budget_s=None, with_quant=False, formats=None):
+def sweep(groups, device, log=sys.stderr, budget_s=None, with_quant=False, formats=None, ms=None):
     stream = torch.cuda.Stream(device=device)
     results = []
     t_start = time.time()
@@ -180,13 +195,18 @@ def sweep(groups, device, log=sys.stderr, budget_s=None, with_quant=False, forma
         fmt, M, N, K = key
         if formats is not None and fmt not in formats:
             continue
+        if ms is not None and M not in ms:
+            continue
         sh = Shape(fmt, M, N, K, device, with_quant=with_quant)
         big = sh.flops > 2e11
         best = None
         tried = 0
+        timed = []
         for v in candidates(fmt, M, N, K):
             us = sh.time_us(v, stream, calls=(4 if big else None), replays=(3 if big else 8))
             tried += 1
+            if us is not None:
+                timed.append((us, v))
             if us is not None and (best is None or us < best[0]):
                 best = (us, v)
         # re-time the winner (and the runner-up choice is implicit) to reduce noise
@@ -194,7 +214,8 @@ def sweep(groups, device, log=sys.stderr, budget_s=None, with_quant=False, forma
         gbs = sh.bytes / (us * 1e-6) / 1e9
         tf = sh.flops / (us * 1e-6) / 1e12
         rec = dict(fmt=FMT_NAMES[fmt], M=M, N=N, K=K, us=round(us, 3), gbs=round(gbs, 1), tflops=round(tf, 2),
-                   variant=best[1].as_dict(), candidates=tried)
+                   variant=best[1].as_dict(), candidates=tried,
+                   top=[dict(us=round(u, 3), variant=v.as_dict()) for u, v in sorted(timed, key=lambda x: x[0])[:5]])
         results.append(rec)
         print(json.dumps(rec), file=log, flush=True)
         del sh
@@ -274,6 +295,7 @@ def main():
     ap.add_argument("--inc-only", action="store_true", help="only regenerate the .inc from an existing table")
     ap.add_argument("--budget-s", type=float, default=None)
     ap.add_argument("--formats", default=None, help="comma-separated subset, e.g. fp8_dynamic")
+    ap.add_argument("--ms", default=None, help="comma-separated subset of M values, e.g. 256")
     ap.add_argument("--merge", default=None, metavar="TABLE",
                     help="merge the measured entries into TABLE (same key: replaced) and write the result to --out")
     ap.add_argument("--with-quant", action="store_true",
@@ -287,7 +309,8 @@ def main():
     lq.init_device(0)
     lq.load_dispatch_table(None)
     fmts = None if a.formats is None else {lq.FORMATS[f] for f in a.formats.split(",")}
-    res = sweep(set(a.configs.split(",")), device, budget_s=a.budget_s, with_quant=a.with_quant, formats=fmts)
+    ms = None if a.ms is None else {int(m) for m in a.ms.split(",")}
+    res = sweep(set(a.configs.split(",")), device, budget_s=a.budget_s, with_quant=a.with_quant, formats=fmts, ms=ms)
     if a.merge:
         tmp = a.out + ".new"
         write_table(res, tmp)

@@ -107,7 +107,7 @@ def test_empty_problem_is_a_noop():
 
 
 @pytest.mark.parametrize("field,value", [
-    ("split_k", 3), ("split_k", 512), ("split_k", 0), ("swap_ab", 2), ("tile_n", 48),
+    ("split_k", 3), ("split_k", 512), ("split_k", 0), ("split_k", -4), ("swap_ab", 2), ("tile_n", 48),
     ("stages", 1), ("stages", 15), ("reduce", 3), ("pdl", 5),
 ])
 def test_variant_checks(field, value):
@@ -118,11 +118,20 @@ def test_variant_checks(field, value):
 
 def test_persistent_variant_rules():
     """persistent = 1 (one-SM tiles), 2 (CTA pairs) and 3 (stream-K; both
-    tile_n 128 / 256) need the Standard orientation, one split and FP8 / INT8."""
+    tile_n 128 / 256) need the Standard orientation and FP8 / INT8; one
+    split, except CTA pairs, which take any split count with reduce 0."""
     for pers in (1, 2, 3):
         ok = lq.make_variant(swap_ab=0, tile_n=256, split_k=1, persistent=pers)
         assert _mm(variant=ok, C=MISALIGNED) == ALIGN    # accepted up to the pointer checks
-    for bad in (dict(swap_ab=1, tile_n=16, persistent=1), dict(swap_ab=0, tile_n=128, split_k=2, persistent=1),
+    for S in (2, 3, 5, 7, 256):
+        ok = lq.make_variant(swap_ab=0, tile_n=256, split_k=S, reduce=0, persistent=2)
+        assert _mm(variant=ok, C=MISALIGNED) == ALIGN, S
+    for bad in (dict(swap_ab=0, tile_n=256, split_k=2, reduce=1, persistent=2),
+                dict(swap_ab=0, tile_n=256, split_k=2, reduce=2, persistent=2),
+                dict(swap_ab=0, tile_n=256, split_k=257, reduce=0, persistent=2),
+                dict(swap_ab=0, tile_n=256, split_k=3, reduce=0, persistent=1),
+                dict(swap_ab=0, tile_n=256, split_k=3, reduce=0, persistent=0),
+                dict(swap_ab=1, tile_n=16, persistent=1), dict(swap_ab=0, tile_n=128, split_k=2, persistent=1),
                 dict(swap_ab=0, tile_n=128, persistent=4), dict(swap_ab=0, tile_n=256, stages=5, persistent=1),
                 dict(swap_ab=0, tile_n=64, persistent=2), dict(swap_ab=1, tile_n=32, persistent=2),
                 dict(swap_ab=0, tile_n=64, persistent=3), dict(swap_ab=0, tile_n=256, split_k=2, persistent=3)):

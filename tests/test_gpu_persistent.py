@@ -207,6 +207,164 @@ def test_pair_int8_exact_bias_and_graph(cuda_device):
     assert lq.device_status(0) == 0
 
 
+# ------------------------------------------------ CTA pairs with Split-K (persistent = 2, reduce 0)
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
+@pytest.mark.parametrize("tn", [128, 256])
+def test_pair_split_equals_one_sm_split(cuda_device, fmt, tn):
+    """Split s covers the same K blocks in both kernels and the partials are
+    summed by the same reduction, so CTA pairs with split 2 and 4 give the
+    bits of the one-SM split; ragged M, N and K (K = 1040: a short last K
+    tile); M = 1100 with split 4 has more units than pairs."""
+    for (M, N, K, S) in ((300, 1000, 1040, 2), (1100, 4096, 1024, 4)):
+        prob = make_problem(fmt, M, N, K, seed=430 + S + tn, outliers=False)
+        A, sa, B, sb = prob.device()
+        vp = lq.make_variant(swap_ab=0, tile_n=tn, split_k=S, reduce=0, persistent=2)
+        v1 = lq.make_variant(swap_ab=0, tile_n=tn, split_k=S, reduce=0)
+        Cp = lq.scaled_mm(prob.fmt, A, sa, B, sb, variant=vp)
+        C1 = lq.scaled_mm(prob.fmt, A, sa, B, sb, variant=v1)
+        torch.cuda.synchronize()
+        assert lq.device_status(0) == 0
+        assert torch.equal(Cp, C1), (M, N, K, S)
+        if M == 300:
+            assert_close(Cp, prob.reference(), f"pair split {S} tn={tn}")
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
+@pytest.mark.parametrize("S", [3, 5, 12])
+def test_pair_split_any_count_and_empty_splits(cuda_device, fmt, S):
+    """Split counts that are not powers of two, and S = 12 > T = 9 K tiles
+    (three splits own no K block and contribute zero partials): within
+    tolerance of the oracle, reproducible, and for W8A8_INT8 the exact
+    accumulators."""
+    prob = make_problem(fmt, 300, 1000, 1040, seed=440 + S)
+    A, sa, B, sb = prob.device()
+    v = lq.make_variant(swap_ab=0, tile_n=256, split_k=S, reduce=0, persistent=2)
+    C0 = lq.scaled_mm(prob.fmt, A, sa, B, sb, variant=v).clone()
+    C1 = lq.scaled_mm(prob.fmt, A, sa, B, sb, variant=v)
+    torch.cuda.synchronize()
+    assert lq.device_status(0) == 0
+    assert torch.equal(C0, C1)
+    assert_close(C0, prob.reference(), f"pair split {S}")
+    if fmt == lq.W8A8_INT8:
+        C2, acc = lq.scaled_mm_i32acc(A, sa, B, sb, variant=v)
+        torch.cuda.synchronize()
+        assert torch.equal(C2, C0)
+        assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.acc_exact(O.FMT_W8A8_INT8, prob.qa, prob.qb))
+
+
+def test_pair_split_bias_graph_and_noalloc(cuda_device):
+    """Bias through the reduction, graph replay of the two launches, and the
+    allocation-free entry point (its fixed scratch array) with the same bits."""
+    fmt = lq.FP8_DYNAMIC
+    prob = make_problem(fmt, 256, 1024, 2560, seed=450)
+    A, sa, B, sb = prob.device()
+    v = lq.make_variant(swap_ab=0, tile_n=256, split_k=3, reduce=0, persistent=2)
+    lq.reserve_workspace(0, lq.workspace_bytes(fmt, 256, 1024, 2560, v))
+    C = lq.scaled_mm(fmt, A, sa, B, sb, variant=v)
+    g = torch.Generator().manual_seed(451)
+    bias = (torch.randn(1024, generator=g) * 0.5).to(torch.bfloat16).cuda()
+    Cb = lq.scaled_mm_bias(fmt, A, sa, B, sb, bias, variant=v)
+    Cn = lq.scaled_mm_noalloc(fmt, A, sa, B, sb, variant=v)
+    torch.cuda.synchronize()
+    assert_close(C, prob.reference(), "pair split 3")
+    assert_close(Cb, prob.reference() + bias.double().cpu().numpy()[None, :], "pair split bias")
+    assert torch.equal(Cn, C)
+    out = torch.empty_like(C)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(gr, stream=s):
+            lq.scaled_mm(fmt, A, sa, B, sb, C=out, variant=v, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(2):
+        out.zero_()
+        gr.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, C)
+    del gr
+    assert lq.device_status(0) == 0
+
+
+# ------------------------------------ fp32-scale Block_FP8 on CTA pairs (persistent = 2, tile_n 128)
+def test_block_pair_equals_one_sm(cuda_device):
+    """The pair kernel promotes each 128-K block's partial with the one-SM
+    kernel's expression (fmaf of the partial and a_s * b_s, in K order), so
+    one split and split 2 (same K blocks per split, same reduction) give the
+    one-SM kernel's bits; M = 300 leaves the second CTA's rows partly past M,
+    M = 1100 gives several tiles per pair and reuses all four accumulator
+    buffers; within tolerance of the oracle."""
+    fmt = lq.BLOCK_FP8
+    for (M, N, K) in ((300, 1024, 1280), (1100, 2048, 1024)):
+        prob = make_problem(fmt, M, N, K, seed=460 + M, outliers=(M == 300))
+        A, sa, B, sb = prob.device()
+        for S in (1, 2):
+            vp = lq.make_variant(swap_ab=0, tile_n=128, split_k=S, reduce=0, persistent=2)
+            v1 = lq.make_variant(swap_ab=0, tile_n=128, split_k=S, reduce=0)
+            Cp = lq.scaled_mm(fmt, A, sa, B, sb, variant=vp)
+            C1 = lq.scaled_mm(fmt, A, sa, B, sb, variant=v1)
+            torch.cuda.synchronize()
+            assert lq.device_status(0) == 0
+            assert torch.equal(Cp, C1), (M, N, K, S)
+        if M == 300:
+            assert_close(Cp, prob.reference(), "block pair")
+        else:
+            rows = np.array([0, 127, 128, 255, 256, 700, 1023, 1024, 1099])
+            cols = np.array([0, 7, 127, 128, 1023, 2047])
+            ok, worst = O.within_tolerance(Cp.float().cpu().numpy().astype(np.float64)[np.ix_(rows, cols)],
+                                           prob.reference(rows, cols))
+            assert ok, worst
+
+
+@pytest.mark.parametrize("S", [3, 12])
+def test_block_pair_split_counts_bias_and_graph(cuda_device, S):
+    """Split 3, and split 12 over T = 10 K blocks (two empty splits): within
+    tolerance of the oracle; the bias epilogue (and bias through the
+    reduction); a graph replay gives the same bits."""
+    fmt = lq.BLOCK_FP8
+    prob = make_problem(fmt, 300, 1024, 1280, seed=470 + S)
+    A, sa, B, sb = prob.device()
+    v1 = lq.make_variant(swap_ab=0, tile_n=128, persistent=2)
+    vs = lq.make_variant(swap_ab=0, tile_n=128, split_k=S, reduce=0, persistent=2)
+    lq.reserve_workspace(0, lq.workspace_bytes(fmt, 300, 1024, 1280, vs))
+    C = lq.scaled_mm(fmt, A, sa, B, sb, variant=vs)
+    g = torch.Generator().manual_seed(471)
+    bias = (torch.randn(1024, generator=g) * 0.5).to(torch.bfloat16).cuda()
+    Cb1 = lq.scaled_mm_bias(fmt, A, sa, B, sb, bias, variant=v1)
+    Cbs = lq.scaled_mm_bias(fmt, A, sa, B, sb, bias, variant=vs)
+    torch.cuda.synchronize()
+    assert lq.device_status(0) == 0
+    assert_close(C, prob.reference(), f"block pair split {S}")
+    refb = prob.reference() + bias.double().cpu().numpy()[None, :]
+    assert_close(Cb1, refb, "block pair bias")
+    assert_close(Cbs, refb, f"block pair split {S} bias")
+    out = torch.empty_like(C)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(gr, stream=s):
+            lq.scaled_mm(fmt, A, sa, B, sb, C=out, variant=vs, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(2):
+        out.zero_()
+        gr.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, C)
+    del gr
+    assert lq.device_status(0) == 0
+
+
+def test_block_pair_refuses_other_tiles(cuda_device):
+    fmt = lq.BLOCK_FP8
+    prob = make_problem(fmt, 256, 512, 512, seed=480)
+    A, sa, B, sb = prob.device()
+    for bad in (dict(swap_ab=0, tile_n=256, persistent=2), dict(swap_ab=0, tile_n=128, persistent=1),
+                dict(swap_ab=0, tile_n=128, persistent=3)):
+        with pytest.raises(lq.LQError):
+            lq.scaled_mm(fmt, A, sa, B, sb, variant=lq.make_variant(**bad))
+
+
 # --------------------------------------------------------------- stream-K (persistent = 3)
 @pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS)
 @pytest.mark.parametrize("tn", [128, 256])
