@@ -320,18 +320,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                   tmem_ld_32x32b_x32(t_buf + c0, v0);
                   tmem_ld_32x32b_x32(t_buf + c0 + CH, v1);
                   tmem_ld_wait();
+                  if (c0 + 2 * CH == TN) {
+                    // The block's partial is in registers: the pair's MMA may refill
+                    // the buffer (before the last multiply-adds: the MMA-epilogue
+                    // hand-off per block is what bounds this kernel).  The arrive
+                    // publishes no memory writes, so it needs no release fence (one
+                    // per block and warp cost hundreds of cycles).
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + static_cast<uint32_t>(b * 8));
+                  }
 #pragma unroll
                   for (int jj = 0; jj < CH; ++jj) {
                     accr[c0 + jj] = fmaf(__uint_as_float(v0[jj]), cur[e], accr[c0 + jj]);
                     accr[c0 + CH + jj] = fmaf(__uint_as_float(v1[jj]), cur[e], accr[c0 + CH + jj]);
                   }
                 }
-                // The block's partial is in registers: the pair's MMA may refill the
-                // buffer.  The arrive publishes no memory writes, so it needs no
-                // release fence (one per block and warp cost hundreds of cycles).
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + static_cast<uint32_t>(b * 8));
               }
             }
           }
