@@ -540,6 +540,18 @@ lq_status lq_set_trace(uint64_t *device_buffer);
  */
 lq_status lq_test_inject_stall(int k_tile, uint64_t wait_limit_ns);
 
+/*
+ * Test hook for the SiLU of lq_silu_and_mul_dynamic_per_token_quant and
+ * lq_silu_and_mul_per_block_quant: out[i] = bf16(silu(gate[i])), silu(g) =
+ * g / (1 + e^-g) rounded once to bf16 from its exact value (24-ai.news
+ * report, section "vLLMに統合されたカーネル"), computed by the same device
+ * code as those kernels.  gate and out: device bf16 [n], 2-byte aligned,
+ * owned by the caller; asynchronous on `stream`.
+ * Errors: LQ_ERR_INVALID_ARG (n < 0, NULL pointer with n > 0),
+ * LQ_ERR_ALIGNMENT, LQ_ERR_CUDA.
+ */
+lq_status lq_test_silu_bf16(const void *gate, void *out, int64_t n, lq_stream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *lq_status_string(lq_status status);
 

@@ -671,6 +671,18 @@ lq_status lq_test_inject_stall(int k_tile, uint64_t wait_limit_ns) {
   return LQ_OK;
 }
 
+lq_status lq_test_silu_bf16(const void* gate, void* out, int64_t n, lq_stream_t stream) {
+  if (n < 0) return LQ_ERR_INVALID_ARG;
+  if (n == 0) return LQ_OK;
+  if (!gate || !out) return LQ_ERR_INVALID_ARG;
+  if (!aligned(gate, 2) || !aligned(out, 2)) return LQ_ERR_ALIGNMENT;
+  DeviceState* d = nullptr;
+  const lq_status ds = device_state(reinterpret_cast<cudaStream_t>(stream), &d);
+  if (ds != LQ_OK) return ds;
+  return lq::launch_silu_bf16(gate, out, n, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? LQ_OK
+                                                                                                  : LQ_ERR_CUDA;
+}
+
 int lq_declare_static_weights(int static_weights) {
   return g_static_weights.exchange(static_weights ? 1 : 0);
 }

@@ -93,6 +93,8 @@ cudaError_t launch_quant_group128(const void* x, void* q, void* scales, int64_t 
 // Producer-side fused quantizers (producer_quant.cu); rows of at most
 // producer_max_row() outputs.
 int64_t producer_max_row();
+// bf16(silu(g)) of n bf16 gates, by the producer kernels' own tiers (a test hook).
+cudaError_t launch_silu_bf16(const void* g, void* out, int64_t n, cudaStream_t stream);
 cudaError_t launch_rms_norm_quant(int fmt, bool per_block, const void* x, void* residual, const void* weight,
                                   float eps, void* q, float* scales, int64_t M, int64_t K, int* status,
                                   uint64_t wait_limit_ns, cudaStream_t stream);

@@ -45,7 +45,39 @@ __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 lo, __nv_bfloat16 
   return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
 }
 
-// silu(g) rounded once to bf16.  The fp32 estimate g / (1 + expf(-g)) has a
+// Two fp32 values rounded to bf16 (to nearest, ties to even) by one
+// conversion instruction; a in the low half.
+__device__ __forceinline__ uint32_t bf16x2_rn(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return static_cast<uint32_t>(__bfloat16_as_ushort(v.x)) | (static_cast<uint32_t>(__bfloat16_as_ushort(v.y)) << 16);
+}
+
+// silu(g) rounded once to bf16, in three tiers: each returns a bf16 value
+// and clears *ok where it cannot vouch for it; the next tier then recomputes.
+// Every finite bf16 gate is checked against the exactly rounded value on the
+// device (lq_test_silu_bf16 runs the tiers the producer kernels run).
+//
+// Tier 1, the hot loop's: e^-g = 2^(-g log2 e) with log2 e split as
+// Lh + Ll, Lh = 47274 / 2^15: g Lh is exact in fp32 (a bf16 gate has 8
+// significant bits, Lh 16), 2^(-g Lh) comes from ex2.approx, and the factor
+// 2^(-g Ll) = 1 - g Ll ln2 + ... from one fma (the next term is below
+// 2^-23.5 for |g| < 80).  The quotient uses the approximate reciprocal
+// (__fdividef).  The estimate is then within a few units of 2^-23 of the
+// exact quotient (the argument's rounding, which grows with |g| in the plain
+// ex2(g log2 e), is gone), and the Ziv test keeps its rounding unless its
+// low 16 bits lie within 16 of a bf16 midpoint.  Returns the fp32 estimate;
+// its bf16 rounding is the result where *ok.
+__device__ __forceinline__ float silu_est_ex2(float g, bool* ok) {
+  float eh;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(eh) : "f"(g * -1.44268798828125f));
+  const float e = __fmaf_rn(eh, g * -4.8884952e-6f, eh);   // times 2^(-g Ll), Ll ln2 = 4.8885e-6
+  const float s = __fdividef(g, 1.f + e);
+  const uint32_t low = __float_as_uint(s) & 0xFFFFu;
+  *ok = g > -80.f && low + 16u - 0x8000u > 32u && fabsf(s) >= 0x1p-100f;
+  return s;
+}
+
+// Tier 2.  The fp32 estimate g / (1 + expf(-g)) has a
 // relative error of at most about 2.25 * 2^-22: expf is within 2 ulp (2^-22
 // relative), the add within half an ulp, and __fdividef within 2 ulp for a
 // divisor in [2^-126, 2^126] (here 1 + e^-g lies in [1, e^80]).  That is at
@@ -77,20 +109,33 @@ __device__ __forceinline__ __nv_bfloat16 silu_bf16_f64(float g) {
   return __double2bfloat16(__ddiv_rn(gd, __dadd_rn(1.0, exp(-gd))));
 }
 
+// Tiers 2 and 3, for a gate that tier 1 could not vouch for.
+__device__ __noinline__ __nv_bfloat16 silu_bf16_slow(float g) {
+  bool ok;
+  const __nv_bfloat16 a = silu_bf16_fast(g, &ok);
+  return ok ? a : silu_bf16_f64(g);
+}
+
+// All three tiers.
+__device__ __forceinline__ __nv_bfloat16 silu_bf16(float g) {
+  bool ok;
+  const float s = silu_est_ex2(g, &ok);
+  return ok ? __float2bfloat16_rn(s) : silu_bf16_slow(g);
+}
+
+// Block reductions with one barrier: every warp reduces the per-warp values
+// itself.  An xor butterfly pairs each lane with a partner that adds the
+// same two values, so all lanes (and all warps) hold the same bits.  `red`
+// is written again only by the next row, after the next barrier of the
+// caller's row loop (one row per CTA in the one-shot kernel).
 template <int kThreads>
 __device__ __forceinline__ double block_sum_f64(double v, double* red) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) red[warp] = v;
   __syncthreads();
-  if (warp == 0) {
-    v = lane < kThreads / 32 ? red[lane] : 0.0;
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[0] = v;
-  }
-  __syncthreads();
-  const double t = red[0];
-  __syncthreads();   // red is reused by the next reduction
+  double t = lane < kThreads / 32 ? red[lane] : 0.0;
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
   return t;
 }
 
@@ -100,13 +145,9 @@ __device__ __forceinline__ float block_max_f32(float v, float* red) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) red[warp] = v;
   __syncthreads();
-  if (warp == 0) {
-    v = lane < kThreads / 32 ? red[lane] : 0.f;
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (lane == 0) red[0] = v;
-  }
-  __syncthreads();
-  return red[0];
+  float m = lane < kThreads / 32 ? red[lane] : 0.f;
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  return m;
 }
 
 enum : int { kOpRmsNorm = 0, kOpSiluMul = 1 };
@@ -144,8 +185,7 @@ __device__ __forceinline__ void quantize_row(int64_t row, const uint4* in_row, c
           uint32_t hw[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            hw[j] = pack_bf16x2(__float2bfloat16_rn(__fadd_rn(bf(xw[j], 0), bf(rw[j], 0))),
-                                __float2bfloat16_rn(__fadd_rn(bf(xw[j], 1), bf(rw[j], 1))));
+            hw[j] = bf16x2_rn(__fadd_rn(bf(xw[j], 0), bf(rw[j], 0)), __fadd_rn(bf(xw[j], 1), bf(rw[j], 1)));
           h = make_uint4(hw[0], hw[1], hw[2], hw[3]);
           res_out[idx] = h;
         }
@@ -169,13 +209,8 @@ __device__ __forceinline__ void quantize_row(int64_t row, const uint4* in_row, c
         uint32_t out[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          __nv_bfloat16 o[2];
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const __nv_bfloat16 n = __float2bfloat16_rn(__fmul_rn(bf(hw[j], k), r));
-            o[k] = __float2bfloat16_rn(__fmul_rn(__bfloat162float(n), bf(ww[j], k)));
-          }
-          out[j] = pack_bf16x2(o[0], o[1]);
+          const uint32_t n = bf16x2_rn(__fmul_rn(bf(hw[j], 0), r), __fmul_rn(bf(hw[j], 1), r));
+          out[j] = bf16x2_rn(__fmul_rn(bf(n, 0), bf(ww[j], 0)), __fmul_rn(bf(n, 1), bf(ww[j], 1)));
         }
         y[i] = make_uint4(out[0], out[1], out[2], out[3]);
       }
@@ -195,21 +230,19 @@ __device__ __forceinline__ void quantize_row(int64_t row, const uint4* in_row, c
         uint32_t out[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          __nv_bfloat16 o[2];
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            bool ok;
-            const __nv_bfloat16 a = silu_bf16_fast(bf(gw[j], k), &ok);
-            if (!ok) redo |= 1u << (8 * i + 2 * j + k);
-            o[k] = __float2bfloat16_rn(__fmul_rn(__bfloat162float(a), bf(uw[j], k)));   // exact product
-          }
-          out[j] = pack_bf16x2(o[0], o[1]);
+          bool ok0, ok1;
+          const float s0 = silu_est_ex2(bf(gw[j], 0), &ok0), s1 = silu_est_ex2(bf(gw[j], 1), &ok1);
+          if (!ok0) redo |= 1u << (8 * i + 2 * j);
+          if (!ok1) redo |= 1u << (8 * i + 2 * j + 1);
+          const uint32_t a = bf16x2_rn(s0, s1);   // the two SiLUs in bf16
+          // products of two bf16 values are exact in fp32
+          out[j] = bf16x2_rn(__fmul_rn(bf(a, 0), bf(uw[j], 0)), __fmul_rn(bf(a, 1), bf(uw[j], 1)));
         }
         y[i] = make_uint4(out[0], out[1], out[2], out[3]);
       }
     }
-    // Cold pass: the few elements whose fp32 estimate could round the wrong
-    // way are recomputed from their inputs in fp64.
+    // Cold pass: the few elements whose tier-1 estimate could round the wrong
+    // way are recomputed from their inputs by the later tiers.
     if (redo) {
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
@@ -222,7 +255,7 @@ __device__ __forceinline__ void quantize_row(int64_t row, const uint4* in_row, c
           for (int e = 0; e < 8; ++e) {
             if ((redo >> (8 * i + e)) & 1u) {
               const int j = e >> 1, k = e & 1;
-              const __nv_bfloat16 a = silu_bf16_f64(bf(gw[j], k));
+              const __nv_bfloat16 a = silu_bf16_slow(bf(gw[j], k));
               const uint32_t v =
                   __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__bfloat162float(a), bf(uw[j], k))));
               yw[j] = k ? ((yw[j] & 0x0000FFFFu) | (v << 16)) : ((yw[j] & 0xFFFF0000u) | v);
@@ -347,21 +380,28 @@ __global__ void __launch_bounds__(kRowThreads) producer_quant_staged_kernel(
     bulk_copy_g2s(dst, in + r * in_len, in_bytes, &bar[b]);
     if (residual) bulk_copy_g2s(dst + in_bytes, residual + r * Kout, static_cast<uint32_t>(Kout * 2), &bar[b]);
   };
+  // Rows it and it + 1 are in flight while row it is worked on: both
+  // buffers are filled up front, and the copy of row it + 1 into buffer
+  // (it + 1) & 1 is issued once every thread has passed iteration it's
+  // barrier, i.e. has left iteration it - 1, the last reader of that buffer.
   if (threadIdx.x == 0 && blockIdx.x < M) issue(blockIdx.x, 0);
+  if (threadIdx.x == 0 && blockIdx.x + gridDim.x < M) issue(blockIdx.x + gridDim.x, 1);
   int it = 0;
+  int issued = 2;   // copies issued (for the drain after a timeout)
   bool failed = false;
   for (int64_t row = blockIdx.x; row < M; row += gridDim.x, ++it) {
     const int b = it & 1;
-    if (threadIdx.x == 0 && row + gridDim.x < M) {
-      // buffer b ^ 1 was last read in the previous iteration, which every
-      // thread has left (barrier at its end)
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue(row + gridDim.x, b ^ 1);
-    }
     const bool landed = mbar_wait(&bar[b], static_cast<uint32_t>(it >> 1) & 1u, wait_limit_ns);
     if (!__syncthreads_and(landed)) {
       failed = true;
       break;
+    }
+    if (it > 0) {
+      if (threadIdx.x == 0 && row + gridDim.x < M) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue(row + gridDim.x, b ^ 1);
+      }
+      issued = it + 2;
     }
     const uint8_t* buf = rows + static_cast<size_t>(b) * row_bytes;
     uint4* rout = residual ? reinterpret_cast<uint4*>(residual + row * Kout) : nullptr;
@@ -369,13 +409,11 @@ __global__ void __launch_bounds__(kRowThreads) producer_quant_staged_kernel(
         row, reinterpret_cast<const uint4*>(buf),
         residual ? reinterpret_cast<const uint4*>(buf + in_bytes) : nullptr, rout, wv, eps, q, scales, Kout, red_d,
         red_f);
-    __syncthreads();   // buffer b is free for the copy issued next iteration
   }
   if (failed && threadIdx.x == 0) {
     if (status) atomicOr(status, 1 << 12);
     // wait (bounded) for the copies this CTA may still have in flight
-    for (int k = 0; k < 2; ++k) {
-      const int jt = it + k;
+    for (int jt = it; jt < issued; ++jt) {
       const int64_t r = blockIdx.x + static_cast<int64_t>(jt) * gridDim.x;
       if (r < M) mbar_wait(&bar[jt & 1], static_cast<uint32_t>(jt >> 1) & 1u, wait_limit_ns);
     }
@@ -477,9 +515,25 @@ cudaError_t launch_rows(const void* in, void* residual, const void* weight, floa
   return cudaErrorInvalidValue;
 }
 
+// The SiLU of the producer kernels, element by element (a test hook).
+__global__ void __launch_bounds__(256) silu_bf16_kernel(const __nv_bfloat16* __restrict__ g,
+                                                        __nv_bfloat16* __restrict__ out, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = silu_bf16(__bfloat162float(g[i]));
+}
+
 }  // namespace
 
 int64_t producer_max_row() { return kMaxRow; }
+
+cudaError_t launch_silu_bf16(const void* g, void* out, int64_t n, cudaStream_t stream) {
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  silu_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(g),
+                                                                       static_cast<__nv_bfloat16*>(out), n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_rms_norm_quant(int fmt, bool per_block, const void* x, void* residual, const void* weight,
                                   float eps, void* q, float* scales, int64_t M, int64_t K, int* status,

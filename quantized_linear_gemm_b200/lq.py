@@ -37,6 +37,7 @@ EXPORTED = (
     "lq_quant_weight_block128", "lq_select_variant", "lq_load_dispatch_table", "lq_dispatch_table_size",
     "lq_init_device", "lq_reserve_workspace", "lq_workspace_bytes", "lq_device_status",
     "lq_status_string", "lq_version", "lq_set_trace", "lq_scaled_mm_noalloc", "lq_test_inject_stall",
+    "lq_test_silu_bf16",
     "lq_quant_scaled_mm", "lq_set_fuse_limit", "lq_rms_norm_dynamic_per_token_quant",
     "lq_rms_norm_per_block_quant", "lq_silu_and_mul_dynamic_per_token_quant", "lq_silu_and_mul_per_block_quant",
     "lq_grouped_scaled_mm", "lq_quant_per_token_group128_ue8m0", "lq_quant_weight_block128_ue8m0",
@@ -107,6 +108,8 @@ def lib() -> ctypes.CDLL:
             L.lq_status_string.restype = ctypes.c_char_p
             L.lq_test_inject_stall.argtypes = [_i32, ctypes.c_uint64]
             L.lq_test_inject_stall.restype = _i32
+            L.lq_test_silu_bf16.argtypes = [_vp, _vp, _i64, _vp]
+            L.lq_test_silu_bf16.restype = _i32
             L.lq_set_trace.argtypes = [_vp]
             L.lq_set_trace.restype = _i32
             L.lq_declare_static_weights.argtypes = [_i32]
@@ -532,6 +535,15 @@ def test_inject_stall(k_tile: int, wait_limit_ns: int = 0) -> None:
     """Test hook: leave K tile `k_tile` of every CTA unloaded so that a bounded
     wait runs out (-1 = off); `wait_limit_ns` > 0 shortens every wait."""
     _check("lq_test_inject_stall", lib().lq_test_inject_stall(int(k_tile), int(wait_limit_ns)))
+
+
+def test_silu_bf16(gate: torch.Tensor, stream=None) -> torch.Tensor:
+    """Test hook: bf16(silu(gate)) by the producer kernels' own device code."""
+    if gate.dtype != torch.bfloat16 or not gate.is_cuda or not gate.is_contiguous():
+        raise ValueError("gate must be a contiguous bf16 CUDA tensor")
+    out = torch.empty_like(gate)
+    _check("lq_test_silu_bf16", lib().lq_test_silu_bf16(_ptr(gate), _ptr(out), gate.numel(), _stream(stream)))
+    return out
 
 
 def status_string(code: int) -> str:

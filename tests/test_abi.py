@@ -247,6 +247,14 @@ def test_stall_hook_argument_check():
     assert lq.lib().lq_test_inject_stall(-1, 0) == OK
 
 
+def test_silu_hook_argument_check():
+    f = lq.lib().lq_test_silu_bf16
+    assert f(FAKE, FAKE, -1, None) == INVALID
+    assert f(None, None, 0, None) == OK
+    assert f(None, FAKE, 8, None) == INVALID
+    assert f(FAKE + 1, FAKE, 8, None) == ALIGN
+
+
 def test_i32acc_needs_an_output():
     L = lq.lib()
     assert L.lq_scaled_mm_i32acc(FAKE, FAKE, FAKE, FAKE, FAKE, None, 4, 128, 128, None, None) == INVALID

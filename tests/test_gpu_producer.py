@@ -122,6 +122,27 @@ def test_silu_rounding_paths(cuda_device):
         assert np.array_equal(q.cpu().numpy(), q_ref), uval
 
 
+def test_silu_bf16_every_gate(cuda_device):
+    """The producer kernels' SiLU (all of its tiers, through the test hook)
+    on every finite bf16 gate: bf16(silu(g)) bit for bit equal to the
+    oracle's value rounded once from the exact quotient.  Codes can hide a
+    wrong last bit of the SiLU; this compares the SiLU itself."""
+    bits = torch.arange(1 << 16, dtype=torch.int32)
+    g = (bits << 16).view(torch.float32)
+    g = g[torch.isfinite(g)].to(torch.bfloat16)
+    out = lq.test_silu_bf16(g.cuda())
+    torch.cuda.synchronize()
+    ref = P.silu_bf16(g.double().numpy())
+    got = out.double().cpu().numpy()
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert same.all(), (g[~torch.from_numpy(same)][:8], got[~same][:8], ref[~same][:8])
+    # the same gates again in another order (the kernel's grid-stride loop splits them differently)
+    perm = torch.randperm(g.numel(), generator=torch.Generator().manual_seed(7))
+    out2 = lq.test_silu_bf16(g[perm].contiguous().cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(out2.cpu(), out.cpu()[perm])
+
+
 def test_silu_ties_of_tiny_gates(cuda_device):
     """Gates 0 < |g| < 2^-125 where g / 2 lies halfway between two bf16
     values (odd multiples of 2^-133, both signs), alone in a row so that the
