@@ -95,7 +95,7 @@ typedef enum {
  *            1 = Swap-AB: C^T = B . A^T is computed, 128 weight rows on the M
  *            side and tile_n tokens on the N side; the epilogue transposes
  *            back on store.
- *  split_k : 1, 2, 4, ..., 256 (CTA pairs with reduce 0: any of 1..256).
+ *  split_k : 1..256; a power of two with reduce 2.
  *            Split s owns the 128-wide K tiles
  *            [floor(s*T/S), floor((s+1)*T/S)), T = ceil(K/128); a split may
  *            be empty.  Partials are summed in the fixed order s = 0..S-1,

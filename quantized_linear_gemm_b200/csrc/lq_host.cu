@@ -414,8 +414,9 @@ dim3 pair_grid(int fmt, int64_t M, int64_t gy, int split_k, int tile_n, bool bia
 lq_status check_variant(int fmt, const lq_variant& v) {
   if (v.swap_ab != 0 && v.swap_ab != 1) return LQ_ERR_INVALID_ARG;
   if (v.split_k < 1 || v.split_k > 256) return LQ_ERR_INVALID_ARG;
-  // any split count for CTA pairs with the separate reduction; powers of two elsewhere
-  if (!is_pow2(v.split_k) && !(v.persistent == 2 && v.reduce == 0)) return LQ_ERR_INVALID_ARG;
+  // the cluster reduction gives each CTA tile_n / split_k columns: powers of two; the
+  // workspace reductions take any split count
+  if (!is_pow2(v.split_k) && v.reduce == 2) return LQ_ERR_INVALID_ARG;
   if (v.reduce < 0 || v.reduce > 2) return LQ_ERR_INVALID_ARG;
   if (v.reduce == 2 && v.split_k > 16) return LQ_ERR_INVALID_ARG;   // a cluster holds at most 16 CTAs
   if (v.pdl < 0 || v.pdl > 2) return LQ_ERR_INVALID_ARG;

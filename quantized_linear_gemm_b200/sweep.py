@@ -79,7 +79,7 @@ def candidates(fmt, M, N, K):
         out.append(lq.make_variant(**kw))
 
     if M <= 64:
-        tns = [tn for tn in (16, 32, 64) if tn >= M][:2] or [64]
+        tns = [16, 32] if M <= 32 else [32, 64]   # M = 24, 32 also as two 16-token tiles
         for tn in tns:
             for S in (1, 2, 4, 8, 16):
                 if S > T:
@@ -94,6 +94,12 @@ def candidates(fmt, M, N, K):
                 if S <= T // 2:
                     add(swap_ab=1, tile_n=tn, split_k=S, stages=2, reduce=1, pdl=2)
                     add(swap_ab=1, tile_n=tn, split_k=S, stages=2, reduce=0, pdl=2)
+            for S in (3, 5, 6):   # split counts that fill the SMs where powers of two leave a partial wave
+                if S <= T:
+                    per = -(-T // S)
+                    for st in sorted({min(per, 3), min(per, 4), min(per, 6)}):
+                        if st >= 2:
+                            add(swap_ab=1, tile_n=tn, split_k=S, stages=st, reduce=1, pdl=2)
     if M >= 16:
         tns = (64, 128) if fmt == lq.BLOCK_FP8 else (64, 128, 256)   # fp32-scale Block_FP8: up to 128
         for tn in tns:
@@ -103,6 +109,11 @@ def candidates(fmt, M, N, K):
                 for st in (3, 4, 6, 0):
                     for pdl in (1, 2):
                         add(swap_ab=0, tile_n=tn, split_k=S, stages=st, reduce=2, pdl=pdl)
+            if -(-M // 128) * -(-N // tn) < 148:   # few tiles: split counts between the powers of two
+                for S in (3, 5, 6, 7):
+                    if S <= T:
+                        for st in (3, 4, 0):
+                            add(swap_ab=0, tile_n=tn, split_k=S, stages=st, reduce=1, pdl=2)
             if fmt == lq.BLOCK_FP8 and tn == 128:   # fp32-scale Block_FP8 on CTA pairs (256 x 128 tiles)
                 for st in (4, 6, 0):
                     for pdl in (1, 2):

@@ -95,7 +95,7 @@ def test_default_variant_waits_before_reading_weights():
 def test_quant_scaled_mm_checks_the_variant_before_launching():
     """The two-kernel path checks the caller's variant before it launches the
     quantization kernel: an invalid one launches nothing."""
-    v = lq.make_variant(swap_ab=1, split_k=3, tile_n=16)
+    v = lq.make_variant(swap_ab=1, split_k=3, tile_n=16, reduce=2)   # split 3: not with the cluster reduction
     assert lq.lib().lq_quant_scaled_mm(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 128, 1024,
                                        ctypes.byref(v), None) == INVALID
 
@@ -107,13 +107,24 @@ def test_empty_problem_is_a_noop():
 
 
 @pytest.mark.parametrize("field,value", [
-    ("split_k", 3), ("split_k", 512), ("split_k", 0), ("split_k", -4), ("swap_ab", 2), ("tile_n", 48),
-    ("stages", 1), ("stages", 15), ("reduce", 3), ("pdl", 5),
+    ("split_k", 3), ("split_k", 512), ("split_k", 257), ("split_k", 0), ("split_k", -4), ("swap_ab", 2),
+    ("tile_n", 48), ("stages", 1), ("stages", 15), ("reduce", 3), ("pdl", 5),
 ])
 def test_variant_checks(field, value):
-    v = lq.make_variant(swap_ab=1, split_k=2, tile_n=32)
+    v = lq.make_variant(swap_ab=1, split_k=2, tile_n=32, reduce=2)   # split 3: not with the cluster reduction
     setattr(v, field, value)
     assert _mm(variant=v) == INVALID
+
+
+def test_split_counts_by_reduction():
+    """Any split count 1..256 with the workspace reductions (0, 1); powers of
+    two (at most 16) with the cluster reduction."""
+    for S in (3, 5, 7, 12, 100, 256):
+        for reduce in (0, 1):
+            for sw, tn in ((1, 16), (0, 128)):
+                v = lq.make_variant(swap_ab=sw, split_k=S, tile_n=tn, reduce=reduce)
+                assert _mm(variant=v, C=MISALIGNED) == ALIGN, (S, reduce, sw)
+        assert _mm(variant=lq.make_variant(swap_ab=1, split_k=S, tile_n=16, reduce=2)) == INVALID, S
 
 
 def test_persistent_variant_rules():
@@ -130,7 +141,7 @@ def test_persistent_variant_rules():
                 dict(swap_ab=0, tile_n=256, split_k=2, reduce=2, persistent=2),
                 dict(swap_ab=0, tile_n=256, split_k=257, reduce=0, persistent=2),
                 dict(swap_ab=0, tile_n=256, split_k=3, reduce=0, persistent=1),
-                dict(swap_ab=0, tile_n=256, split_k=3, reduce=0, persistent=0),
+                dict(swap_ab=0, tile_n=256, split_k=3, reduce=2, persistent=0),
                 dict(swap_ab=1, tile_n=16, persistent=1), dict(swap_ab=0, tile_n=128, split_k=2, persistent=1),
                 dict(swap_ab=0, tile_n=128, persistent=4), dict(swap_ab=0, tile_n=256, stages=5, persistent=1),
                 dict(swap_ab=0, tile_n=64, persistent=2), dict(swap_ab=1, tile_n=32, persistent=2),
@@ -303,7 +314,7 @@ def test_dispatch_table_file(tmp_path):
         # workspace need follows the selected variant
         assert lq.workspace_bytes("fp8_dynamic", 5, 4096, 4096) == 8 * 5 * 4096 * 4
         bad = tmp_path / "bad.txt"
-        bad.write_text("fp8_dynamic 8 4096 4096 1 3 16 4 0 1\n")   # split_k 3 is not a power of two
+        bad.write_text("fp8_dynamic 8 4096 4096 1 3 16 4 2 1\n")   # split_k 3 with the cluster reduction
         with pytest.raises(lq.LQError) as e:
             lq.load_dispatch_table(str(bad))
         assert e.value.code == TABLE

@@ -91,6 +91,34 @@ def test_split_k_with_empty_splits(cuda_device, S):
             assert_close(_run(prob, v), prob.reference(), f"S={S} reduce={reduce} fmt={fmt}")
 
 
+@pytest.mark.parametrize("fmt", [lq.FP8_DYNAMIC, lq.W8A8_INT8, lq.BLOCK_FP8, lq.BLOCK_FP8_UE8M0],
+                         ids=["fp8", "int8", "block", "ue8m0"])
+@pytest.mark.parametrize("swap,tn", [(1, 16), (1, 32), (0, 128)])
+def test_split_counts_not_powers_of_two(cuda_device, fmt, swap, tn):
+    """Split counts 3, 5, 7 and 12 (K = 2304: 18 K tiles, splits of one to
+    six tiles) with the separate reduction and with the last arriver: the
+    same partials summed in the same order, so identical bits; within
+    tolerance of the oracle; W8A8_INT8 accumulators exact."""
+    M, N, K = (40, 512, 2304) if swap else (200, 512, 2304)
+    prob = make_problem(fmt, M, N, K, seed=16 + tn)
+    A, sa, B, sb = prob.device()
+    ref = prob.reference()
+    for S in (3, 5, 7, 12):
+        outs = []
+        for red in (0, 1):
+            v = lq.make_variant(swap_ab=swap, tile_n=tn, split_k=S, stages=2, reduce=red)
+            lq.reserve_workspace(0, lq.workspace_bytes(fmt, M, N, K, v))
+            outs.append(lq.scaled_mm(fmt, A, sa, B, sb, variant=v).clone())
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0], outs[1]), f"S={S}"
+        assert_close(outs[0], ref, f"S={S}")
+        if fmt == lq.W8A8_INT8:
+            _, acc = lq.scaled_mm_i32acc(A, sa, B, sb, variant=v)
+            torch.cuda.synchronize()
+            assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.acc_exact(O.FMT_W8A8_INT8, prob.qa, prob.qb))
+    assert lq.device_status(0) == 0
+
+
 def test_config0_fp8_standard(cuda_device):
     """FP8_Dynamic, M = 16, N = K = 2048, A ~ N(0,1), B ~ N(0,0.02), Standard."""
     x = inputs.activations(16, 2048, seed=0, outliers=False).float().numpy()
