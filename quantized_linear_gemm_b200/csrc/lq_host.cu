@@ -324,7 +324,7 @@ int pair_capacity(int fmt, int tile_n, bool bias, int smem_bytes) {
   const int n = fmt == lq::kFmtFp8    ? lq::pair_capacity_fp8(tile_n, bias, smem_bytes)
                 : fmt == lq::kFmtInt8  ? lq::pair_capacity_int8(tile_n, bias, smem_bytes)
                 : fmt == lq::kFmtBlock ? lq::pair_capacity_block(tile_n, bias, smem_bytes)
-                                       : 0;
+                                       : lq::pair_capacity_block_e8m0(tile_n, bias, smem_bytes);
   cache.emplace_back(key, n);
   return n;
 }
@@ -397,7 +397,7 @@ bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
 // never wait for each other's columns.
 int pair_launch_smem(int fmt, int tile_n, int stages) {
   const int bytes = lq::pair_smem_bytes_for(tile_n, stages);
-  const bool all_columns = tile_n == 256 || fmt == lq::kFmtBlock;
+  const bool all_columns = tile_n == 256 || lq::is_block_fmt(fmt);
   return all_columns && bytes < 116 * 1024 ? 116 * 1024 : bytes;
 }
 
@@ -430,9 +430,9 @@ lq_status check_variant(int fmt, const lq_variant& v) {
   if (v.persistent < 0 || v.persistent > 3) return LQ_ERR_INVALID_ARG;
   if (v.persistent) {
     // Standard orientation, FP8_Dynamic / W8A8_INT8 (CTA pairs and stream-K: tile_n 128 or 256), and
-    // fp32-scale Block_FP8 on CTA pairs with tile_n 128; one split, except CTA pairs, which take Split-K
-    // with the separate reduction
-    const bool block_pair = fmt == lq::kFmtBlock && v.persistent == 2 && v.tile_n == 128;
+    // Block_FP8 (fp32 or UE8M0 scales) on CTA pairs with tile_n 128; one split, except CTA pairs, which
+    // take Split-K with the separate reduction
+    const bool block_pair = (fmt == lq::kFmtBlock || fmt == lq::kFmtBlockE8m0) && v.persistent == 2 && v.tile_n == 128;
     if (v.swap_ab || (fmt != lq::kFmtFp8 && fmt != lq::kFmtInt8 && !block_pair)) return LQ_ERR_INVALID_ARG;
     if (v.split_k != 1 && !(v.persistent == 2 && v.reduce == 0)) return LQ_ERR_INVALID_ARG;
     if (v.persistent >= 2 && v.tile_n == 64) return LQ_ERR_INVALID_ARG;

@@ -83,7 +83,8 @@ int pair_smem_bytes_for(int tile_n, int stages);
 // Largest number of co-resident CTA pairs of the pair kernel (0 if unknown).
 int pair_capacity_fp8(int tile_n, bool bias, int smem_bytes);
 int pair_capacity_int8(int tile_n, bool bias, int smem_bytes);
-int pair_capacity_block(int tile_n, bool bias, int smem_bytes);   // tile_n 128
+int pair_capacity_block(int tile_n, bool bias, int smem_bytes);        // tile_n 128
+int pair_capacity_block_e8m0(int tile_n, bool bias, int smem_bytes);   // tile_n 128
 
 // Quantization kernels (quant_kernels.cu).
 cudaError_t launch_quant_per_token(int fmt, const void* x, void* q, float* scales, int64_t M, int64_t K,

@@ -116,7 +116,7 @@ int pair_capacity(int tile_n, bool bias, int smem_bytes) {
       default: return 0;
     }
   }
-  if constexpr (FMT == kFmtBlock) {
+  if constexpr (FMT == kFmtBlock || FMT == kFmtBlockE8m0) {
     if (tile_n == 128) return bias ? max_pairs<FMT, 128, true>(smem_bytes) : max_pairs<FMT, 128, false>(smem_bytes);
   }
   return 0;

@@ -1,6 +1,7 @@
 // Persistent scaled_mm on CTA pairs (tcgen05 cta_group::2) for large M:
-// Standard orientation, FP8_Dynamic, W8A8_INT8 and Block_FP8 with fp32
-// scales, one split or Split-K with the separate fixed-order reduction.
+// Standard orientation, FP8_Dynamic, W8A8_INT8, Block_FP8 with fp32 scales
+// and Block_FP8 with UE8M0 scales, one split or Split-K with the separate
+// fixed-order reduction.
 //
 // A cluster of two CTAs (two SMs) computes 256 x TN output tiles with one
 // MMA of M = 256: each CTA loads its own 128 rows of A and half (TN / 2 rows)
@@ -24,7 +25,19 @@
 // it, times a_s[m, kb] * b_s[n / 128, kb], into fp32 registers (fmaf in K
 // order, as the one-SM kernel does: the same bits).  Per SM a 128-K block
 // then moves 24 KB of operands from L2 instead of the one-SM 128 x 128
-// tile's 32 KB, which is what bounds that tile.  Synchronisation:
+// tile's 32 KB, which is what bounds that tile.
+//
+// Block_FP8 with UE8M0 scales (256 x 128 tiles): the tensor core's block
+// scaling (tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale), one
+// accumulator per tile as for FP8.  Each CTA's tensor memory holds, at the
+// same addresses, the scale factors of its own 128 rows of A and of all 128
+// rows of B, in four slots of four K blocks each (row e at lane e mod 32,
+// column e / 32, the same in all four lane quarters; block t of a group in
+// bits [8t, 8t + 8)).  Four more warps per CTA fill the slots, so that the
+// epilogue warps, busy with the previous tile, never hold up the MMA:
+//   xfull[g]  first CTA only: slot g written by both CTAs' scale warps;
+//   wfull[g]  both CTAs: slot g read by the tensor core (commit multicast).
+// Synchronisation:
 //   full[s]   first CTA only: both CTAs' TMA loads of slot s count their
 //             bytes here (the first CTA announces the pair's total);
 //   empty[s]  both CTAs: slot s read by the tensor core (commit multicast);
@@ -56,18 +69,30 @@ __host__ __device__ constexpr int pair_smem_bytes(int stages) {
   return 1024 + stages * PairShape<TN>::kStageBytes + kCtlBytes + kPersistentScaleBytes;
 }
 
+// Threads of a pair CTA: producer, MMA and four epilogue warps, and for the
+// UE8M0 format four scale-factor warps.
+__host__ __device__ constexpr int pair_threads(int fmt) { return fmt == kFmtBlockE8m0 ? kThreads + 128 : kThreads; }
+
+constexpr int kPairSfSlots = 4;
+
 template <int FMT, int TN, bool BIAS>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(pair_threads(FMT), 1)
     scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const GemmParams p) {
-  static_assert(FMT == kFmtFp8 || FMT == kFmtInt8 || FMT == kFmtBlock, "pair kernel: FP8, INT8, Block_FP8");
+  static_assert(FMT == kFmtFp8 || FMT == kFmtInt8 || FMT == kFmtBlock || FMT == kFmtBlockE8m0,
+                "pair kernel: FP8, INT8, Block_FP8 (fp32 or UE8M0 scales)");
   static_assert(TN == 128 || TN == 256, "pair tiles: 256 x 128 or 256 x 256");
   constexpr bool kPromote = FMT == kFmtBlock;
+  constexpr bool kMX = FMT == kFmtBlockE8m0;
   static_assert(!kPromote || TN == 128, "Block_FP8 pairs: 256 x 128 tiles (TN fp32 accumulators per thread)");
+  static_assert(!kMX || TN == 128, "UE8M0 pairs: 256 x 128 tiles (two accumulators and the scale factors)");
   using Shape = PairShape<TN>;
   constexpr bool kInt8 = FMT == kFmtInt8;
   constexpr int kNBuf = kPromote ? 4 : 2;     // tensor-memory accumulator buffers
-  constexpr int kTmemCols = kNBuf * TN;
+  constexpr int kSfBase = kNBuf * TN;         // UE8M0: scale-factor slots after the accumulators
+  constexpr int kSfSlotCols = 8;              // A: 4 columns (128 rows), B: 4 columns (TN = 128 rows)
+  constexpr int kTmemCols = kMX ? 512 : kNBuf * TN;
+  static_assert(!kMX || kSfBase + kPairSfSlots * kSfSlotCols <= kTmemCols, "tensor memory");
   constexpr int CH = 32;
   constexpr uint16_t kPairMask = 0x3;
 
@@ -82,7 +107,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   c.tfull = bars + 2 * stages;
   c.tempty = c.tfull + kNBuf;
   c.mma_done = c.tempty + kNBuf;
-  c.tmem_slot = reinterpret_cast<uint32_t*>(c.mma_done + 1);
+  c.xfull = c.mma_done + 1;              // UE8M0 scale-factor slots (unused otherwise)
+  c.wfull = c.xfull + kPairSfSlots;
+  c.tmem_slot = reinterpret_cast<uint32_t*>(c.wfull + kPairSfSlots);
   c.abort_flag = reinterpret_cast<volatile int*>(c.tmem_slot + 1);
   c.last_flag = c.abort_flag + 1;
   float* colsc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kCtlBytes);   // [2][256]
@@ -120,6 +147,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&c.tempty[b], 2 * kEpiThreads / 32);
     }
     mbar_init(c.mma_done, 1);
+    for (int g = 0; g < kPairSfSlots; ++g) {
+      mbar_init(&c.xfull[g], 8);   // four scale warps in each CTA
+      mbar_init(&c.wfull[g], 1);
+    }
     *c.abort_flag = 0;
     *c.last_flag = 0;
     fence_barrier_init();
@@ -189,6 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------ MMA issuer (first CTA)
     if (leader && lane == 0) {
       constexpr uint32_t idesc = make_idesc<kInt8>(kPairTileM, TN);
+      constexpr uint32_t idesc_mx = make_idesc_mx(kPairTileM, TN);
       bool issued_any = false;
       bool go = true;
       int64_t it = 0;
@@ -225,6 +257,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // UE8M0: the scale-factor slot of the current group of four K blocks
+      // (groups start at each unit's first block), its use count, its address
+      int64_t sf_group = -1;
+      uint32_t sf_addr = tmem_base + static_cast<uint32_t>(kSfBase);
+      int sf_slot = 0;
       for (int64_t j = 0; j < my_tiles && go && !kPromote; ++j) {
         const int b = static_cast<int>(j & 1);
         const uint32_t use = static_cast<uint32_t>(j >> 1);
@@ -236,6 +273,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kb_lo = kb_begin(sp);
         const int kb_hi = kb_begin(sp + 1);
         for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
+          if (kMX && ((kb - kb_lo) & 3) == 0) {   // both CTAs' scale factors of blocks kb .. kb+3
+            ++sf_group;
+            sf_slot = static_cast<int>(sf_group % kPairSfSlots);
+            sf_addr = tmem_base + static_cast<uint32_t>(kSfBase + sf_slot * kSfSlotCols);
+            const uint32_t sf_ph = static_cast<uint32_t>(sf_group / kPairSfSlots) & 1u;
+            if (!wait_bar<true>(&c.xfull[sf_slot], sf_ph, p, c, 13)) {
+              go = false;
+              break;
+            }
+          }
           const int s = static_cast<int>(it % stages);
           const uint32_t ph = static_cast<uint32_t>(it / stages) & 1u;
           if (!wait_bar(&c.full[s], ph, p, c, 2)) {
@@ -250,13 +297,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kTileK / kMmaK; ++kk) {
             const uint32_t acc = (kb > kb_lo || kk > 0);
-            if (kInt8)
+            if constexpr (kMX) {
+              const uint32_t t = static_cast<uint32_t>((kb - kb_lo) & 3);   // this block's byte in the slot
+              mma_mxf8f6f4_block_scale_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc_with_sf_ids(idesc_mx, t, t),
+                                            sf_addr, sf_addr + 4, acc);
+            } else if (kInt8) {
               mma_i8_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, acc);
-            else
+            } else {
               mma_f8f6f4_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+            }
           }
           issued_any = true;
           mma_commit_pair_multicast(&c.empty[s], kPairMask);
+          if (kMX && (((kb - kb_lo) & 3) == 3 || kb + 1 == kb_hi))
+            mma_commit_pair_multicast(&c.wfull[sf_slot], kPairMask);   // the slot is read
         }
         // (a unit with no K blocks commits at once; its epilogue stores zeros)
         if (go) mma_commit_pair_multicast(&c.tfull[b], kPairMask);
@@ -266,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // arrives once every MMA issued so far has finished (at once if none was)
       if (my_tiles > 0) mma_commit_pair_multicast(c.mma_done, kPairMask);
     }
-  } else {
+  } else if (warp < kThreads / 32) {
     // ------------------------------------------------------------ epilogue
     grid_dependency_wait();   // the scales may come from the previous kernel
     const int q = warp & 3;
@@ -376,10 +430,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int sp = split_of(j);
       const bool empty_unit = kb_begin(sp + 1) == kb_begin(sp);
       float* cs = colsc + b * 256;
-      if (!split_mode)
+      // (UE8M0: the accumulator carries its scales, and the scale arrays hold bytes)
+      if (!split_mode && !kMX)
         for (int col = r; col < TN; col += kEpiThreads) cs[col] = n0 + col < p.N ? __ldg(p.b_s + n0 + col) : 0.f;
       const int64_t m = m0 + rank * kTileM + r;
-      const float as_r = (m < p.M && !split_mode) ? __ldg(p.a_s + m) : 0.f;
+      const float as_r = (m < p.M && !split_mode && !kMX) ? __ldg(p.a_s + m) : 0.f;
       named_barrier_sync(2, kEpiThreads);
       if (ok) ok = __all_sync(0xffffffffu, wait_bar(&c.tfull[b], use & 1u, p, c, 5) && !*c.abort_flag);
       if (!ok) continue;
@@ -415,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 const float a = kInt8 ? static_cast<float>(static_cast<int32_t>(v[j8 + e])) : __uint_as_float(v[j8 + e]);
-                f[e] = a * as_r * cs[c0 + j8 + e];
+                f[e] = kMX ? a : a * as_r * cs[c0 + j8 + e];
               }
               if constexpr (BIAS) {
 #pragma unroll
@@ -435,6 +490,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (warp == 2 && lane == 0) trace_stamp(p, 6);
+  } else if constexpr (kMX) {
+    // --------------------------------------------- UE8M0 scale-factor warps
+    // Per group of four K blocks of each unit (the MMA warp's grouping):
+    // wait until the slot's previous group has been read (wfull, from the
+    // pair's commits), write the UE8M0 bytes of this CTA's 128 A rows and of
+    // the tile's 128 B rows to this warp's lane quarter of the slot, and
+    // arrive on the first CTA's xfull (release: the tensor-memory stores,
+    // complete after tcgen05.wait::st, come before the MMA that reads them).
+    grid_dependency_wait();   // the scales may come from the previous kernel
+    const int q = warp & 3;   // warps 6..9: lane quarters 2, 3, 0, 1
+    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t xfull0 = dsmem_map(smem_addr(c.xfull), 0);   // the first CTA's xfull[0]
+    const uint8_t* a_b = reinterpret_cast<const uint8_t*>(p.a_s);   // [M, KB]
+    const uint8_t* b_b = reinterpret_cast<const uint8_t*>(p.b_s);   // [N / 128, KB]
+    bool ok = true;
+    int64_t group = -1;
+    for (int64_t j = 0; j < my_tiles && ok; ++j) {
+      int64_t m0, n0;
+      tile_origin(j, &m0, &n0);
+      const int sp = split_of(j);
+      const int kb_hi = kb_begin(sp + 1);
+      for (int kb0 = kb_begin(sp); kb0 < kb_hi; kb0 += 4) {
+        ++group;
+        const int slot = static_cast<int>(group % kPairSfSlots);
+        if (group >= kPairSfSlots) {
+          const uint32_t ph = static_cast<uint32_t>(group / kPairSfSlots - 1) & 1u;
+          ok = __all_sync(0xffffffffu, wait_bar(&c.wfull[slot], ph, p, c, 14) && !*c.abort_flag);
+          if (!ok) break;
+        }
+        uint32_t wa[4], wb[4];
+#pragma unroll
+        for (int col = 0; col < 4; ++col) {
+          const int64_t m = m0 + rank * kTileM + col * 32 + lane;
+          const int64_t n = n0 + col * 32 + lane;
+          uint32_t xa = 0, xb = 0;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int kb = kb0 + t;   // past the unit's blocks or the matrix: 127 (a factor of one)
+            const uint32_t ba = (kb < kb_hi && m < p.M) ? a_b[m * p.KB + kb] : 127u;
+            const uint32_t bb = (kb < kb_hi && n < p.N) ? b_b[(n >> 7) * p.KB + kb] : 127u;
+            xa |= ba << (8 * t);
+            xb |= bb << (8 * t);
+          }
+          wa[col] = xa;
+          wb[col] = xb;
+        }
+        tc_fence_after_sync();
+        const uint32_t col0 = t_row + static_cast<uint32_t>(kSfBase + slot * kSfSlotCols);
+        tmem_st_32x32b_x4(col0, wa);
+        tmem_st_32x32b_x4(col0 + 4, wb);
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(xfull0 + static_cast<uint32_t>(slot * 8));
+      }
+    }
   }
 
   // -------------------------------------------------------------- teardown
@@ -462,7 +573,7 @@ cudaError_t launch_pair_tc(const GemmLaunch& l) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = l.grid;
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(pair_threads(FMT), 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(l.smem_bytes);
   cfg.stream = l.stream;
   cudaLaunchAttribute attr[2];
@@ -489,7 +600,7 @@ int max_pairs(int smem_bytes) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(pair_threads(FMT), 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -515,7 +626,7 @@ cudaError_t launch_pair(const GemmLaunch& l, int tile_n) {
       default: return cudaErrorInvalidValue;
     }
   }
-  if constexpr (FMT == kFmtBlock) {
+  if constexpr (FMT == kFmtBlock || FMT == kFmtBlockE8m0) {
     if (tile_n == 128) return launch_pair_tc<FMT, 128, BIAS>(l);
   }
   return cudaErrorInvalidValue;

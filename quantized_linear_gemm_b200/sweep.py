@@ -114,7 +114,7 @@ def candidates(fmt, M, N, K):
                     if S <= T:
                         for st in (3, 4, 0):
                             add(swap_ab=0, tile_n=tn, split_k=S, stages=st, reduce=1, pdl=2)
-            if fmt == lq.BLOCK_FP8 and tn == 128:   # fp32-scale Block_FP8 on CTA pairs (256 x 128 tiles)
+            if fmt in (lq.BLOCK_FP8, lq.BLOCK_FP8_UE8M0) and tn == 128:   # Block_FP8 on CTA pairs (256 x 128 tiles)
                 for st in (4, 6, 0):
                     for pdl in (1, 2):
                         add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=2)
@@ -126,7 +126,7 @@ def candidates(fmt, M, N, K):
                             add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=2)
                             add(swap_ab=0, tile_n=tn, split_k=1, stages=st, pdl=pdl, persistent=3)
             # CTA pairs with Split-K where the 256-row tiles alone leave pairs idle
-            pair_ok = tn == 128 if fmt == lq.BLOCK_FP8 else (tn >= 128 and fmt != lq.BLOCK_FP8_UE8M0)
+            pair_ok = tn == 128 if fmt in (lq.BLOCK_FP8, lq.BLOCK_FP8_UE8M0) else tn >= 128
             tiles = -(-M // 256) * -(-N // tn)
             if pair_ok and tiles < PAIRS:
                 for S in range(2, 9):

@@ -149,6 +149,10 @@ def test_persistent_variant_rules():
         assert _mm(variant=lq.make_variant(**bad)) == INVALID, bad
     for fmt in (2, 3):
         assert _mm(fmt=fmt, K=256, N=256, variant=lq.make_variant(swap_ab=0, tile_n=128, persistent=1)) == INVALID
+        # Block_FP8 (fp32 or UE8M0 scales) on CTA pairs: 256 x 128 tiles only
+        ok = lq.make_variant(swap_ab=0, tile_n=128, persistent=2)
+        assert _mm(fmt=fmt, K=256, N=256, variant=ok, C=MISALIGNED) == ALIGN
+        assert _mm(fmt=fmt, K=256, N=256, variant=lq.make_variant(swap_ab=0, tile_n=256, persistent=2)) == INVALID
 
 
 def test_variant_tile_rules():

@@ -363,6 +363,84 @@ def test_block_pair_refuses_other_tiles(cuda_device):
                 dict(swap_ab=0, tile_n=128, persistent=3)):
         with pytest.raises(lq.LQError):
             lq.scaled_mm(fmt, A, sa, B, sb, variant=lq.make_variant(**bad))
+    ue = make_problem(lq.BLOCK_FP8_UE8M0, 256, 512, 512, seed=481)
+    A, sa, B, sb = ue.device()
+    with pytest.raises(lq.LQError):   # UE8M0 pairs: 256 x 128 tiles
+        lq.scaled_mm(lq.BLOCK_FP8_UE8M0, A, sa, B, sb, variant=lq.make_variant(swap_ab=0, tile_n=256, persistent=2))
+
+
+# ------------------------------------------ UE8M0 Block_FP8 on CTA pairs (persistent = 2, tile_n 128)
+def test_ue8m0_pair_against_oracle_and_one_sm(cuda_device):
+    """Block-scaled MMA over a CTA pair (each CTA's tensor memory holds the
+    scale factors of its own A rows and of all B rows of the tile, filled by
+    four scale-factor warps): ragged M = 300 (the second CTA's rows partly
+    past M) within tolerance of the oracle; M = 1100, N = 2048 with several
+    tiles per pair, scale-factor slots and both accumulators reused, on
+    sampled outputs; split 2 against the one-SM kernel's split 2 (the same K
+    blocks per split and the same reduction)."""
+    fmt = lq.BLOCK_FP8_UE8M0
+    prob = make_problem(fmt, 300, 1024, 1280, seed=490)
+    A, sa, B, sb = prob.device()
+    vp = lq.make_variant(swap_ab=0, tile_n=128, persistent=2)
+    C0 = lq.scaled_mm(fmt, A, sa, B, sb, variant=vp).clone()
+    C1 = lq.scaled_mm(fmt, A, sa, B, sb, variant=vp)
+    C2 = lq.scaled_mm(fmt, A, sa, B, sb, variant=lq.make_variant(swap_ab=0, tile_n=128, split_k=2, reduce=0,
+                                                                   persistent=2))
+    Cs = lq.scaled_mm(fmt, A, sa, B, sb, variant=lq.make_variant(swap_ab=0, tile_n=128, split_k=2, reduce=0))
+    torch.cuda.synchronize()
+    assert lq.device_status(0) == 0
+    assert torch.equal(C0, C1)
+    assert_close(C0, prob.reference(), "ue8m0 pair")
+    assert torch.equal(C2, Cs)
+    assert_close(C2, prob.reference(), "ue8m0 pair split 2")
+    big = make_problem(fmt, 1100, 2048, 1024, seed=491, outliers=False)
+    A, sa, B, sb = big.device()
+    Cb = lq.scaled_mm(fmt, A, sa, B, sb, variant=vp)
+    torch.cuda.synchronize()
+    assert lq.device_status(0) == 0
+    rows = np.array([0, 127, 128, 255, 256, 700, 1023, 1024, 1099])
+    cols = np.array([0, 7, 127, 128, 1023, 2047])
+    ok, worst = O.within_tolerance(Cb.float().cpu().numpy().astype(np.float64)[np.ix_(rows, cols)],
+                                   big.reference(rows, cols))
+    assert ok, worst
+
+
+@pytest.mark.parametrize("S", [3, 12])
+def test_ue8m0_pair_split_counts_bias_and_graph(cuda_device, S):
+    """Split 3, and split 12 over T = 10 K blocks (empty splits); bias with
+    and without Split-K; a graph replay gives the same bits."""
+    fmt = lq.BLOCK_FP8_UE8M0
+    prob = make_problem(fmt, 300, 1024, 1280, seed=495 + S)
+    A, sa, B, sb = prob.device()
+    v1 = lq.make_variant(swap_ab=0, tile_n=128, persistent=2)
+    vs = lq.make_variant(swap_ab=0, tile_n=128, split_k=S, reduce=0, persistent=2)
+    lq.reserve_workspace(0, lq.workspace_bytes(fmt, 300, 1024, 1280, vs))
+    C = lq.scaled_mm(fmt, A, sa, B, sb, variant=vs)
+    g = torch.Generator().manual_seed(496)
+    bias = (torch.randn(1024, generator=g) * 0.5).to(torch.bfloat16).cuda()
+    Cb1 = lq.scaled_mm_bias(fmt, A, sa, B, sb, bias, variant=v1)
+    Cbs = lq.scaled_mm_bias(fmt, A, sa, B, sb, bias, variant=vs)
+    torch.cuda.synchronize()
+    assert lq.device_status(0) == 0
+    assert_close(C, prob.reference(), f"ue8m0 pair split {S}")
+    refb = prob.reference() + bias.double().cpu().numpy()[None, :]
+    assert_close(Cb1, refb, "ue8m0 pair bias")
+    assert_close(Cbs, refb, f"ue8m0 pair split {S} bias")
+    out = torch.empty_like(C)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(gr, stream=s):
+            lq.scaled_mm(fmt, A, sa, B, sb, C=out, variant=vs, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(2):
+        out.zero_()
+        gr.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, C)
+    del gr
+    assert lq.device_status(0) == 0
 
 
 # --------------------------------------------------------------- stream-K (persistent = 3)
