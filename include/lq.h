@@ -119,8 +119,13 @@ typedef enum {
  *            overlaps the next tile's mainloop; 2 = the same on CTA pairs
  *            (clusters of two, one MMA of 256 rows over both SMs with
  *            tcgen05 cta_group::2; each CTA loads 128 rows of A and half of
- *            the tile's tile_n (128 or 256) weight rows).  Same results bit
- *            for bit.  Pairs also take split_k > 1 with reduce 0: the units
+ *            the tile's tile_n weight rows): FP8_DYNAMIC / W8A8_INT8 with
+ *            tile_n 128 or 256, and BLOCK_FP8 / BLOCK_FP8_UE8M0 with tile_n
+ *            128 (fp32 scales: promotion per 128-K block in four
+ *            tensor-memory buffers; UE8M0 scales: the tensor core's block
+ *            scaling over the pair).  Same results bit for bit as the one-SM
+ *            kernels with the same K grouping.  Pairs also take split_k > 1
+ *            with reduce 0: the units
  *            (256-row tile, split) are spread over the pairs and the
  *            separate reduction sums the workspace partials, as for the
  *            one-SM tiles; 3 = stream-K (tile_n 128 or 256): one CTA per SM,
