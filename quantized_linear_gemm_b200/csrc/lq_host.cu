@@ -391,14 +391,24 @@ bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, lq_variant* out) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
 
-// Dynamic shared memory of a CTA-pair launch.  A pair kernel that takes all
-// 512 tensor-memory columns (tile_n 256, or the four Block_FP8 buffers)
-// asks for at least 116 KB, so that two of its CTAs never share an SM and
-// never wait for each other's columns.
+// Dynamic shared memory of a launch whose CTAs each allocate `cols` tensor-
+// memory columns, raised where needed so that no more CTAs fit on an SM
+// (228 KB of shared memory, 1 KB reserved per CTA) than its 512 columns
+// hold.  A CTA's tcgen05.alloc waits until enough columns are free, so two
+// CTAs waiting for columns held by each other's cluster peers (Split-K
+// clusters, stream-K chains) would never proceed.
+int tmem_bounded_smem(int smem_bytes, int cols) {
+  if (cols <= 0 || cols >= 512) cols = 512;
+  const int fit = 512 / cols;                           // CTAs whose columns fit together
+  const int floor_bytes = (228 * 1024) / (fit + 1) - 1024 + 1;   // fit + 1 CTAs exceed the SM
+  return smem_bytes < floor_bytes ? floor_bytes : smem_bytes;
+}
+
+// Dynamic shared memory of a CTA-pair launch: the pair kernels that take all
+// 512 tensor-memory columns (tile_n 256, both Block_FP8 forms) never share an
+// SM with another of their CTAs, tile_n 128 pairs at most two.
 int pair_launch_smem(int fmt, int tile_n, int stages) {
-  const int bytes = lq::pair_smem_bytes_for(tile_n, stages);
-  const bool all_columns = tile_n == 256 || lq::is_block_fmt(fmt);
-  return all_columns && bytes < 116 * 1024 ? 116 * 1024 : bytes;
+  return tmem_bounded_smem(lq::pair_smem_bytes_for(tile_n, stages), lq::tmem_cols_per_cta(fmt, tile_n, 2));
 }
 
 // Grid of a CTA-pair launch: one pair per (256-row tile, split) unit, at most
@@ -556,18 +566,21 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
   }
   l.fuse = fused ? 1 : 0;
   l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
-  l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce, fused);
+  l.smem_bytes = tmem_bounded_smem(lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce, fused),
+                                   lq::tmem_cols_per_cta(fmt, v.tile_n, 0));
   if (v.persistent == 1) {   // one CTA per SM (at most one per tile), each looping over tiles
     const int64_t tiles = gx * gy;
     const int64_t ctas = tiles < sm_count() ? tiles : sm_count();
     l.grid = dim3(static_cast<unsigned>(ctas), 1, 1);
-    l.smem_bytes = lq::persistent_smem_bytes_for(v.tile_n, v.stages);
+    l.smem_bytes = tmem_bounded_smem(lq::persistent_smem_bytes_for(v.tile_n, v.stages),
+                                     lq::tmem_cols_per_cta(fmt, v.tile_n, 1));
     l.persistent = 1;
   } else if (v.persistent == 3) {   // stream-K: one CTA per SM splitting tiles x K blocks
     const int64_t iters = ((M + 127) / 128) * gy * p.T;
     const int64_t ctas = iters < sm_count() ? iters : sm_count();
     l.grid = dim3(static_cast<unsigned>(ctas), 1, 1);
-    l.smem_bytes = lq::persistent_smem_bytes_for(v.tile_n, v.stages);
+    l.smem_bytes = tmem_bounded_smem(lq::persistent_smem_bytes_for(v.tile_n, v.stages),
+                                     lq::tmem_cols_per_cta(fmt, v.tile_n, 3));
     l.persistent = 3;
   } else if (v.persistent == 2) {   // clusters of two CTAs, 256-row tiles, each pair looping over units
     l.smem_bytes = pair_launch_smem(fmt, v.tile_n, v.stages);
@@ -783,7 +796,8 @@ lq_status lq_grouped_scaled_mm(lq_fmt fmt_, const void* A, const float* a_scales
   p.num_experts = static_cast<int>(E);
   if (!encode_operand(&l.tmX, B, E * N, K, 128) || !encode_operand(&l.tmY, A, T, K, v.tile_n)) return LQ_ERR_CUDA;
   l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
-  l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce);
+  l.smem_bytes = tmem_bounded_smem(lq::gemm_smem_bytes_for(v.tile_n, v.stages, cluster_reduce),
+                                   lq::tmem_cols_per_cta(fmt, v.tile_n, 0));
   l.pdl = v.pdl != 0;
   l.cluster_z = cluster_reduce ? v.split_k : 1;
   l.grouped = 1;
@@ -1187,12 +1201,14 @@ extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const floa
       !encode_operand(&l.tmY, y_ptr, y_rows, K, v.persistent == 2 ? v.tile_n / 2 : v.tile_n))
     return LQ_ERR_CUDA;
   l.grid = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(v.split_k));
-  l.smem_bytes = lq::gemm_smem_bytes_for(v.tile_n, v.stages, false);
+  l.smem_bytes = tmem_bounded_smem(lq::gemm_smem_bytes_for(v.tile_n, v.stages, false),
+                                   lq::tmem_cols_per_cta(fmt, v.tile_n, 0));
   if (v.persistent == 1) {   // split_k 1: no scratch; one CTA per SM looping over tiles
     const int64_t tiles = gx * gy;
     const int64_t ctas = tiles < sm_count() ? tiles : sm_count();
     l.grid = dim3(static_cast<unsigned>(ctas), 1, 1);
-    l.smem_bytes = lq::persistent_smem_bytes_for(v.tile_n, v.stages);
+    l.smem_bytes = tmem_bounded_smem(lq::persistent_smem_bytes_for(v.tile_n, v.stages),
+                                     lq::tmem_cols_per_cta(fmt, v.tile_n, 1));
     l.persistent = 1;
   } else if (v.persistent == 2) {   // clusters of two CTAs, 256-row tiles, each pair looping over units
     l.smem_bytes = pair_launch_smem(fmt, v.tile_n, v.stages);

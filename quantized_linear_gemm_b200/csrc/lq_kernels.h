@@ -84,6 +84,9 @@ int pair_smem_bytes_for(int tile_n, int stages);
 int pair_capacity_fp8(int tile_n, bool bias, int smem_bytes);
 int pair_capacity_int8(int tile_n, bool bias, int smem_bytes);
 int pair_capacity_block(int tile_n, bool bias, int smem_bytes);        // tile_n 128
+// Tensor-memory columns one CTA allocates: the one-SM kernel (persistent 0),
+// the persistent and stream-K kernels (1, 3), CTA pairs (2: all 512).
+int tmem_cols_per_cta(int fmt, int tile_n, int persistent);
 int pair_capacity_block_e8m0(int tile_n, bool bias, int smem_bytes);   // tile_n 128
 
 // Quantization kernels (quant_kernels.cu).

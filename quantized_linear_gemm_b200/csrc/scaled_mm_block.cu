@@ -1,9 +1,33 @@
 // Block_FP8 instantiations of the scaled_mm kernel and the Split-K reduction.
+#include <type_traits>
+
 #include "scaled_mm_launch.cuh"
 namespace lq {
 cudaError_t launch_scaled_mm_block(const GemmLaunch& l, int swap_ab, int tile_n) {
   return launch_format<kFmtBlock>(l, swap_ab, tile_n);
 }
+int tmem_cols_per_cta(int fmt, int tile_n, int persistent) {
+  if (persistent == 1 || persistent == 3) return tmem_cols_for(2 * tile_n);   // two accumulators
+  if (persistent == 2) return (is_block_fmt(fmt) || tile_n == 256) ? 512 : 2 * tile_n;   // CTA pairs
+  auto one = [&](auto fmt_c) -> int {
+    constexpr int F = decltype(fmt_c)::value;
+    switch (tile_n) {
+      case 16: return tc_tmem_cols<F, 16>();
+      case 32: return tc_tmem_cols<F, 32>();
+      case 64: return tc_tmem_cols<F, 64>();
+      case 128: return tc_tmem_cols<F, 128>();
+      case 256: return tc_tmem_cols<F, 256>();
+      default: return 512;
+    }
+  };
+  switch (fmt) {
+    case kFmtFp8: return one(std::integral_constant<int, kFmtFp8>{});
+    case kFmtInt8: return one(std::integral_constant<int, kFmtInt8>{});
+    case kFmtBlock: return one(std::integral_constant<int, kFmtBlock>{});
+    default: return one(std::integral_constant<int, kFmtBlockE8m0>{});
+  }
+}
+
 int pair_capacity_block(int tile_n, bool bias, int smem_bytes) {
   return pair_capacity<kFmtBlock>(tile_n, bias, smem_bytes);
 }

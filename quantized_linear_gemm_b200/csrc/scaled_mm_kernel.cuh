@@ -77,6 +77,13 @@ struct MxSf {
 // are the ring's xfull / wfull entries).
 __device__ __forceinline__ int mx_slots(int stages) { return stages < 4 ? stages : 4; }
 
+// Tensor-memory columns one CTA of scaled_mm_tc_kernel<FMT, *, TN, ...>
+// allocates (the host bounds the CTAs per SM by them).
+template <int FMT, int TN>
+__host__ __device__ constexpr int tc_tmem_cols() {
+  return FMT == kFmtBlockE8m0 ? tmem_cols_for(MxSf<TN>::kEnd) : tmem_cols_for(TN * (FMT == kFmtBlock ? 2 : 1));
+}
+
 // Cluster Split-K reduction.  Tiles up to 64 wide push: every CTA sends its
 // partial columns, from registers, into slots in the shared memory of the
 // CTA that owns those columns (st.async, completion counted in bytes on the
@@ -199,7 +206,8 @@ __global__ void __launch_bounds__(kThreads, SWAP ? 2 : 1)   // Swap-AB: two CTAs
   constexpr bool kMX = FMT == kFmtBlockE8m0;
   constexpr bool kPromote = kBlocked && !kMX;
   constexpr int kAccBufs = kPromote ? 2 : 1;
-  constexpr int kTmemCols = kMX ? tmem_cols_for(MxSf<TN>::kEnd) : tmem_cols_for(TN * kAccBufs);
+  constexpr int kTmemCols = tc_tmem_cols<FMT, TN>();
+  static_assert(kTmemCols >= TN * kAccBufs, "tensor memory");
   constexpr int CH = TN < 32 ? TN : 32;   // TMEM columns per tcgen05.ld
 
   extern __shared__ uint8_t smem_raw[];
@@ -687,8 +695,33 @@ __global__ void __launch_bounds__(kThreads, SWAP ? 2 : 1)   // Swap-AB: two CTAs
         const int64_t n = y_row0 + e;
         return n < N ? b_b[(n >> 7) * p.KB + kb] : 127u;
       };
+      // A row's four bytes of a whole, 4-byte aligned group are one 32-bit
+      // load (a quarter of the load instructions and cache-line requests
+      // of byte loads, which share the L1 / shared-memory path with the MMA's
+      // operand reads); otherwise byte by byte.
+      const bool words = (p.KB & 3) == 0 && ((reinterpret_cast<uintptr_t>(a_b) | reinterpret_cast<uintptr_t>(b_b)) & 3u) == 0;
+      auto a_word = [&](int64_t m, int64_t kb0) -> uint32_t {
+        return m < M ? __ldg(reinterpret_cast<const uint32_t*>(a_b + m * p.KB + kb0)) : 0x7F7F7F7Fu;
+      };
+      auto b_word = [&](int64_t n, int64_t kb0) -> uint32_t {
+        return n < N ? __ldg(reinterpret_cast<const uint32_t*>(b_b + (n >> 7) * p.KB + kb0)) : 0x7F7F7F7Fu;
+      };
       uint32_t wx[Sf::kXCols], wy[Sf::kYCols];
       auto gather = [&](int g) {
+        const int64_t kb0 = kb_lo + 4 * g;
+        if (words && (kb0 & 3) == 0 && 4 * g + 4 <= nkb) {
+#pragma unroll
+          for (int col = 0; col < Sf::kXCols; ++col) {
+            const int e = col * 32 + lane;
+            wx[col] = SWAP ? b_word(x_row0 + e, kb0) : a_word(x_row0 + e, kb0);
+          }
+#pragma unroll
+          for (int col = 0; col < Sf::kYCols; ++col) {
+            const int e = col * 32 + lane;
+            wy[col] = e >= TN ? 0x7F7F7F7Fu : (SWAP ? a_word(y_row0 + e, kb0) : b_word(y_row0 + e, kb0));
+          }
+          return;
+        }
 #pragma unroll
         for (int col = 0; col < Sf::kXCols; ++col) {
           uint32_t w = 0;
