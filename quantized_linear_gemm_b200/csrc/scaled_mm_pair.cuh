@@ -504,6 +504,7 @@ __global__ void __launch_bounds__(pair_threads(FMT), 1)
     const uint32_t xfull0 = dsmem_map(smem_addr(c.xfull), 0);   // the first CTA's xfull[0]
     const uint8_t* a_b = reinterpret_cast<const uint8_t*>(p.a_s);   // [M, KB]
     const uint8_t* b_b = reinterpret_cast<const uint8_t*>(p.b_s);   // [N / 128, KB]
+    const bool words = (p.KB & 3) == 0 && ((reinterpret_cast<uintptr_t>(a_b) | reinterpret_cast<uintptr_t>(b_b)) & 3u) == 0;
     bool ok = true;
     int64_t group = -1;
     for (int64_t j = 0; j < my_tiles && ok; ++j) {
@@ -520,10 +521,17 @@ __global__ void __launch_bounds__(pair_threads(FMT), 1)
           if (!ok) break;
         }
         uint32_t wa[4], wb[4];
+        // a row's four bytes as one 32-bit load where the group is whole and aligned
+        const bool word = words && (kb0 & 3) == 0 && kb0 + 4 <= kb_hi;
 #pragma unroll
         for (int col = 0; col < 4; ++col) {
           const int64_t m = m0 + rank * kTileM + col * 32 + lane;
           const int64_t n = n0 + col * 32 + lane;
+          if (word) {
+            wa[col] = m < p.M ? __ldg(reinterpret_cast<const uint32_t*>(a_b + m * p.KB + kb0)) : 0x7F7F7F7Fu;
+            wb[col] = n < p.N ? __ldg(reinterpret_cast<const uint32_t*>(b_b + (n >> 7) * p.KB + kb0)) : 0x7F7F7F7Fu;
+            continue;
+          }
           uint32_t xa = 0, xb = 0;
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
