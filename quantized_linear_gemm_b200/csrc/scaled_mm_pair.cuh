@@ -332,6 +332,9 @@ __global__ void __launch_bounds__(pair_threads(FMT), 1)
       // Block scale products of this thread's row, a group of kPre K blocks
       // ahead (the loads' latency hides behind a group of promotions).
       constexpr int kPre = 8;
+      static_assert(kPre == 8, "two float4 scale loads per group");
+      const bool vec_scales = (p.KB & 3) == 0 &&
+                              ((reinterpret_cast<uintptr_t>(p.a_s) | reinterpret_cast<uintptr_t>(p.b_s)) & 15u) == 0;
       int64_t g = 0;   // running K block over all units: buffer g mod kNBuf
       for (int64_t j = 0; j < my_tiles; ++j) {
         int64_t m0, n0;
@@ -347,15 +350,36 @@ __global__ void __launch_bounds__(pair_threads(FMT), 1)
           const float sb = __ldg(p.b_s + nb * p.KB + kb);
           return (m < p.M ? __ldg(p.a_s + m * p.KB + kb) : 0.f) * sb;
         };
+        // The kPre products of blocks i .. i + kPre - 1: where the group lies
+        // inside the unit and its first block is 16-byte aligned, a row's
+        // scales come as two float4 loads (a quarter of the load requests,
+        // each warp instruction touching one cache line per row, on the L1 /
+        // shared-memory path the MMA's operands use).  The same products.
+        auto load_group = [&](int i, float (&out)[kPre]) {
+          const int64_t kb0 = kb_lo + i;
+          if (vec_scales && (kb0 & 3) == 0 && i + kPre <= nkb) {
+            const float4* bp = reinterpret_cast<const float4*>(p.b_s + nb * p.KB + kb0);
+            const float4 b0 = __ldg(bp), b1 = __ldg(bp + 1);
+            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+            if (m < p.M) {
+              const float4* ap = reinterpret_cast<const float4*>(p.a_s + m * p.KB + kb0);
+              a0 = __ldg(ap);
+              a1 = __ldg(ap + 1);
+            }
+            out[0] = a0.x * b0.x; out[1] = a0.y * b0.y; out[2] = a0.z * b0.z; out[3] = a0.w * b0.w;
+            out[4] = a1.x * b1.x; out[5] = a1.y * b1.y; out[6] = a1.z * b1.z; out[7] = a1.w * b1.w;
+            return;
+          }
+#pragma unroll
+          for (int e = 0; e < kPre; ++e) out[e] = load_scale(i + e);
+        };
         float accr[TN];
 #pragma unroll
         for (int e = 0; e < TN; ++e) accr[e] = 0.f;
         float cur[kPre], nxt[kPre];
-#pragma unroll
-        for (int e = 0; e < kPre; ++e) cur[e] = load_scale(e);
+        load_group(0, cur);
         for (int i0 = 0; i0 < nkb; i0 += kPre) {
-#pragma unroll
-          for (int e = 0; e < kPre; ++e) nxt[e] = load_scale(i0 + kPre + e);
+          load_group(i0 + kPre, nxt);
 #pragma unroll
           for (int e = 0; e < kPre; ++e) {
             if (i0 + e < nkb) {   // the same for every epilogue thread
