@@ -187,7 +187,8 @@ typedef struct {
  *   stream   : CUDA stream.
  *
  * Errors: LQ_ERR_INVALID_ARG / LQ_ERR_ALIGNMENT / LQ_ERR_UNSUPPORTED_SHAPE
- * before any launch; LQ_ERR_WORKSPACE when split_k > 1 needs a larger
+ * before any launch (an explicit variant is checked first, before the
+ * pointers and sizes); LQ_ERR_WORKSPACE when split_k > 1 needs a larger
  * workspace while `stream` is capturing; LQ_ERR_CUDA when a launch fails.
  * A Split-K call with reduce 0 or 1 uses the library's per-device workspace:
  * such calls on different streams of one device must not overlap in time on

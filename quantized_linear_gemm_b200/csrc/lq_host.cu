@@ -481,7 +481,12 @@ lq_status scaled_mm_impl(int fmt, const void* A, const float* a_s, const void* B
                          cudaStream_t stream, const void* x_fused = nullptr, void* codes_out = nullptr,
                          float* scales_out = nullptr, const void* bias = nullptr) {
   const bool fused = x_fused != nullptr;
-  lq_status rc = fused ? LQ_OK : check_gemm_args(fmt, A, a_s, B, b_s, C, M, N, K);
+  lq_status rc = LQ_OK;
+  if (!fused && variant && fmt >= 0 && fmt <= 3) {   // an explicit variant is checked before the pointers
+    rc = check_variant(fmt, *variant);
+    if (rc != LQ_OK) return rc;
+  }
+  rc = fused ? LQ_OK : check_gemm_args(fmt, A, a_s, B, b_s, C, M, N, K);
   if (rc != LQ_OK) return rc;
   if (acc_out && !aligned(acc_out, 16)) return LQ_ERR_ALIGNMENT;
   if (M == 0 || N == 0) return LQ_OK;
@@ -1142,18 +1147,26 @@ extern "C" lq_status lq_scaled_mm_noalloc(lq_fmt fmt_, const void* A, const floa
                                           const lq_variant* variant, lq_stream_t stream_) {
   const int fmt = static_cast<int>(fmt_);
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  lq_status rc = check_gemm_args(fmt, A, a_scales, B, b_scales, C, M, N, K);
+  // Split-K partials always go through the scratch array and the separate
+  // fixed-order reduction kernel (no arrival counters, nothing to re-arm);
+  // stream-K, whose partials need a workspace, runs as persistent CTAs.
+  auto noalloc_form = [](lq_variant v) {
+    if (v.split_k > 1) v.reduce = 0;
+    if (v.persistent == 3) v.persistent = 1;
+    return v;
+  };
+  lq_status rc = LQ_OK;
+  if (variant && fmt >= 0 && fmt <= 3) {   // an explicit variant is checked before the pointers
+    rc = check_variant(fmt, noalloc_form(*variant));
+    if (rc != LQ_OK) return rc;
+  }
+  rc = check_gemm_args(fmt, A, a_scales, B, b_scales, C, M, N, K);
   if (rc != LQ_OK) return rc;
   if (M == 0 || N == 0) return LQ_OK;
   if (K == 0)
     return lq::launch_fill_zero_bf16(static_cast<__nv_bfloat16*>(C), M * N, stream) == cudaSuccess ? LQ_OK
                                                                                                   : LQ_ERR_CUDA;
-  lq_variant v = variant ? *variant : default_variant(fmt, M, N, K);
-  // Split-K partials always go through the scratch array and the separate
-  // fixed-order reduction kernel (no arrival counters, nothing to re-arm);
-  // stream-K, whose partials need a workspace, runs as persistent CTAs.
-  if (v.split_k > 1) v.reduce = 0;
-  if (v.persistent == 3) v.persistent = 1;
+  lq_variant v = noalloc_form(variant ? *variant : default_variant(fmt, M, N, K));
   rc = check_variant(fmt, v);
   if (rc != LQ_OK) return rc;
   const size_t need = v.split_k > 1 ? static_cast<size_t>(v.split_k) * static_cast<size_t>(M) *

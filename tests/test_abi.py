@@ -116,6 +116,22 @@ def test_variant_checks(field, value):
     assert _mm(variant=v) == INVALID
 
 
+def test_explicit_variant_is_checked_before_the_pointers():
+    """So that a valid variant with a misaligned C reports the pointer
+    (LQ_ERR_ALIGNMENT: the variant was accepted) and an invalid one reports
+    the variant whatever the pointers; the same for the allocation-free
+    entry point, which applies its own reduction first."""
+    bad = lq.make_variant(swap_ab=1, split_k=3, tile_n=16, reduce=2)
+    good = lq.make_variant(swap_ab=1, split_k=3, tile_n=16, reduce=1)
+    assert _mm(variant=bad, C=MISALIGNED) == INVALID
+    assert _mm(variant=good, C=MISALIGNED) == ALIGN
+    assert _mm(variant=bad, A=None) == INVALID
+    f = lq.lib().lq_scaled_mm_noalloc
+    assert f(0, FAKE, FAKE, FAKE, FAKE, MISALIGNED, 16, 128, 128, ctypes.byref(bad), None) == ALIGN   # reduce 0 there
+    worse = lq.make_variant(swap_ab=1, split_k=2, tile_n=48)
+    assert f(0, FAKE, FAKE, FAKE, FAKE, MISALIGNED, 16, 128, 128, ctypes.byref(worse), None) == INVALID
+
+
 def test_split_counts_by_reduction():
     """Any split count 1..256 with the workspace reductions (0, 1); powers of
     two (at most 16) with the cluster reduction."""
